@@ -1,0 +1,193 @@
+/*
+ * loopvq_oracle.c -- CPU checker for the LoopVQ encode / decode-attention path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or constant with the CUDA library, and the CUDA library never
+ * calls it.
+ *
+ * It states what the method computes in the most direct way: plain loops, one
+ * element at a time, in the order the definitions are written.
+ *
+ *   encode     nearest codebook entry of each coupled sub-vector, squared
+ *              distance accumulated in fp32 over the coordinates in ascending
+ *              order, first (lowest) index kept on ties.
+ *              LoopVQ paper, Sec. 2 "Vector quantization of the KV cache",
+ *              eq. (2); Sec. 4.1 "Loop-axis vector quantization", eq. (4).
+ *   dequant    loop step m of a block copies coordinate i*Tc + m of the
+ *              selected entry into channel g*c + i, for i < c.
+ *              LoopVQ paper, Sec. 4.1 eq. (5); Sec. 4.3 "Attention"; App. A.2.
+ *   rope       half-split rotary embedding in fp64 applied to reconstructed
+ *              keys only, pairs (f, f + D/2), angle p * theta^(-2f/D).
+ *              LoopVQ paper, Sec. 2 (keys quantized before RoPE); App. C.
+ *   attention  softmax attention of one query over the reconstructed cache in
+ *              fp64, two passes (max, then sum); lse = max + ln(sum).
+ *              LoopVQ paper, Sec. 4.3 "Attention".
+ *   splits     the same attention computed per split of the tokens and merged
+ *              through the log-sum-exp of each split (Flash-Decoding merge),
+ *              which the pages state recovers the exact softmax.
+ *              LoopVQ paper, Sec. 4.3 "Attention".
+ *
+ * Array conventions (all dense, row-major, caller-owned):
+ *   x   float  [Tc][N][D]   one block of Tc loop steps of one (layer, head, K|V)
+ *   E   float  [K][G]       codebook, G = c*Tc, coordinate i*Tc + m
+ *   idx uint8  [N][D/c]     code of channel group g (channels g*c .. g*c+c-1)
+ *   q   double [D]          query, already rotated at its own position
+ * Inputs that are bf16 in the method are passed as the exactly widened floats.
+ *
+ * Parity pins live in tests/test_oracle_pins.py; every function here is pinned
+ * there by a check that does not re-use this file's arithmetic.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+/* Coupled vector of token n, channel group g (eq. 4):
+ *   z[i*Tc + m] = x[m][n][g*c + i],  i < c, m < Tc. */
+static void coupled_vector(const float *x, int Tc, int N, int D, int c, int n, int g, float *z)
+{
+    for (int i = 0; i < c; ++i)
+        for (int m = 0; m < Tc; ++m)
+            z[i * Tc + m] = x[((size_t)m * N + n) * D + (size_t)g * c + i];
+}
+
+/* Nearest entry (eq. 2) of every coupled vector; fp32 distances, lowest index on ties. */
+void ora_encode(const float *x, int Tc, int N, int D, int c, const float *E, int K, uint8_t *idx)
+{
+    const int G = c * Tc;
+    const int ng = D / c;
+    float z[256];
+    for (int n = 0; n < N; ++n) {
+        for (int g = 0; g < ng; ++g) {
+            coupled_vector(x, Tc, N, D, c, n, g, z);
+            int best = 0;
+            float best_d = INFINITY;
+            for (int r = 0; r < K; ++r) {
+                float d = 0.0f;
+                for (int k = 0; k < G; ++k) {
+                    float diff = z[k] - E[(size_t)r * G + k];
+                    float sq = diff * diff;
+                    d = d + sq;
+                }
+                if (d < best_d) { best_d = d; best = r; }
+            }
+            idx[(size_t)n * ng + g] = (uint8_t)best;
+        }
+    }
+}
+
+/* fp64 squared distance between coupled vector (n, g) and entry r; used to judge near-ties. */
+double ora_dist64(const float *x, int Tc, int N, int D, int c, const float *E, int n, int g, int r)
+{
+    const int G = c * Tc;
+    float z[256];
+    coupled_vector(x, Tc, N, D, c, n, g, z);
+    double d = 0.0;
+    for (int k = 0; k < G; ++k) {
+        double diff = (double)z[k] - (double)E[(size_t)r * G + k];
+        d += diff * diff;
+    }
+    return d;
+}
+
+/* Reconstruction of loop step m of the block (eq. 5): out[n][g*c + i] = E[idx[n][g]][i*Tc + m]. */
+void ora_dequant(const uint8_t *idx, int N, int D, int c, int Tc, int m, const float *E, double *out)
+{
+    const int G = c * Tc;
+    const int ng = D / c;
+    for (int n = 0; n < N; ++n)
+        for (int g = 0; g < ng; ++g) {
+            int r = idx[(size_t)n * ng + g];
+            for (int i = 0; i < c; ++i)
+                out[(size_t)n * D + (size_t)g * c + i] = (double)E[(size_t)r * G + i * Tc + m];
+        }
+}
+
+/* Half-split RoPE in fp64 at positions pos0 + n (App. C; pairs (f, f + D/2)). */
+void ora_rope(double *x, int N, int D, double theta, int pos0)
+{
+    const int h = D / 2;
+    for (int n = 0; n < N; ++n) {
+        double p = (double)(pos0 + n);
+        for (int f = 0; f < h; ++f) {
+            double omega = pow(theta, -2.0 * (double)f / (double)D);
+            double ang = p * omega;
+            double cs = cos(ang), sn = sin(ang);
+            double a = x[(size_t)n * D + f];
+            double b = x[(size_t)n * D + f + h];
+            x[(size_t)n * D + f] = a * cs - b * sn;
+            x[(size_t)n * D + f + h] = b * cs + a * sn;
+        }
+    }
+}
+
+/* Softmax attention of q over N keys/values in fp64, two passes.  N == 0 gives out = 0, lse = -inf. */
+void ora_attention(const double *q, const double *k, const double *v, int N, int D, double scale,
+                   double *out, double *lse)
+{
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    if (N <= 0) { *lse = -INFINITY; return; }
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double mx = -INFINITY;
+    for (int n = 0; n < N; ++n) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += q[d] * k[(size_t)n * D + d];
+        s[n] = dot * scale;
+        if (s[n] > mx) mx = s[n];
+    }
+    double sum = 0.0;
+    for (int n = 0; n < N; ++n) {
+        double p = exp(s[n] - mx);
+        sum += p;
+        for (int d = 0; d < D; ++d) out[d] += p * v[(size_t)n * D + d];
+    }
+    for (int d = 0; d < D; ++d) out[d] /= sum;
+    *lse = mx + log(sum);
+    free(s);
+}
+
+/* The same attention split at bounds[0] = 0 < ... < bounds[nsplit] = N: each split is attended on its
+ * own, giving (out_s, lse_s); the splits are merged by weights exp(lse_s - max_s lse_s). */
+void ora_attention_splits(const double *q, const double *k, const double *v, int N, int D, double scale,
+                          const int *bounds, int nsplit, double *out, double *lse)
+{
+    double *os = (double *)malloc(sizeof(double) * (size_t)D * (size_t)(nsplit > 0 ? nsplit : 1));
+    double *ls = (double *)malloc(sizeof(double) * (size_t)(nsplit > 0 ? nsplit : 1));
+    double mx = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) {
+        int a = bounds[s], b = bounds[s + 1];
+        ora_attention(q, k + (size_t)a * D, v + (size_t)a * D, b - a, D, scale, os + (size_t)s * D, &ls[s]);
+        if (ls[s] > mx) mx = ls[s];
+    }
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    if (mx == -INFINITY) { *lse = -INFINITY; free(os); free(ls); return; }
+    double wsum = 0.0;
+    for (int s = 0; s < nsplit; ++s) {
+        if (ls[s] == -INFINITY) continue;
+        double w = exp(ls[s] - mx);
+        wsum += w;
+        for (int d = 0; d < D; ++d) out[d] += w * os[(size_t)s * D + d];
+    }
+    for (int d = 0; d < D; ++d) out[d] /= wsum;
+    *lse = mx + log(wsum);
+    free(os);
+    free(ls);
+}
+
+/* Decode attention of one query at loop step m of a block over a coded cache of N tokens
+ * (Sec. 4.3): reconstruct keys (eq. 5), rotate them at positions 0..N-1, reconstruct values,
+ * attend.  Scratch is allocated here; the checker is not a hot path. */
+void ora_decode(const double *q, const uint8_t *idx_k, const uint8_t *idx_v, const float *E_k,
+                const float *E_v, int N, int D, int c, int Tc, int m, double theta, double scale,
+                double *out, double *lse)
+{
+    size_t nd = (size_t)(N > 0 ? N : 1) * (size_t)D;
+    double *kh = (double *)malloc(sizeof(double) * nd);
+    double *vh = (double *)malloc(sizeof(double) * nd);
+    ora_dequant(idx_k, N, D, c, Tc, m, E_k, kh);
+    ora_rope(kh, N, D, theta, 0);
+    ora_dequant(idx_v, N, D, c, Tc, m, E_v, vh);
+    ora_attention(q, kh, vh, N, D, scale, out, lse);
+    free(kh);
+    free(vh);
+}
