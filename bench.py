@@ -1,0 +1,364 @@
+#!/usr/bin/env python
+"""Benchmark of the LoopVQ decode hot path on B200.
+
+A step is one decode step of the looped model over the whole batch: decode
+attention for every (loop step, layer), loop-step-major as the looped forward
+runs them (T x L calls of loopvq_decode_attn), against a cache that was
+encoded on the GPU (loopvq_encode) from seeded synthetic keys and values.
+
+Default workload (ctx32k): 24 layers, 16 KV / 16 query heads of dimension 128,
+4 loop steps coded as one block, c = 4 (G = 16, K = 256: 0.5 bit per element),
+batch 8, 32768-token cache, per-sequence lengths uniform in [16384, 32768].
+
+The JSON line reports algorithmic cache bytes per second (whole job), the time
+per step and per call, the roofline of the dominant call, the clocks seen while
+timing, an end-to-end figure through the public API with host buffers, and the
+CPU checker timed on a bounded sample as a reported baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl loopvq|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, lengths, random_indices, queries, bf16_bits_to_f32, codebook  # noqa: E402
+
+METRIC = "LoopVQ decode-attn µs/step & GB/s at 32K ctx, 0.5 bit; % of roofline"
+SMEM_BYTES_PER_CLK_SM = 128
+N_SM = 148
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="ctx32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="loopvq", choices=["loopvq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def workload_desc(w):
+    return {
+        "workload": f"{w.name}: looped decoder, {w.L} layers x {w.T} loop steps (blocks of {w.Tc}), "
+                    f"{w.Hkv} KV / {w.Hq} q heads, D={w.D}, c={w.c} (G={w.G}, K={w.K}, {8 / w.G:g} bit), "
+                    f"batch {w.B}, cache {w.Nmax} tokens",
+        "batch": w.B, "context": w.Nmax,
+        "lengths": (f"uniform in [{w.len_lo}, {w.Nmax}] (seeded)" if w.len_lo >= 0 else "all full"),
+        "layers": w.L, "loop_steps": w.T, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
+        "bits_per_element": 8 / w.G,
+        "l2": "inputs larger than L2: every call streams its layer's index words (> 126 MB), "
+              "successive calls touch different layers",
+    }
+
+
+def call_bytes(w, lens):
+    """Algorithmic bytes of one decode call: index words, codebook slices, query, output, lse."""
+    idx = int(np.sum(lens)) * w.Hkv * 2 * (w.D // w.c)
+    slices = 2 * w.Hkv * w.K * w.c * 2
+    q = w.B * w.Hq * w.D * 2
+    out = w.B * w.Hq * w.D * 4 + w.B * w.Hq * 4
+    return idx + slices + q + out
+
+
+def gather_bytes(w, lens):
+    """Shared-memory gather bytes of one call: D bf16 key and D bf16 value per token and KV head."""
+    return int(np.sum(lens)) * w.Hkv * 2 * w.D * 2
+
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.f = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except FileNotFoundError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        self.p.wait()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def cpu_sample(w, seconds, layer=0, t=1):
+    """Time the CPU checker's decode on (sequence, query head) units of one call until `seconds` pass.
+    Codes for the sampled units are regenerated uniform codes of the same shape (the checker's
+    work does not depend on code values); regeneration is not timed."""
+    from oracle import oracle as O
+    lens = lengths(w)
+    blk, m = t // w.Tc, t % w.Tc
+    qpk = w.Hq // w.Hkv
+    total_s, nbytes, units = 0.0, 0, 0
+    order = [(b, hq) for b in range(w.B) for hq in range(w.Hq)]
+    for b, hq in order:
+        h = hq // qpk
+        n = int(lens[b])
+        ik = random_indices(w, layer, blk, 0, b, h, range(n))
+        iv = random_indices(w, layer, blk, 1, b, h, range(n))
+        q = bf16_bits_to_f32(queries(w, layer, t, b=[b], hq=[hq])[0, 0]).astype(np.float64)
+        Ek = bf16_bits_to_f32(codebook(w, layer, blk, 0, h))
+        Ev = bf16_bits_to_f32(codebook(w, layer, blk, 1, h))
+        t0 = time.perf_counter()
+        O.decode(q, ik, iv, Ek, Ev, w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        total_s += time.perf_counter() - t0
+        nbytes += n * 2 * (w.D // w.c)
+        units += 1
+        if total_s >= seconds:
+            break
+    return total_s, nbytes, units
+
+
+def run_reference(args):
+    """The CPU checker as the reference arm: each step decodes a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    per_step = max(0.2, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_sample(w, per_step)
+    tot_s, tot_b, tot_u = 0.0, 0, 0
+    for _ in range(args.steps):
+        s, b, u = cpu_sample(w, per_step)
+        tot_s, tot_b, tot_u = tot_s + s, tot_b + b, tot_u + u
+    gbs = tot_b / tot_s / 1e9
+    sample = (f"{tot_u} (sequence, query head) units of the layer-0, loop-step-2 call over {args.steps} steps; "
+              f"fp64 dequant, RoPE and softmax per unit; single thread")
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_desc(w),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import looped_lm_decode_b200 as LQ
+    from synth import gpu as SG
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+
+    # ---------------- set-up: codebooks, slices, RoPE table, GPU encode of every (layer, block)
+    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, device=dev)
+    SG.fill_codebook(w, cache.codebook)
+    LQ.prepare(cache)
+    xk = torch.empty((w.Tc, w.B, w.Nmax, w.Hkv, w.D), dtype=torch.bfloat16, device=dev)
+    xv = torch.empty_like(xk)
+    enc_ms = []
+    for layer in range(w.L):
+        for blk in range(w.NB):
+            SG.fill_kv(w, layer, 0, blk * w.Tc, blk * w.Tc + w.Tc - 1, xk)
+            SG.fill_kv(w, layer, 1, blk * w.Tc, blk * w.Tc + w.Tc - 1, xv)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            LQ.encode(cache, layer, blk, xk, xv)
+            e1.record()
+            torch.cuda.synchronize()
+            enc_ms.append(e0.elapsed_time(e1))
+    del xk, xv
+    torch.cuda.empty_cache()
+
+    lens_np = lengths(w)
+    lens = torch.from_numpy(lens_np).to(dev)
+    max_len = int(lens_np.max())
+    ncall = w.L * w.T
+    qs = torch.empty((ncall, w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    for t in range(w.T):
+        for layer in range(w.L):
+            SG.fill_q(w, layer, t, qs[t * w.L + layer])
+    out = torch.empty((ncall, w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+    lse = torch.empty((ncall, w.B, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(LQ.decode_workspace_bytes(cache, max_len), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        for t in range(w.T):
+            for layer in range(w.L):
+                i = t * w.L + layer
+                if evs is not None:
+                    evs[2 * i].record(stream)
+                LQ.decode_attn(cache, layer, t, qs[i], lens, max_len, 0.0, out=out[i], lse=lse[i], workspace=ws,
+                               stream=stream)
+                if evs is not None:
+                    evs[2 * i + 1].record(stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    call_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * ncall)] for _ in range(args.steps)]
+    clocks = Clocks(local)
+    barrier()
+    clocks.start()
+    time.sleep(0.3)                       # let the sampler start before the timed region
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(call_evs[k])
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    call_ms = [call_evs[k][2 * i].elapsed_time(call_evs[k][2 * i + 1])
+               for k in range(args.steps) for i in range(ncall)]
+    ms_step_local = ms_total / args.steps
+
+    # ---------------- end to end through the public API with host buffers
+    q_host = torch.empty(qs.shape, dtype=qs.dtype, pin_memory=True)
+    q_host.copy_(qs)
+    lens_host = torch.from_numpy(lens_np.copy()).pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        qs.copy_(q_host, non_blocking=True)
+        lens.copy_(lens_host, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    barrier()
+    e2e_ms_local = a0.elapsed_time(a1) / e2e_steps
+    h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * 4
+    d2h = out_host.numel() * 4 + lse_host.numel() * 4
+
+    def allmax(x):
+        if dist is None:
+            return x
+        tt = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        return float(tt.item())
+
+    ms_step = allmax(ms_step_local)
+    e2e_ms = allmax(e2e_ms_local)
+    avg_call_ms = allmax(statistics.fmean(call_ms))
+
+    if rank == 0:
+        cb = call_bytes(w, lens_np)
+        gb = gather_bytes(w, lens_np)
+        step_bytes = cb * ncall
+        value = world * step_bytes / (ms_step * 1e-3) / 1e9
+        hbm_peak, peak_kind = peaks()
+        achieved = cb / (avg_call_ms * 1e-3) / 1e9
+        sm_mhz = clk.get("sm_mhz") or 1965.0
+        smem_peak = SMEM_BYTES_PER_CLK_SM * N_SM * sm_mhz * 1e6 / 1e9
+        smem_achieved = gb / (avg_call_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": dict(workload_desc(w), parallelism=("replicas" if world > 1 else "single GPU")),
+            "us_per_step": ms_step * 1e3, "us_per_call": avg_call_ms * 1e3, "calls_per_step": ncall,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "one loopvq_decode_attn call (split kernel + merge kernel)",
+                         "bytes_per_launch": cb},
+            "smem_gather": {"achieved": smem_achieved, "peak": smem_peak, "unit": "GB/s",
+                            "frac": smem_achieved / smem_peak, "bytes_per_launch": gb,
+                            "peak_kind": f"derived: {SMEM_BYTES_PER_CLK_SM} B/clk/SM x {N_SM} SMs x median SM clock"},
+            "clocks": clk,
+            "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps * ncall * 2,
+            "encode": {"ms_per_layer_block": statistics.median(enc_ms),
+                       "tokens_per_s": w.B * w.Nmax / (statistics.median(enc_ms) * 1e-3),
+                       "input_gbs": 2 * w.Tc * w.B * w.Nmax * w.Hkv * w.D * 2 / (statistics.median(enc_ms) * 1e-3) / 1e9,
+                       "kernel": "encode_direct (fp32 exact argmin on CUDA cores)"},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            s, nb, u = cpu_sample(w, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": nb / s / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"{u} (sequence, query head) units of the layer-0, loop-step-2 call, "
+                                              f"{s:.1f} s single-threaded"}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * loopvq.h -- C ABI of the LoopVQ hot path on B200 (sm_100a).
+ *
+ * LoopVQ codes a looped transformer's KV cache along the loop axis: a coupled
+ * sub-vector takes the same c channels from each of the Tc loop steps of a
+ * block, G = c*Tc elements, and is stored as the index of its nearest entry in
+ * a K-entry codebook, b/G bits per element, one index shared by the Tc loop
+ * steps.  Decode attention at loop step t reads the shared indices through
+ * that step's slice of the codebook, applies RoPE to the rebuilt keys and runs
+ * split-K online-softmax attention merged by log-sum-exp.
+ *   LoopVQ paper ("LoopVQ: Sub 1-bit KV Cache Quantization for Looped
+ *   Transformers"), Sec. 2 eq. (2); Sec. 4.1 eq. (4)-(5); Sec. 4.3
+ *   "Cache layout", "Encoding", "Attention"; App. C.
+ *
+ * Conventions for every call:
+ *   - Pointers named in loopvq_cache and every array argument are DEVICE
+ *     memory owned by the caller, unless the argument says otherwise.  The
+ *     library allocates nothing on any call.
+ *   - Calls are asynchronous on the caller's CUDA stream (cudaStream_t passed
+ *     as void*; NULL is the legacy default stream).  No call synchronises.
+ *   - Arguments are validated on the host before any launch; a failed check
+ *     returns a status and launches nothing.  loopvq_last_error() then gives a
+ *     message (thread-local, valid until the next call on this thread).
+ *   - A CUDA launch error returns LOOPVQ_ERR_CUDA with the CUDA error string.
+ *
+ * Supported shapes: D in {64, 128}; c in {4, 8}; Tc in {1, 2, 4} with
+ * G = c*Tc <= 32; 1 <= K <= 256; Hq a multiple of Hkv with Hq/Hkv in
+ * {1, 2, 4, 8}; T a multiple of Tc; Nmax a multiple of 4.
+ */
+#ifndef LOOPVQ_H
+#define LOOPVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LOOPVQ_OK = 0,
+    LOOPVQ_ERR_INVALID_ARG = 1,   /* null pointer, out-of-range index or size */
+    LOOPVQ_ERR_UNSUPPORTED = 2,   /* valid but not built: D, c, Tc, Hq/Hkv outside the supported set */
+    LOOPVQ_ERR_WORKSPACE = 3,     /* workspace missing or smaller than loopvq_decode_workspace_bytes */
+    LOOPVQ_ERR_CUDA = 4           /* a launch failed; loopvq_last_error() holds the CUDA message */
+} loopvq_status;
+
+enum { LOOPVQ_BF16 = 0, LOOPVQ_FP32 = 1 };
+
+/*
+ * The coded cache of one model (all layers), described by shape and by four
+ * caller-owned device buffers.  NB = T / Tc blocks, NP = D / (2c) pair-groups.
+ *
+ * idx       uint32 words, [L][NB][B][Hkv][Nmax/4][NP][4].  Word (token n,
+ *           pair-group p) sits at tile n/4, slot n%4 and packs four 8-bit
+ *           codes: byte0 = K code of channel group p, byte1 = K code of group
+ *           p + NP (the group holding the RoPE partners of group p), byte2 =
+ *           V code of group p, byte3 = V code of group p + NP.  Channel group
+ *           g covers channels g*c .. g*c+c-1.  One word serves all Tc loop
+ *           steps of its block (Sec. 4.3 "Cache layout": one index row per
+ *           block).  2*D/c bytes per token, head and block.
+ * codebook  bf16 [L][NB][2][Hkv][K][G], 2 = {K, V}; coordinate i*Tc + m of an
+ *           entry belongs to channel i at loop step m of the block (eq. 4).
+ *           One codebook per (layer, block, KV head, K|V), shared by all
+ *           channel groups.
+ * slices    bf16 [L][T][2][Hkv][K][c]: loop step t = beta*Tc + m keeps
+ *           coordinates i*Tc + m, i < c, of every entry (Sec. 4.3 "Attention":
+ *           the slice B_t, cut once when the model is loaded).  Written by
+ *           loopvq_prepare.
+ * rope      fp32 [Nmax][D]: row p holds cos(p*w_f) in [0, D/2) and sin(p*w_f)
+ *           in [D/2, D), w_f = theta^(-2f/D), angles in fp64 (App. C: one row
+ *           of D values per position).  Written by loopvq_prepare.
+ */
+typedef struct loopvq_cache {
+    int32_t L, T, Tc, Hkv, Hq, D, c, K;
+    int32_t B, Nmax;
+    float theta;                 /* RoPE base, e.g. 1e4 */
+    uint32_t *idx;
+    const uint16_t *codebook;
+    uint16_t *slices;
+    float *rope;
+} loopvq_cache;
+
+/* Element counts of the four buffers (0 if the shape is invalid). */
+size_t loopvq_idx_words(const loopvq_cache *cache);
+size_t loopvq_codebook_elems(const loopvq_cache *cache);
+size_t loopvq_slice_elems(const loopvq_cache *cache);
+size_t loopvq_rope_elems(const loopvq_cache *cache);
+
+/*
+ * Load-time preparation (Sec. 4.3 "Attention"; App. C): cut every loop
+ * step's codebook slice from the codebooks, and fill the RoPE table.
+ * Reads cache->codebook, writes cache->slices and cache->rope.
+ */
+loopvq_status loopvq_prepare(const loopvq_cache *cache, void *stream);
+
+/*
+ * Encode (Sec. 4.3 "Encoding"; eq. 2 and 4): for the sequences
+ * b0 .. b0+nb-1 and tokens tok0 .. tok0+ntok-1, build every coupled vector of
+ * block `block` of layer `layer` for keys and values and store the index of
+ * its nearest codebook entry (squared Euclidean distance, lowest index on
+ * ties) into cache->idx.
+ *
+ * xk, xv    pre-RoPE keys / values of the Tc loop steps of the block, dtype
+ *           LOOPVQ_BF16 or LOOPVQ_FP32.  Element (m, b, n, h, d) is at
+ *           x[m*s[0] + (b-b0)*s[1] + (n-tok0)*s[2] + h*s[3] + d]; strides s are
+ *           in elements, d is contiguous.  Both use the same strides.
+ * Only the words of the named sequences and tokens are written; every word
+ * is rewritten whole (K and V codes of both groups of a pair).
+ */
+loopvq_status loopvq_encode(const loopvq_cache *cache, int layer, int block,
+                            const void *xk, const void *xv, int x_dtype,
+                            const int64_t x_strides[4],
+                            int b0, int nb, int tok0, int ntok, void *stream);
+
+/* Workspace bytes loopvq_decode_attn needs for caches of up to max_len tokens. */
+size_t loopvq_decode_workspace_bytes(const loopvq_cache *cache, int max_len);
+
+/*
+ * Decode attention at loop step t (0-based) of layer `layer`
+ * (Sec. 4.3 "Attention"; App. C):
+ *   for every sequence b and query head hq (KV head hq / (Hq/Hkv)):
+ *     k_n = RoPE(rebuilt key of token n, position n), v_n = rebuilt value,
+ *     s_n = scale * <q, k_n>,  out = sum_n softmax(s)_n v_n,
+ *     lse = ln sum_n exp(s_n),  over tokens n < len_b.
+ * Tokens are cut into splits, each attended by its own thread blocks; the
+ * splits are combined through their log-sum-exp, which is exact.
+ *
+ * q         bf16 [B][Hq][D], already rotated at the query position.
+ * lens      int32 [B] device; each length is clamped to [0, max_len].
+ * max_len   host-side upper bound of the lengths, 0 <= max_len <= Nmax.
+ * scale     score scale; <= 0 selects 1/sqrt(D).
+ * out       fp32 [B][Hq][D]; len_b == 0 gives zeros.
+ * lse       fp32 [B][Hq] natural-log log-sum-exp, -inf for len_b == 0; may be NULL.
+ * workspace device scratch of at least loopvq_decode_workspace_bytes(cache, max_len)
+ *           bytes, 16-byte aligned; its contents on entry do not matter.
+ */
+loopvq_status loopvq_decode_attn(const loopvq_cache *cache, int layer, int t,
+                                 const uint16_t *q, const int32_t *lens, int max_len,
+                                 float scale, float *out, float *lse,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Explicit reconstruction for checking (eq. 5): for sequence b, tokens
+ * tok0 .. tok0+ntok-1 and every KV head, the loop-step-t reconstruction of
+ * keys (kv = 0) or values (kv = 1); keys are rotated by RoPE at their
+ * positions when apply_rope != 0.
+ * out       fp32 [Hkv][ntok][D].
+ */
+loopvq_status loopvq_dequant_debug(const loopvq_cache *cache, int layer, int t, int kv,
+                                   int b, int tok0, int ntok, int apply_rope,
+                                   float *out, void *stream);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char *loopvq_last_error(void);
+
+/* ABI version, bumped on any incompatible change. */
+int loopvq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOOPVQ_H */

@@ -1,0 +1,7 @@
+"""LoopVQ hot path on B200: loop-axis VQ encode and decode attention over the coded cache.
+
+The compute runs in libloopvq.so (CUDA, sm_100a) behind the C ABI in
+include/loopvq.h; this package is its thin Python binding.
+"""
+from .loopvq import (Cache, CacheDesc, LoopVQError, prepare, encode, decode_attn, decode_workspace_bytes,  # noqa: F401
+                     dequant_debug, default_scale, lib, LIB_PATH, EXPORTS)

@@ -1,0 +1,183 @@
+// C ABI of libloopvq: host-side validation, then launches on the caller's stream.
+// Every entry point checks its arguments before launching anything and never
+// allocates or synchronises.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "loopvq_internal.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+loopvq_status fail(loopvq_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+loopvq_status cuda_fail(cudaError_t e, const char *where) {
+    return fail(LOOPVQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by every call.
+loopvq_status check_shape(const loopvq_cache *cc) {
+    if (!cc) return fail(LOOPVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (cc->L <= 0 || cc->T <= 0 || cc->Tc <= 0 || cc->Hkv <= 0 || cc->Hq <= 0 || cc->D <= 0 || cc->c <= 0 ||
+        cc->K <= 0 || cc->B <= 0 || cc->Nmax <= 0)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "all shape fields must be positive");
+    if (cc->T % cc->Tc != 0) return fail(LOOPVQ_ERR_INVALID_ARG, "T=%d is not a multiple of Tc=%d", cc->T, cc->Tc);
+    if (cc->Hq % cc->Hkv != 0) return fail(LOOPVQ_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", cc->Hq, cc->Hkv);
+    if (cc->K > 256) return fail(LOOPVQ_ERR_INVALID_ARG, "K=%d exceeds 256 (8-bit codes)", cc->K);
+    if (cc->Nmax % 4 != 0) return fail(LOOPVQ_ERR_INVALID_ARG, "Nmax=%d is not a multiple of 4", cc->Nmax);
+    if (cc->D != 64 && cc->D != 128) return fail(LOOPVQ_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", cc->D);
+    if (cc->c != 4 && cc->c != 8) return fail(LOOPVQ_ERR_UNSUPPORTED, "c=%d (supported: 4, 8)", cc->c);
+    if (cc->Tc != 1 && cc->Tc != 2 && cc->Tc != 4) return fail(LOOPVQ_ERR_UNSUPPORTED, "Tc=%d (supported: 1, 2, 4)", cc->Tc);
+    const int qpk = cc->Hq / cc->Hkv;
+    if (qpk != 1 && qpk != 2 && qpk != 4 && qpk != 8)
+        return fail(LOOPVQ_ERR_UNSUPPORTED, "Hq/Hkv=%d (supported: 1, 2, 4, 8)", qpk);
+    if (!(cc->theta > 0.f) || !std::isfinite(cc->theta)) return fail(LOOPVQ_ERR_INVALID_ARG, "theta must be positive");
+    return LOOPVQ_OK;
+}
+
+loopvq_status check_ptr(const void *p, const char *name) {
+    if (!p) return fail(LOOPVQ_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(p)) return fail(LOOPVQ_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return LOOPVQ_OK;
+}
+
+#define LQ_TRY(x)                              \
+    do {                                       \
+        loopvq_status _s = (x);                \
+        if (_s != LOOPVQ_OK) return _s;        \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t loopvq_idx_words(const loopvq_cache *cc) {
+    if (check_shape(cc) != LOOPVQ_OK) return 0;
+    return (size_t)cc->L * (cc->T / cc->Tc) * cc->B * cc->Hkv * (size_t)cc->Nmax * (cc->D / (2 * cc->c));
+}
+
+size_t loopvq_codebook_elems(const loopvq_cache *cc) {
+    if (check_shape(cc) != LOOPVQ_OK) return 0;
+    return (size_t)cc->L * (cc->T / cc->Tc) * 2 * cc->Hkv * (size_t)cc->K * cc->c * cc->Tc;
+}
+
+size_t loopvq_slice_elems(const loopvq_cache *cc) {
+    if (check_shape(cc) != LOOPVQ_OK) return 0;
+    return (size_t)cc->L * cc->T * 2 * cc->Hkv * (size_t)cc->K * cc->c;
+}
+
+size_t loopvq_rope_elems(const loopvq_cache *cc) {
+    if (check_shape(cc) != LOOPVQ_OK) return 0;
+    return (size_t)cc->Nmax * cc->D;
+}
+
+loopvq_status loopvq_prepare(const loopvq_cache *cc, void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_shape(cc));
+    LQ_TRY(check_ptr(cc->codebook, "codebook"));
+    LQ_TRY(check_ptr(cc->slices, "slices"));
+    LQ_TRY(check_ptr(cc->rope, "rope"));
+    cudaError_t e = loopvq::launch_prepare(*cc, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_prepare");
+    return LOOPVQ_OK;
+}
+
+loopvq_status loopvq_encode(const loopvq_cache *cc, int layer, int block, const void *xk, const void *xv,
+                            int x_dtype, const int64_t x_strides[4], int b0, int nb, int tok0, int ntok,
+                            void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_shape(cc));
+    LQ_TRY(check_ptr(cc->idx, "idx"));
+    LQ_TRY(check_ptr(cc->codebook, "codebook"));
+    if (layer < 0 || layer >= cc->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, cc->L);
+    if (block < 0 || block >= cc->T / cc->Tc)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "block=%d out of [0, %d)", block, cc->T / cc->Tc);
+    if (x_dtype != LOOPVQ_BF16 && x_dtype != LOOPVQ_FP32) return fail(LOOPVQ_ERR_INVALID_ARG, "x_dtype=%d", x_dtype);
+    if (nb < 0 || ntok < 0 || b0 < 0 || tok0 < 0 || b0 + nb > cc->B || tok0 + ntok > cc->Nmax)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "sequence range [%d, %d) or token range [%d, %d) outside the cache",
+                    b0, b0 + nb, tok0, tok0 + ntok);
+    if (nb == 0 || ntok == 0) return LOOPVQ_OK;
+    if (!xk || !xv) return fail(LOOPVQ_ERR_INVALID_ARG, "xk / xv is NULL");
+    if (!x_strides) return fail(LOOPVQ_ERR_INVALID_ARG, "x_strides is NULL");
+    for (int i = 0; i < 4; ++i)
+        if (x_strides[i] < 0) return fail(LOOPVQ_ERR_INVALID_ARG, "negative stride %d", i);
+    const size_t es = x_dtype == LOOPVQ_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(xk) | reinterpret_cast<uintptr_t>(xv)) % es)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "xk / xv not aligned to the element size");
+    cudaError_t e = loopvq::launch_encode(*cc, layer, block, xk, xv, x_dtype, x_strides, b0, nb, tok0, ntok,
+                                          (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_encode");
+    return LOOPVQ_OK;
+}
+
+size_t loopvq_decode_workspace_bytes(const loopvq_cache *cc, int max_len) {
+    if (check_shape(cc) != LOOPVQ_OK || max_len < 0 || max_len > cc->Nmax) return 0;
+    return loopvq::plan_decode(*cc, max_len).ws_bytes;
+}
+
+loopvq_status loopvq_decode_attn(const loopvq_cache *cc, int layer, int t, const uint16_t *q,
+                                 const int32_t *lens, int max_len, float scale, float *out, float *lse,
+                                 void *workspace, size_t ws_bytes, void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_shape(cc));
+    LQ_TRY(check_ptr(cc->idx, "idx"));
+    LQ_TRY(check_ptr(cc->slices, "slices"));
+    LQ_TRY(check_ptr(cc->rope, "rope"));
+    LQ_TRY(check_ptr(q, "q"));
+    LQ_TRY(check_ptr(lens, "lens"));
+    LQ_TRY(check_ptr(out, "out"));
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(LOOPVQ_ERR_INVALID_ARG, "lse not 4-byte aligned");
+    if (layer < 0 || layer >= cc->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, cc->L);
+    if (t < 0 || t >= cc->T) return fail(LOOPVQ_ERR_INVALID_ARG, "t=%d out of [0, %d)", t, cc->T);
+    if (max_len < 0 || max_len > cc->Nmax)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "max_len=%d out of [0, Nmax=%d]", max_len, cc->Nmax);
+    if (!std::isfinite(scale)) return fail(LOOPVQ_ERR_INVALID_ARG, "scale is not finite");
+    if (scale <= 0.f) scale = 1.0f / std::sqrt((float)cc->D);
+    const loopvq::DecodePlan plan = loopvq::plan_decode(*cc, max_len);
+    if (plan.nsplit > 65535) return fail(LOOPVQ_ERR_UNSUPPORTED, "too many splits");
+    if (!workspace || ws_bytes < plan.ws_bytes)
+        return fail(LOOPVQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws_bytes,
+                    workspace ? ws_bytes : (size_t)0);
+    if (!aligned16(workspace)) return fail(LOOPVQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    cudaError_t e = loopvq::launch_decode(*cc, plan, layer, t, q, lens, max_len, scale, out, lse, workspace,
+                                          (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_decode_attn");
+    return LOOPVQ_OK;
+}
+
+loopvq_status loopvq_dequant_debug(const loopvq_cache *cc, int layer, int t, int kv, int b, int tok0, int ntok,
+                                   int apply_rope, float *out, void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_shape(cc));
+    LQ_TRY(check_ptr(cc->idx, "idx"));
+    LQ_TRY(check_ptr(cc->slices, "slices"));
+    LQ_TRY(check_ptr(cc->rope, "rope"));
+    if (layer < 0 || layer >= cc->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, cc->L);
+    if (t < 0 || t >= cc->T) return fail(LOOPVQ_ERR_INVALID_ARG, "t=%d out of [0, %d)", t, cc->T);
+    if (kv != 0 && kv != 1) return fail(LOOPVQ_ERR_INVALID_ARG, "kv=%d (0 = keys, 1 = values)", kv);
+    if (b < 0 || b >= cc->B) return fail(LOOPVQ_ERR_INVALID_ARG, "b=%d out of [0, %d)", b, cc->B);
+    if (tok0 < 0 || ntok < 0 || tok0 + ntok > cc->Nmax)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "token range [%d, %d) outside [0, %d)", tok0, tok0 + ntok, cc->Nmax);
+    if (ntok == 0) return LOOPVQ_OK;
+    if (!out) return fail(LOOPVQ_ERR_INVALID_ARG, "out is NULL");
+    cudaError_t e = loopvq::launch_dequant(*cc, layer, t, kv, b, tok0, ntok, apply_rope, out, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_dequant_debug");
+    return LOOPVQ_OK;
+}
+
+const char *loopvq_last_error(void) { return g_err; }
+
+int loopvq_abi_version(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// Encode: nearest-entry coding of loop-axis coupled vectors.
+//
+// LoopVQ paper, Sec. 4.1 eq. (4): the coupled vector of token n, channel group g
+// takes channel g*c + i at loop step m of the block as coordinate i*Tc + m;
+// Sec. 2 eq. (2): it is stored as the index of its nearest codebook entry.
+// Sec. 4.3 "Encoding": a block is encoded once its last loop step exists.
+//
+// This direct kernel evaluates the squared distance to every entry in fp32,
+// coordinate by coordinate in ascending order with separately rounded
+// subtract / multiply / add, and keeps the first minimum, so its indices are the
+// exact nearest entries under that arithmetic.  One thread owns one index word:
+// the K and V codes of a channel group and of its RoPE partner group.
+#include <math_constants.h>
+
+#include "loopvq_internal.cuh"
+
+namespace loopvq {
+
+struct EncodeArgs {
+    const void *xk, *xv;
+    int64_t s0, s1, s2, s3;   // element strides of (m, b, n, h)
+    uint32_t *idx;            // words of (layer, block, b = 0, h = 0)
+    const uint16_t *cb;       // codebook of (layer, block, kv = 0, h = 0): [2][Hkv][K][G]
+    int Hkv, K, Nmax, b0, tok0, ntok;
+};
+
+template <typename XT>
+__device__ __forceinline__ float ld_x(const XT *p);
+template <>
+__device__ __forceinline__ float ld_x<uint16_t>(const uint16_t *p) { return bf16_to_f32(__ldg(p)); }
+template <>
+__device__ __forceinline__ float ld_x<float>(const float *p) { return __ldg(p); }
+
+template <int D, int C, int TC, typename XT>
+__global__ void __launch_bounds__(128) encode_direct_kernel(const EncodeArgs a) {
+    constexpr int G = C * TC;
+    constexpr int NP = D / (2 * C);
+    extern __shared__ __align__(16) float ecb[];           // [2][K][G] fp32: K codebook then V
+    const int h = blockIdx.y;
+    const int brel = blockIdx.z;
+    const int b = a.b0 + brel;
+    const int K = a.K;
+
+    for (int e = threadIdx.x; e < 2 * K * G; e += blockDim.x) {
+        const int kv = e / (K * G);
+        const int rem = e % (K * G);
+        ecb[e] = bf16_to_f32(a.cb[((size_t)kv * a.Hkv + h) * (size_t)K * G + rem]);
+    }
+    __syncthreads();
+
+    const int wl = blockIdx.x * blockDim.x + threadIdx.x;  // word within this (b, h) request
+    if (wl >= a.ntok * NP) return;
+    const int nrel = wl / NP;
+    const int p = wl % NP;
+    const int n = a.tok0 + nrel;
+
+    // coupled vectors of groups p and p + NP, keys and values
+    float z[4][G];
+    const XT *xk = reinterpret_cast<const XT *>(a.xk);
+    const XT *xv = reinterpret_cast<const XT *>(a.xv);
+    const size_t base = (size_t)brel * a.s1 + (size_t)nrel * a.s2 + (size_t)h * a.s3;
+#pragma unroll
+    for (int m = 0; m < TC; ++m)
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+            const size_t off = base + (size_t)m * a.s0;
+            z[0][i * TC + m] = ld_x(xk + off + p * C + i);
+            z[1][i * TC + m] = ld_x(xk + off + (p + NP) * C + i);
+            z[2][i * TC + m] = ld_x(xv + off + p * C + i);
+            z[3][i * TC + m] = ld_x(xv + off + (p + NP) * C + i);
+        }
+
+    float best[4] = {CUDART_INF_F, CUDART_INF_F, CUDART_INF_F, CUDART_INF_F};
+    int bi[4] = {0, 0, 0, 0};
+    const float *ek = ecb;
+    const float *ev = ecb + (size_t)K * G;
+    for (int r = 0; r < K; ++r) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < G; ++k) {
+            const float e0 = ek[r * G + k];
+            const float e1 = ev[r * G + k];
+            float t;
+            t = __fsub_rn(z[0][k], e0); d[0] = __fadd_rn(d[0], __fmul_rn(t, t));
+            t = __fsub_rn(z[1][k], e0); d[1] = __fadd_rn(d[1], __fmul_rn(t, t));
+            t = __fsub_rn(z[2][k], e1); d[2] = __fadd_rn(d[2], __fmul_rn(t, t));
+            t = __fsub_rn(z[3][k], e1); d[3] = __fadd_rn(d[3], __fmul_rn(t, t));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (d[u] < best[u]) { best[u] = d[u]; bi[u] = r; }
+    }
+    const uint32_t word = (uint32_t)bi[0] | ((uint32_t)bi[1] << 8) | ((uint32_t)bi[2] << 16) | ((uint32_t)bi[3] << 24);
+    a.idx[((size_t)b * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C) + idx_word(n, p, NP)] = word;
+}
+
+template <int D, int C, int TC>
+static cudaError_t launch_ct(const EncodeArgs &a, int x_dtype, int nb, cudaStream_t s) {
+    constexpr int NP = D / (2 * C);
+    const size_t smem = 2 * (size_t)a.K * C * TC * sizeof(float);
+    dim3 grid((a.ntok * NP + 127) / 128, a.Hkv, nb);
+    if (x_dtype == LOOPVQ_BF16) {
+        auto k = encode_direct_kernel<D, C, TC, uint16_t>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k<<<grid, 128, smem, s>>>(a);
+    } else {
+        auto k = encode_direct_kernel<D, C, TC, float>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k<<<grid, 128, smem, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t dispatch_c(int c, int tc, const EncodeArgs &a, int x_dtype, int nb, cudaStream_t s) {
+    if (c == 4) {
+        if (tc == 4) return launch_ct<D, 4, 4>(a, x_dtype, nb, s);
+        if (tc == 2) return launch_ct<D, 4, 2>(a, x_dtype, nb, s);
+        if (tc == 1) return launch_ct<D, 4, 1>(a, x_dtype, nb, s);
+    } else if (c == 8) {
+        if (tc == 4) return launch_ct<D, 8, 4>(a, x_dtype, nb, s);
+        if (tc == 2) return launch_ct<D, 8, 2>(a, x_dtype, nb, s);
+        if (tc == 1) return launch_ct<D, 8, 1>(a, x_dtype, nb, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_encode(const loopvq_cache &cc, int layer, int block, const void *xk, const void *xv,
+                          int x_dtype, const int64_t *strides, int b0, int nb, int tok0, int ntok,
+                          cudaStream_t s) {
+    if (nb == 0 || ntok == 0) return cudaSuccess;
+    EncodeArgs a{};
+    a.xk = xk;
+    a.xv = xv;
+    a.s0 = strides[0];
+    a.s1 = strides[1];
+    a.s2 = strides[2];
+    a.s3 = strides[3];
+    a.idx = cc.idx + idx_base(cc, layer, block, 0, 0);
+    a.cb = cc.codebook + codebook_base(cc, layer, block, 0, 0);
+    a.Hkv = cc.Hkv;
+    a.K = cc.K;
+    a.Nmax = cc.Nmax;
+    a.b0 = b0;
+    a.tok0 = tok0;
+    a.ntok = ntok;
+    if (cc.D == 128) return dispatch_c<128>(cc.c, cc.Tc, a, x_dtype, nb, s);
+    if (cc.D == 64) return dispatch_c<64>(cc.c, cc.Tc, a, x_dtype, nb, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace loopvq

@@ -1,0 +1,60 @@
+// Internal declarations shared by the CUDA translation units of libloopvq.
+// Layout arithmetic for the buffers described in include/loopvq.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/loopvq.h"
+
+namespace loopvq {
+
+// Offsets (in elements) of the first element of a sub-array.
+__host__ __device__ inline size_t idx_words_per_bh(int Nmax, int D, int c) {
+    return (size_t)Nmax * (size_t)(D / (2 * c));
+}
+// idx base of (layer, block, b, h)
+__host__ __device__ inline size_t idx_base(const loopvq_cache &cc, int layer, int block, int b, int h) {
+    const int NB = cc.T / cc.Tc;
+    return ((((size_t)layer * NB + block) * cc.B + b) * cc.Hkv + h) * idx_words_per_bh(cc.Nmax, cc.D, cc.c);
+}
+// word of token n, pair-group p within a (layer, block, b, h) run
+__host__ __device__ inline size_t idx_word(int n, int p, int NP) {
+    return (((size_t)(n >> 2) * NP + p) << 2) + (n & 3);
+}
+// slice base of (layer, t, kv, h): [K][c] bf16
+__host__ __device__ inline size_t slice_base(const loopvq_cache &cc, int layer, int t, int kv, int h) {
+    return ((((size_t)layer * cc.T + t) * 2 + kv) * cc.Hkv + h) * (size_t)cc.K * cc.c;
+}
+// codebook base of (layer, block, kv, h): [K][G] bf16
+__host__ __device__ inline size_t codebook_base(const loopvq_cache &cc, int layer, int block, int kv, int h) {
+    const int NB = cc.T / cc.Tc;
+    return ((((size_t)layer * NB + block) * 2 + kv) * cc.Hkv + h) * (size_t)cc.K * (cc.c * cc.Tc);
+}
+
+// bf16 bit pattern -> fp32 (exact)
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+// Launchers (host); each returns a cudaError_t from the launch.
+cudaError_t launch_prepare(const loopvq_cache &cc, cudaStream_t s);
+cudaError_t launch_encode(const loopvq_cache &cc, int layer, int block, const void *xk, const void *xv,
+                          int x_dtype, const int64_t *strides, int b0, int nb, int tok0, int ntok,
+                          cudaStream_t s);
+cudaError_t launch_dequant(const loopvq_cache &cc, int layer, int t, int kv, int b, int tok0, int ntok,
+                           int apply_rope, float *out, cudaStream_t s);
+
+struct DecodePlan {
+    int split_len;      // tokens per split (multiple of 4)
+    int nsplit;         // splits covering max_len
+    int nbt;            // sequences per thread block
+    int nchunk;         // ceil(B / nbt)
+    size_t ws_bytes;    // workspace needed
+};
+DecodePlan plan_decode(const loopvq_cache &cc, int max_len);
+cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
+                          const uint16_t *q, const int32_t *lens, int max_len, float scale,
+                          float *out, float *lse, void *workspace, cudaStream_t s);
+
+}  // namespace loopvq

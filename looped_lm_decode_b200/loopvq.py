@@ -1,0 +1,170 @@
+"""Python binding of libloopvq (the C ABI in include/loopvq.h).
+
+Argument marshalling only: torch provides device memory and streams, and
+every step of the path runs in the library's CUDA kernels.  Loading fails
+loudly if the library has not been built; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libloopvq.so")
+
+LOOPVQ_OK, LOOPVQ_ERR_INVALID_ARG, LOOPVQ_ERR_UNSUPPORTED, LOOPVQ_ERR_WORKSPACE, LOOPVQ_ERR_CUDA = range(5)
+LOOPVQ_BF16, LOOPVQ_FP32 = 0, 1
+
+EXPORTS = ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "loopvq_rope_elems",
+           "loopvq_prepare", "loopvq_encode", "loopvq_decode_workspace_bytes", "loopvq_decode_attn",
+           "loopvq_dequant_debug", "loopvq_last_error", "loopvq_abi_version")
+
+
+class CacheDesc(C.Structure):
+    """Mirror of struct loopvq_cache."""
+    _fields_ = [("L", C.c_int32), ("T", C.c_int32), ("Tc", C.c_int32), ("Hkv", C.c_int32),
+                ("Hq", C.c_int32), ("D", C.c_int32), ("c", C.c_int32), ("K", C.c_int32),
+                ("B", C.c_int32), ("Nmax", C.c_int32), ("theta", C.c_float),
+                ("idx", C.c_void_p), ("codebook", C.c_void_p), ("slices", C.c_void_p), ("rope", C.c_void_p)]
+
+
+class LoopVQError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"loopvq status {status}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with looped_lm_decode_b200/build.py "
+                               "(nvcc, sm_100a); there is no CPU fallback")
+        L = C.CDLL(LIB_PATH)
+        P = C.POINTER(CacheDesc)
+        vp, i, sz, f = C.c_void_p, C.c_int, C.c_size_t, C.c_float
+        for name in ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "loopvq_rope_elems"):
+            getattr(L, name).argtypes = [P]
+            getattr(L, name).restype = sz
+        L.loopvq_prepare.argtypes = [P, vp]
+        L.loopvq_encode.argtypes = [P, i, i, vp, vp, i, C.POINTER(C.c_int64), i, i, i, i, vp]
+        L.loopvq_decode_workspace_bytes.argtypes = [P, i]
+        L.loopvq_decode_workspace_bytes.restype = sz
+        L.loopvq_decode_attn.argtypes = [P, i, i, vp, vp, i, f, vp, vp, vp, sz, vp]
+        L.loopvq_dequant_debug.argtypes = [P, i, i, i, i, i, i, i, vp, vp]
+        for name in ("loopvq_prepare", "loopvq_encode", "loopvq_decode_attn", "loopvq_dequant_debug"):
+            getattr(L, name).restype = i
+        L.loopvq_last_error.argtypes = []
+        L.loopvq_last_error.restype = C.c_char_p
+        L.loopvq_abi_version.restype = i
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != LOOPVQ_OK:
+        raise LoopVQError(status, lib().loopvq_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+class Cache:
+    """Shape plus the four device buffers of a coded cache (see include/loopvq.h)."""
+
+    def __init__(self, L, T, Tc, Hkv, Hq, D, c, K, B, Nmax, theta=1.0e4, device="cuda", alloc=True):
+        self.desc = CacheDesc(L, T, Tc, Hkv, Hq, D, c, K, B, Nmax, theta, None, None, None, None)
+        self.L, self.T, self.Tc, self.Hkv, self.Hq, self.D, self.c, self.K = L, T, Tc, Hkv, Hq, D, c, K
+        self.B, self.Nmax, self.theta = B, Nmax, theta
+        self.idx = self.codebook = self.slices = self.rope = None
+        if alloc:
+            n_idx = lib().loopvq_idx_words(C.byref(self.desc))
+            if n_idx == 0:
+                raise LoopVQError(LOOPVQ_ERR_INVALID_ARG, "invalid or unsupported cache shape")
+            self.idx = torch.zeros(n_idx, dtype=torch.int32, device=device)
+            self.codebook = torch.zeros(lib().loopvq_codebook_elems(C.byref(self.desc)), dtype=torch.int16, device=device)
+            self.slices = torch.zeros(lib().loopvq_slice_elems(C.byref(self.desc)), dtype=torch.int16, device=device)
+            self.rope = torch.zeros(lib().loopvq_rope_elems(C.byref(self.desc)), dtype=torch.float32, device=device)
+            self._sync_desc()
+
+    def _sync_desc(self):
+        self.desc.idx = self.idx.data_ptr() if self.idx is not None else None
+        self.desc.codebook = self.codebook.data_ptr() if self.codebook is not None else None
+        self.desc.slices = self.slices.data_ptr() if self.slices is not None else None
+        self.desc.rope = self.rope.data_ptr() if self.rope is not None else None
+
+    @property
+    def NB(self):
+        return self.T // self.Tc
+
+    @property
+    def NP(self):
+        return self.D // (2 * self.c)
+
+    def ref(self):
+        self._sync_desc()
+        return C.byref(self.desc)
+
+
+def prepare(cache: Cache, stream=None):
+    _check(lib().loopvq_prepare(cache.ref(), _stream(stream)))
+
+
+def encode(cache: Cache, layer: int, block: int, xk: torch.Tensor, xv: torch.Tensor, b0: int = 0, tok0: int = 0,
+           stream=None):
+    """xk, xv: [Tc][nb][ntok][Hkv][D] (bf16 or fp32, innermost dim contiguous, same strides)."""
+    assert xk.shape == xv.shape and xk.stride() == xv.stride() and xk.dtype == xv.dtype
+    Tc, nb, ntok, Hkv, D = xk.shape
+    assert xk.stride(4) == 1
+    dt = {torch.bfloat16: LOOPVQ_BF16, torch.float32: LOOPVQ_FP32}[xk.dtype]
+    strides = (C.c_int64 * 4)(*xk.stride()[:4])
+    _check(lib().loopvq_encode(cache.ref(), layer, block, _ptr(xk), _ptr(xv), dt, strides, b0, nb, tok0, ntok,
+                               _stream(stream)))
+
+
+def decode_workspace_bytes(cache: Cache, max_len: int) -> int:
+    return lib().loopvq_decode_workspace_bytes(cache.ref(), max_len)
+
+
+def decode_attn(cache: Cache, layer: int, t: int, q: torch.Tensor, lens: torch.Tensor, max_len: int,
+                scale: float = 0.0, out=None, lse=None, workspace=None, stream=None):
+    """q bf16 [B][Hq][D] (post-RoPE), lens int32 [B]; returns (out fp32 [B][Hq][D], lse fp32 [B][Hq])."""
+    B, Hq, D = cache.B, cache.Hq, cache.D
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    need = decode_workspace_bytes(cache, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().loopvq_decode_attn(cache.ref(), layer, t, _ptr(q), _ptr(lens), max_len, scale, _ptr(out),
+                                    _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)))
+    return out, lse
+
+
+def dequant_debug(cache: Cache, layer: int, t: int, kv: int, b: int, tok0: int, ntok: int, apply_rope: bool = False,
+                  out=None, stream=None):
+    if out is None:
+        out = torch.empty((cache.Hkv, ntok, cache.D), dtype=torch.float32, device="cuda")
+    _check(lib().loopvq_dequant_debug(cache.ref(), layer, t, kv, b, tok0, ntok, int(bool(apply_rope)), _ptr(out),
+                                      _stream(stream)))
+    return out
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

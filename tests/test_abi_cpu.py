@@ -1,0 +1,96 @@
+"""The C-ABI library loads without a GPU, exports every declared symbol, and validates arguments
+on the host before any launch."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import looped_lm_decode_b200 as LQ
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "loopvq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(loopvq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 11
+    lib = LQ.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(LQ.EXPORTS)
+    assert lib.loopvq_abi_version() == 1
+
+
+def _cache(**kw):
+    args = dict(L=2, T=4, Tc=4, Hkv=16, Hq=16, D=128, c=4, K=256, B=8, Nmax=1024)
+    args.update(kw)
+    return LQ.Cache(**args, alloc=False)
+
+
+def test_buffer_sizes():
+    lib = LQ.lib()
+    c = _cache()
+    assert lib.loopvq_idx_words(c.ref()) == 2 * 1 * 8 * 16 * 1024 * 16
+    assert lib.loopvq_codebook_elems(c.ref()) == 2 * 1 * 2 * 16 * 256 * 16
+    assert lib.loopvq_slice_elems(c.ref()) == 2 * 4 * 2 * 16 * 256 * 4
+    assert lib.loopvq_rope_elems(c.ref()) == 1024 * 128
+    # 2*D/c bytes per token, head and block: 0.5 bit per element over Tc loop steps of K and V
+    bits = lib.loopvq_idx_words(c.ref()) * 32 / (2 * 8 * 16 * 1024 * 4 * 2 * 128)
+    assert bits == 0.5
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), 2), (dict(c=16), 2), (dict(Tc=3, T=6), 2), (dict(Hq=48), 2), (dict(Hq=17), 1),
+    (dict(T=6), 1), (dict(K=300), 1), (dict(Nmax=1022), 1), (dict(B=0), 1)])
+def test_shape_validation(kw, status):
+    lib = LQ.lib()
+    c = _cache(**kw)
+    assert lib.loopvq_idx_words(c.ref()) == 0
+    st = lib.loopvq_decode_attn(c.ref(), 0, 0, None, None, 0, 0.0, None, None, None, 0, None)
+    assert st == status, lib.loopvq_last_error()
+
+
+def test_argument_validation_before_launch():
+    lib = LQ.lib()
+    assert lib.loopvq_prepare(None, None) == 1
+    assert b"NULL" in lib.loopvq_last_error()
+    c = _cache()
+    # fake, aligned, never-dereferenced pointers: every call must be refused on the host
+    c.desc.idx = c.desc.slices = c.desc.rope = c.desc.codebook = 0x10000
+    c.ref = lambda: C.byref(c.desc)          # keep the fake pointers in the descriptor
+    fake = C.c_void_p(0x20000)
+    assert lib.loopvq_decode_attn(c.ref(), 2, 0, fake, fake, 0, 0.0, fake, None, fake, 1 << 30, None) == 1
+    assert b"layer" in lib.loopvq_last_error()
+    assert lib.loopvq_decode_attn(c.ref(), 0, 4, fake, fake, 0, 0.0, fake, None, fake, 1 << 30, None) == 1
+    assert lib.loopvq_decode_attn(c.ref(), 0, 0, fake, fake, 2000, 0.0, fake, None, fake, 1 << 30, None) == 1
+    assert b"max_len" in lib.loopvq_last_error()
+    need = lib.loopvq_decode_workspace_bytes(c.ref(), 1024)
+    assert need > 0
+    assert lib.loopvq_decode_attn(c.ref(), 0, 0, fake, fake, 1024, 0.0, fake, None, fake, need - 1, None) == 3
+    assert lib.loopvq_decode_attn(c.ref(), 0, 0, fake, fake, 1024, 0.0, fake, None, None, need, None) == 3
+    assert lib.loopvq_decode_attn(c.ref(), 0, 0, C.c_void_p(0x20002), fake, 1024, 0.0, fake, None, fake, need,
+                                  None) == 1
+    assert b"aligned" in lib.loopvq_last_error()
+    assert lib.loopvq_dequant_debug(c.ref(), 0, 0, 2, 0, 0, 4, 0, fake, None) == 1
+    assert lib.loopvq_dequant_debug(c.ref(), 0, 0, 0, 8, 0, 4, 0, fake, None) == 1
+    strides = (C.c_int64 * 4)(1, 1, 1, 1)
+    assert lib.loopvq_encode(c.ref(), 0, 1, fake, fake, 0, strides, 0, 1, 0, 4, None) == 1
+    assert lib.loopvq_encode(c.ref(), 0, 0, fake, fake, 7, strides, 0, 1, 0, 4, None) == 1
+    assert lib.loopvq_encode(c.ref(), 0, 0, fake, fake, 0, strides, 7, 2, 0, 4, None) == 1
+    # an empty request is a no-op that succeeds without touching the device
+    assert lib.loopvq_encode(c.ref(), 0, 0, None, None, 0, strides, 0, 0, 0, 0, None) == 0
+
+
+def test_workspace_grows_with_context():
+    lib = LQ.lib()
+    c = _cache(Nmax=32768)
+    a = lib.loopvq_decode_workspace_bytes(c.ref(), 1024)
+    b = lib.loopvq_decode_workspace_bytes(c.ref(), 32768)
+    assert 0 < a <= b
+    assert lib.loopvq_decode_workspace_bytes(c.ref(), 40000) == 0

@@ -1,0 +1,89 @@
+"""Full-size workloads in the launch configuration the benchmark times, checked on sampled outputs.
+
+A cache of one layer has exactly the per-call launch configuration of every layer
+of the full model (grid and splits depend on batch, heads, head size, code width
+and max length only), so each workload runs at its full batch, head count and
+context.  Bulk inputs come from the CUDA generator; the checker regenerates the
+sampled slices on the CPU from the same counters.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import looped_lm_decode_b200 as LQ
+from oracle import oracle as O
+from synth import WORKLOADS, lengths, random_indices, queries, kv_loops, bf16_bits_to_f32
+from synth import gpu as SG
+from tests.helpers import unpack_words, words_view, np_codebook_f32, attn_tolerance_ok
+
+pytestmark = pytest.mark.gpu
+
+SAMPLES = {"ctx32k": [(0, 0), (3, 7), (7, 15)], "ctx4k": [(0, 0), (31, 15)], "gqa16k": [(0, 0), (63, 13)],
+           "deep32": [(1, 39), (0, 17)]}
+
+
+def _full_cache(w):
+    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta)
+    SG.fill_codebook(w, cache.codebook)
+    LQ.prepare(cache)
+    return cache
+
+
+@pytest.mark.parametrize("name", list(SAMPLES))
+def test_decode_full_size_sampled(name):
+    w = WORKLOADS[name].replace(L=1)
+    cache = _full_cache(w)
+    t = w.T - 2                        # a loop step that is not the first of its block
+    blk, m = t // w.Tc, t % w.Tc
+    per_lb = w.B * w.Hkv * w.Nmax * cache.NP
+    SG.fill_idx(w, 0, blk, cache.idx[blk * per_lb:(blk + 1) * per_lb])
+    lens = lengths(w)
+    qd = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    SG.fill_q(w, 0, t, qd)
+    out, lse = LQ.decode_attn(cache, 0, t, qd.view(torch.int16), torch.from_numpy(lens).cuda(), int(lens.max()))
+    torch.cuda.synchronize()
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    qpk = w.Hq // w.Hkv
+    for b, hq in SAMPLES[name]:
+        h = hq // qpk
+        n = int(lens[b])
+        ik = random_indices(w, 0, blk, 0, b, h, range(n))
+        iv = random_indices(w, 0, blk, 1, b, h, range(n))
+        qb = queries(w, 0, t, b=[b], hq=[hq])[0, 0]
+        ref, lref = O.decode(bf16_bits_to_f32(qb).astype(np.float64), ik, iv, np_codebook_f32(w, 0, blk, 0, h),
+                             np_codebook_f32(w, 0, blk, 1, h), w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        ok, msg = attn_tolerance_ok(out[b, hq], ref, lse[b, hq:hq + 1], np.array([lref]))
+        assert ok, f"{name} (b={b}, hq={hq}): {msg}"
+
+
+def test_encode_full_size_sampled():
+    """deep32 prefill encode of one (layer, block) at full size: 2 x 8192 tokens x 40 heads, K and V."""
+    w = WORKLOADS["deep32"].replace(L=1)
+    cache = _full_cache(w)
+    blk = 3
+    xs = []
+    for kv in range(2):
+        x = torch.empty((w.Tc, w.B, w.Nmax, w.Hkv, w.D), dtype=torch.bfloat16, device="cuda")
+        SG.fill_kv(w, 0, kv, blk * w.Tc, blk * w.Tc + w.Tc - 1, x)
+        xs.append(x)
+    LQ.encode(cache, 0, blk, xs[0], xs[1])
+    torch.cuda.synchronize()
+    toks = np.array([0, 1, 2, 3, 1000, 4095, 4096, 8190, 8191])
+    ties = 0
+    for b, h in [(0, 0), (1, 39), (0, 21)]:
+        words = words_view(cache, 0, blk, b, h).cpu().numpy().view(np.uint32)
+        ck, cv = unpack_words(words, w.Nmax, cache.NP)
+        for kv, codes in ((0, ck), (1, cv)):
+            x = kv_loops(w, 0, kv, blk * w.Tc, blk * w.Tc + w.Tc - 1, [b], toks, [h])[:, 0, :, 0, :]
+            xf = np.ascontiguousarray(bf16_bits_to_f32(x))
+            E = np_codebook_f32(w, 0, blk, kv, h)
+            ref = O.encode(xf, E, w.c)
+            for i, n in enumerate(toks):
+                for g in np.nonzero(codes[n] != ref[i])[0]:
+                    dg = O.dist64(xf, E, w.c, i, g, int(codes[n, g]))
+                    do = O.dist64(xf, E, w.c, i, g, int(ref[i, g]))
+                    assert abs(dg - do) <= 1e-5 * max(dg, do)
+                    ties += 1
+    print(f"near-ties: {ties}")
