@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--impl", default="loopvq", choices=["loopvq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     return ap.parse_args()
 
 
@@ -135,24 +136,34 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+_CPU_INPUTS = {}
+
+
+def _cpu_inputs(w, layer, t, b, hq):
+    key = (w.name, layer, t, b, hq)
+    if key not in _CPU_INPUTS:
+        blk = t // w.Tc
+        h = hq // (w.Hq // w.Hkv)
+        n = int(lengths(w)[b])
+        _CPU_INPUTS[key] = (
+            bf16_bits_to_f32(queries(w, layer, t, b=[b], hq=[hq])[0, 0]).astype(np.float64),
+            random_indices(w, layer, blk, 0, b, h, range(n)), random_indices(w, layer, blk, 1, b, h, range(n)),
+            bf16_bits_to_f32(codebook(w, layer, blk, 0, h)), bf16_bits_to_f32(codebook(w, layer, blk, 1, h)))
+    return _CPU_INPUTS[key]
+
+
 def cpu_sample(w, seconds, layer=0, t=1):
     """Time the CPU checker's decode on (sequence, query head) units of one call until `seconds` pass.
     Codes for the sampled units are regenerated uniform codes of the same shape (the checker's
     work does not depend on code values); regeneration is not timed."""
     from oracle import oracle as O
     lens = lengths(w)
-    blk, m = t // w.Tc, t % w.Tc
-    qpk = w.Hq // w.Hkv
+    m = t % w.Tc
     total_s, nbytes, units = 0.0, 0, 0
     order = [(b, hq) for b in range(w.B) for hq in range(w.Hq)]
     for b, hq in order:
-        h = hq // qpk
         n = int(lens[b])
-        ik = random_indices(w, layer, blk, 0, b, h, range(n))
-        iv = random_indices(w, layer, blk, 1, b, h, range(n))
-        q = bf16_bits_to_f32(queries(w, layer, t, b=[b], hq=[hq])[0, 0]).astype(np.float64)
-        Ek = bf16_bits_to_f32(codebook(w, layer, blk, 0, h))
-        Ev = bf16_bits_to_f32(codebook(w, layer, blk, 1, h))
+        q, ik, iv, Ek, Ev = _cpu_inputs(w, layer, t, b, hq)
         t0 = time.perf_counter()
         O.decode(q, ik, iv, Ek, Ev, w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
         total_s += time.perf_counter() - t0
@@ -169,7 +180,7 @@ def run_reference(args):
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
-    per_step = max(0.2, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.1, min(2.0, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_sample(w, per_step)
     tot_s, tot_b, tot_u = 0.0, 0, 0
@@ -209,6 +220,8 @@ def main():
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     w = WORKLOADS[args.workload]
+    if args.layers > 0:
+        w = w.replace(L=args.layers)
 
     # ---------------- set-up: codebooks, slices, RoPE table, GPU encode of every (layer, block)
     cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, device=dev)

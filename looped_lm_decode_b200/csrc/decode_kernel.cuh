@@ -1,0 +1,364 @@
+// Split-K decode attention over the loop-axis coded cache (kernel templates).
+//
+// LoopVQ paper, Sec. 4.3 "Attention" and App. C: at loop step t every index is
+// looked up in that step's codebook slice B_t held in shared memory, keys are
+// rebuilt before RoPE and rotated from per-position cos/sin values, and the
+// quantized tokens are cut into splits processed by separate thread blocks whose
+// partial outputs are merged through their log-sum-exp (exact softmax).
+//
+// B200 design (not the pages' kernel):
+//  * One CTA per (token split, KV head, sequence).  The head's K and V slices are
+//    staged as bank-private replicas: row r (256 bytes) holds entry r of the K
+//    slice in bytes [0,128) and of the V slice in [128,256), replicated so that
+//    the 8-byte piece a lane reads sits in its own bank pair: lane l reads bytes
+//    (l % 16) * 8 of the half-row.  For c = 4 that is replica l % 16 of the
+//    8-byte entry; for c = 8 it is half (l % 2) of replica (l % 16) / 2 of the
+//    16-byte entry.  A gather by 16 lanes of random entries is conflict-free,
+//    and its address is one byte permute of the index word (code -> bits 8..15,
+//    the lane's column -> bits 0..7).
+//  * Every lane owns 8 channels: 4 of a channel group g < D/(2c) and the 4
+//    RoPE partners in group g + D/(2c), so it rotates its own rebuilt keys.  A
+//    token slot of D/8 lanes covers the head dimension and handles 4-token
+//    tiles; the 4 partial scores are reduce-scattered over the slot so each lane
+//    finishes one token and takes one exponent.
+//  * Each thread keeps a DEPTH-deep queue of its own 16-byte index-word loads in
+//    flight with cp.async (it reads back only what it copied, so no barrier is
+//    involved).
+//  * RoPE: one table row per tile, then exact one-position rotations.
+//  * Online softmax with a lazy maximum; fp32 math in packed pairs (FFMA2).
+#pragma once
+
+#include <math_constants.h>
+
+#include "loopvq_internal.cuh"
+
+namespace loopvq {
+
+struct DecodeArgs {
+    const uint32_t *idx;     // words of (layer, block, b = 0, h = 0)
+    const uint16_t *slk;     // K slices of (layer, t, h = 0): [Hkv][K][c]
+    const uint16_t *slv;     // V slices of (layer, t, h = 0)
+    const float *rope;       // [Nmax][D]
+    const uint16_t *q;       // [B][Hq][D] bf16
+    const int32_t *lens;     // [B]
+    float *ws_o;             // [B][Hq][nsplit][D]  unnormalised split outputs
+    float2 *ws_ml;           // [B][Hq][nsplit]     (reference max, sum) in log2 units
+    float *out;              // [B][Hq][D]
+    float *lse;              // [B][Hq] or null
+    int B, Hkv, Hq, K, Nmax, max_len, split_len, nsplit;
+    float qscale;            // scale * log2(e)
+};
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 unpack2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+
+__device__ __forceinline__ uint2 lds64(const unsigned char *smem, uint32_t off) {
+    return *reinterpret_cast<const uint2 *>(smem + off);
+}
+
+__device__ __forceinline__ uint32_t word_k(const uint4 &w, int k) {
+    return k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));
+}
+
+// Per-thread asynchronous prefetch queue: each thread copies, and later reads, only its own 16-byte
+// entries, so completion is tracked with its own commit groups and no CTA barrier is involved.
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH>
+__global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const DecodeArgs a) {
+    constexpr int NP = D / (2 * C);                        // pair-groups = index words per token
+    constexpr int HALVES = C / 4;                          // lanes sharing one pair-group
+    constexpr int NL = D / 8;                              // lanes per token slot
+    constexpr int SPW = 32 / NL;                           // slots per warp
+    constexpr int NSLOT = WARPS * SPW;
+    constexpr int NT = WARPS * 32;
+    constexpr int EB = 2 * C;                              // bytes of one slice entry
+    constexpr int REPL = 128 / EB;                         // replicas per half-row
+    constexpr int STRIDE = NSLOT * 4;                      // tokens between two tiles of a slot
+    static_assert(C == 4 || C == 8, "c");
+    static_assert(NL >= 4 && NL <= 16, "slot width");
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tok_begin = split * a.split_len;
+    const int len = min(max(__ldg(a.lens + b), 0), a.max_len);
+    if (tok_begin >= len) return;                          // the merge never reads this split
+    const int tok_end = min(tok_begin + a.split_len, len);
+
+    const int ls = lane % NL;                              // lane within the slot
+    const int gp = ls / HALVES;                            // pair-group
+    const int half = ls % HALVES;                          // which 4 channels of the group
+    const int slot = warp * SPW + lane / NL;
+    const unsigned slot_mask = ((1u << NL) - 1u) << (lane & ~(NL - 1));
+    const int slot_lane0 = lane & ~(NL - 1);
+    const uint32_t colk = (uint32_t)((lane % 16) * 8);     // byte 0 of every K gather address
+    const uint32_t colv = colk + 128u;                     // ... of every V gather address
+    const int ch = gp * C + half * 4;                      // first of this lane's 4 low channels
+    const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP + ((size_t)gp << 2);
+    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) + 65536u + (uint32_t)tid * 16u;
+
+    // queue the first DEPTH tiles of this slot before staging the slices
+    const int pfirst = tok_begin + slot * 4;
+#pragma unroll
+    for (int d = 0; d < DEPTH; ++d) {
+        const int p = pfirst + d * STRIDE;
+        if (p < tok_end) cp_async16(ring + (uint32_t)(d * NT * 16), idx_b + (size_t)(p >> 2) * NP * 4);
+        cp_async_commit();
+    }
+
+    // stage the K and V slices as bank-private replicas (rows >= K zeroed)
+    {
+        const uint16_t *sk = a.slk + (size_t)h * a.K * C;
+        const uint16_t *sv = a.slv + (size_t)h * a.K * C;
+        for (int it = tid; it < 256 * 2 * REPL; it += NT) {
+            const int rep = it % REPL;
+            const int kv = (it / REPL) & 1;
+            const int r = it / (2 * REPL);
+            unsigned char *dst = smem + r * 256 + kv * 128 + rep * EB;
+            const uint16_t *src = (kv ? sv : sk) + (size_t)r * C;
+            if constexpr (C == 4) {
+                uint2 v = make_uint2(0u, 0u);
+                if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(src));
+                *reinterpret_cast<uint2 *>(dst) = v;
+            } else {
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (r < a.K) v = __ldg(reinterpret_cast<const uint4 *>(src));
+                *reinterpret_cast<uint4 *>(dst) = v;
+            }
+        }
+    }
+
+    float2 qlo[QPK][2], qhi[QPK][2];
+#pragma unroll
+    for (int j = 0; j < QPK; ++j) {
+        const uint16_t *qp = a.q + ((size_t)b * a.Hq + h * QPK + j) * D;
+        const uint2 lo = *reinterpret_cast<const uint2 *>(qp + ch);
+        const uint2 hi = *reinterpret_cast<const uint2 *>(qp + D / 2 + ch);
+        qlo[j][0] = f2(bf16lo(lo.x) * a.qscale, bf16hi(lo.x) * a.qscale);
+        qlo[j][1] = f2(bf16lo(lo.y) * a.qscale, bf16hi(lo.y) * a.qscale);
+        qhi[j][0] = f2(bf16lo(hi.x) * a.qscale, bf16hi(hi.x) * a.qscale);
+        qhi[j][1] = f2(bf16lo(hi.y) * a.qscale, bf16hi(hi.y) * a.qscale);
+    }
+    // one-position rotation of this lane's 4 frequencies (RoPE table row 1)
+    float2 c1[2], s1[2];
+    {
+        const float4 cv = __ldg(reinterpret_cast<const float4 *>(a.rope + D + ch));
+        const float4 sv = __ldg(reinterpret_cast<const float4 *>(a.rope + D + D / 2 + ch));
+        c1[0] = f2(cv.x, cv.y);
+        c1[1] = f2(cv.z, cv.w);
+        s1[0] = f2(sv.x, sv.y);
+        s1[1] = f2(sv.z, sv.w);
+    }
+    float m_[QPK], l_[QPK];
+    float2 olo[QPK][2], ohi[QPK][2];
+#pragma unroll
+    for (int j = 0; j < QPK; ++j) {
+        m_[j] = -CUDART_INF_F;
+        l_[j] = 0.f;
+        olo[j][0] = olo[j][1] = ohi[j][0] = ohi[j][1] = f2(0.f, 0.f);
+    }
+    const bool hb = (ls & (NL / 2)) != 0;
+    const bool mb = (ls & (NL / 4)) != 0;
+    const int tk = (hb ? 2 : 0) + (mb ? 1 : 0);            // token of the tile this lane finishes
+
+    // RoPE row of each tile's first token, loaded one tile ahead
+    float4 ra_c, ra_s;
+    {
+        const float *row = a.rope + (size_t)min(pfirst, a.Nmax - 4) * D + ch;
+        ra_c = __ldg(reinterpret_cast<const float4 *>(row));
+        ra_s = __ldg(reinterpret_cast<const float4 *>(row + D / 2));
+    }
+    __syncthreads();
+
+    int stage = 0;
+    for (int p0 = pfirst; p0 < tok_end; p0 += STRIDE) {
+        cp_async_wait<DEPTH - 1>();                        // this thread's oldest queued tile has landed
+        uint4 w4;
+        {
+            const uint32_t addr = ring + (uint32_t)(stage * NT * 16);
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w4.x), "=r"(w4.y), "=r"(w4.z), "=r"(w4.w) : "r"(addr) : "memory");
+        }
+        float2 cs[2] = {f2(ra_c.x, ra_c.y), f2(ra_c.z, ra_c.w)};
+        float2 sn[2] = {f2(ra_s.x, ra_s.y), f2(ra_s.z, ra_s.w)};
+        {
+            const float *row = a.rope + (size_t)min(p0 + STRIDE, a.Nmax - 4) * D + ch;
+            ra_c = __ldg(reinterpret_cast<const float4 *>(row));
+            ra_s = __ldg(reinterpret_cast<const float4 *>(row + D / 2));
+        }
+
+        // ---- keys: rebuild, rotate, partial dot per query head
+        float ps[QPK][4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (k > 0) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float2 cn = __ffma2_rn(cs[i], c1[i], neg2(__fmul2_rn(sn[i], s1[i])));
+                    const float2 snn = __ffma2_rn(sn[i], c1[i], __fmul2_rn(cs[i], s1[i]));
+                    cs[i] = cn;
+                    sn[i] = snn;
+                }
+            }
+            const uint32_t w = word_k(w4, k);
+            const uint2 elo = lds64(smem, __byte_perm(w, colk, 0x7604));
+            const uint2 ehi = lds64(smem, __byte_perm(w, colk, 0x7614));
+            const uint32_t el[2] = {elo.x, elo.y}, eh[2] = {ehi.x, ehi.y};
+            float2 rlo[2], rhi[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float2 kl = unpack2(el[i]);
+                const float2 kh = unpack2(eh[i]);
+                rlo[i] = __ffma2_rn(kl, cs[i], neg2(__fmul2_rn(kh, sn[i])));   // kl*cos - kh*sin
+                rhi[i] = __ffma2_rn(kh, cs[i], __fmul2_rn(kl, sn[i]));         // kh*cos + kl*sin
+            }
+#pragma unroll
+            for (int j = 0; j < QPK; ++j) {
+                float2 acc = __fmul2_rn(qlo[j][0], rlo[0]);
+                acc = __ffma2_rn(qhi[j][0], rhi[0], acc);
+                acc = __ffma2_rn(qlo[j][1], rlo[1], acc);
+                acc = __ffma2_rn(qhi[j][1], rhi[1], acc);
+                ps[j][k] = acc.x + acc.y;
+            }
+        }
+        // the queue entry has been consumed: queue the tile DEPTH steps ahead into it
+        {
+            const int pq = p0 + DEPTH * STRIDE;
+            if (pq < tok_end) cp_async16(ring + (uint32_t)(stage * NT * 16), idx_b + (size_t)(pq >> 2) * NP * 4);
+            cp_async_commit();
+            stage = stage + 1 == DEPTH ? 0 : stage + 1;
+        }
+
+        // ---- reduce-scatter the 4 scores over the slot, online-softmax update
+        float pe[QPK];
+#pragma unroll
+        for (int j = 0; j < QPK; ++j) {
+            float keep0 = hb ? ps[j][2] : ps[j][0], keep1 = hb ? ps[j][3] : ps[j][1];
+            const float send0 = hb ? ps[j][0] : ps[j][2], send1 = hb ? ps[j][1] : ps[j][3];
+            keep0 += __shfl_xor_sync(slot_mask, send0, NL / 2);
+            keep1 += __shfl_xor_sync(slot_mask, send1, NL / 2);
+            float keep = mb ? keep1 : keep0;
+            const float send = mb ? keep0 : keep1;
+            keep += __shfl_xor_sync(slot_mask, send, NL / 4);
+#pragma unroll
+            for (int o = NL / 8; o >= 1; o >>= 1) keep += __shfl_xor_sync(slot_mask, keep, o);
+            const float s = (p0 + tk < tok_end) ? keep : -CUDART_INF_F;
+            // Lazy maximum: the reference only has to stay within 2^8 of the running maximum for
+            // the weights to stay finite, so it moves (with an exact rescale) only when a score of
+            // the tile exceeds it by more than 8 in log2 units.
+            if (__any_sync(slot_mask, s > m_[j] + 8.f)) {
+                float tmax = fmaxf(s, __shfl_xor_sync(slot_mask, s, NL / 4));
+                tmax = fmaxf(tmax, __shfl_xor_sync(slot_mask, tmax, NL / 2));
+                const float corr = ex2(m_[j] - tmax);
+                l_[j] *= corr;
+                const float2 c2 = f2(corr, corr);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    olo[j][i] = __fmul2_rn(olo[j][i], c2);
+                    ohi[j][i] = __fmul2_rn(ohi[j][i], c2);
+                }
+                m_[j] = tmax;
+            }
+            pe[j] = ex2(s - m_[j]);
+            l_[j] += pe[j];
+        }
+
+        // ---- values: rebuild and accumulate with each token's weight
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int src = slot_lane0 + (k >> 1) * (NL / 2) + (k & 1) * (NL / 4);
+            const uint32_t w = word_k(w4, k);
+            const uint2 vlo = lds64(smem, __byte_perm(w, colv, 0x7624));
+            const uint2 vhi = lds64(smem, __byte_perm(w, colv, 0x7634));
+            const uint32_t vl[2] = {vlo.x, vlo.y}, vh[2] = {vhi.x, vhi.y};
+#pragma unroll
+            for (int j = 0; j < QPK; ++j) {
+                const float pk = __shfl_sync(slot_mask, pe[j], src);
+                const float2 p2 = f2(pk, pk);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    olo[j][i] = __ffma2_rn(p2, unpack2(vl[i]), olo[j][i]);
+                    ohi[j][i] = __ffma2_rn(p2, unpack2(vh[i]), ohi[j][i]);
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+
+    // ---- combine the slots of this CTA, write the split's partial result
+    __syncthreads();                                       // slices no longer needed
+    constexpr int RS = D + 4;                              // floats per (slot, query head) record
+    float *red = reinterpret_cast<float *>(smem);
+#pragma unroll
+    for (int j = 0; j < QPK; ++j) {
+        float lsum = l_[j] + __shfl_xor_sync(slot_mask, l_[j], NL / 4);
+        lsum += __shfl_xor_sync(slot_mask, lsum, NL / 2);
+        float *rec = red + ((size_t)slot * QPK + j) * RS;
+        *reinterpret_cast<float4 *>(rec + ch) = make_float4(olo[j][0].x, olo[j][0].y, olo[j][1].x, olo[j][1].y);
+        *reinterpret_cast<float4 *>(rec + D / 2 + ch) = make_float4(ohi[j][0].x, ohi[j][0].y, ohi[j][1].x, ohi[j][1].y);
+        if (ls == 0) {
+            rec[D] = m_[j];
+            rec[D + 1] = lsum;
+        }
+    }
+    __syncthreads();
+    for (int it = tid; it < QPK * D; it += NT) {
+        const int d = it % D;
+        const int j = it / D;
+        float mx = -CUDART_INF_F;
+        for (int s2 = 0; s2 < NSLOT; ++s2) mx = fmaxf(mx, red[((size_t)s2 * QPK + j) * RS + D]);
+        float acc = 0.f, lsum = 0.f;
+        if (mx != -CUDART_INF_F) {
+            for (int s2 = 0; s2 < NSLOT; ++s2) {
+                const float *rec = red + ((size_t)s2 * QPK + j) * RS;
+                const float wgt = ex2(rec[D] - mx);
+                acc += rec[d] * wgt;
+                lsum += rec[D + 1] * wgt;
+            }
+        }
+        const size_t bh = (size_t)b * a.Hq + h * QPK + j;
+        a.ws_o[(bh * a.nsplit + split) * D + d] = acc;
+        if (d == 0) a.ws_ml[bh * a.nsplit + split] = f2(mx, lsum);
+    }
+}
+
+// Log-sum-exp merge of the splits of every (sequence, query head).
+template <int D>
+__global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
+    const int bh = blockIdx.x;
+    const int b = bh / a.Hq;
+    const int d = threadIdx.x;
+    const int len = min(max(a.lens[b], 0), a.max_len);
+    const int ns = len > 0 ? (len + a.split_len - 1) / a.split_len : 0;
+    const float2 *ml = a.ws_ml + (size_t)bh * a.nsplit;
+    float mx = -CUDART_INF_F;
+    for (int s = 0; s < ns; ++s) mx = fmaxf(mx, ml[s].x);
+    float acc = 0.f, lsum = 0.f;
+    if (mx != -CUDART_INF_F) {
+        const float *o = a.ws_o + (size_t)bh * a.nsplit * D + d;
+        for (int s = 0; s < ns; ++s) {
+            const float wgt = ex2(ml[s].x - mx);
+            acc += o[(size_t)s * D] * wgt;
+            lsum += ml[s].y * wgt;
+        }
+    }
+    const bool any = (mx != -CUDART_INF_F) && lsum > 0.f;
+    a.out[(size_t)bh * D + d] = any ? acc / lsum : 0.f;
+    if (a.lse != nullptr && d == 0)
+        a.lse[bh] = any ? (mx + log2f(lsum)) * 0.69314718055994530942f : -CUDART_INF_F;
+}
+
+}  // namespace loopvq
