@@ -151,6 +151,42 @@ loopvq_status loopvq_dequant_debug(const loopvq_cache *cache, int layer, int t, 
                                    int b, int tok0, int ntok, int apply_rope,
                                    float *out, void *stream);
 
+/*
+ * Size in bytes of the built-in split scratch used by loopvq_decode_attn_noalloc.
+ */
+#define LOOPVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+size_t loopvq_noalloc_scratch_bytes(void);
+
+/*
+ * Decode attention without any caller workspace.  (The LoopVQ paper has no
+ * counterpart: this is a deployment convenience of this library.)
+ *
+ * Some callers cannot allocate device memory at all: plain C hosts with no
+ * device allocator of their own, plug-ins whose host application owns every
+ * byte of the device through its own allocator, and serving loops that must
+ * not call cudaMalloc because it can synchronise the device.  This entry
+ * point computes exactly what loopvq_decode_attn computes (same kernels, same
+ * arguments minus the workspace) but keeps the split partials in a fixed
+ * 8 MiB array compiled into the library (LOOPVQ_NOALLOC_SCRATCH_BYTES).
+ *
+ *  - Every GPU that loads the library holds that array until the process
+ *    exits.  Nothing is allocated or freed by this call (no cudaMalloc, no
+ *    cudaFree, no allocating library routine).
+ *  - The first call on a device looks up the array's device address on the
+ *    current device (cudaGetSymbolAddress) and caches it; make that first call
+ *    before any stream capture.
+ *  - A call whose split scratch, loopvq_decode_workspace_bytes(cache, max_len),
+ *    exceeds the array is rejected with LOOPVQ_ERR_WORKSPACE and a message
+ *    naming both sizes; nothing is launched.
+ *  - All calls in the process share the one array per device and it keeps the
+ *    last call's contents (no call needs it cleared: every partial that is read
+ *    is written by the same call first).  Calls that overlap on the GPU, for
+ *    example on two streams, race on it: issue them in order on one stream.
+ */
+loopvq_status loopvq_decode_attn_noalloc(const loopvq_cache *cache, int layer, int t,
+                                         const uint16_t *q, const int32_t *lens, int max_len,
+                                         float scale, float *out, float *lse, void *stream);
+
 /* Message of the last failed call on this thread ("" if none). */
 const char *loopvq_last_error(void);
 

@@ -60,6 +60,10 @@ loopvq_status check_ptr(const void *p, const char *name) {
 
 }  // namespace
 
+namespace loopvq {
+void set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace loopvq
+
 extern "C" {
 
 size_t loopvq_idx_words(const loopvq_cache *cc) {

@@ -37,6 +37,9 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
+// Sets the thread-local message returned by loopvq_last_error().
+void set_last_error(const char *msg);
+
 // Launchers (host); each returns a cudaError_t from the launch.
 cudaError_t launch_prepare(const loopvq_cache &cc, cudaStream_t s);
 cudaError_t launch_encode(const loopvq_cache &cc, int layer, int block, const void *xk, const void *xv,

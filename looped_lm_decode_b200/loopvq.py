@@ -20,7 +20,8 @@ LOOPVQ_BF16, LOOPVQ_FP32 = 0, 1
 
 EXPORTS = ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "loopvq_rope_elems",
            "loopvq_prepare", "loopvq_encode", "loopvq_decode_workspace_bytes", "loopvq_decode_attn",
-           "loopvq_dequant_debug", "loopvq_last_error", "loopvq_abi_version")
+           "loopvq_dequant_debug", "loopvq_last_error", "loopvq_abi_version",
+           "loopvq_decode_attn_noalloc", "loopvq_noalloc_scratch_bytes")
 
 
 class CacheDesc(C.Structure):
@@ -58,6 +59,10 @@ def lib():
         L.loopvq_decode_workspace_bytes.restype = sz
         L.loopvq_decode_attn.argtypes = [P, i, i, vp, vp, i, f, vp, vp, vp, sz, vp]
         L.loopvq_dequant_debug.argtypes = [P, i, i, i, i, i, i, i, vp, vp]
+        L.loopvq_decode_attn_noalloc.argtypes = [P, i, i, vp, vp, i, f, vp, vp, vp]
+        L.loopvq_decode_attn_noalloc.restype = i
+        L.loopvq_noalloc_scratch_bytes.argtypes = []
+        L.loopvq_noalloc_scratch_bytes.restype = sz
         for name in ("loopvq_prepare", "loopvq_encode", "loopvq_decode_attn", "loopvq_dequant_debug"):
             getattr(L, name).restype = i
         L.loopvq_last_error.argtypes = []
@@ -154,6 +159,19 @@ def decode_attn(cache: Cache, layer: int, t: int, q: torch.Tensor, lens: torch.T
     _check(lib().loopvq_decode_attn(cache.ref(), layer, t, _ptr(q), _ptr(lens), max_len, scale, _ptr(out),
                                     _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                     _stream(stream)))
+    return out, lse
+
+
+def decode_attn_noalloc(cache: Cache, layer: int, t: int, q: torch.Tensor, lens: torch.Tensor, max_len: int,
+                        scale: float = 0.0, out=None, lse=None, stream=None):
+    """decode_attn with the library's built-in scratch array instead of a caller workspace."""
+    B, Hq, D = cache.B, cache.Hq, cache.D
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check(lib().loopvq_decode_attn_noalloc(cache.ref(), layer, t, _ptr(q), _ptr(lens), max_len, scale, _ptr(out),
+                                            _ptr(lse), _stream(stream)))
     return out, lse
 
 
