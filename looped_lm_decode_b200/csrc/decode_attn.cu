@@ -16,7 +16,7 @@ namespace loopvq {
 static constexpr int kWarps = 8;
 static constexpr int kMinBlocks = 2;
 static constexpr int kDepth = 4;
-static constexpr long kTargetCtas = 148L * 2 * 6;
+static constexpr long kTargetCtas = 148L * 2 * 4;
 
 static size_t ring_smem_bytes() { return 65536 + (size_t)kDepth * kWarps * 32 * 16; }
 
@@ -44,7 +44,8 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStr
     const size_t red = (size_t)NSLOT * QPK * (D + 4) * sizeof(float);
     const size_t smem = ring_smem_bytes();
     if (red > smem) return cudaErrorInvalidConfiguration;   // the slot records reuse slices and queue
-    auto kern = decode_split_kernel<D, C, QPK, kWarps, kMinBlocks, kDepth>;
+    // one query head per KV head: rotate the query (cheaper than rotating every key); GQA rotates keys once
+    auto kern = decode_split_kernel<D, C, QPK, kWarps, kMinBlocks, kDepth, QPK == 1, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (plan.nsplit > 0) {

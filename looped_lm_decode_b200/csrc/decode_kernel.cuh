@@ -17,14 +17,19 @@
 //    and its address is one byte permute of the index word (code -> bits 8..15,
 //    the lane's column -> bits 0..7).
 //  * Every lane owns 8 channels: 4 of a channel group g < D/(2c) and the 4
-//    RoPE partners in group g + D/(2c), so it rotates its own rebuilt keys.  A
-//    token slot of D/8 lanes covers the head dimension and handles 4-token
-//    tiles; the 4 partial scores are reduce-scattered over the slot so each lane
-//    finishes one token and takes one exponent.
+//    RoPE partners in group g + D/(2c), so all RoPE arithmetic stays in the
+//    lane.  A token slot of D/8 lanes covers the head dimension and handles
+//    4-token tiles; the 4 partial scores are reduce-scattered over the slot so
+//    each lane finishes one token and takes one exponent.
+//  * With one query head per KV head the query is rotated instead of the keys
+//    (ROTQ): per pair f the score term is Re(Z) k_f + Im(Z) k_{f+D/2} with
+//    Z = (q_f + i q_{f+D/2}) e^{-i p w_f}, and Z advances one position by one
+//    complex multiply.  With several query heads the rebuilt keys are rotated
+//    once and shared.
 //  * Each thread keeps a DEPTH-deep queue of its own 16-byte index-word loads in
 //    flight with cp.async (it reads back only what it copied, so no barrier is
 //    involved).
-//  * RoPE: one table row per tile, then exact one-position rotations.
+//  * RoPE values: one table row per tile, then exact one-position rotations.
 //  * Online softmax with a lazy maximum; fp32 math in packed pairs (FFMA2).
 #pragma once
 
@@ -76,7 +81,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH>
+template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, bool ROTQ, bool K32>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const DecodeArgs a) {
     constexpr int NP = D / (2 * C);                        // pair-groups = index words per token
     constexpr int HALVES = C / 4;                          // lanes sharing one pair-group
@@ -84,10 +89,12 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     constexpr int SPW = 32 / NL;                           // slots per warp
     constexpr int NSLOT = WARPS * SPW;
     constexpr int NT = WARPS * 32;
-    constexpr int EB = 2 * C;                              // bytes of one slice entry
-    constexpr int REPL = 128 / EB;                         // replicas per half-row
+    constexpr int EB = 2 * C;                              // bytes of one bf16 slice entry
+    constexpr int REPL = 128 / EB;                         // bf16 replicas per half-row
+    constexpr int REPLK = K32 ? 128 / (4 * C) : REPL;      // K replicas (fp32 entries when K32)
     constexpr int STRIDE = NSLOT * 4;                      // tokens between two tiles of a slot
     static_assert(C == 4 || C == 8, "c");
+    static_assert(!ROTQ || QPK == 1, "query rotation is for one query head per KV head");
     static_assert(NL >= 4 && NL <= 16, "slot width");
 
     extern __shared__ __align__(128) unsigned char smem[];
@@ -104,8 +111,9 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     const int slot = warp * SPW + lane / NL;
     const unsigned slot_mask = ((1u << NL) - 1u) << (lane & ~(NL - 1));
     const int slot_lane0 = lane & ~(NL - 1);
-    const uint32_t colk = (uint32_t)((lane % 16) * 8);     // byte 0 of every K gather address
-    const uint32_t colv = colk + 128u;                     // ... of every V gather address
+    const uint32_t colk = K32 ? (uint32_t)((lane % 8) * 16)   // fp32 keys: 16-byte pieces, 8 per wavefront
+                              : (uint32_t)((lane % 16) * 8);  // bf16: 8-byte pieces, 16 per wavefront
+    const uint32_t colv = (uint32_t)((lane % 16) * 8) + 128u; // byte 0 of every V gather address
     const int ch = gp * C + half * 4;                      // first of this lane's 4 low channels
     const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP + ((size_t)gp << 2);
     const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) + 65536u + (uint32_t)tid * 16u;
@@ -123,9 +131,22 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     {
         const uint16_t *sk = a.slk + (size_t)h * a.K * C;
         const uint16_t *sv = a.slv + (size_t)h * a.K * C;
+        if constexpr (K32) {
+            // K half-rows: REPLK replicas of the entry widened to fp32 (4C bytes)
+            for (int it = tid; it < 256 * REPLK * (C / 4); it += NT) {
+                const int q4 = it % (C / 4);
+                const int rep = (it / (C / 4)) % REPLK;
+                const int r = it / (REPLK * (C / 4));
+                uint2 v = make_uint2(0u, 0u);
+                if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(sk + (size_t)r * C + q4 * 4));
+                *reinterpret_cast<float4 *>(smem + r * 256 + rep * 4 * C + q4 * 16) =
+                    make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+            }
+        }
         for (int it = tid; it < 256 * 2 * REPL; it += NT) {
             const int rep = it % REPL;
             const int kv = (it / REPL) & 1;
+            if (K32 && kv == 0) continue;
             const int r = it / (2 * REPL);
             unsigned char *dst = smem + r * 256 + kv * 128 + rep * EB;
             const uint16_t *src = (kv ? sv : sk) + (size_t)r * C;
@@ -162,6 +183,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         s1[0] = f2(sv.x, sv.y);
         s1[1] = f2(sv.z, sv.w);
     }
+    const float2 ns1[2] = {neg2(s1[0]), neg2(s1[1])};
+    const float2 nqlo[2] = {neg2(qlo[0][0]), neg2(qlo[0][1])};
     float m_[QPK], l_[QPK];
     float2 olo[QPK][2], ohi[QPK][2];
 #pragma unroll
@@ -202,36 +225,73 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 
         // ---- keys: rebuild, rotate, partial dot per query head
         float ps[QPK][4];
+        // ROTQ: rotate the query instead of every key.  With Z = (q_f + i q_{f+D/2}) e^{-i p w_f},
+        // the score term of pair f is Re(Z) k_f + Im(Z) k_{f+D/2}; Z of the next position is Z times
+        // e^{-i w_f}.  Otherwise keys are rotated by (cos, sin), advanced one position per token.
+        float2 zu[2], zw[2];
+        if constexpr (ROTQ) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                zu[i] = __ffma2_rn(qlo[0][i], cs[i], __fmul2_rn(qhi[0][i], sn[i]));
+                zw[i] = __ffma2_rn(qhi[0][i], cs[i], __fmul2_rn(nqlo[i], sn[i]));
+            }
+        }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             if (k > 0) {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    const float2 cn = __ffma2_rn(cs[i], c1[i], neg2(__fmul2_rn(sn[i], s1[i])));
-                    const float2 snn = __ffma2_rn(sn[i], c1[i], __fmul2_rn(cs[i], s1[i]));
-                    cs[i] = cn;
-                    sn[i] = snn;
+                    if constexpr (ROTQ) {
+                        const float2 un = __ffma2_rn(zu[i], c1[i], __fmul2_rn(zw[i], s1[i]));
+                        const float2 wn = __ffma2_rn(zw[i], c1[i], __fmul2_rn(zu[i], ns1[i]));
+                        zu[i] = un;
+                        zw[i] = wn;
+                    } else {
+                        const float2 cn = __ffma2_rn(cs[i], c1[i], __fmul2_rn(sn[i], ns1[i]));
+                        const float2 snn = __ffma2_rn(sn[i], c1[i], __fmul2_rn(cs[i], s1[i]));
+                        cs[i] = cn;
+                        sn[i] = snn;
+                    }
                 }
             }
             const uint32_t w = word_k(w4, k);
-            const uint2 elo = lds64(smem, __byte_perm(w, colk, 0x7604));
-            const uint2 ehi = lds64(smem, __byte_perm(w, colk, 0x7614));
-            const uint32_t el[2] = {elo.x, elo.y}, eh[2] = {ehi.x, ehi.y};
-            float2 rlo[2], rhi[2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const float2 kl = unpack2(el[i]);
-                const float2 kh = unpack2(eh[i]);
-                rlo[i] = __ffma2_rn(kl, cs[i], neg2(__fmul2_rn(kh, sn[i])));   // kl*cos - kh*sin
-                rhi[i] = __ffma2_rn(kh, cs[i], __fmul2_rn(kl, sn[i]));         // kh*cos + kl*sin
+            float2 kl[2], kh[2];
+            if constexpr (K32) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(smem + __byte_perm(w, colk, 0x7604));
+                const float4 b4 = *reinterpret_cast<const float4 *>(smem + __byte_perm(w, colk, 0x7614));
+                kl[0] = f2(a4.x, a4.y);
+                kl[1] = f2(a4.z, a4.w);
+                kh[0] = f2(b4.x, b4.y);
+                kh[1] = f2(b4.z, b4.w);
+            } else {
+                const uint2 elo = lds64(smem, __byte_perm(w, colk, 0x7604));
+                const uint2 ehi = lds64(smem, __byte_perm(w, colk, 0x7614));
+                kl[0] = unpack2(elo.x);
+                kl[1] = unpack2(elo.y);
+                kh[0] = unpack2(ehi.x);
+                kh[1] = unpack2(ehi.y);
             }
+            if constexpr (ROTQ) {
+                float2 acc = __fmul2_rn(zu[0], kl[0]);
+                acc = __ffma2_rn(zw[0], kh[0], acc);
+                acc = __ffma2_rn(zu[1], kl[1], acc);
+                acc = __ffma2_rn(zw[1], kh[1], acc);
+                ps[0][k] = acc.x + acc.y;
+            } else {
+                float2 rlo[2], rhi[2];
 #pragma unroll
-            for (int j = 0; j < QPK; ++j) {
-                float2 acc = __fmul2_rn(qlo[j][0], rlo[0]);
-                acc = __ffma2_rn(qhi[j][0], rhi[0], acc);
-                acc = __ffma2_rn(qlo[j][1], rlo[1], acc);
-                acc = __ffma2_rn(qhi[j][1], rhi[1], acc);
-                ps[j][k] = acc.x + acc.y;
+                for (int i = 0; i < 2; ++i) {
+                    rlo[i] = __ffma2_rn(kl[i], cs[i], __fmul2_rn(kh[i], neg2(sn[i])));   // kl*cos - kh*sin
+                    rhi[i] = __ffma2_rn(kh[i], cs[i], __fmul2_rn(kl[i], sn[i]));         // kh*cos + kl*sin
+                }
+#pragma unroll
+                for (int j = 0; j < QPK; ++j) {
+                    float2 acc = __fmul2_rn(qlo[j][0], rlo[0]);
+                    acc = __ffma2_rn(qhi[j][0], rhi[0], acc);
+                    acc = __ffma2_rn(qlo[j][1], rlo[1], acc);
+                    acc = __ffma2_rn(qhi[j][1], rhi[1], acc);
+                    ps[j][k] = acc.x + acc.y;
+                }
             }
         }
         // the queue entry has been consumed: queue the tile DEPTH steps ahead into it
