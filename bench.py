@@ -64,6 +64,24 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def profiled_traffic(workload_name):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if that summary was
+    taken from the kernel sources as they are now (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"decode_split_{workload_name}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        prof = json.load(f)
+    h = hashlib.sha256()
+    for src in ("decode_kernel.cuh", "decode_attn.cu"):
+        with open(os.path.join(ROOT, "looped_lm_decode_b200", "csrc", src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != prof.get("kernel_sources_sha256_16"):
+        return None
+    return prof["dram_bytes_read_per_launch"] + prof["dram_bytes_write_per_launch"]
+
+
 def workload_desc(w):
     return {
         "workload": f"{w.name}: looped decoder, {w.L} layers x {w.T} loop steps (blocks of {w.Tc}), "
@@ -347,7 +365,7 @@ def main():
             "config": dict(workload_desc(w), parallelism=("replicas" if world > 1 else "single GPU")),
             "us_per_step": ms_step * 1e3, "us_per_call": avg_call_ms * 1e3, "calls_per_step": ncall,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": None, "peak_kind": peak_kind,
+                         "frac": achieved / hbm_peak, "traffic": profiled_traffic(w.name), "peak_kind": peak_kind,
                          "kernel": "one loopvq_decode_attn call (split kernel + merge kernel)",
                          "bytes_per_launch": cb},
             "smem_gather": {"achieved": smem_achieved, "peak": smem_peak, "unit": "GB/s",
