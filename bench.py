@@ -378,7 +378,7 @@ def main():
             "encode": {"ms_per_layer_block": statistics.median(enc_ms),
                        "tokens_per_s": w.B * w.Nmax / (statistics.median(enc_ms) * 1e-3),
                        "input_gbs": 2 * w.Tc * w.B * w.Nmax * w.Hkv * w.D * 2 / (statistics.median(enc_ms) * 1e-3) / 1e9,
-                       "kernel": "encode_direct (fp32 exact argmin on CUDA cores)"},
+                       "kernel": "encode_tc_kernel (tcgen05 bf16 distance contraction + TMEM arg-max)"},
         }
         if world == 1 and not args.no_cpu_baseline:
             s, nb, u = cpu_sample(w, args.cpu_seconds)

@@ -127,10 +127,19 @@ static cudaError_t dispatch_c(int c, int tc, const EncodeArgs &a, int x_dtype, i
     return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_encode_tc(const loopvq_cache &cc, int layer, int block, const void *xk, const void *xv,
+                             const int64_t *strides, int b0, int nb, int tok0, int ntok, cudaStream_t s);
+
 cudaError_t launch_encode(const loopvq_cache &cc, int layer, int block, const void *xk, const void *xv,
                           int x_dtype, const int64_t *strides, int b0, int nb, int tok0, int ntok,
                           cudaStream_t s) {
     if (nb == 0 || ntok == 0) return cudaSuccess;
+    // bf16 inputs with a tensor-core instantiation go to the tcgen05 contraction; fp32 inputs (not
+    // representable as bf16 MMA operands) and other shapes use the exact CUDA-core kernel below
+    if (x_dtype == LOOPVQ_BF16) {
+        const cudaError_t e = launch_encode_tc(cc, layer, block, xk, xv, strides, b0, nb, tok0, ntok, s);
+        if (e != cudaErrorNotSupported) return e;
+    }
     EncodeArgs a{};
     a.xk = xk;
     a.xv = xv;

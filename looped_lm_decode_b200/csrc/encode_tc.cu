@@ -1,0 +1,366 @@
+// Encode on the 5th-generation tensor cores (tcgen05): nearest codebook entry as a distance contraction.
+//
+// LoopVQ paper, Sec. 4.3 "Encoding": a block is encoded by computing the distances to all
+// codebook entries as a matrix product on tensor cores, then selecting the nearest entry;
+// Sec. 4.1 eq. (4) for the coupled vectors, Sec. 2 eq. (2) for the nearest-entry rule.
+//
+// ||z - e_r||^2 = ||z||^2 - 2 (z.e_r - ||e_r||^2 / 2), so the nearest entry maximises
+// s_r = z.e_r - h_r with h_r = ||e_r||^2 / 2.  The contraction computes s directly: every
+// coupled vector is extended with three ones and every entry with -h_r split exactly into three
+// bf16 parts, so one bf16 MMA (fp32 accumulate) per 16 coordinates yields s in tensor memory and the
+// epilogue is a plain arg-max (first maximum, i.e. lowest index on ties) per TMEM lane.
+//
+// Tile: M = 128 coupled vectors (TOKS tokens x D/c channel groups of one sequence and KV head) by
+// N = 256 entries; keys and values are two MMAs into the same 256 TMEM columns in turn.  Operands are
+// staged in shared memory in the canonical K-major layout without swizzle: 8-row x 16-byte core
+// matrices, the K-direction neighbour 128 bytes on (leading byte offset), the next 8 rows KB*128
+// bytes on (stride byte offset).  One thread issues the MMAs and commits to an mbarrier; every wait
+// on it is bounded in time, and a timeout writes 0xFFFFFFFF words instead of codes.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "loopvq_internal.cuh"
+
+namespace loopvq {
+
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// SWIZZLE_NONE K-major shared-memory matrix descriptor (tcgen05 format, version 1)
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;          // version
+    return d;                         // base offset 0, lbo mode 0, layout type 0 (no swizzle)
+}
+
+// kind::f16 instruction descriptor: D fp32, A and B bf16, both K-major, M x N
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t mbar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the mbarrier phase with the given parity; false after ~2 s.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity) {
+    if (mbar_try(mbar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try(mbar, parity)) return true;
+        if (globaltimer() - t0 > 2000000000ull) return false;
+    }
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
+          "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+          "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+
+}  // namespace tc
+
+struct EncodeTcArgs {
+    const uint16_t *xk, *xv;  // bf16, element (m, b - b0, n - tok0, h, d)
+    int64_t s0, s1, s2, s3;
+    uint32_t *idx;            // words of (layer, block, b = 0, h = 0)
+    const uint16_t *cb;       // codebook of (layer, block, kv = 0, h = 0): [2][Hkv][K][G]
+    int Hkv, K, Nmax, b0, tok0, ntok, tiles_per_cta;
+};
+
+// Shared-memory plan (bytes): B operands for K and V (256 x KD bf16 each), one A operand (128 x KD),
+// an index staging buffer, the mbarrier and the TMEM base address.
+template <int KD>
+struct TcSmem {
+    static constexpr int kB = 256 * KD * 2;
+    static constexpr int kA = 128 * KD * 2;
+    static constexpr int offBK = 0;
+    static constexpr int offBV = kB;
+    static constexpr int offA = 2 * kB;
+    static constexpr int offCodes = offA + kA;          // 2 x 128 bytes
+    static constexpr int offMbar = offCodes + 256;
+    static constexpr int offTmem = offMbar + 8;
+    static constexpr int kUsed = offTmem + 8;
+    static constexpr int kAlloc = 80 * 1024;            // keeps at most two CTAs per SM: 2 x 256 TMEM columns
+};
+
+template <int D, int C, int TC>
+__global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a) {
+    constexpr int G = C * TC;
+    constexpr int KD = ((G + 3 + 15) / 16) * 16;      // contraction length: coordinates + 3, padded
+    constexpr int KB = KD / 8;                          // 16-byte k-blocks per row
+    constexpr int NG = D / C;                           // channel groups per token
+    constexpr int NP = NG / 2;
+    constexpr int TOKS = 128 / NG;                      // tokens per 128-row tile
+    using S = TcSmem<KD>;
+    static_assert(128 % NG == 0, "tile rows");
+    static_assert(S::kUsed <= S::kAlloc, "shared memory plan");
+
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int h = blockIdx.y, brel = blockIdx.z, b = a.b0 + brel;
+    const uint32_t mbar = tc::smem_u32(smem + S::offMbar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::offTmem);
+    uint8_t *codes = smem + S::offCodes;
+
+    // ---- TMEM (256 columns) and the mbarrier
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc::smem_u32(tmem_slot)),
+                     "r"(256));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        tc::mbar_init(mbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+
+    // ---- B operands: entry r -> [e_r (G coords), -h_hi, -h_mid, -h_lo, 0 ...], h = ||e_r||^2 / 2
+    for (int it = tid; it < 2 * 256; it += 128) {
+        const int kv = it >> 8, r = it & 255;
+        uint16_t row[KD];
+#pragma unroll
+        for (int k = 0; k < KD; ++k) row[k] = 0;
+        if (r < a.K) {
+            const uint16_t *e = a.cb + ((size_t)kv * a.Hkv + h) * (size_t)a.K * G + (size_t)r * G;
+            double hh = 0.0;
+#pragma unroll
+            for (int k = 0; k < G; ++k) {
+                row[k] = e[k];
+                const double v = (double)bf16_to_f32(e[k]);
+                hh += v * v;
+            }
+            hh *= 0.5;
+            const float p1 = __bfloat162float(__float2bfloat16_rn((float)hh));
+            const double r1 = hh - (double)p1;
+            const float p2 = __bfloat162float(__float2bfloat16_rn((float)r1));
+            const double r2 = r1 - (double)p2;
+            row[G] = tc::bf16_bits_rn(-p1);
+            row[G + 1] = tc::bf16_bits_rn(-p2);
+            row[G + 2] = tc::bf16_bits_rn((float)-r2);
+        } else {
+            row[G] = tc::bf16_bits_rn(-1.0e30f);       // entries past K never win
+        }
+        unsigned char *base = smem + (kv ? S::offBV : S::offBK) + ((r >> 3) * KB) * 128 + (r & 7) * 16;
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+            uint4 v;
+            v.x = row[kb * 8 + 0] | ((uint32_t)row[kb * 8 + 1] << 16);
+            v.y = row[kb * 8 + 2] | ((uint32_t)row[kb * 8 + 3] << 16);
+            v.z = row[kb * 8 + 4] | ((uint32_t)row[kb * 8 + 5] << 16);
+            v.w = row[kb * 8 + 6] | ((uint32_t)row[kb * 8 + 7] << 16);
+            *reinterpret_cast<uint4 *>(base + kb * 128) = v;
+        }
+    }
+    tc::fence_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const uint32_t idesc = tc::idesc_bf16(128, 256);
+    const uint32_t aaddr = tc::smem_u32(smem + S::offA);
+    const uint32_t bkaddr = tc::smem_u32(smem + S::offBK), bvaddr = tc::smem_u32(smem + S::offBV);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int row = tid;                                   // TMEM lane == tile row == thread
+    const int rtok = row / NG, rg = row % NG;
+    const int ntiles = (a.ntok + TOKS - 1) / TOKS;
+    const int t_begin = blockIdx.x * a.tiles_per_cta;
+    const int t_end = min(t_begin + a.tiles_per_cta, ntiles);
+    uint32_t *idx_bh = a.idx + ((size_t)b * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C);
+
+    for (int tile = t_begin; tile < t_end; ++tile) {
+        const int nrel = tile * TOKS + rtok;               // this row's token, relative to tok0
+        const bool valid = nrel < a.ntok;
+#pragma unroll 1
+        for (int kv = 0; kv < 2; ++kv) {
+            // ---- A operand: this row's coupled vector, extended by three ones
+            {
+                uint16_t zr[KD];
+#pragma unroll
+                for (int k = 0; k < KD; ++k) zr[k] = 0;
+                if (valid) {
+                    const uint16_t *x = (kv ? a.xv : a.xk) + (size_t)brel * a.s1 + (size_t)nrel * a.s2 +
+                                        (size_t)h * a.s3 + rg * C;
+#pragma unroll
+                    for (int m = 0; m < TC; ++m)
+#pragma unroll
+                        for (int i = 0; i < C; ++i) zr[i * TC + m] = __ldg(x + (size_t)m * a.s0 + i);
+                }
+                zr[G] = zr[G + 1] = zr[G + 2] = 0x3F80;       // bf16 1.0
+                unsigned char *base = smem + S::offA + ((row >> 3) * KB) * 128 + (row & 7) * 16;
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+                    uint4 v;
+                    v.x = zr[kb * 8 + 0] | ((uint32_t)zr[kb * 8 + 1] << 16);
+                    v.y = zr[kb * 8 + 2] | ((uint32_t)zr[kb * 8 + 3] << 16);
+                    v.z = zr[kb * 8 + 4] | ((uint32_t)zr[kb * 8 + 5] << 16);
+                    v.w = zr[kb * 8 + 6] | ((uint32_t)zr[kb * 8 + 7] << 16);
+                    *reinterpret_cast<uint4 *>(base + kb * 128) = v;
+                }
+            }
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            __syncthreads();
+            // ---- s = [z, 1, 1, 1] . [e, -h] for all 256 entries, into TMEM columns [0, 256)
+            if (tid == 0) {
+                tc::tc_fence_after();
+                const uint32_t baddr = kv ? bvaddr : bkaddr;
+#pragma unroll
+                for (int ks = 0; ks < KD / 16; ++ks) {
+                    const uint64_t ad = tc::smem_desc(aaddr + ks * 256, 128, KB * 128);
+                    const uint64_t bd = tc::smem_desc(baddr + ks * 256, 128, KB * 128);
+                    tc::mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(mbar);
+            }
+            // every thread waits (bounded); the CTA continues only if all of them saw the MMAs complete
+            ok = __syncthreads_and(tc::mbar_wait_bounded(mbar, phase) ? 1 : 0) != 0;
+            phase ^= 1u;
+            if (!ok) break;
+            tc::tc_fence_after();
+            // ---- arg-max over the entries of this row (first maximum wins)
+            float best = -CUDART_INF_F;
+            int bi = 0;
+            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < 256; c0 += 64) {
+                uint32_t va[32], vb[32];
+                tc::tmem_ld32(taddr + c0, va);
+                tc::tmem_ld32(taddr + c0 + 32, vb);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float v = __uint_as_float(va[j]);
+                    if (v > best && c0 + j < a.K) { best = v; bi = c0 + j; }
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float v = __uint_as_float(vb[j]);
+                    if (v > best && c0 + 32 + j < a.K) { best = v; bi = c0 + 32 + j; }
+                }
+            }
+            codes[kv * 128 + row] = (uint8_t)bi;
+            tc::tc_fence_before();
+            __syncthreads();                               // TMEM and the A operand are free again
+        }
+        // ---- pack {K p, K p+NP, V p, V p+NP} words and store them (sentinel words after a timeout)
+        if (tid < TOKS * NP) {
+            const int t = tid / NP, p = tid % NP;
+            const int nr = tile * TOKS + t;
+            if (nr < a.ntok) {
+                const uint32_t w = ok ? ((uint32_t)codes[t * NG + p] | ((uint32_t)codes[t * NG + p + NP] << 8) |
+                                         ((uint32_t)codes[128 + t * NG + p] << 16) |
+                                         ((uint32_t)codes[128 + t * NG + p + NP] << 24))
+                                      : 0xFFFFFFFFu;
+                idx_bh[idx_word(a.tok0 + nr, p, NP)] = w;
+            }
+        }
+        __syncthreads();
+        if (!ok) break;
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+}
+
+template <int D, int C, int TC>
+static cudaError_t launch_tc_ct(const EncodeTcArgs &a0, int nb, cudaStream_t s) {
+    constexpr int NG = D / C;
+    constexpr int TOKS = 128 / NG;
+    constexpr int KD = ((C * TC + 3 + 15) / 16) * 16;
+    EncodeTcArgs a = a0;
+    const int ntiles = (a.ntok + TOKS - 1) / TOKS;
+    // enough CTAs per (sequence, head) to fill the GPU twice over, each looping over its tiles
+    const long units = (long)a.Hkv * nb;
+    long per = (2L * 148 + units - 1) / units;
+    if (per < 1) per = 1;
+    if (per > ntiles) per = ntiles;
+    a.tiles_per_cta = (int)((ntiles + per - 1) / per);
+    const int gx = (ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+    auto k = encode_tc_kernel<D, C, TC>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSmem<KD>::kAlloc);
+    if (e != cudaSuccess) return e;
+    dim3 grid(gx, a.Hkv, nb);
+    k<<<grid, 128, TcSmem<KD>::kAlloc, s>>>(a);
+    return cudaGetLastError();
+}
+
+// Returns cudaErrorNotSupported when the shape has no tensor-core instantiation.
+cudaError_t launch_encode_tc(const loopvq_cache &cc, int layer, int block, const void *xk, const void *xv,
+                             const int64_t *strides, int b0, int nb, int tok0, int ntok, cudaStream_t s) {
+    EncodeTcArgs a{};
+    a.xk = reinterpret_cast<const uint16_t *>(xk);
+    a.xv = reinterpret_cast<const uint16_t *>(xv);
+    a.s0 = strides[0];
+    a.s1 = strides[1];
+    a.s2 = strides[2];
+    a.s3 = strides[3];
+    a.idx = cc.idx + idx_base(cc, layer, block, 0, 0);
+    a.cb = cc.codebook + codebook_base(cc, layer, block, 0, 0);
+    a.Hkv = cc.Hkv;
+    a.K = cc.K;
+    a.Nmax = cc.Nmax;
+    a.b0 = b0;
+    a.tok0 = tok0;
+    a.ntok = ntok;
+    const int G = cc.c * cc.Tc;
+    if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4>(a, nb, s);
+    if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4>(a, nb, s);
+    if (cc.D == 64 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<64, 4, 4>(a, nb, s);
+    if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4>(a, nb, s);
+    (void)G;
+    return cudaErrorNotSupported;
+}
+
+}  // namespace loopvq
