@@ -64,6 +64,21 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def max_over_ranks(x, dist=None, device="cpu"):
+    """Maximum of a per-rank float over all ranks (the slowest rank sets every timed figure)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, bytes_per_step_per_rank, ms_per_step_max):
+    """Whole-job algorithmic bytes per second (GB/s) under weak scaling: every rank serves its own batch."""
+    return world * bytes_per_step_per_rank / (ms_per_step_max * 1e-3) / 1e9
+
+
 def profiled_traffic(workload_name):
     """DRAM bytes per launch of the decode kernel from the committed ncu summary, if that summary was
     taken from the kernel sources as they are now (else None)."""
@@ -337,22 +352,15 @@ def main():
     h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * 4
     d2h = out_host.numel() * 4 + lse_host.numel() * 4
 
-    def allmax(x):
-        if dist is None:
-            return x
-        tt = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        return float(tt.item())
-
-    ms_step = allmax(ms_step_local)
-    e2e_ms = allmax(e2e_ms_local)
-    avg_call_ms = allmax(statistics.fmean(call_ms))
+    ms_step = max_over_ranks(ms_step_local, dist, dev)
+    e2e_ms = max_over_ranks(e2e_ms_local, dist, dev)
+    avg_call_ms = max_over_ranks(statistics.fmean(call_ms), dist, dev)
 
     if rank == 0:
         cb = call_bytes(w, lens_np)
         gb = gather_bytes(w, lens_np)
         step_bytes = cb * ncall
-        value = world * step_bytes / (ms_step * 1e-3) / 1e9
+        value = job_throughput(world, step_bytes, ms_step)
         hbm_peak, peak_kind = peaks()
         achieved = cb / (avg_call_ms * 1e-3) / 1e9
         sm_mhz = clk.get("sm_mhz") or 1965.0
@@ -372,7 +380,7 @@ def main():
                             "frac": smem_achieved / smem_peak, "bytes_per_launch": gb,
                             "peak_kind": f"derived: {SMEM_BYTES_PER_CLK_SM} B/clk/SM x {N_SM} SMs x median SM clock"},
             "clocks": clk,
-            "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "e2e": {"value": job_throughput(world, step_bytes, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * ncall * 2,
             "encode": {"ms_per_layer_block": statistics.median(enc_ms),

@@ -16,13 +16,14 @@ namespace loopvq {
 static constexpr int kWarps = 8;
 static constexpr int kMinBlocks = 2;
 static constexpr int kDepth = 4;
+static constexpr int kWords = 1;                          // index words per lane per iteration (4-token tiles)
 static constexpr long kTargetCtas = 148L * 2 * 4;
 
-static size_t ring_smem_bytes() { return 65536 + (size_t)kDepth * kWarps * 32 * 16; }
+static size_t ring_smem_bytes() { return 65536 + (size_t)kDepth * kWarps * 32 * 16 * kWords; }
 
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len) {
     DecodePlan p{};
-    const int stride = 4 * kWarps * (32 / (cc.D / 8));    // tokens between two tiles of one slot
+    const int stride = 4 * kWords * kWarps * (32 / (cc.D / 8));   // tokens between two iterations of a slot
     p.nbt = 1;
     p.nchunk = cc.B;
     const long units = (long)cc.Hkv * cc.B;
@@ -44,8 +45,7 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStr
     const size_t red = (size_t)NSLOT * QPK * (D + 4) * sizeof(float);
     const size_t smem = ring_smem_bytes();
     if (red > smem) return cudaErrorInvalidConfiguration;   // the slot records reuse slices and queue
-    // one query head per KV head: rotate the query (cheaper than rotating every key); GQA rotates keys once
-    auto kern = decode_split_kernel<D, C, QPK, kWarps, kMinBlocks, kDepth, QPK == 1, false>;
+    auto kern = decode_split_kernel<D, C, QPK, kWarps, kMinBlocks, kDepth, kWords>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (plan.nsplit > 0) {

@@ -81,21 +81,79 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, bool ROTQ, bool K32>
+// Sum of the T partial scores of a lane over the NL lanes of its slot, scattered so that each lane
+// ends with the full score of one token: log2(T) halving exchanges, then butterflies over the
+// remaining lane bits.  The token a lane finishes is given by tile_token().
+template <int T, int NL>
+__device__ __forceinline__ float reduce_scatter(const float (&v)[T], int ls, unsigned mask) {
+    static_assert(T == 4 || T == 8, "tile");
+    float a[T / 2];
+    constexpr int o1 = NL / 2;
+    const bool b1 = (ls & o1) != 0;
+#pragma unroll
+    for (int i = 0; i < T / 2; ++i) {
+        const float keep = b1 ? v[T / 2 + i] : v[i];
+        const float send = b1 ? v[i] : v[T / 2 + i];
+        a[i] = keep + __shfl_xor_sync(mask, send, o1);
+    }
+    float c[T / 4];
+    constexpr int o2 = NL / 4;
+    const bool b2 = (ls & o2) != 0;
+#pragma unroll
+    for (int i = 0; i < T / 4; ++i) {
+        const float keep = b2 ? a[T / 4 + i] : a[i];
+        const float send = b2 ? a[i] : a[T / 4 + i];
+        c[i] = keep + __shfl_xor_sync(mask, send, o2);
+    }
+    float r;
+    int obut;
+    if constexpr (T == 8) {
+        constexpr int o3 = NL / 8;
+        const bool b3 = (ls & o3) != 0;
+        const float keep = b3 ? c[1] : c[0];
+        const float send = b3 ? c[0] : c[1];
+        r = keep + __shfl_xor_sync(mask, send, o3);
+        obut = NL / 16;
+    } else {
+        r = c[0];
+        obut = NL / 8;
+    }
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1)
+        if (o <= obut) r += __shfl_xor_sync(mask, r, o);
+    return r;
+}
+
+template <int T, int NL>
+__device__ __forceinline__ int tile_token(int ls) {
+    int t = ((ls & (NL / 2)) ? T / 2 : 0) + ((ls & (NL / 4)) ? T / 4 : 0);
+    if constexpr (T == 8) t += (ls & (NL / 8)) ? 1 : 0;
+    return t;
+}
+
+template <int T, int NL>
+__device__ __forceinline__ int tile_owner(int t) {          // a lane of the slot that finishes token t
+    int l = ((t & (T / 2)) ? NL / 2 : 0) + ((t & (T / 4)) ? NL / 4 : 0);
+    if constexpr (T == 8) l += (t & 1) ? NL / 8 : 0;
+    return l;
+}
+
+template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, int NW>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const DecodeArgs a) {
+    constexpr bool ROTQ = QPK == 1;                        // rotate the query, not every key
     constexpr int NP = D / (2 * C);                        // pair-groups = index words per token
     constexpr int HALVES = C / 4;                          // lanes sharing one pair-group
     constexpr int NL = D / 8;                              // lanes per token slot
     constexpr int SPW = 32 / NL;                           // slots per warp
     constexpr int NSLOT = WARPS * SPW;
     constexpr int NT = WARPS * 32;
-    constexpr int EB = 2 * C;                              // bytes of one bf16 slice entry
-    constexpr int REPL = 128 / EB;                         // bf16 replicas per half-row
-    constexpr int REPLK = K32 ? 128 / (4 * C) : REPL;      // K replicas (fp32 entries when K32)
-    constexpr int STRIDE = NSLOT * 4;                      // tokens between two tiles of a slot
+    constexpr int EB = 2 * C;                              // bytes of one slice entry
+    constexpr int REPL = 128 / EB;                         // replicas per half-row
+    constexpr int TT = 4 * NW;                             // tokens per slot iteration
+    constexpr int STRIDE = NSLOT * TT;                     // tokens between two iterations of a slot
+    constexpr int QB = NT * 16 * NW;                       // bytes of one prefetch-queue stage
     static_assert(C == 4 || C == 8, "c");
-    static_assert(!ROTQ || QPK == 1, "query rotation is for one query head per KV head");
-    static_assert(NL >= 4 && NL <= 16, "slot width");
+    static_assert(NL >= 8 && NL <= 16, "slot width");
 
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -111,19 +169,21 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     const int slot = warp * SPW + lane / NL;
     const unsigned slot_mask = ((1u << NL) - 1u) << (lane & ~(NL - 1));
     const int slot_lane0 = lane & ~(NL - 1);
-    const uint32_t colk = K32 ? (uint32_t)((lane % 8) * 16)   // fp32 keys: 16-byte pieces, 8 per wavefront
-                              : (uint32_t)((lane % 16) * 8);  // bf16: 8-byte pieces, 16 per wavefront
-    const uint32_t colv = (uint32_t)((lane % 16) * 8) + 128u; // byte 0 of every V gather address
+    const uint32_t colk = (uint32_t)((lane % 16) * 8);     // byte 0 of every K gather address
+    const uint32_t colv = colk + 128u;                     // ... of every V gather address
     const int ch = gp * C + half * 4;                      // first of this lane's 4 low channels
     const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP + ((size_t)gp << 2);
     const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) + 65536u + (uint32_t)tid * 16u;
 
-    // queue the first DEPTH tiles of this slot before staging the slices
-    const int pfirst = tok_begin + slot * 4;
+    // queue the first DEPTH iterations of this slot before staging the slices
+    const int pfirst = tok_begin + slot * TT;
 #pragma unroll
     for (int d = 0; d < DEPTH; ++d) {
         const int p = pfirst + d * STRIDE;
-        if (p < tok_end) cp_async16(ring + (uint32_t)(d * NT * 16), idx_b + (size_t)(p >> 2) * NP * 4);
+#pragma unroll
+        for (int u = 0; u < NW; ++u)
+            if (p + 4 * u < tok_end)
+                cp_async16(ring + (uint32_t)(d * QB + u * NT * 16), idx_b + (size_t)((p >> 2) + u) * NP * 4);
         cp_async_commit();
     }
 
@@ -131,22 +191,9 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     {
         const uint16_t *sk = a.slk + (size_t)h * a.K * C;
         const uint16_t *sv = a.slv + (size_t)h * a.K * C;
-        if constexpr (K32) {
-            // K half-rows: REPLK replicas of the entry widened to fp32 (4C bytes)
-            for (int it = tid; it < 256 * REPLK * (C / 4); it += NT) {
-                const int q4 = it % (C / 4);
-                const int rep = (it / (C / 4)) % REPLK;
-                const int r = it / (REPLK * (C / 4));
-                uint2 v = make_uint2(0u, 0u);
-                if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(sk + (size_t)r * C + q4 * 4));
-                *reinterpret_cast<float4 *>(smem + r * 256 + rep * 4 * C + q4 * 16) =
-                    make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-            }
-        }
         for (int it = tid; it < 256 * 2 * REPL; it += NT) {
             const int rep = it % REPL;
             const int kv = (it / REPL) & 1;
-            if (K32 && kv == 0) continue;
             const int r = it / (2 * REPL);
             unsigned char *dst = smem + r * 256 + kv * 128 + rep * EB;
             const uint16_t *src = (kv ? sv : sk) + (size_t)r * C;
@@ -193,11 +240,9 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         l_[j] = 0.f;
         olo[j][0] = olo[j][1] = ohi[j][0] = ohi[j][1] = f2(0.f, 0.f);
     }
-    const bool hb = (ls & (NL / 2)) != 0;
-    const bool mb = (ls & (NL / 4)) != 0;
-    const int tk = (hb ? 2 : 0) + (mb ? 1 : 0);            // token of the tile this lane finishes
+    const int tk = tile_token<TT, NL>(ls);                 // token of the iteration this lane finishes
 
-    // RoPE row of each tile's first token, loaded one tile ahead
+    // RoPE row of each iteration's first token, loaded one iteration ahead
     float4 ra_c, ra_s;
     {
         const float *row = a.rope + (size_t)min(pfirst, a.Nmax - 4) * D + ch;
@@ -208,12 +253,23 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 
     int stage = 0;
     for (int p0 = pfirst; p0 < tok_end; p0 += STRIDE) {
-        cp_async_wait<DEPTH - 1>();                        // this thread's oldest queued tile has landed
-        uint4 w4;
-        {
-            const uint32_t addr = ring + (uint32_t)(stage * NT * 16);
+        cp_async_wait<DEPTH - 1>();                        // this thread's oldest queued stage has landed
+        uint4 w4[NW];
+#pragma unroll
+        for (int u = 0; u < NW; ++u) {
+            const uint32_t addr = ring + (uint32_t)(stage * QB + u * NT * 16);
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w4.x), "=r"(w4.y), "=r"(w4.z), "=r"(w4.w) : "r"(addr) : "memory");
+                         : "=r"(w4[u].x), "=r"(w4[u].y), "=r"(w4[u].z), "=r"(w4[u].w) : "r"(addr) : "memory");
+        }
+        // the stage has been read into registers: queue the iteration DEPTH steps ahead into it
+        {
+            const int pq = p0 + DEPTH * STRIDE;
+#pragma unroll
+            for (int u = 0; u < NW; ++u)
+                if (pq + 4 * u < tok_end)
+                    cp_async16(ring + (uint32_t)(stage * QB + u * NT * 16), idx_b + (size_t)((pq >> 2) + u) * NP * 4);
+            cp_async_commit();
+            stage = stage + 1 == DEPTH ? 0 : stage + 1;
         }
         float2 cs[2] = {f2(ra_c.x, ra_c.y), f2(ra_c.z, ra_c.w)};
         float2 sn[2] = {f2(ra_s.x, ra_s.y), f2(ra_s.z, ra_s.w)};
@@ -223,11 +279,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             ra_s = __ldg(reinterpret_cast<const float4 *>(row + D / 2));
         }
 
-        // ---- keys: rebuild, rotate, partial dot per query head
-        float ps[QPK][4];
-        // ROTQ: rotate the query instead of every key.  With Z = (q_f + i q_{f+D/2}) e^{-i p w_f},
-        // the score term of pair f is Re(Z) k_f + Im(Z) k_{f+D/2}; Z of the next position is Z times
-        // e^{-i w_f}.  Otherwise keys are rotated by (cos, sin), advanced one position per token.
+        // ---- keys: rebuild, score.  ROTQ: per pair f the term is Re(Z) k_f + Im(Z) k_{f+D/2} with
+        // Z = (q_f + i q_{f+D/2}) e^{-i p w_f}, advanced one position per token by one complex multiply.
+        // Otherwise the rebuilt keys are rotated by (cos, sin), advanced the same way, and shared.
+        float ps[QPK][TT];
         float2 zu[2], zw[2];
         if constexpr (ROTQ) {
 #pragma unroll
@@ -237,7 +292,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             }
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < TT; ++k) {
             if (k > 0) {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
@@ -254,23 +309,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                     }
                 }
             }
-            const uint32_t w = word_k(w4, k);
-            float2 kl[2], kh[2];
-            if constexpr (K32) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(smem + __byte_perm(w, colk, 0x7604));
-                const float4 b4 = *reinterpret_cast<const float4 *>(smem + __byte_perm(w, colk, 0x7614));
-                kl[0] = f2(a4.x, a4.y);
-                kl[1] = f2(a4.z, a4.w);
-                kh[0] = f2(b4.x, b4.y);
-                kh[1] = f2(b4.z, b4.w);
-            } else {
-                const uint2 elo = lds64(smem, __byte_perm(w, colk, 0x7604));
-                const uint2 ehi = lds64(smem, __byte_perm(w, colk, 0x7614));
-                kl[0] = unpack2(elo.x);
-                kl[1] = unpack2(elo.y);
-                kh[0] = unpack2(ehi.x);
-                kh[1] = unpack2(ehi.y);
-            }
+            const uint32_t w = word_k(w4[k >> 2], k & 3);
+            const uint2 elo = lds64(smem, __byte_perm(w, colk, 0x7604));
+            const uint2 ehi = lds64(smem, __byte_perm(w, colk, 0x7614));
+            const float2 kl[2] = {unpack2(elo.x), unpack2(elo.y)};
+            const float2 kh[2] = {unpack2(ehi.x), unpack2(ehi.y)};
             if constexpr (ROTQ) {
                 float2 acc = __fmul2_rn(zu[0], kl[0]);
                 acc = __ffma2_rn(zw[0], kh[0], acc);
@@ -294,34 +337,21 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 }
             }
         }
-        // the queue entry has been consumed: queue the tile DEPTH steps ahead into it
-        {
-            const int pq = p0 + DEPTH * STRIDE;
-            if (pq < tok_end) cp_async16(ring + (uint32_t)(stage * NT * 16), idx_b + (size_t)(pq >> 2) * NP * 4);
-            cp_async_commit();
-            stage = stage + 1 == DEPTH ? 0 : stage + 1;
-        }
 
-        // ---- reduce-scatter the 4 scores over the slot, online-softmax update
+        // ---- reduce-scatter the scores over the slot, online-softmax update
         float pe[QPK];
 #pragma unroll
         for (int j = 0; j < QPK; ++j) {
-            float keep0 = hb ? ps[j][2] : ps[j][0], keep1 = hb ? ps[j][3] : ps[j][1];
-            const float send0 = hb ? ps[j][0] : ps[j][2], send1 = hb ? ps[j][1] : ps[j][3];
-            keep0 += __shfl_xor_sync(slot_mask, send0, NL / 2);
-            keep1 += __shfl_xor_sync(slot_mask, send1, NL / 2);
-            float keep = mb ? keep1 : keep0;
-            const float send = mb ? keep0 : keep1;
-            keep += __shfl_xor_sync(slot_mask, send, NL / 4);
-#pragma unroll
-            for (int o = NL / 8; o >= 1; o >>= 1) keep += __shfl_xor_sync(slot_mask, keep, o);
+            const float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
             const float s = (p0 + tk < tok_end) ? keep : -CUDART_INF_F;
             // Lazy maximum: the reference only has to stay within 2^8 of the running maximum for
             // the weights to stay finite, so it moves (with an exact rescale) only when a score of
-            // the tile exceeds it by more than 8 in log2 units.
+            // the iteration exceeds it by more than 8 in log2 units.
             if (__any_sync(slot_mask, s > m_[j] + 8.f)) {
-                float tmax = fmaxf(s, __shfl_xor_sync(slot_mask, s, NL / 4));
-                tmax = fmaxf(tmax, __shfl_xor_sync(slot_mask, tmax, NL / 2));
+                float tmax = s;
+#pragma unroll
+                for (int o = NL / 2; o >= NL / TT; o >>= 1)
+                    tmax = fmaxf(tmax, __shfl_xor_sync(slot_mask, tmax, o));
                 const float corr = ex2(m_[j] - tmax);
                 l_[j] *= corr;
                 const float2 c2 = f2(corr, corr);
@@ -338,9 +368,9 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 
         // ---- values: rebuild and accumulate with each token's weight
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int src = slot_lane0 + (k >> 1) * (NL / 2) + (k & 1) * (NL / 4);
-            const uint32_t w = word_k(w4, k);
+        for (int k = 0; k < TT; ++k) {
+            const int src = slot_lane0 + tile_owner<TT, NL>(k);
+            const uint32_t w = word_k(w4[k >> 2], k & 3);
             const uint2 vlo = lds64(smem, __byte_perm(w, colv, 0x7624));
             const uint2 vhi = lds64(smem, __byte_perm(w, colv, 0x7634));
             const uint32_t vl[2] = {vlo.x, vlo.y}, vh[2] = {vhi.x, vhi.y};
@@ -359,13 +389,16 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     cp_async_wait<0>();
 
     // ---- combine the slots of this CTA, write the split's partial result
-    __syncthreads();                                       // slices no longer needed
+    __syncthreads();                                       // slices and queue no longer needed
     constexpr int RS = D + 4;                              // floats per (slot, query head) record
+    // l_ sums the weights of the tokens this lane finished: add the other token positions of the slot
+    constexpr int TOKBITS = (TT == 8) ? 3 : 2;
     float *red = reinterpret_cast<float *>(smem);
 #pragma unroll
     for (int j = 0; j < QPK; ++j) {
-        float lsum = l_[j] + __shfl_xor_sync(slot_mask, l_[j], NL / 4);
-        lsum += __shfl_xor_sync(slot_mask, lsum, NL / 2);
+        float lsum = l_[j];
+#pragma unroll
+        for (int sb = 0; sb < TOKBITS; ++sb) lsum += __shfl_xor_sync(slot_mask, lsum, NL >> (1 + sb));
         float *rec = red + ((size_t)slot * QPK + j) * RS;
         *reinterpret_cast<float4 *>(rec + ch) = make_float4(olo[j][0].x, olo[j][0].y, olo[j][1].x, olo[j][1].y);
         *reinterpret_cast<float4 *>(rec + D / 2 + ch) = make_float4(ohi[j][0].x, ohi[j][0].y, ohi[j][1].x, ohi[j][1].y);

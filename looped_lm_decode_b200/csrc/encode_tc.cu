@@ -218,24 +218,40 @@ __global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a)
     const int t_end = min(t_begin + a.tiles_per_cta, ntiles);
     uint32_t *idx_bh = a.idx + ((size_t)b * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C);
 
+    // this row's coupled vectors (keys and values) of the next tile are loaded one tile ahead
+    uint16_t zn[2][G];
+    auto load_row = [&](int tile, uint16_t (&z)[2][G]) {
+        const int nrel = tile * TOKS + rtok;
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+#pragma unroll
+            for (int k = 0; k < G; ++k) z[kv][k] = 0;
+            if (tile < t_end && nrel < a.ntok) {
+                const uint16_t *x = (kv ? a.xv : a.xk) + (size_t)brel * a.s1 + (size_t)nrel * a.s2 +
+                                    (size_t)h * a.s3 + rg * C;
+#pragma unroll
+                for (int m = 0; m < TC; ++m)
+#pragma unroll
+                    for (int i = 0; i < C; ++i) z[kv][i * TC + m] = __ldg(x + (size_t)m * a.s0 + i);
+            }
+        }
+    };
+    load_row(t_begin, zn);
+
     for (int tile = t_begin; tile < t_end; ++tile) {
-        const int nrel = tile * TOKS + rtok;               // this row's token, relative to tok0
-        const bool valid = nrel < a.ntok;
+        uint16_t zc[2][G];
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv)
+#pragma unroll
+            for (int k = 0; k < G; ++k) zc[kv][k] = zn[kv][k];
+        load_row(tile + 1, zn);
 #pragma unroll 1
         for (int kv = 0; kv < 2; ++kv) {
             // ---- A operand: this row's coupled vector, extended by three ones
             {
                 uint16_t zr[KD];
 #pragma unroll
-                for (int k = 0; k < KD; ++k) zr[k] = 0;
-                if (valid) {
-                    const uint16_t *x = (kv ? a.xv : a.xk) + (size_t)brel * a.s1 + (size_t)nrel * a.s2 +
-                                        (size_t)h * a.s3 + rg * C;
-#pragma unroll
-                    for (int m = 0; m < TC; ++m)
-#pragma unroll
-                        for (int i = 0; i < C; ++i) zr[i * TC + m] = __ldg(x + (size_t)m * a.s0 + i);
-                }
+                for (int k = 0; k < KD; ++k) zr[k] = k < G ? (kv ? zc[1][k] : zc[0][k]) : 0;
                 zr[G] = zr[G + 1] = zr[G + 2] = 0x3F80;       // bf16 1.0
                 unsigned char *base = smem + S::offA + ((row >> 3) * KB) * 128 + (row & 7) * 16;
 #pragma unroll
@@ -278,15 +294,16 @@ __global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a)
                 tc::tmem_ld32(taddr + c0, va);
                 tc::tmem_ld32(taddr + c0 + 32, vb);
                 tc::tmem_wait_ld();
+                // entries at or past K score -1e30 through their extended coordinate, so they never win
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const float v = __uint_as_float(va[j]);
-                    if (v > best && c0 + j < a.K) { best = v; bi = c0 + j; }
+                    if (v > best) { best = v; bi = c0 + j; }
                 }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const float v = __uint_as_float(vb[j]);
-                    if (v > best && c0 + 32 + j < a.K) { best = v; bi = c0 + 32 + j; }
+                    if (v > best) { best = v; bi = c0 + 32 + j; }
                 }
             }
             codes[kv * 128 + row] = (uint8_t)bi;
