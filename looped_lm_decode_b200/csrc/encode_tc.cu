@@ -100,12 +100,92 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Wait for this thread's outstanding tcgen05.ld; the registers are named so that no read of them can be
+// scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&v)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                   "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                   "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                   "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
+                   "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+                 :
+                 : "memory");
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ uint16_t bf16_bits_rn(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+
+// Exact arg-max of a TMEM lane's scores in two passes over the same columns.  Pass 1 takes the maximum
+// M with three-input max.  Pass 2 finds the first column whose score is >= M (so == M): in each run of
+// 32 columns, column j adds set(s_j >= M) * 2^-(j mod 32) to one of two accumulators of 16 columns, so
+// each accumulator is an exact sum of distinct powers of two whose exponent names its lowest hit.
+__device__ __forceinline__ float max3f(float x, float y, float z) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(x), "f"(y), "f"(z));
+    return r;
+}
+
+__device__ __forceinline__ float ge_one(float x, float m) {      // 1.0f if x >= m, else 0.0f
+    float r;
+    asm("set.ge.f32.f32 %0, %1, %2;" : "=f"(r) : "f"(x), "f"(m));
+    return r;
+}
+
+// maximum of NCOLS columns from column col0 (64 columns per wait)
+template <int NCOLS>
+__device__ __forceinline__ float cols_max(uint32_t taddr, int col0) {
+    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, m2 = -CUDART_INF_F, m3 = -CUDART_INF_F;
+#pragma unroll 1
+    for (int c = 0; c < NCOLS; c += 64) {
+        uint32_t va[32], vb[32];
+        tmem_ld32(taddr + col0 + c, va);
+        tmem_ld32(taddr + col0 + c + 32, vb);
+        tmem_wait_ld(va);
+        tmem_wait_ld(vb);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            m0 = max3f(m0, __uint_as_float(va[j]), __uint_as_float(va[j + 1]));
+            m1 = max3f(m1, __uint_as_float(va[j + 2]), __uint_as_float(va[j + 3]));
+            m2 = max3f(m2, __uint_as_float(vb[j]), __uint_as_float(vb[j + 1]));
+            m3 = max3f(m3, __uint_as_float(vb[j + 2]), __uint_as_float(vb[j + 3]));
+        }
+    }
+    return max3f(m0, m1, fmaxf(m2, m3));
+}
+
+// first of 32 columns (from c0) with score >= M, or -1
+__device__ __forceinline__ int first_hit32(const uint32_t (&v)[32], float M, int c0) {
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        acc0 = fmaf(ge_one(__uint_as_float(v[j]), M), __int_as_float((127 - j) << 23), acc0);
+        acc1 = fmaf(ge_one(__uint_as_float(v[16 + j]), M), __int_as_float((127 - 16 - j) << 23), acc1);
+    }
+    const float r = fmaxf(acc0, acc1);       // 0, or in [2^-31, 2): exponent 127 - (lowest hit)
+    return r > 0.f ? c0 + 127 - (int)(__float_as_uint(r) >> 23) : -1;
+}
+
+// first of NCOLS columns from col0 with score >= M, or -1
+template <int NCOLS>
+__device__ __forceinline__ int cols_first(uint32_t taddr, int col0, float M) {
+    int best = -1;
+#pragma unroll 1
+    for (int c = 0; c < NCOLS; c += 64) {
+        uint32_t va[32], vb[32];
+        tmem_ld32(taddr + col0 + c, va);
+        tmem_ld32(taddr + col0 + c + 32, vb);
+        tmem_wait_ld(va);
+        tmem_wait_ld(vb);
+        const int ia = first_hit32(va, M, col0 + c);
+        const int ib = first_hit32(vb, M, col0 + c + 32);
+        const int i = ia >= 0 ? ia : ib;
+        if (best < 0) best = i;
+    }
+    return best;
+}
 
 }  // namespace tc
 
@@ -114,27 +194,33 @@ struct EncodeTcArgs {
     int64_t s0, s1, s2, s3;
     uint32_t *idx;            // words of (layer, block, b = 0, h = 0)
     const uint16_t *cb;       // codebook of (layer, block, kv = 0, h = 0): [2][Hkv][K][G]
-    int Hkv, K, Nmax, b0, tok0, ntok, tiles_per_cta;
+    int Hkv, K, Nmax, b0, nb, tok0, ntok;
+    long long units_per_cta;  // flattened (head, sequence, tile) units, head-major, per CTA
 };
 
-// Shared-memory plan (bytes): B operands for K and V (256 x KD bf16 each), one A operand (128 x KD),
-// an index staging buffer, the mbarrier and the TMEM base address.
+// Shared-memory plan (bytes): B operands for K and V (256 x KD bf16 each), A operands for K and V
+// (128 x KD each), the code staging buffer, a per-row exchange area, the mbarrier and the TMEM address.
 template <int KD>
 struct TcSmem {
     static constexpr int kB = 256 * KD * 2;
     static constexpr int kA = 128 * KD * 2;
     static constexpr int offBK = 0;
     static constexpr int offBV = kB;
-    static constexpr int offA = 2 * kB;
-    static constexpr int offCodes = offA + kA;          // 2 x 128 bytes
-    static constexpr int offMbar = offCodes + 256;
+    static constexpr int offA = 2 * kB;                 // A operand of the keys
+    static constexpr int offA2 = offA + kA;             // A operand of the values
+    static constexpr int offCodes = offA2 + kA;         // 2 x 128 bytes
+    static constexpr int offRed = offCodes + 256;       // per-row exchange: [2][128] float, [2][128] int
+    static constexpr int offMbar = offRed + 2048;
     static constexpr int offTmem = offMbar + 8;
     static constexpr int kUsed = offTmem + 8;
     static constexpr int kAlloc = 80 * 1024;            // keeps at most two CTAs per SM: 2 x 256 TMEM columns
 };
 
+// Threads: 256.  Thread (half, row) owns tile row `row` (= its TMEM lane, row = tid % 128): it stages
+// the row's key (half 0) or value (half 1) coupled vector, and takes the arg-max over TMEM columns
+// [128 * half, 128 * half + 128); the two halves combine through shared memory.
 template <int D, int C, int TC>
-__global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a) {
+__global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a) {
     constexpr int G = C * TC;
     constexpr int KD = ((G + 3 + 15) / 16) * 16;      // contraction length: coordinates + 3, padded
     constexpr int KB = KD / 8;                          // 16-byte k-blocks per row
@@ -147,10 +233,12 @@ __global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a)
 
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int h = blockIdx.y, brel = blockIdx.z, b = a.b0 + brel;
+    const int row = tid & 127, half = tid >> 7;
     const uint32_t mbar = tc::smem_u32(smem + S::offMbar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::offTmem);
     uint8_t *codes = smem + S::offCodes;
+    float *red_m = reinterpret_cast<float *>(smem + S::offRed);
+    int *red_i = reinterpret_cast<int *>(smem + S::offRed + 1024);
 
     // ---- TMEM (256 columns) and the mbarrier
     if (warp == 0) {
@@ -163,113 +251,136 @@ __global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
 
-    // ---- B operands: entry r -> [e_r (G coords), -h_hi, -h_mid, -h_lo, 0 ...], h = ||e_r||^2 / 2
-    for (int it = tid; it < 2 * 256; it += 128) {
-        const int kv = it >> 8, r = it & 255;
-        uint16_t row[KD];
+    // ---- B operands of head h: entry r -> [e_r (G coords), -h_hi, -h_mid, -h_lo, 0 ...], h_r = ||e_r||^2 / 2
+    auto build_b = [&](int h) {
+        for (int it = tid; it < 2 * 256; it += 256) {
+            const int kv = it >> 8, r = it & 255;
+            uint16_t rw[KD];
 #pragma unroll
-        for (int k = 0; k < KD; ++k) row[k] = 0;
-        if (r < a.K) {
-            const uint16_t *e = a.cb + ((size_t)kv * a.Hkv + h) * (size_t)a.K * G + (size_t)r * G;
-            double hh = 0.0;
+            for (int k = 0; k < KD; ++k) rw[k] = 0;
+            if (r < a.K) {
+                const uint16_t *e = a.cb + ((size_t)kv * a.Hkv + h) * (size_t)a.K * G + (size_t)r * G;
+                double hh = 0.0;
 #pragma unroll
-            for (int k = 0; k < G; ++k) {
-                row[k] = e[k];
-                const double v = (double)bf16_to_f32(e[k]);
-                hh += v * v;
+                for (int k = 0; k < G; ++k) {
+                    rw[k] = e[k];
+                    const double v = (double)bf16_to_f32(e[k]);
+                    hh += v * v;
+                }
+                hh *= 0.5;
+                const float p1 = __bfloat162float(__float2bfloat16_rn((float)hh));
+                const double r1 = hh - (double)p1;
+                const float p2 = __bfloat162float(__float2bfloat16_rn((float)r1));
+                const double r2 = r1 - (double)p2;
+                rw[G] = tc::bf16_bits_rn(-p1);
+                rw[G + 1] = tc::bf16_bits_rn(-p2);
+                rw[G + 2] = tc::bf16_bits_rn((float)-r2);
+            } else {
+                rw[G] = tc::bf16_bits_rn(-1.0e30f);        // entries past K never win
             }
-            hh *= 0.5;
-            const float p1 = __bfloat162float(__float2bfloat16_rn((float)hh));
-            const double r1 = hh - (double)p1;
-            const float p2 = __bfloat162float(__float2bfloat16_rn((float)r1));
-            const double r2 = r1 - (double)p2;
-            row[G] = tc::bf16_bits_rn(-p1);
-            row[G + 1] = tc::bf16_bits_rn(-p2);
-            row[G + 2] = tc::bf16_bits_rn((float)-r2);
-        } else {
-            row[G] = tc::bf16_bits_rn(-1.0e30f);       // entries past K never win
-        }
-        unsigned char *base = smem + (kv ? S::offBV : S::offBK) + ((r >> 3) * KB) * 128 + (r & 7) * 16;
+            unsigned char *base = smem + (kv ? S::offBV : S::offBK) + ((r >> 3) * KB) * 128 + (r & 7) * 16;
 #pragma unroll
-        for (int kb = 0; kb < KB; ++kb) {
-            uint4 v;
-            v.x = row[kb * 8 + 0] | ((uint32_t)row[kb * 8 + 1] << 16);
-            v.y = row[kb * 8 + 2] | ((uint32_t)row[kb * 8 + 3] << 16);
-            v.z = row[kb * 8 + 4] | ((uint32_t)row[kb * 8 + 5] << 16);
-            v.w = row[kb * 8 + 6] | ((uint32_t)row[kb * 8 + 7] << 16);
-            *reinterpret_cast<uint4 *>(base + kb * 128) = v;
+            for (int kb = 0; kb < KB; ++kb) {
+                uint4 v;
+                v.x = rw[kb * 8 + 0] | ((uint32_t)rw[kb * 8 + 1] << 16);
+                v.y = rw[kb * 8 + 2] | ((uint32_t)rw[kb * 8 + 3] << 16);
+                v.z = rw[kb * 8 + 4] | ((uint32_t)rw[kb * 8 + 5] << 16);
+                v.w = rw[kb * 8 + 6] | ((uint32_t)rw[kb * 8 + 7] << 16);
+                *reinterpret_cast<uint4 *>(base + kb * 128) = v;
+            }
         }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+    };
+
+    // ---- this CTA's run of units u = (h * nb + brel) * ntiles + tile, walked without divisions
+    const long long ntiles = (a.ntok + TOKS - 1) / TOKS;
+    const long long total = ntiles * a.nb * a.Hkv;
+    const long long u_begin = (long long)blockIdx.x * a.units_per_cta;
+    const long long u_end = u_begin + a.units_per_cta < total ? u_begin + a.units_per_cta : total;
+    struct Pos {
+        int h, brel, tile;
+    };
+    Pos cur;
+    {
+        const long long hb = u_begin / ntiles;
+        cur.tile = (int)(u_begin - hb * ntiles);
+        cur.h = (int)(hb / a.nb);
+        cur.brel = (int)(hb - (long long)cur.h * a.nb);
     }
-    tc::fence_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    const uint32_t idesc = tc::idesc_bf16(128, 256);
-    const uint32_t aaddr = tc::smem_u32(smem + S::offA);
-    const uint32_t bkaddr = tc::smem_u32(smem + S::offBK), bvaddr = tc::smem_u32(smem + S::offBV);
-    uint32_t phase = 0;
-    bool ok = true;
-    const int row = tid;                                   // TMEM lane == tile row == thread
-    const int rtok = row / NG, rg = row % NG;
-    const int ntiles = (a.ntok + TOKS - 1) / TOKS;
-    const int t_begin = blockIdx.x * a.tiles_per_cta;
-    const int t_end = min(t_begin + a.tiles_per_cta, ntiles);
-    uint32_t *idx_bh = a.idx + ((size_t)b * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C);
-
-    // this row's coupled vectors (keys and values) of the next tile are loaded one tile ahead
-    uint16_t zn[2][G];
-    auto load_row = [&](int tile, uint16_t (&z)[2][G]) {
-        const int nrel = tile * TOKS + rtok;
-#pragma unroll
-        for (int kv = 0; kv < 2; ++kv) {
-#pragma unroll
-            for (int k = 0; k < G; ++k) z[kv][k] = 0;
-            if (tile < t_end && nrel < a.ntok) {
-                const uint16_t *x = (kv ? a.xv : a.xk) + (size_t)brel * a.s1 + (size_t)nrel * a.s2 +
-                                    (size_t)h * a.s3 + rg * C;
-#pragma unroll
-                for (int m = 0; m < TC; ++m)
-#pragma unroll
-                    for (int i = 0; i < C; ++i) z[kv][i * TC + m] = __ldg(x + (size_t)m * a.s0 + i);
+    auto advance = [&](Pos &p) {
+        if (++p.tile == (int)ntiles) {
+            p.tile = 0;
+            if (++p.brel == a.nb) {
+                p.brel = 0;
+                ++p.h;
             }
         }
     };
-    load_row(t_begin, zn);
 
-    for (int tile = t_begin; tile < t_end; ++tile) {
-        uint16_t zc[2][G];
+    int cur_h = cur.h;
+    build_b(cur_h);                                        // also publishes the TMEM address
+    const uint32_t tmem = *tmem_slot;
+
+    const uint32_t idesc = tc::idesc_bf16(128, 256);
+    const uint32_t bkaddr = tc::smem_u32(smem + S::offBK), bvaddr = tc::smem_u32(smem + S::offBV);
+    uint32_t phase = 0;
+    bool ok = true;
+    const int rtok = row / NG, rg = row % NG;
+
+    // this thread's coupled vector (key for half 0, value for half 1) of the next unit, one unit ahead
+    uint16_t zn[G];
+    auto load_row = [&](bool valid, const Pos &p, uint16_t (&z)[G]) {
+        const int nrel = p.tile * TOKS + rtok;
 #pragma unroll
-        for (int kv = 0; kv < 2; ++kv)
+        for (int k = 0; k < G; ++k) z[k] = 0;
+        if (valid && nrel < a.ntok) {
+            const uint16_t *x = (half ? a.xv : a.xk) + (size_t)p.brel * a.s1 + (size_t)nrel * a.s2 +
+                                (size_t)p.h * a.s3 + rg * C;
 #pragma unroll
-            for (int k = 0; k < G; ++k) zc[kv][k] = zn[kv][k];
-        load_row(tile + 1, zn);
+            for (int m = 0; m < TC; ++m)
+#pragma unroll
+                for (int i = 0; i < C; ++i) z[i * TC + m] = __ldg(x + (size_t)m * a.s0 + i);
+        }
+    };
+    load_row(u_begin < u_end, cur, zn);
+
+    for (long long u = u_begin; u < u_end; ++u) {
+        const int tile = cur.tile, brel = cur.brel, h = cur.h;
+        advance(cur);
+        if (h != cur_h) {                                  // previous MMAs have completed: B may be rewritten
+            build_b(h);
+            cur_h = h;
+        }
+        // ---- A operand of this thread's half: the coupled vector extended by three ones
+        {
+            uint16_t zr[KD];
+#pragma unroll
+            for (int k = 0; k < KD; ++k) zr[k] = k < G ? zn[k] : 0;
+            zr[G] = zr[G + 1] = zr[G + 2] = 0x3F80;           // bf16 1.0
+            unsigned char *base = smem + (half ? S::offA2 : S::offA) + ((row >> 3) * KB) * 128 + (row & 7) * 16;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+                uint4 v;
+                v.x = zr[kb * 8 + 0] | ((uint32_t)zr[kb * 8 + 1] << 16);
+                v.y = zr[kb * 8 + 2] | ((uint32_t)zr[kb * 8 + 3] << 16);
+                v.z = zr[kb * 8 + 4] | ((uint32_t)zr[kb * 8 + 5] << 16);
+                v.w = zr[kb * 8 + 6] | ((uint32_t)zr[kb * 8 + 7] << 16);
+                *reinterpret_cast<uint4 *>(base + kb * 128) = v;
+            }
+        }
+        load_row(u + 1 < u_end, cur, zn);
 #pragma unroll 1
         for (int kv = 0; kv < 2; ++kv) {
-            // ---- A operand: this row's coupled vector, extended by three ones
-            {
-                uint16_t zr[KD];
-#pragma unroll
-                for (int k = 0; k < KD; ++k) zr[k] = k < G ? (kv ? zc[1][k] : zc[0][k]) : 0;
-                zr[G] = zr[G + 1] = zr[G + 2] = 0x3F80;       // bf16 1.0
-                unsigned char *base = smem + S::offA + ((row >> 3) * KB) * 128 + (row & 7) * 16;
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    uint4 v;
-                    v.x = zr[kb * 8 + 0] | ((uint32_t)zr[kb * 8 + 1] << 16);
-                    v.y = zr[kb * 8 + 2] | ((uint32_t)zr[kb * 8 + 3] << 16);
-                    v.z = zr[kb * 8 + 4] | ((uint32_t)zr[kb * 8 + 5] << 16);
-                    v.w = zr[kb * 8 + 6] | ((uint32_t)zr[kb * 8 + 7] << 16);
-                    *reinterpret_cast<uint4 *>(base + kb * 128) = v;
-                }
-            }
             tc::fence_async_smem();
             tc::tc_fence_before();
             __syncthreads();
             // ---- s = [z, 1, 1, 1] . [e, -h] for all 256 entries, into TMEM columns [0, 256)
             if (tid == 0) {
                 tc::tc_fence_after();
+                const uint32_t aaddr = tc::smem_u32(smem + (kv ? S::offA2 : S::offA));
                 const uint32_t baddr = kv ? bvaddr : bkaddr;
 #pragma unroll
                 for (int ks = 0; ks < KD / 16; ++ks) {
@@ -284,32 +395,21 @@ __global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a)
             phase ^= 1u;
             if (!ok) break;
             tc::tc_fence_after();
-            // ---- arg-max over the entries of this row (first maximum wins)
-            float best = -CUDART_INF_F;
-            int bi = 0;
-            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 64) {
-                uint32_t va[32], vb[32];
-                tc::tmem_ld32(taddr + c0, va);
-                tc::tmem_ld32(taddr + c0 + 32, vb);
-                tc::tmem_wait_ld();
-                // entries at or past K score -1e30 through their extended coordinate, so they never win
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float v = __uint_as_float(va[j]);
-                    if (v > best) { best = v; bi = c0 + j; }
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float v = __uint_as_float(vb[j]);
-                    if (v > best) { best = v; bi = c0 + 32 + j; }
-                }
-            }
-            codes[kv * 128 + row] = (uint8_t)bi;
+            // ---- exact arg-max of the row: maximum over both halves, then the first column equal to it
+            const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+            red_m[half * 128 + row] = tc::cols_max<128>(taddr, half * 128);
+            __syncthreads();
+            const float M = fmaxf(red_m[row], red_m[128 + row]);
+            red_i[half * 128 + row] = tc::cols_first<128>(taddr, half * 128, M);
             tc::tc_fence_before();
-            __syncthreads();                               // TMEM and the A operand are free again
+            __syncthreads();                               // TMEM is free again
+            if (half == 0) {
+                // a row without a hit has only NaN scores; it takes entry 0
+                const int i0 = red_i[row], i1 = red_i[128 + row];
+                codes[kv * 128 + row] = (uint8_t)(i0 >= 0 ? i0 : (i1 >= 0 ? i1 : 0));
+            }
         }
+        __syncthreads();
         // ---- pack {K p, K p+NP, V p, V p+NP} words and store them (sentinel words after a timeout)
         if (tid < TOKS * NP) {
             const int t = tid / NP, p = tid % NP;
@@ -319,10 +419,10 @@ __global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a)
                                          ((uint32_t)codes[128 + t * NG + p] << 16) |
                                          ((uint32_t)codes[128 + t * NG + p + NP] << 24))
                                       : 0xFFFFFFFFu;
+                uint32_t *idx_bh = a.idx + ((size_t)(a.b0 + brel) * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C);
                 idx_bh[idx_word(a.tok0 + nr, p, NP)] = w;
             }
         }
-        __syncthreads();
         if (!ok) break;
     }
 
@@ -332,24 +432,37 @@ __global__ void __launch_bounds__(128, 1) encode_tc_kernel(const EncodeTcArgs a)
 }
 
 template <int D, int C, int TC>
-static cudaError_t launch_tc_ct(const EncodeTcArgs &a0, int nb, cudaStream_t s) {
+static cudaError_t launch_tc_ct(const EncodeTcArgs &a0, cudaStream_t s) {
     constexpr int NG = D / C;
     constexpr int TOKS = 128 / NG;
     constexpr int KD = ((C * TC + 3 + 15) / 16) * 16;
     EncodeTcArgs a = a0;
-    const int ntiles = (a.ntok + TOKS - 1) / TOKS;
-    // enough CTAs per (sequence, head) to fill the GPU twice over, each looping over its tiles
-    const long units = (long)a.Hkv * nb;
-    long per = (2L * 148 + units - 1) / units;
-    if (per < 1) per = 1;
-    if (per > ntiles) per = ntiles;
-    a.tiles_per_cta = (int)((ntiles + per - 1) / per);
-    const int gx = (ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
     auto k = encode_tc_kernel<D, C, TC>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSmem<KD>::kAlloc);
     if (e != cudaSuccess) return e;
-    dim3 grid(gx, a.Hkv, nb);
-    k<<<grid, 128, TcSmem<KD>::kAlloc, s>>>(a);
+    // CTAs resident per SM, from the limits that bind here: shared memory, registers and tensor memory
+    // (each CTA allocates 256 of the SM's 512 TMEM columns)
+    int dev = 0, sms = 0, smem_sm = 0, resv = 0;
+    cudaFuncAttributes fa{};
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess)
+        return e;
+    if ((e = cudaDeviceGetAttribute(&resv, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa, k)) != cudaSuccess) return e;
+    const int by_smem = smem_sm / (TcSmem<KD>::kAlloc + (int)fa.sharedSizeBytes + resv);
+    const int by_regs = 65536 / (((fa.numRegs + 7) / 8) * 8 * 256);
+    int per_sm = by_smem < by_regs ? by_smem : by_regs;
+    if (per_sm > 2) per_sm = 2;
+    if (per_sm < 1) return cudaErrorNotSupported;
+    // persistent grid: one wave of CTAs, each taking an equal run of the head-major units
+    const long long ntiles = (a.ntok + TOKS - 1) / TOKS;
+    const long long total = ntiles * a.nb * a.Hkv;
+    long long ctas = (long long)sms * per_sm;
+    if (ctas > total) ctas = total;
+    a.units_per_cta = (total + ctas - 1) / ctas;
+    ctas = (total + a.units_per_cta - 1) / a.units_per_cta;
+    k<<<(unsigned)ctas, 256, TcSmem<KD>::kAlloc, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -369,13 +482,14 @@ cudaError_t launch_encode_tc(const loopvq_cache &cc, int layer, int block, const
     a.K = cc.K;
     a.Nmax = cc.Nmax;
     a.b0 = b0;
+    a.nb = nb;
     a.tok0 = tok0;
     a.ntok = ntok;
     const int G = cc.c * cc.Tc;
-    if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4>(a, nb, s);
-    if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4>(a, nb, s);
-    if (cc.D == 64 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<64, 4, 4>(a, nb, s);
-    if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4>(a, nb, s);
+    if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4>(a, s);
+    if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4>(a, s);
+    if (cc.D == 64 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<64, 4, 4>(a, s);
+    if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4>(a, s);
     (void)G;
     return cudaErrorNotSupported;
 }
