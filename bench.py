@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size (profiling runs)")
     return ap.parse_args()
 
 
@@ -255,6 +256,8 @@ def main():
     w = WORKLOADS[args.workload]
     if args.layers > 0:
         w = w.replace(L=args.layers)
+    if args.batch > 0:
+        w = w.replace(B=args.batch)
 
     # ---------------- set-up: codebooks, slices, RoPE table, GPU encode of every (layer, block)
     cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, device=dev)
