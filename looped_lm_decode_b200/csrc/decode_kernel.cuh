@@ -29,7 +29,11 @@
 //  * Each thread keeps a DEPTH-deep queue of its own 16-byte index-word loads in
 //    flight with cp.async (it reads back only what it copied, so no barrier is
 //    involved).
-//  * RoPE values: one table row per tile, then exact one-position rotations.
+//  * RoPE values: one table row per tile; the next position is one complex multiply away, and the
+//    rest of the tile follows the three-term recurrence X_{k+1} = 2 cos(w) X_k - X_{k-1}, which holds
+//    for every sequence X_k = A e^{-i k w} and needs one fused multiply-add per component.
+//  * The tile's value gathers are issued before the key arithmetic, so their shared-memory latency
+//    overlaps the score, reduction and softmax work.
 //  * Online softmax with a lazy maximum; fp32 math in packed pairs (FFMA2).
 #pragma once
 
@@ -231,6 +235,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         s1[1] = f2(sv.z, sv.w);
     }
     const float2 ns1[2] = {neg2(s1[0]), neg2(s1[1])};
+    const float2 tc1[2] = {f2(2.f * c1[0].x, 2.f * c1[0].y), f2(2.f * c1[1].x, 2.f * c1[1].y)};   // 2 cos(w)
     const float2 nqlo[2] = {neg2(qlo[0][0]), neg2(qlo[0][1])};
     float m_[QPK], l_[QPK];
     float2 olo[QPK][2], ohi[QPK][2];
@@ -279,11 +284,24 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             ra_s = __ldg(reinterpret_cast<const float4 *>(row + D / 2));
         }
 
+        // ---- values of the tile: gathered now and used after the softmax when registers allow
+        // (one or two query heads per KV head); otherwise gathered in the value loop
+        constexpr bool VEARLY = QPK <= 2;
+        uint2 vraw[TT][2];
+        if constexpr (VEARLY) {
+#pragma unroll
+            for (int k = 0; k < TT; ++k) {
+                const uint32_t w = word_k(w4[k >> 2], k & 3);
+                vraw[k][0] = lds64(smem, __byte_perm(w, colv, 0x7624));
+                vraw[k][1] = lds64(smem, __byte_perm(w, colv, 0x7634));
+            }
+        }
+
         // ---- keys: rebuild, score.  ROTQ: per pair f the term is Re(Z) k_f + Im(Z) k_{f+D/2} with
-        // Z = (q_f + i q_{f+D/2}) e^{-i p w_f}, advanced one position per token by one complex multiply.
-        // Otherwise the rebuilt keys are rotated by (cos, sin), advanced the same way, and shared.
+        // Z = (q_f + i q_{f+D/2}) e^{-i p w_f}, advanced along the tile (see the header).  Otherwise the
+        // rebuilt keys are rotated by (cos, sin), advanced the same way, and shared by the query heads.
         float ps[QPK][TT];
-        float2 zu[2], zw[2];
+        float2 zu[2], zw[2], xu[2], xw[2];                // X_k and X_{k-1} of the advanced pair
         if constexpr (ROTQ) {
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
@@ -296,17 +314,21 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             if (k > 0) {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    if constexpr (ROTQ) {
-                        const float2 un = __ffma2_rn(zu[i], c1[i], __fmul2_rn(zw[i], s1[i]));
-                        const float2 wn = __ffma2_rn(zw[i], c1[i], __fmul2_rn(zu[i], ns1[i]));
-                        zu[i] = un;
-                        zw[i] = wn;
+                    // the pair (re, im) advanced by one position: ROTQ by e^{-iw}, else by e^{+iw}
+                    float2 &re = ROTQ ? zu[i] : cs[i];
+                    float2 &im = ROTQ ? zw[i] : sn[i];
+                    float2 nre, nim;
+                    if (k == 1) {
+                        nre = ROTQ ? __ffma2_rn(re, c1[i], __fmul2_rn(im, s1[i])) : __ffma2_rn(re, c1[i], __fmul2_rn(im, ns1[i]));
+                        nim = ROTQ ? __ffma2_rn(im, c1[i], __fmul2_rn(re, ns1[i])) : __ffma2_rn(im, c1[i], __fmul2_rn(re, s1[i]));
                     } else {
-                        const float2 cn = __ffma2_rn(cs[i], c1[i], __fmul2_rn(sn[i], ns1[i]));
-                        const float2 snn = __ffma2_rn(sn[i], c1[i], __fmul2_rn(cs[i], s1[i]));
-                        cs[i] = cn;
-                        sn[i] = snn;
+                        nre = __ffma2_rn(tc1[i], re, neg2(xu[i]));
+                        nim = __ffma2_rn(tc1[i], im, neg2(xw[i]));
                     }
+                    xu[i] = re;
+                    xw[i] = im;
+                    re = nre;
+                    im = nim;
                 }
             }
             const uint32_t w = word_k(w4[k >> 2], k & 3);
@@ -370,10 +392,12 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 #pragma unroll
         for (int k = 0; k < TT; ++k) {
             const int src = slot_lane0 + tile_owner<TT, NL>(k);
-            const uint32_t w = word_k(w4[k >> 2], k & 3);
-            const uint2 vlo = lds64(smem, __byte_perm(w, colv, 0x7624));
-            const uint2 vhi = lds64(smem, __byte_perm(w, colv, 0x7634));
-            const uint32_t vl[2] = {vlo.x, vlo.y}, vh[2] = {vhi.x, vhi.y};
+            if constexpr (!VEARLY) {
+                const uint32_t w = word_k(w4[k >> 2], k & 3);
+                vraw[k][0] = lds64(smem, __byte_perm(w, colv, 0x7624));
+                vraw[k][1] = lds64(smem, __byte_perm(w, colv, 0x7634));
+            }
+            const uint32_t vl[2] = {vraw[k][0].x, vraw[k][0].y}, vh[2] = {vraw[k][1].x, vraw[k][1].y};
 #pragma unroll
             for (int j = 0; j < QPK; ++j) {
                 const float pk = __shfl_sync(slot_mask, pe[j], src);
