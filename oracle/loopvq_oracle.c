@@ -27,6 +27,12 @@
  *              through the log-sum-exp of each split (Flash-Decoding merge),
  *              which the pages state recovers the exact softmax.
  *              LoopVQ paper, Sec. 4.3 "Attention".
+ *   windowed   attention of one query over a cache whose sink and recent
+ *              tokens are kept in bf16 (keys stored already rotated) and whose
+ *              other tokens lo <= n < hi are coded: the coded keys are rebuilt
+ *              and rotated at their absolute positions, all keys are put in
+ *              one list, and one softmax runs over the list.
+ *              LoopVQ paper, Sec. 4.3 "Cache layout" and "Attention".
  *
  * Array conventions (all dense, row-major, caller-owned):
  *   x   float  [Tc][N][D]   one block of Tc loop steps of one (layer, head, K|V)
@@ -187,6 +193,33 @@ void ora_decode(const double *q, const uint8_t *idx_k, const uint8_t *idx_v, con
     ora_dequant(idx_k, N, D, c, Tc, m, E_k, kh);
     ora_rope(kh, N, D, theta, 0);
     ora_dequant(idx_v, N, D, c, Tc, m, E_v, vh);
+    ora_attention(q, kh, vh, N, D, scale, out, lse);
+    free(kh);
+    free(vh);
+}
+
+/* Attention of one query over NW bf16 window tokens (keys kw already rotated, values vw, both
+ * [NW][D]) together with the coded tokens lo <= n < hi, whose codes are rows 0 .. hi-lo-1 of
+ * idx_k / idx_v (Sec. 4.3 "Cache layout": sink and recent tokens in bf16, the rest coded).  The
+ * coded keys are rebuilt (eq. 5) and rotated at positions lo .. hi-1; then one softmax runs over the
+ * concatenated key list: window tokens first, coded tokens after. */
+void ora_decode_windowed(const double *q, const double *kw, const double *vw, int NW, const uint8_t *idx_k,
+                         const uint8_t *idx_v, const float *E_k, const float *E_v, int lo, int hi, int D, int c,
+                         int Tc, int m, double theta, double scale, double *out, double *lse)
+{
+    const int NC = hi > lo ? hi - lo : 0;
+    const int N = NW + NC;
+    size_t nd = (size_t)(N > 0 ? N : 1) * (size_t)D;
+    double *kh = (double *)malloc(sizeof(double) * nd);
+    double *vh = (double *)malloc(sizeof(double) * nd);
+    for (size_t i = 0; i < (size_t)NW * D; ++i) {
+        kh[i] = kw[i];
+        vh[i] = vw[i];
+    }
+    double *kc = kh + (size_t)NW * D, *vc = vh + (size_t)NW * D;
+    ora_dequant(idx_k, NC, D, c, Tc, m, E_k, kc);
+    ora_rope(kc, NC, D, theta, lo);
+    ora_dequant(idx_v, NC, D, c, Tc, m, E_v, vc);
     ora_attention(q, kh, vh, N, D, scale, out, lse);
     free(kh);
     free(vh);

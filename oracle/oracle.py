@@ -39,6 +39,9 @@ def lib():
         _lib.ora_attention_splits.restype = None
         _lib.ora_decode.argtypes = [f64p, u8p, u8p, f32p, f32p, I, I, I, I, I, D_, D_, f64p, C.POINTER(D_)]
         _lib.ora_decode.restype = None
+        _lib.ora_decode_windowed.argtypes = [f64p, f64p, f64p, I, u8p, u8p, f32p, f32p, I, I, I, I, I, I, D_, D_,
+                                             f64p, C.POINTER(D_)]
+        _lib.ora_decode_windowed.restype = None
     return _lib
 
 
@@ -124,4 +127,26 @@ def decode(q, idx_k, idx_v, E_k, E_v, c: int, Tc: int, m: int, theta: float = 1.
     lse = C.c_double(0.0)
     lib().ora_decode(q, idx_k if N else np.zeros((1, D // c), np.uint8), idx_v if N else np.zeros((1, D // c), np.uint8),
                      _f32(E_k), _f32(E_v), N, D, c, Tc, m, theta, scale, out, C.byref(lse))
+    return out, lse.value
+
+
+def decode_windowed(q, k_win, v_win, idx_k, idx_v, E_k, E_v, c: int, Tc: int, m: int, lo: int,
+                    theta: float = 1.0e4, scale: float = None):
+    """One query over NW bf16 window tokens (k_win already rotated, v_win: [NW][D]) and the coded
+    tokens lo .. lo + len(idx_k) - 1 (codes idx_k / idx_v [n][D/c]) at loop step m of the block."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    D = q.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    kw = np.ascontiguousarray(k_win, dtype=np.float64).reshape(-1, D)
+    vw = np.ascontiguousarray(v_win, dtype=np.float64).reshape(-1, D)
+    idx_k = np.ascontiguousarray(idx_k, dtype=np.uint8).reshape(-1, D // c)
+    idx_v = np.ascontiguousarray(idx_v, dtype=np.uint8).reshape(-1, D // c)
+    NW, NC = kw.shape[0], idx_k.shape[0]
+    out = np.zeros(D, dtype=np.float64)
+    lse = C.c_double(0.0)
+    z64 = np.zeros((1, D), np.float64)
+    z8 = np.zeros((1, D // c), np.uint8)
+    lib().ora_decode_windowed(q, kw if NW else z64, vw if NW else z64, NW, idx_k if NC else z8, idx_v if NC else z8,
+                              _f32(E_k), _f32(E_v), lo, lo + NC, D, c, Tc, m, theta, scale, out, C.byref(lse))
     return out, lse.value

@@ -300,3 +300,61 @@ def test_keys_are_rotated_values_are_not():
     np.testing.assert_allclose(out, ro, rtol=1e-11, atol=1e-12)
     wrong, _ = _softmax_attention_np(q, k, _rope_complex(v, np.arange(N)), 0.125)
     assert np.abs(wrong - out).max() > 1e-3
+
+
+# ---------------------------------------------------------------- bf16 window + coded tokens
+
+def _window_case(NW=5, lo=9, NC=23, D=64, c=4, Tc=4, m=1):
+    E_k, E_v = _rand_bf16((256, c * Tc)), _rand_bf16((256, c * Tc))
+    ik = RNG.integers(0, 256, (NC, D // c)).astype(np.uint8)
+    iv = RNG.integers(0, 256, (NC, D // c)).astype(np.uint8)
+    kw, vw = _rand_bf16((NW, D)), _rand_bf16((NW, D))
+    q = RNG.standard_normal(D)
+    return q, kw, vw, ik, iv, E_k, E_v, c, Tc, m, lo
+
+
+def test_windowed_is_one_softmax_over_window_and_rotated_coded_tokens():
+    """Sec. 4.3 "Cache layout": window keys are taken as stored, coded keys are rebuilt and rotated at
+    their absolute positions lo..hi-1; one softmax runs over all of them (numpy complex RoPE here)."""
+    q, kw, vw, ik, iv, E_k, E_v, c, Tc, m, lo = _window_case()
+    out, lse = O.decode_windowed(q, kw, vw, ik, iv, E_k, E_v, c, Tc, m, lo, 1e4, 0.2)
+    kc = _rope_complex(O.dequant(ik, E_k, c, Tc, m), lo + np.arange(len(ik)))
+    vc = O.dequant(iv, E_v, c, Tc, m)
+    ro, rl = _softmax_attention_np(q, np.concatenate([kw, kc]), np.concatenate([vw, vc]), 0.2)
+    np.testing.assert_allclose(out, ro, rtol=1e-11, atol=1e-12)
+    assert abs(lse - rl) < 1e-11
+
+
+def test_windowed_equals_merge_of_its_parts():
+    """The two-kernel split of Sec. 4.3 "Attention": attention over the window alone and over the coded
+    range alone, combined through their log-sum-exps (scipy), equals the windowed attention."""
+    q, kw, vw, ik, iv, E_k, E_v, c, Tc, m, lo = _window_case(NW=8, lo=8, NC=40)
+    out, lse = O.decode_windowed(q, kw, vw, ik, iv, E_k, E_v, c, Tc, m, lo, 1e4, 0.125)
+    oa, la = O.attention(q, kw, vw, 0.125)
+    ob, lb = O.decode_windowed(q, np.zeros((0, 64)), np.zeros((0, 64)), ik, iv, E_k, E_v, c, Tc, m, lo, 1e4, 0.125)
+    L = logsumexp([la, lb])
+    np.testing.assert_allclose(out, math.exp(la - L) * oa + math.exp(lb - L) * ob, rtol=1e-11, atol=1e-12)
+    assert abs(lse - L) < 1e-11
+
+
+def test_windowed_with_coded_prefix_as_window_equals_plain_decode():
+    """Holding tokens 0..lo-1 in the window as their rotated reconstructions must give the same result
+    as decoding all tokens from codes: pins the absolute positions of the coded part."""
+    q, _, _, ik, iv, E_k, E_v, c, Tc, m, _ = _window_case(NC=30)
+    lo = 6
+    kw = _rope_complex(O.dequant(ik[:lo], E_k, c, Tc, m), np.arange(lo))
+    vw = O.dequant(iv[:lo], E_v, c, Tc, m)
+    out, lse = O.decode_windowed(q, kw, vw, ik[lo:], iv[lo:], E_k, E_v, c, Tc, m, lo, 1e4, 0.1)
+    ro, rl = O.decode(q, ik, iv, E_k, E_v, c, Tc, m, 1e4, 0.1)
+    np.testing.assert_allclose(out, ro, rtol=1e-10, atol=1e-12)
+    assert abs(lse - rl) < 1e-10
+
+
+def test_windowed_special_cases():
+    q, kw, vw, ik, iv, E_k, E_v, c, Tc, m, lo = _window_case()
+    z = np.zeros((0, 64))
+    out, lse = O.decode_windowed(q, kw, vw, ik[:0], iv[:0], E_k, E_v, c, Tc, m, lo, 1e4, 0.3)
+    ro, rl = _softmax_attention_np(q, kw, vw, 0.3)
+    np.testing.assert_allclose(out, ro, rtol=1e-11, atol=1e-12)
+    out, lse = O.decode_windowed(q, z, z, ik[:0], iv[:0], E_k, E_v, c, Tc, m, lo, 1e4, 0.3)
+    assert lse == -math.inf and (out == 0).all()
