@@ -141,6 +141,77 @@ loopvq_status loopvq_decode_attn(const loopvq_cache *cache, int layer, int t,
                                  void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Decode attention over a token range of the coded cache (Sec. 4.3 "Cache
+ * layout" and "Attention"): the same as loopvq_decode_attn, over tokens
+ * start_b <= n < len_b.  This is the coded part of a cache whose first n_s
+ * (sink) and last n_r (recent) tokens are kept in bf16.  Combine it with
+ * loopvq_bf16_decode_attn over the bf16 tokens through loopvq_merge2.
+ *
+ * starts    int32 [B] device, or NULL for all 0; each start is clamped to
+ *           [0, len_b].  Any start works: index words are read in 4-token tiles
+ *           and the tile tokens before the start are masked.
+ * Positions for RoPE stay absolute (token index n).  Workspace as for
+ * loopvq_decode_attn.  len_b <= start_b gives zeros and lse = -inf.
+ */
+loopvq_status loopvq_decode_attn_range(const loopvq_cache *cache, int layer, int t,
+                                       const uint16_t *q, const int32_t *starts, const int32_t *lens,
+                                       int max_len, float scale, float *out, float *lse,
+                                       void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * A bf16 KV cache: the unquantized layout that LoopVQ is compared against
+ * (Sec. 5.3), and the store of the sink and recent tokens (Sec. 4.3 "Cache
+ * layout").  Keys are stored as the model attends to them, already rotated
+ * by RoPE at their positions.  Caller-owned device buffers:
+ *   k, v      bf16 [B][Hkv][Nmax][D], 16-byte aligned.
+ * D in {64, 128}; Hq a multiple of Hkv with Hq / Hkv in {1, 2, 4, 8}.
+ */
+typedef struct loopvq_bf16_cache {
+    int32_t B, Hkv, Hq, D, Nmax;
+    const uint16_t *k;
+    const uint16_t *v;
+} loopvq_bf16_cache;
+
+/* Workspace bytes loopvq_bf16_decode_attn needs for up to max_len tokens per sequence. */
+size_t loopvq_bf16_decode_workspace_bytes(const loopvq_bf16_cache *cache, int max_len);
+
+/*
+ * Decode attention over a bf16 cache (the bf16 kernel of Sec. 4.3
+ * "Attention"): for every sequence b and query head hq (KV head
+ * hq / (Hq/Hkv)), s_n = scale * <q, k_n>, out = sum_n softmax(s)_n v_n,
+ * lse = ln sum_n exp(s_n), over tokens start_b <= n < len_b.  Split over
+ * tokens and merged by log-sum-exp like loopvq_decode_attn.
+ *
+ * q         bf16 [B][Hq][D], rotated at the query position.
+ * starts    int32 [B] device or NULL (all 0); lens int32 [B] device; both
+ *           clamped as in loopvq_decode_attn_range.  max_len <= Nmax is a host
+ *           upper bound of the lengths.
+ * scale     <= 0 selects 1/sqrt(D).
+ * out, lse, workspace as for loopvq_decode_attn.
+ */
+loopvq_status loopvq_bf16_decode_attn(const loopvq_bf16_cache *cache, const uint16_t *q,
+                                      const int32_t *starts, const int32_t *lens, int max_len,
+                                      float scale, float *out, float *lse,
+                                      void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Log-sum-exp merge of two attentions of the same queries over disjoint
+ * token sets (Sec. 4.3 "Attention": the bf16 and the quantized kernels'
+ * results are combined exactly):
+ *   m = max(lse_a, lse_b), w_x = exp(lse_x - m),
+ *   out = (w_a out_a + w_b out_b) / (w_a + w_b),  lse = m + ln(w_a + w_b).
+ * A part with lse = -inf (no tokens) contributes nothing; both empty gives
+ * zeros and -inf.
+ *
+ * out_a, out_b, out   fp32 [rows][D]; lse_a, lse_b, lse fp32 [rows] (lse may be
+ * NULL).  out may alias out_a or out_b and lse may alias lse_a or lse_b.
+ * D in {64, 128}.
+ */
+loopvq_status loopvq_merge2(const float *out_a, const float *lse_a, const float *out_b,
+                            const float *lse_b, int rows, int D, float *out, float *lse,
+                            void *stream);
+
+/*
  * Explicit reconstruction for checking (eq. 5): for sequence b, tokens
  * tok0 .. tok0+ntok-1 and every KV head, the loop-step-t reconstruction of
  * keys (kv = 0) or values (kv = 1); keys are rotated by RoPE at their

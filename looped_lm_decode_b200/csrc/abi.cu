@@ -130,9 +130,9 @@ size_t loopvq_decode_workspace_bytes(const loopvq_cache *cc, int max_len) {
     return loopvq::plan_decode(*cc, max_len).ws_bytes;
 }
 
-loopvq_status loopvq_decode_attn(const loopvq_cache *cc, int layer, int t, const uint16_t *q,
-                                 const int32_t *lens, int max_len, float scale, float *out, float *lse,
-                                 void *workspace, size_t ws_bytes, void *stream) {
+static loopvq_status decode_common(const char *fn, const loopvq_cache *cc, int layer, int t, const uint16_t *q,
+                                   const int32_t *starts, const int32_t *lens, int max_len, float scale, float *out,
+                                   float *lse, void *workspace, size_t ws_bytes, void *stream) {
     g_err[0] = 0;
     LQ_TRY(check_shape(cc));
     LQ_TRY(check_ptr(cc->idx, "idx"));
@@ -141,6 +141,8 @@ loopvq_status loopvq_decode_attn(const loopvq_cache *cc, int layer, int t, const
     LQ_TRY(check_ptr(q, "q"));
     LQ_TRY(check_ptr(lens, "lens"));
     LQ_TRY(check_ptr(out, "out"));
+    if (starts && (reinterpret_cast<uintptr_t>(starts) & 3u))
+        return fail(LOOPVQ_ERR_INVALID_ARG, "starts not 4-byte aligned");
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(LOOPVQ_ERR_INVALID_ARG, "lse not 4-byte aligned");
     if (layer < 0 || layer >= cc->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, cc->L);
     if (t < 0 || t >= cc->T) return fail(LOOPVQ_ERR_INVALID_ARG, "t=%d out of [0, %d)", t, cc->T);
@@ -154,9 +156,84 @@ loopvq_status loopvq_decode_attn(const loopvq_cache *cc, int layer, int t, const
         return fail(LOOPVQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws_bytes,
                     workspace ? ws_bytes : (size_t)0);
     if (!aligned16(workspace)) return fail(LOOPVQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
-    cudaError_t e = loopvq::launch_decode(*cc, plan, layer, t, q, lens, max_len, scale, out, lse, workspace,
+    cudaError_t e = loopvq::launch_decode(*cc, plan, layer, t, q, starts, lens, max_len, scale, out, lse, workspace,
                                           (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "loopvq_decode_attn");
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return LOOPVQ_OK;
+}
+
+loopvq_status loopvq_decode_attn(const loopvq_cache *cc, int layer, int t, const uint16_t *q,
+                                 const int32_t *lens, int max_len, float scale, float *out, float *lse,
+                                 void *workspace, size_t ws_bytes, void *stream) {
+    return decode_common("loopvq_decode_attn", cc, layer, t, q, nullptr, lens, max_len, scale, out, lse, workspace,
+                         ws_bytes, stream);
+}
+
+loopvq_status loopvq_decode_attn_range(const loopvq_cache *cc, int layer, int t, const uint16_t *q,
+                                       const int32_t *starts, const int32_t *lens, int max_len, float scale,
+                                       float *out, float *lse, void *workspace, size_t ws_bytes, void *stream) {
+    return decode_common("loopvq_decode_attn_range", cc, layer, t, q, starts, lens, max_len, scale, out, lse,
+                         workspace, ws_bytes, stream);
+}
+
+static loopvq_status check_bf16(const loopvq_bf16_cache *c) {
+    if (!c) return fail(LOOPVQ_ERR_INVALID_ARG, "cache is NULL");
+    if (c->B <= 0 || c->Hkv <= 0 || c->Hq <= 0 || c->D <= 0 || c->Nmax <= 0)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "all shape fields must be positive");
+    if (c->Hq % c->Hkv != 0) return fail(LOOPVQ_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", c->Hq, c->Hkv);
+    if (c->D != 64 && c->D != 128) return fail(LOOPVQ_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", c->D);
+    const int qpk = c->Hq / c->Hkv;
+    if (qpk != 1 && qpk != 2 && qpk != 4 && qpk != 8)
+        return fail(LOOPVQ_ERR_UNSUPPORTED, "Hq/Hkv=%d (supported: 1, 2, 4, 8)", qpk);
+    LQ_TRY(check_ptr(c->k, "k"));
+    LQ_TRY(check_ptr(c->v, "v"));
+    return LOOPVQ_OK;
+}
+
+size_t loopvq_bf16_decode_workspace_bytes(const loopvq_bf16_cache *c, int max_len) {
+    if (check_bf16(c) != LOOPVQ_OK || max_len < 0 || max_len > c->Nmax) return 0;
+    return loopvq::plan_bf16(*c, max_len).ws_bytes;
+}
+
+loopvq_status loopvq_bf16_decode_attn(const loopvq_bf16_cache *c, const uint16_t *q, const int32_t *starts,
+                                      const int32_t *lens, int max_len, float scale, float *out, float *lse,
+                                      void *workspace, size_t ws_bytes, void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_bf16(c));
+    LQ_TRY(check_ptr(q, "q"));
+    LQ_TRY(check_ptr(lens, "lens"));
+    LQ_TRY(check_ptr(out, "out"));
+    if (starts && (reinterpret_cast<uintptr_t>(starts) & 3u))
+        return fail(LOOPVQ_ERR_INVALID_ARG, "starts not 4-byte aligned");
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(LOOPVQ_ERR_INVALID_ARG, "lse not 4-byte aligned");
+    if (max_len < 0 || max_len > c->Nmax)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "max_len=%d out of [0, Nmax=%d]", max_len, c->Nmax);
+    if (!std::isfinite(scale)) return fail(LOOPVQ_ERR_INVALID_ARG, "scale is not finite");
+    if (scale <= 0.f) scale = 1.0f / std::sqrt((float)c->D);
+    const loopvq::DecodePlan plan = loopvq::plan_bf16(*c, max_len);
+    if (plan.nsplit > 65535) return fail(LOOPVQ_ERR_UNSUPPORTED, "too many splits");
+    if (!workspace || ws_bytes < plan.ws_bytes)
+        return fail(LOOPVQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws_bytes,
+                    workspace ? ws_bytes : (size_t)0);
+    if (!aligned16(workspace)) return fail(LOOPVQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    cudaError_t e = loopvq::launch_bf16_decode(*c, plan, q, starts, lens, max_len, scale, out, lse, workspace,
+                                               (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_bf16_decode_attn");
+    return LOOPVQ_OK;
+}
+
+loopvq_status loopvq_merge2(const float *out_a, const float *lse_a, const float *out_b, const float *lse_b,
+                            int rows, int D, float *out, float *lse, void *stream) {
+    g_err[0] = 0;
+    if (rows < 0) return fail(LOOPVQ_ERR_INVALID_ARG, "rows=%d is negative", rows);
+    if (D != 64 && D != 128) return fail(LOOPVQ_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", D);
+    if (rows == 0) return LOOPVQ_OK;
+    if (!out_a || !lse_a || !out_b || !lse_b || !out) return fail(LOOPVQ_ERR_INVALID_ARG, "NULL input or output");
+    const void *ptrs[6] = {out_a, lse_a, out_b, lse_b, out, lse};
+    for (const void *p : ptrs)
+        if (p && (reinterpret_cast<uintptr_t>(p) & 3u)) return fail(LOOPVQ_ERR_INVALID_ARG, "pointer not 4-byte aligned");
+    cudaError_t e = loopvq::launch_merge2(out_a, lse_a, out_b, lse_b, rows, D, out, lse, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_merge2");
     return LOOPVQ_OK;
 }
 

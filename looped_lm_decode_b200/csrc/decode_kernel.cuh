@@ -50,6 +50,7 @@ struct DecodeArgs {
     const float *rope;       // [Nmax][D]
     const uint16_t *q;       // [B][Hq][D] bf16
     const int32_t *lens;     // [B]
+    const int32_t *starts;   // [B] first attended token, or null for 0
     float *ws_o;             // [B][Hq][nsplit][D]  unnormalised split outputs
     float2 *ws_ml;           // [B][Hq][nsplit]     (reference max, sum) in log2 units
     float *out;              // [B][Hq][D]
@@ -162,8 +163,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     extern __shared__ __align__(128) unsigned char smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tok_begin = split * a.split_len;
     const int len = min(max(__ldg(a.lens + b), 0), a.max_len);
+    // tokens [st, len) are attended; splits start from st rounded down to a 4-token tile, and the
+    // tokens of that tile before st are masked
+    const int st = a.starts ? min(max(__ldg(a.starts + b), 0), len) : 0;
+    const int tok_begin = (st & ~3) + split * a.split_len;
     if (tok_begin >= len) return;                          // the merge never reads this split
     const int tok_end = min(tok_begin + a.split_len, len);
 
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 #pragma unroll
         for (int j = 0; j < QPK; ++j) {
             const float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
-            const float s = (p0 + tk < tok_end) ? keep : -CUDART_INF_F;
+            const float s = (p0 + tk < tok_end && p0 + tk >= st) ? keep : -CUDART_INF_F;
             // Lazy maximum: the reference only has to stay within 2^8 of the running maximum for
             // the weights to stay finite, so it moves (with an exact rescale) only when a score of
             // the iteration exceeds it by more than 8 in log2 units.
@@ -459,7 +463,9 @@ __global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
     const int b = bh / a.Hq;
     const int d = threadIdx.x;
     const int len = min(max(a.lens[b], 0), a.max_len);
-    const int ns = len > 0 ? (len + a.split_len - 1) / a.split_len : 0;
+    const int st = a.starts ? min(max(a.starts[b], 0), len) : 0;
+    const int span = len - (st & ~3);                      // tokens covered by the splits
+    const int ns = len > st ? (span + a.split_len - 1) / a.split_len : 0;
     const float2 *ml = a.ws_ml + (size_t)bh * a.nsplit;
     float mx = -CUDART_INF_F;
     for (int s = 0; s < ns; ++s) mx = fmaxf(mx, ml[s].x);

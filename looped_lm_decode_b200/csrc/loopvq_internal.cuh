@@ -57,7 +57,13 @@ struct DecodePlan {
 };
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len);
 cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
-                          const uint16_t *q, const int32_t *lens, int max_len, float scale,
+                          const uint16_t *q, const int32_t *starts, const int32_t *lens, int max_len, float scale,
                           float *out, float *lse, void *workspace, cudaStream_t s);
+DecodePlan plan_bf16(const loopvq_bf16_cache &c, int max_len);
+cudaError_t launch_bf16_decode(const loopvq_bf16_cache &c, const DecodePlan &plan, const uint16_t *q,
+                               const int32_t *starts, const int32_t *lens, int max_len, float scale, float *out,
+                               float *lse, void *workspace, cudaStream_t s);
+cudaError_t launch_merge2(const float *out_a, const float *lse_a, const float *out_b, const float *lse_b, int rows,
+                          int D, float *out, float *lse, cudaStream_t s);
 
 }  // namespace loopvq

@@ -21,7 +21,8 @@ LOOPVQ_BF16, LOOPVQ_FP32 = 0, 1
 EXPORTS = ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "loopvq_rope_elems",
            "loopvq_prepare", "loopvq_encode", "loopvq_decode_workspace_bytes", "loopvq_decode_attn",
            "loopvq_dequant_debug", "loopvq_last_error", "loopvq_abi_version",
-           "loopvq_decode_attn_noalloc", "loopvq_noalloc_scratch_bytes")
+           "loopvq_decode_attn_noalloc", "loopvq_noalloc_scratch_bytes", "loopvq_decode_attn_range",
+           "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn", "loopvq_merge2")
 
 
 class CacheDesc(C.Structure):
@@ -30,6 +31,12 @@ class CacheDesc(C.Structure):
                 ("Hq", C.c_int32), ("D", C.c_int32), ("c", C.c_int32), ("K", C.c_int32),
                 ("B", C.c_int32), ("Nmax", C.c_int32), ("theta", C.c_float),
                 ("idx", C.c_void_p), ("codebook", C.c_void_p), ("slices", C.c_void_p), ("rope", C.c_void_p)]
+
+
+class Bf16CacheDesc(C.Structure):
+    """Mirror of struct loopvq_bf16_cache."""
+    _fields_ = [("B", C.c_int32), ("Hkv", C.c_int32), ("Hq", C.c_int32), ("D", C.c_int32), ("Nmax", C.c_int32),
+                ("k", C.c_void_p), ("v", C.c_void_p)]
 
 
 class LoopVQError(RuntimeError):
@@ -61,6 +68,15 @@ def lib():
         L.loopvq_dequant_debug.argtypes = [P, i, i, i, i, i, i, i, vp, vp]
         L.loopvq_decode_attn_noalloc.argtypes = [P, i, i, vp, vp, i, f, vp, vp, vp]
         L.loopvq_decode_attn_noalloc.restype = i
+        L.loopvq_decode_attn_range.argtypes = [P, i, i, vp, vp, vp, i, f, vp, vp, vp, sz, vp]
+        L.loopvq_decode_attn_range.restype = i
+        PB = C.POINTER(Bf16CacheDesc)
+        L.loopvq_bf16_decode_workspace_bytes.argtypes = [PB, i]
+        L.loopvq_bf16_decode_workspace_bytes.restype = sz
+        L.loopvq_bf16_decode_attn.argtypes = [PB, vp, vp, vp, i, f, vp, vp, vp, sz, vp]
+        L.loopvq_bf16_decode_attn.restype = i
+        L.loopvq_merge2.argtypes = [vp, vp, vp, vp, i, i, vp, vp, vp]
+        L.loopvq_merge2.restype = i
         L.loopvq_noalloc_scratch_bytes.argtypes = []
         L.loopvq_noalloc_scratch_bytes.restype = sz
         for name in ("loopvq_prepare", "loopvq_encode", "loopvq_decode_attn", "loopvq_dequant_debug"):
@@ -172,6 +188,75 @@ def decode_attn_noalloc(cache: Cache, layer: int, t: int, q: torch.Tensor, lens:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     _check(lib().loopvq_decode_attn_noalloc(cache.ref(), layer, t, _ptr(q), _ptr(lens), max_len, scale, _ptr(out),
                                             _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+def decode_attn_range(cache: Cache, layer: int, t: int, q: torch.Tensor, starts, lens: torch.Tensor,
+                      max_len: int, scale: float = 0.0, out=None, lse=None, workspace=None, stream=None):
+    """decode_attn over tokens starts[b] <= n < lens[b] (starts int32 [B] or None for 0)."""
+    B, Hq, D = cache.B, cache.Hq, cache.D
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    need = decode_workspace_bytes(cache, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().loopvq_decode_attn_range(cache.ref(), layer, t, _ptr(q), _ptr(starts), _ptr(lens), max_len, scale,
+                                          _ptr(out), _ptr(lse), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse
+
+
+class Bf16Cache:
+    """A bf16 KV cache: k, v bf16 [B][Hkv][Nmax][D], keys already rotated (see include/loopvq.h)."""
+
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, Hq: int):
+        assert k.shape == v.shape and k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16
+        assert k.is_contiguous() and v.is_contiguous()
+        self.k, self.v = k, v
+        self.B, self.Hkv, self.Nmax, self.D = k.shape
+        self.Hq = Hq
+        self.desc = Bf16CacheDesc(self.B, self.Hkv, Hq, self.D, self.Nmax, k.data_ptr(), v.data_ptr())
+
+    def ref(self):
+        self.desc.k, self.desc.v = self.k.data_ptr(), self.v.data_ptr()
+        return C.byref(self.desc)
+
+
+def bf16_decode_workspace_bytes(cache: Bf16Cache, max_len: int) -> int:
+    return lib().loopvq_bf16_decode_workspace_bytes(cache.ref(), max_len)
+
+
+def bf16_decode_attn(cache: Bf16Cache, q: torch.Tensor, lens: torch.Tensor, max_len: int, starts=None,
+                     scale: float = 0.0, out=None, lse=None, workspace=None, stream=None):
+    """q bf16 [B][Hq][D]; attends tokens starts[b] <= n < lens[b]; returns (out, lse) like decode_attn."""
+    B, Hq, D = cache.B, cache.Hq, cache.D
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    need = bf16_decode_workspace_bytes(cache, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().loopvq_bf16_decode_attn(cache.ref(), _ptr(q), _ptr(starts), _ptr(lens), max_len, scale, _ptr(out),
+                                         _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         _stream(stream)))
+    return out, lse
+
+
+def merge2(out_a, lse_a, out_b, lse_b, out=None, lse=None, stream=None):
+    """Log-sum-exp merge of two attentions over disjoint token sets; out may alias out_a / out_b."""
+    D = out_a.shape[-1]
+    rows = out_a.numel() // D
+    if out is None:
+        out = torch.empty_like(out_a)
+    if lse is None:
+        lse = torch.empty_like(lse_a)
+    _check(lib().loopvq_merge2(_ptr(out_a), _ptr(lse_a), _ptr(out_b), _ptr(lse_b), rows, D, _ptr(out), _ptr(lse),
+                               _stream(stream)))
     return out, lse
 
 

@@ -94,3 +94,59 @@ def test_workspace_grows_with_context():
     b = lib.loopvq_decode_workspace_bytes(c.ref(), 32768)
     assert 0 < a <= b
     assert lib.loopvq_decode_workspace_bytes(c.ref(), 40000) == 0
+
+
+def _bf16_desc(**kw):
+    args = dict(B=8, Hkv=16, Hq=16, D=128, Nmax=1024)
+    args.update(kw)
+    return LQ.Bf16CacheDesc(args["B"], args["Hkv"], args["Hq"], args["D"], args["Nmax"], 0x10000, 0x30000)
+
+
+@pytest.mark.parametrize("kw,status", [(dict(D=96), 2), (dict(Hq=48), 2), (dict(Hq=17), 1), (dict(B=0), 1),
+                                       (dict(Nmax=0), 1)])
+def test_bf16_shape_validation(kw, status):
+    lib = LQ.lib()
+    d = _bf16_desc(**kw)
+    fake = C.c_void_p(0x20000)
+    assert lib.loopvq_bf16_decode_workspace_bytes(C.byref(d), 0) == 0
+    st = lib.loopvq_bf16_decode_attn(C.byref(d), fake, None, fake, 0, 0.0, fake, None, fake, 1 << 30, None)
+    assert st == status, lib.loopvq_last_error()
+
+
+def test_bf16_argument_validation_before_launch():
+    lib = LQ.lib()
+    d = _bf16_desc()
+    fake = C.c_void_p(0x20000)
+    need = lib.loopvq_bf16_decode_workspace_bytes(C.byref(d), 1024)
+    assert need > 0
+    assert lib.loopvq_bf16_decode_attn(C.byref(d), fake, None, fake, 1025, 0.0, fake, None, fake, need, None) == 1
+    assert b"max_len" in lib.loopvq_last_error()
+    assert lib.loopvq_bf16_decode_attn(C.byref(d), fake, None, fake, 1024, 0.0, fake, None, fake, need - 1, None) == 3
+    assert lib.loopvq_bf16_decode_attn(C.byref(d), fake, C.c_void_p(0x20002), fake, 1024, 0.0, fake, None, fake,
+                                       need, None) == 1
+    assert b"starts" in lib.loopvq_last_error()
+    d.k = 0x10008
+    assert lib.loopvq_bf16_decode_attn(C.byref(d), fake, None, fake, 1024, 0.0, fake, None, fake, need, None) == 1
+    assert b"aligned" in lib.loopvq_last_error()
+    d.k = None
+    assert lib.loopvq_bf16_decode_attn(C.byref(d), fake, None, fake, 1024, 0.0, fake, None, fake, need, None) == 1
+    assert b"NULL" in lib.loopvq_last_error()
+
+
+def test_range_and_merge_validation_before_launch():
+    lib = LQ.lib()
+    c = _cache()
+    c.desc.idx = c.desc.slices = c.desc.rope = c.desc.codebook = 0x10000
+    c.ref = lambda: C.byref(c.desc)
+    fake = C.c_void_p(0x20000)
+    need = lib.loopvq_decode_workspace_bytes(c.ref(), 1024)
+    assert lib.loopvq_decode_attn_range(c.ref(), 0, 0, fake, C.c_void_p(0x20001), fake, 1024, 0.0, fake, None, fake,
+                                        need, None) == 1
+    assert b"starts" in lib.loopvq_last_error()
+    assert lib.loopvq_decode_attn_range(c.ref(), 0, 0, fake, fake, fake, 1024, 0.0, fake, None, fake, need - 1,
+                                        None) == 3
+    assert lib.loopvq_merge2(fake, fake, fake, fake, 4, 96, fake, fake, None) == 2
+    assert lib.loopvq_merge2(fake, fake, fake, fake, -1, 128, fake, fake, None) == 1
+    assert lib.loopvq_merge2(fake, None, fake, fake, 4, 128, fake, fake, None) == 1
+    assert lib.loopvq_merge2(fake, fake, fake, fake, 4, 128, C.c_void_p(0x20002), fake, None) == 1
+    assert lib.loopvq_merge2(None, None, None, None, 0, 128, None, None, None) == 0

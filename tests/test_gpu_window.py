@@ -1,0 +1,192 @@
+"""bf16 decode kernel, coded token ranges and the bf16-window + coded-cache layout vs the CPU checker.
+
+The pages keep the first n_s (sink) and last n_r (recent) tokens of a request in bf16, with keys
+stored already rotated, and code the rest (LoopVQ paper, Sec. 4.3 "Cache layout"); one kernel attends
+to each part and the results are combined through their log-sum-exps ("Attention").  The bars are
+those of the coded decode: max|out - ref| <= 2e-3 * ||ref||_inf, |lse - lse_ref| <= 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import looped_lm_decode_b200 as LQ
+from oracle import oracle as O
+from synth import WORKLOADS, kv_loops, queries, random_indices, bf16_bits_to_f32
+from tests.helpers import pack_words, words_view, make_cache, np_codebook_f32, attn_tolerance_ok
+
+pytestmark = pytest.mark.gpu
+
+N_SINK, N_RECENT = 8, 64            # the pages' serving setting (Sec. 5.3)
+
+
+def _bf16_cache_bits(w, layer, t, n):
+    """bf16 bits [B][Hkv][n][D] of keys (kv = 0) and values (kv = 1): seeded data standing for a bf16
+    cache whose keys were rotated when written."""
+    out = []
+    for kv in range(2):
+        x = kv_loops(w, layer, kv, t, t, range(w.B), range(n), range(w.Hkv))[0]     # [B][n][Hkv][D]
+        out.append(np.ascontiguousarray(x.transpose(0, 2, 1, 3)))
+    return out
+
+
+def _dev_bits(x):
+    return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _dev_i32(x):
+    return torch.from_numpy(np.asarray(x, np.int32)).cuda()
+
+
+BF16_SHAPES = {
+    "mha128": WORKLOADS["ctx4k"].replace(B=3, Hkv=2, Hq=2, Nmax=700),
+    "gqa4": WORKLOADS["gqa16k"].replace(B=2, Hkv=2, Hq=8, Nmax=512),
+    "qpk8": WORKLOADS["ctx4k"].replace(B=2, Hkv=1, Hq=8, Nmax=300),
+    "d64qpk2": WORKLOADS["tiny"].replace(B=3, Hkv=2, Hq=4, Nmax=260),
+}
+
+
+@pytest.mark.parametrize("name", list(BF16_SHAPES))
+@pytest.mark.parametrize("gain", [1.0, 8.0])
+def test_bf16_decode_parity(name, gain):
+    w = BF16_SHAPES[name]
+    kb, vb = _bf16_cache_bits(w, 0, 1, w.Nmax)
+    cache = LQ.Bf16Cache(_dev_bits(kb), _dev_bits(vb), w.Hq)
+    rng = np.random.default_rng(11)
+    lens = rng.integers(0, w.Nmax + 1, w.B).astype(np.int32)
+    lens[0] = w.Nmax
+    if w.B > 2:
+        lens[2] = 1
+    starts = np.array([rng.integers(0, max(int(l), 1)) for l in lens], np.int32)
+    starts[-1] = lens[-1]                                   # an empty range
+    qb = queries(w, 0, 1, gain=gain)
+    max_len = int(lens.max())
+    for with_starts in (False, True):
+        st = starts if with_starts else np.zeros(w.B, np.int32)
+        out, lse = LQ.bf16_decode_attn(cache, _dev_bits(qb), _dev_i32(lens), max_len,
+                                       starts=_dev_i32(st) if with_starts else None)
+        torch.cuda.synchronize()
+        out, lse = out.cpu().numpy(), lse.cpu().numpy()
+        ref = np.zeros((w.B, w.Hq, w.D))
+        lref = np.zeros((w.B, w.Hq))
+        qpk = w.Hq // w.Hkv
+        for b in range(w.B):
+            for hq in range(w.Hq):
+                h = hq // qpk
+                a, e = int(st[b]), int(lens[b])
+                ref[b, hq], lref[b, hq] = O.attention(bf16_bits_to_f32(qb[b, hq]).astype(np.float64),
+                                                      bf16_bits_to_f32(kb[b, h, a:e]), bf16_bits_to_f32(vb[b, h, a:e]),
+                                                      1 / math.sqrt(w.D))
+        ok, msg = attn_tolerance_ok(out, ref, lse, lref)
+        assert ok, f"{name} starts={with_starts}: {msg}"
+
+
+CODED = WORKLOADS["ctx4k"].replace(L=1, B=4, Hkv=2, Hq=2, Nmax=512)
+CODED_GQA = WORKLOADS["gqa16k"].replace(L=1, B=2, Hkv=2, Hq=8, Nmax=256)
+
+
+def _coded_cache(w, layer=0):
+    cache = make_cache(w)
+    codes = {}
+    for blk in range(w.NB):
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                ik = random_indices(w, layer, blk, 0, b, h, range(w.Nmax))
+                iv = random_indices(w, layer, blk, 1, b, h, range(w.Nmax))
+                codes[(blk, b, h)] = (ik, iv)
+                words_view(cache, layer, blk, b, h).copy_(torch.from_numpy(pack_words(ik, iv, cache.NP).view(np.int32)))
+    return cache, codes
+
+
+def _oracle_windowed(w, codes, t, qb, kw_bits, vw_bits, nw, lo, hi, scale):
+    """Per (b, hq): window tokens 0..nw[b]-1 of the bf16 arrays plus coded tokens lo[b]..hi[b]-1."""
+    blk, m = t // w.Tc, t % w.Tc
+    qpk = w.Hq // w.Hkv
+    ref = np.zeros((w.B, w.Hq, w.D))
+    lref = np.zeros((w.B, w.Hq))
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            h = hq // qpk
+            ik, iv = codes[(blk, b, h)]
+            a, e = int(lo[b]), max(int(hi[b]), int(lo[b]))
+            kw = bf16_bits_to_f32(kw_bits[b, h, :nw[b]]) if kw_bits is not None else np.zeros((0, w.D))
+            vw = bf16_bits_to_f32(vw_bits[b, h, :nw[b]]) if vw_bits is not None else np.zeros((0, w.D))
+            ref[b, hq], lref[b, hq] = O.decode_windowed(
+                bf16_bits_to_f32(qb[b, hq]).astype(np.float64), kw, vw, ik[a:e], iv[a:e],
+                np_codebook_f32(w, 0, blk, 0, h), np_codebook_f32(w, 0, blk, 1, h), w.c, w.Tc, m, a, w.theta, scale)
+    return ref, lref
+
+
+@pytest.mark.parametrize("w", [CODED, CODED_GQA], ids=["mha", "gqa"])
+def test_decode_range_parity(w):
+    """Coded tokens start_b <= n < len_b only; starts off the 4-token tiles are masked inside the tile."""
+    cache, codes = _coded_cache(w)
+    starts = np.array([0, 5, 130, 7][:w.B], np.int32)
+    lens = np.array([w.Nmax, 233, 131, 7][:w.B], np.int32)
+    t = 2
+    qb = queries(w, 0, t)
+    out, lse = LQ.decode_attn_range(cache, 0, t, _dev_bits(qb), _dev_i32(starts), _dev_i32(lens), int(lens.max()))
+    torch.cuda.synchronize()
+    ref, lref = _oracle_windowed(w, codes, t, qb, None, None, [0] * w.B, starts, lens, 1 / math.sqrt(w.D))
+    ok, msg = attn_tolerance_ok(out.cpu().numpy(), ref, lse.cpu().numpy(), lref)
+    assert ok, msg
+
+
+@pytest.mark.parametrize("w", [CODED, CODED_GQA], ids=["mha", "gqa"])
+@pytest.mark.parametrize("t", [0, 3])
+def test_windowed_cache_parity(w, t):
+    """Sink tokens 0..7 and recent tokens len-64..len-1 in a bf16 window, the rest coded: bf16 kernel +
+    coded range kernel + merge2 against one softmax over all tokens."""
+    cache, codes = _coded_cache(w)
+    lens = np.array([w.Nmax, 200, 72, 30][:w.B], np.int32)
+    nw = np.minimum(lens, N_SINK + N_RECENT).astype(np.int32)        # window fill
+    lo = np.minimum(lens, N_SINK).astype(np.int32)                     # coded range [lo, hi)
+    hi = np.maximum(lens - N_RECENT, lo).astype(np.int32)
+    W = N_SINK + N_RECENT
+    kw_bits, vw_bits = _bf16_cache_bits(w, 0, t, W)
+    win = LQ.Bf16Cache(_dev_bits(kw_bits), _dev_bits(vw_bits), w.Hq)
+    qb = queries(w, 0, t)
+    q = _dev_bits(qb)
+    ow, lw = LQ.bf16_decode_attn(win, q, _dev_i32(nw), W)
+    oc, lc = LQ.decode_attn_range(cache, 0, t, q, _dev_i32(lo), _dev_i32(hi), int(hi.max()))
+    out, lse = LQ.merge2(oc, lc, ow, lw, out=oc, lse=lc)              # in place
+    torch.cuda.synchronize()
+    ref, lref = _oracle_windowed(w, codes, t, qb, kw_bits, vw_bits, nw, lo, hi, 1 / math.sqrt(w.D))
+    ok, msg = attn_tolerance_ok(out.cpu().numpy(), ref, lse.cpu().numpy(), lref)
+    assert ok, msg
+
+
+def test_merge2_is_attention_over_the_union():
+    """Two disjoint token sets attended separately (by the checker) and merged on the GPU equal one
+    attention over their union; an empty part (lse = -inf) leaves the other unchanged."""
+    rng = np.random.default_rng(3)
+    rows, D = 6, 128
+    q = rng.standard_normal((rows, D))
+    parts = []
+    for n in (40, 25):
+        k, v = rng.standard_normal((rows, n, D)), rng.standard_normal((rows, n, D))
+        parts.append((k, v))
+    res = [[O.attention(q[r], k[r], v[r], 0.1) for r in range(rows)] for k, v in parts]
+    oa = np.array([x[0] for x in res[0]], np.float32)
+    la = np.array([x[1] for x in res[0]], np.float32)
+    ob = np.array([x[0] for x in res[1]], np.float32)
+    lb = np.array([x[1] for x in res[1]], np.float32)
+    ob[4], lb[4] = 0.0, -np.inf                                         # row 4: part b empty
+    oa[5], la[5] = 0.0, -np.inf                                         # row 5: both empty
+    ob[5], lb[5] = 0.0, -np.inf
+    ref, lref = [], []
+    for r in range(rows):
+        ka = parts[0][0][r] if r != 5 else np.zeros((0, D))
+        va = parts[0][1][r] if r != 5 else np.zeros((0, D))
+        kb_ = parts[1][0][r] if r < 4 else np.zeros((0, D))
+        vb_ = parts[1][1][r] if r < 4 else np.zeros((0, D))
+        o, l = O.attention(q[r], np.concatenate([ka, kb_]), np.concatenate([va, vb_]), 0.1)
+        ref.append(o)
+        lref.append(l)
+    ta, tla = torch.from_numpy(oa).cuda(), torch.from_numpy(la).cuda()
+    out, lse = LQ.merge2(ta, tla, torch.from_numpy(ob).cuda(), torch.from_numpy(lb).cuda(), out=ta, lse=tla)
+    torch.cuda.synchronize()
+    ok, msg = attn_tolerance_ok(out.cpu().numpy(), np.array(ref), lse.cpu().numpy(), np.array(lref), rel=1e-5,
+                                lse_tol=1e-5)
+    assert ok, msg
