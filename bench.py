@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--batch", type=int, default=0, help="override the batch size (profiling runs)")
+    ap.add_argument("--no-compare", action="store_true",
+                    help="skip the bf16-cache comparison and the bf16-window layout measurement")
     return ap.parse_args()
 
 
@@ -96,6 +98,84 @@ def profiled_traffic(workload_name):
     if h.hexdigest()[:16] != prof.get("kernel_sources_sha256_16"):
         return None
     return prof["dram_bytes_read_per_launch"] + prof["dram_bytes_write_per_launch"]
+
+
+def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
+    """Same decode calls on a cache held entirely in bf16 (the pages' comparison, LoopVQ paper Sec. 5.3),
+    and on the pages' serving layout: 8 sink + 64 recent tokens in a bf16 window, the rest coded, merged
+    through the log-sum-exps (Sec. 4.3 "Cache layout", "Attention").  Timed per call with CUDA events."""
+    import torch
+    import looped_lm_decode_b200 as LQ
+    from synth import gpu as SG
+    dev = qs.device
+    nl = min(2, w.L)                                # two bf16 layers: every call streams > L2
+    tmp = torch.empty((1, w.B, w.Nmax, w.Hkv, w.D), dtype=torch.bfloat16, device=dev)
+    caches = []
+    for layer in range(nl):
+        kv = []
+        for k in range(2):
+            SG.fill_kv(w, layer, k, 1, 1, tmp)
+            kv.append(tmp[0].permute(0, 2, 1, 3).contiguous())
+        caches.append(LQ.Bf16Cache(kv[0], kv[1], w.Hq))
+    del tmp
+    ws_b = torch.empty(max(LQ.bf16_decode_workspace_bytes(caches[0], max_len), 16), dtype=torch.uint8, device=dev)
+    out_b = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+    lse_b = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+
+    def timed(fn, calls):
+        for i in range(calls):
+            fn(i)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps * calls)]
+        torch.cuda.synchronize()
+        for r in range(reps):
+            for i in range(calls):
+                e0, e1 = evs[r * calls + i]
+                e0.record(stream)
+                fn(i)
+                e1.record(stream)
+        torch.cuda.synchronize()
+        return statistics.fmean(a.elapsed_time(b) for a, b in evs)
+
+    calls = w.T * nl
+    bf_ms = timed(lambda i: LQ.bf16_decode_attn(caches[i % nl], qs[i], lens, max_len, out=out_b, lse=lse_b,
+                                                workspace=ws_b, stream=stream), calls)
+    bf_bytes = int(lens_np.astype(np.int64).sum()) * w.Hkv * 2 * w.D * 2 + w.B * w.Hq * (w.D * 2 + w.D * 4 + 4)
+    del caches
+
+    n_sink, n_recent = 8, 64
+    W = n_sink + n_recent
+    tmp = torch.empty((1, w.B, W, w.Hkv, w.D), dtype=torch.bfloat16, device=dev)
+    win = []
+    for k in range(2):
+        SG.fill_kv(w.replace(Nmax=W), 0, k, 0, 0, tmp)
+        win.append(tmp[0].permute(0, 2, 1, 3).contiguous())
+    wcache = LQ.Bf16Cache(win[0], win[1], w.Hq)
+    lw = torch.from_numpy(np.minimum(lens_np, W).astype(np.int32)).to(dev)
+    lo_np = np.minimum(lens_np, n_sink).astype(np.int32)
+    hi_np = np.maximum(lens_np - n_recent, lo_np).astype(np.int32)
+    lo, hi = torch.from_numpy(lo_np).to(dev), torch.from_numpy(hi_np).to(dev)
+    ws_w = torch.empty(max(LQ.bf16_decode_workspace_bytes(wcache, W), 16), dtype=torch.uint8, device=dev)
+    out_c = torch.empty_like(out_b)
+    lse_c = torch.empty_like(lse_b)
+    hmax = int(hi_np.max())
+
+    def windowed(i):
+        t, layer = divmod(i, w.L)
+        LQ.bf16_decode_attn(wcache, qs[i], lw, W, out=out_b, lse=lse_b, workspace=ws_w, stream=stream)
+        LQ.decode_attn_range(cache, layer, t, qs[i], lo, hi, hmax, out=out_c, lse=lse_c, workspace=ws, stream=stream)
+        LQ.merge2(out_c, lse_c, out_b, lse_b, out=out_c, lse=lse_c, stream=stream)
+
+    win_ms = timed(windowed, w.T * w.L)
+    peak, kind = peaks()
+    return {
+        "bf16_cache": {"us_per_call": bf_ms * 1e3, "gbs": bf_bytes / (bf_ms * 1e-3) / 1e9,
+                       "frac": bf_bytes / (bf_ms * 1e-3) / 1e9 / peak, "peak": peak, "peak_kind": kind,
+                       "bytes_per_call": bf_bytes,
+                       "kernel": "loopvq_bf16_decode_attn over a bf16 cache of the same shape (keys stored rotated)"},
+        "windowed": {"us_per_call": win_ms * 1e3, "sink": n_sink, "recent": n_recent,
+                     "calls": "loopvq_bf16_decode_attn (window) + loopvq_decode_attn_range (coded) + loopvq_merge2"},
+    }
 
 
 def workload_desc(w):
@@ -355,6 +435,10 @@ def main():
     h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * 4
     d2h = out_host.numel() * 4 + lse_host.numel() * 4
 
+    compare = None
+    if not args.no_compare and rank == 0:
+        compare = bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream)
+
     ms_step = max_over_ranks(ms_step_local, dist, dev)
     e2e_ms = max_over_ranks(e2e_ms_local, dist, dev)
     avg_call_ms = max_over_ranks(statistics.fmean(call_ms), dist, dev)
@@ -391,6 +475,10 @@ def main():
                        "input_gbs": 2 * w.Tc * w.B * w.Nmax * w.Hkv * w.D * 2 / (statistics.median(enc_ms) * 1e-3) / 1e9,
                        "kernel": "encode_tc_kernel (tcgen05 bf16 distance contraction + TMEM arg-max)"},
         }
+        if compare is not None:
+            line["bf16_cache"] = compare["bf16_cache"]
+            line["bf16_cache"]["loopvq_speedup"] = compare["bf16_cache"]["us_per_call"] / (avg_call_ms * 1e3)
+            line["windowed"] = compare["windowed"]
         if world == 1 and not args.no_cpu_baseline:
             s, nb, u = cpu_sample(w, args.cpu_seconds)
             line["cpu_baseline"] = {"value": nb / s / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",

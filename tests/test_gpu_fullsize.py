@@ -87,3 +87,34 @@ def test_encode_full_size_sampled():
                     assert abs(dg - do) <= 1e-5 * max(dg, do)
                     ties += 1
     print(f"near-ties: {ties}")
+
+
+@pytest.mark.parametrize("name", ["ctx32k", "gqa16k"])
+def test_bf16_cache_full_size_sampled(name):
+    """The bf16-cache comparison at full size, built as bench.py builds it (loop step 1 of layer 0 as
+    rotated keys / values, [B][Hkv][Nmax][D]); sampled (sequence, query head) outputs vs the checker."""
+    w = WORKLOADS[name].replace(L=1)
+    tmp = torch.empty((1, w.B, w.Nmax, w.Hkv, w.D), dtype=torch.bfloat16, device="cuda")
+    kv = []
+    for k in range(2):
+        SG.fill_kv(w, 0, k, 1, 1, tmp)
+        kv.append(tmp[0].permute(0, 2, 1, 3).contiguous())
+    del tmp
+    cache = LQ.Bf16Cache(kv[0], kv[1], w.Hq)
+    lens = lengths(w)
+    t = 2
+    qd = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    SG.fill_q(w, 0, t, qd)
+    out, lse = LQ.bf16_decode_attn(cache, qd, torch.from_numpy(lens).cuda(), int(lens.max()))
+    torch.cuda.synchronize()
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    qpk = w.Hq // w.Hkv
+    for b, hq in SAMPLES[name]:
+        h = hq // qpk
+        n = int(lens[b])
+        kb = bf16_bits_to_f32(kv_loops(w, 0, 0, 1, 1, [b], range(n), [h])[0, 0, :, 0, :])
+        vb = bf16_bits_to_f32(kv_loops(w, 0, 1, 1, 1, [b], range(n), [h])[0, 0, :, 0, :])
+        qb = queries(w, 0, t, b=[b], hq=[hq])[0, 0]
+        ref, lref = O.attention(bf16_bits_to_f32(qb).astype(np.float64), kb, vb, 1 / math.sqrt(w.D))
+        ok, msg = attn_tolerance_ok(out[b, hq], ref, lse[b, hq:hq + 1], np.array([lref]))
+        assert ok, f"{name} (b={b}, hq={hq}): {msg}"
