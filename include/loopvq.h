@@ -23,9 +23,10 @@
  *     message (thread-local, valid until the next call on this thread).
  *   - A CUDA launch error returns LOOPVQ_ERR_CUDA with the CUDA error string.
  *
- * Supported shapes: D in {64, 128}; c in {4, 8}; Tc in {1, 2, 4} with
- * G = c*Tc <= 32; 1 <= K <= 256; Hq a multiple of Hkv with Hq/Hkv in
- * {1, 2, 4, 8}; T a multiple of Tc; Nmax a multiple of 4.
+ * Supported shapes: D in {64, 128}; c in {4, 8, 16, 32}; Tc in {1, 2, 4}
+ * with G = c*Tc <= 32; 1 <= K <= 256; Hq a multiple of Hkv with Hq/Hkv in
+ * {1, 2, 4, 8}; T a multiple of Tc; Nmax a multiple of 4.  Tc = 1 is plain
+ * per-loop-step coding (CQ, Sec. 2), which runs on the same kernels.
  */
 #ifndef LOOPVQ_H
 #define LOOPVQ_H

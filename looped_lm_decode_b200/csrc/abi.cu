@@ -37,8 +37,11 @@ loopvq_status check_shape(const loopvq_cache *cc) {
     if (cc->K > 256) return fail(LOOPVQ_ERR_INVALID_ARG, "K=%d exceeds 256 (8-bit codes)", cc->K);
     if (cc->Nmax % 4 != 0) return fail(LOOPVQ_ERR_INVALID_ARG, "Nmax=%d is not a multiple of 4", cc->Nmax);
     if (cc->D != 64 && cc->D != 128) return fail(LOOPVQ_ERR_UNSUPPORTED, "D=%d (supported: 64, 128)", cc->D);
-    if (cc->c != 4 && cc->c != 8) return fail(LOOPVQ_ERR_UNSUPPORTED, "c=%d (supported: 4, 8)", cc->c);
+    if (cc->c != 4 && cc->c != 8 && cc->c != 16 && cc->c != 32)
+        return fail(LOOPVQ_ERR_UNSUPPORTED, "c=%d (supported: 4, 8, 16, 32)", cc->c);
     if (cc->Tc != 1 && cc->Tc != 2 && cc->Tc != 4) return fail(LOOPVQ_ERR_UNSUPPORTED, "Tc=%d (supported: 1, 2, 4)", cc->Tc);
+    if (cc->c * cc->Tc > 32)
+        return fail(LOOPVQ_ERR_UNSUPPORTED, "G = c*Tc = %d (supported: up to 32)", cc->c * cc->Tc);
     const int qpk = cc->Hq / cc->Hkv;
     if (qpk != 1 && qpk != 2 && qpk != 4 && qpk != 8)
         return fail(LOOPVQ_ERR_UNSUPPORTED, "Hq/Hkv=%d (supported: 1, 2, 4, 8)", qpk);

@@ -98,8 +98,12 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     const int qpk = cc.Hq / cc.Hkv;
     if (cc.D == 128 && cc.c == 4) return dispatch_qpk<128, 4>(qpk, a, plan, s);
     if (cc.D == 128 && cc.c == 8) return dispatch_qpk<128, 8>(qpk, a, plan, s);
+    if (cc.D == 128 && cc.c == 16) return dispatch_qpk<128, 16>(qpk, a, plan, s);
+    if (cc.D == 128 && cc.c == 32) return dispatch_qpk<128, 32>(qpk, a, plan, s);
     if (cc.D == 64 && cc.c == 4) return dispatch_qpk<64, 4>(qpk, a, plan, s);
     if (cc.D == 64 && cc.c == 8) return dispatch_qpk<64, 8>(qpk, a, plan, s);
+    if (cc.D == 64 && cc.c == 16) return dispatch_qpk<64, 16>(qpk, a, plan, s);
+    if (cc.D == 64 && cc.c == 32) return dispatch_qpk<64, 32>(qpk, a, plan, s);
     return cudaErrorInvalidValue;
 }
 

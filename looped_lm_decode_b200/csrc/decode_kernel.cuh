@@ -12,8 +12,8 @@
 //    slice in bytes [0,128) and of the V slice in [128,256), replicated so that
 //    the 8-byte piece a lane reads sits in its own bank pair: lane l reads bytes
 //    (l % 16) * 8 of the half-row.  For c = 4 that is replica l % 16 of the
-//    8-byte entry; for c = 8 it is half (l % 2) of replica (l % 16) / 2 of the
-//    16-byte entry.  A gather by 16 lanes of random entries is conflict-free,
+//    8-byte entry; for c = 4j it is part l % j of replica (l % 16) / j of the
+//    2c-byte entry (c = 8, 16, 32).  A gather by 16 lanes of random entries is conflict-free,
 //    and its address is one byte permute of the index word (code -> bits 8..15,
 //    the lane's column -> bits 0..7).
 //  * Every lane owns 8 channels: 4 of a channel group g < D/(2c) and the 4
@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     constexpr int TT = 4 * NW;                             // tokens per slot iteration
     constexpr int STRIDE = NSLOT * TT;                     // tokens between two iterations of a slot
     constexpr int QB = NT * 16 * NW;                       // bytes of one prefetch-queue stage
-    static_assert(C == 4 || C == 8, "c");
+    static_assert(C == 4 || C == 8 || C == 16 || C == 32, "c");
     static_assert(NL >= 8 && NL <= 16, "slot width");
 
     extern __shared__ __align__(128) unsigned char smem[];
@@ -210,9 +210,12 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(src));
                 *reinterpret_cast<uint2 *>(dst) = v;
             } else {
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (r < a.K) v = __ldg(reinterpret_cast<const uint4 *>(src));
-                *reinterpret_cast<uint4 *>(dst) = v;
+#pragma unroll
+                for (int u = 0; u < EB / 16; ++u) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < a.K) v = __ldg(reinterpret_cast<const uint4 *>(src) + u);
+                    *reinterpret_cast<uint4 *>(dst + 16 * u) = v;
+                }
             }
         }
     }

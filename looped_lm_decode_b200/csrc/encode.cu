@@ -123,6 +123,11 @@ static cudaError_t dispatch_c(int c, int tc, const EncodeArgs &a, int x_dtype, i
         if (tc == 4) return launch_ct<D, 8, 4>(a, x_dtype, nb, s);
         if (tc == 2) return launch_ct<D, 8, 2>(a, x_dtype, nb, s);
         if (tc == 1) return launch_ct<D, 8, 1>(a, x_dtype, nb, s);
+    } else if (c == 16) {
+        if (tc == 2) return launch_ct<D, 16, 2>(a, x_dtype, nb, s);
+        if (tc == 1) return launch_ct<D, 16, 1>(a, x_dtype, nb, s);
+    } else if (c == 32) {
+        if (tc == 1) return launch_ct<D, 32, 1>(a, x_dtype, nb, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -488,8 +488,12 @@ cudaError_t launch_encode_tc(const loopvq_cache &cc, int layer, int block, const
     const int G = cc.c * cc.Tc;
     if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4>(a, s);
     if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4>(a, s);
+    if (cc.D == 128 && cc.c == 16 && cc.Tc == 1) return launch_tc_ct<128, 16, 1>(a, s);
+    if (cc.D == 128 && cc.c == 32 && cc.Tc == 1) return launch_tc_ct<128, 32, 1>(a, s);
     if (cc.D == 64 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<64, 4, 4>(a, s);
     if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4>(a, s);
+    if (cc.D == 64 && cc.c == 16 && cc.Tc == 1) return launch_tc_ct<64, 16, 1>(a, s);
+    if (cc.D == 64 && cc.c == 32 && cc.Tc == 1) return launch_tc_ct<64, 32, 1>(a, s);
     (void)G;
     return cudaErrorNotSupported;
 }

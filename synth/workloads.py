@@ -8,6 +8,9 @@ Five workload shapes (all K = 256 codes, b = 8 bits):
   gqa16k     24 layers, 4 KV/16 q heads, D = 128, c = 8 (G = 32, 0.25 bit), batch 64, 16384 tokens
   deep32     4 layers, 40 KV heads, T = 32 coded as 8 blocks of 4, D = 128, c = 4,
              batch 2, 8192 tokens
+  ctx32k_cq  ctx32k coded per loop step (CQ: Tc = 1, c = G = 16, 0.5 bit), the
+             baseline the pages compare LoopVQ against at the same bitwidth; same
+             seed as ctx32k, so keys, values, queries and lengths are identical
 
 The model shapes follow the pages' Ouro-1.4B description (24 layers, 16 heads of
 dimension 128, 4 loop steps) and the deep-recurrence variant follows the
@@ -97,6 +100,8 @@ WORKLOADS = {
                        rho=_rho((0.6, 0.8, 0.95), 4)),
     "deep32": Workload("deep32", 4, L=4, T=32, Tc=4, Hkv=40, Hq=40, D=128, c=4, K=256, B=2, Nmax=8192,
                        rho=_rho((0.9,), 32)),
+    "ctx32k_cq": Workload("ctx32k_cq", 2, L=24, T=4, Tc=1, Hkv=16, Hq=16, D=128, c=16, K=256, B=8, Nmax=32768,
+                          rho=_rho((0.7, 0.8, 0.9), 4), len_lo=16384),
 }
 
 

@@ -46,7 +46,7 @@ def test_buffer_sizes():
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(D=96), 2), (dict(c=16), 2), (dict(Tc=3, T=6), 2), (dict(Hq=48), 2), (dict(Hq=17), 1),
+    (dict(D=96), 2), (dict(c=16), 2), (dict(c=64, Tc=1), 2), (dict(c=2), 2), (dict(Tc=3, T=6), 2), (dict(Hq=48), 2), (dict(Hq=17), 1),
     (dict(T=6), 1), (dict(K=300), 1), (dict(Nmax=1022), 1), (dict(B=0), 1)])
 def test_shape_validation(kw, status):
     lib = LQ.lib()

@@ -28,6 +28,10 @@ SMALL = {
     "deep": WORKLOADS["deep32"].replace(L=1, T=8, B=2, Hkv=3, Hq=3, Nmax=256),
     "d64c8": WORKLOADS["tiny"].replace(c=8, Hq=2, B=2, Nmax=128),
     "qpk2": WORKLOADS["ctx4k"].replace(L=1, B=2, Hkv=2, Hq=4, Nmax=256),
+    # plain per-loop-step coding (CQ): Tc = 1, c = G, on the same kernels
+    "cq16": WORKLOADS["ctx4k"].replace(L=1, B=2, Hkv=2, Hq=2, Nmax=256, c=16, Tc=1),
+    "cq32g": WORKLOADS["gqa16k"].replace(L=1, B=2, Hkv=1, Hq=4, Nmax=128, c=32, Tc=1),
+    "cq16d64": WORKLOADS["tiny"].replace(c=16, Tc=2, B=2, Hq=2, Hkv=2, Nmax=128),
 }
 
 
@@ -188,7 +192,8 @@ def _check_codes(w, x_np, dtype, E, codes_gpu, b, h, kv):
 
 
 @pytest.mark.parametrize("name,dtype", [("tiny", "bf16"), ("tiny", "f32"), ("ctx", "bf16"), ("gqa", "bf16"),
-                                        ("deep", "bf16"), ("d64c8", "f32")])
+                                        ("deep", "bf16"), ("d64c8", "f32"), ("cq16", "bf16"), ("cq16", "f32"),
+                                        ("cq32g", "bf16"), ("cq16d64", "bf16")])
 def test_encode_parity(name, dtype):
     w = SMALL[name]
     if name == "ctx":
