@@ -213,6 +213,76 @@ loopvq_status loopvq_merge2(const float *out_a, const float *lse_a, const float 
                             void *stream);
 
 /*
+ * The bf16 window of a coded cache and its decode-time life cycle (Sec. 4.3
+ * "Cache layout": the first n_s (sink) and the most recent n_r tokens of a
+ * request stay in bf16, pages of 8 tokens; "Encoding": during decode the
+ * oldest recent page is encoded once the window holds 8 tokens more than n_r).
+ *
+ * Every sequence b has W = n_sink + n_recent + 8 slots per (layer, loop step):
+ *   slots 0 .. n_sink-1        tokens 0 .. n_sink-1 (the sink, once filled);
+ *   slots n_sink .. fill_b-1   tokens coded_end_b .. coded_end_b + fill_b - n_sink - 1
+ *                              (the recent tokens, oldest first);
+ * and the tokens n_sink <= n < coded_end_b are in the coded cache.  A token is
+ * held twice as a key: rotated at its position (what attention reads) and
+ * before RoPE (what the encoder reads when its page leaves the window, since
+ * keys are coded before RoPE).  Caller-owned device buffers:
+ *   k_rot, k_pre, v   bf16 [L][T][B][Hkv][W][D], 16-byte aligned;
+ *   fill              int32 [B], slots in use (0 .. W);
+ *   coded_end         int32 [B], >= n_sink; starts at n_sink for an empty
+ *                     coded part.
+ * Shapes L, T, B, Hkv, Hq, D must equal those of the coded cache used with it;
+ * n_sink and n_recent are positive multiples of 8.  The caller fills the
+ * window and the counters after prefill (loopvq_encode for the coded part).
+ */
+typedef struct loopvq_window {
+    int32_t L, T, B, Hkv, Hq, D;
+    int32_t n_sink, n_recent;
+    uint16_t *k_rot;
+    uint16_t *k_pre;
+    uint16_t *v;
+    int32_t *fill;
+    int32_t *coded_end;
+} loopvq_window;
+
+/* Slots per (layer, loop step, sequence, KV head): n_sink + n_recent + 8 (0 if invalid). */
+int loopvq_window_slots(const loopvq_window *w);
+
+/*
+ * Start a decode step: for every sequence whose window is full (fill_b == W)
+ * encode its oldest recent page (slots n_sink .. n_sink+7, tokens coded_end_b
+ * .. coded_end_b+7) for every layer and block from k_pre and v into the coded
+ * cache (exact fp32 nearest entries, as loopvq_encode), move the remaining
+ * recent slots down by 8 and set coded_end_b += 8, fill_b -= 8; then reserve
+ * the new token's slot (fill_b += 1) for every sequence.  All decisions are
+ * taken on the device from fill and coded_end; nothing synchronises.  A page
+ * whose tokens would reach past the coded cache's Nmax is not written.
+ */
+loopvq_status loopvq_window_advance(const loopvq_window *w, const loopvq_cache *cache, void *stream);
+
+/*
+ * Write the current token of (layer, t) into slot fill_b - 1 of every
+ * sequence: k_rot (rotated at its position), k_pre (before RoPE) and v are
+ * bf16 [B][Hkv][D], 16-byte aligned.  Call after loopvq_window_advance.
+ */
+loopvq_status loopvq_window_append(const loopvq_window *w, int layer, int t, const uint16_t *k_rot,
+                                   const uint16_t *k_pre, const uint16_t *v, void *stream);
+
+/* Workspace bytes loopvq_window_decode_attn needs with coded parts of up to max_coded tokens. */
+size_t loopvq_window_workspace_bytes(const loopvq_window *w, const loopvq_cache *cache, int max_coded);
+
+/*
+ * Decode attention of (layer, t) over the window and the coded cache: the
+ * bf16 kernel over window slots 0 .. fill_b-1, the coded kernel over tokens
+ * n_sink <= n < coded_end_b, merged through their log-sum-exps (Sec. 4.3
+ * "Attention").  max_coded is a host upper bound of coded_end (<= Nmax).
+ * q, scale, out, lse as for loopvq_decode_attn; workspace of at least
+ * loopvq_window_workspace_bytes(w, cache, max_coded) bytes.
+ */
+loopvq_status loopvq_window_decode_attn(const loopvq_window *w, const loopvq_cache *cache, int layer, int t,
+                                        const uint16_t *q, int max_coded, float scale, float *out,
+                                        float *lse, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Explicit reconstruction for checking (eq. 5): for sequence b, tokens
  * tok0 .. tok0+ntok-1 and every KV head, the loop-step-t reconstruction of
  * keys (kv = 0) or values (kv = 1); keys are rotated by RoPE at their

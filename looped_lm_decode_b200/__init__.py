@@ -6,4 +6,5 @@ include/loopvq.h; this package is its thin Python binding.
 from .loopvq import (Cache, CacheDesc, LoopVQError, prepare, encode, decode_attn, decode_workspace_bytes,  # noqa: F401
                      dequant_debug, default_scale, lib, LIB_PATH, EXPORTS, decode_attn_noalloc,
                      decode_attn_range, Bf16Cache, Bf16CacheDesc, bf16_decode_attn, bf16_decode_workspace_bytes,
-                     merge2)
+                     merge2, Window, WindowDesc, window_advance, window_append, window_workspace_bytes,
+                     window_decode_attn)

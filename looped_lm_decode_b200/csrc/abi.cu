@@ -159,8 +159,8 @@ static loopvq_status decode_common(const char *fn, const loopvq_cache *cc, int l
         return fail(LOOPVQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws_bytes,
                     workspace ? ws_bytes : (size_t)0);
     if (!aligned16(workspace)) return fail(LOOPVQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
-    cudaError_t e = loopvq::launch_decode(*cc, plan, layer, t, q, starts, lens, max_len, scale, out, lse, workspace,
-                                          (cudaStream_t)stream);
+    cudaError_t e = loopvq::launch_decode(*cc, plan, layer, t, q, starts, 0, lens, max_len, scale, out, lse,
+                                          workspace, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, fn);
     return LOOPVQ_OK;
 }
@@ -237,6 +237,92 @@ loopvq_status loopvq_merge2(const float *out_a, const float *lse_a, const float 
         if (p && (reinterpret_cast<uintptr_t>(p) & 3u)) return fail(LOOPVQ_ERR_INVALID_ARG, "pointer not 4-byte aligned");
     cudaError_t e = loopvq::launch_merge2(out_a, lse_a, out_b, lse_b, rows, D, out, lse, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "loopvq_merge2");
+    return LOOPVQ_OK;
+}
+
+static loopvq_status check_window(const loopvq_window *w, const loopvq_cache *cc) {
+    if (!w) return fail(LOOPVQ_ERR_INVALID_ARG, "window is NULL");
+    LQ_TRY(check_shape(cc));
+    if (w->L != cc->L || w->T != cc->T || w->B != cc->B || w->Hkv != cc->Hkv || w->Hq != cc->Hq || w->D != cc->D)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "window shape (L, T, B, Hkv, Hq, D) differs from the cache's");
+    if (w->n_sink <= 0 || w->n_recent <= 0 || w->n_sink % 8 != 0 || w->n_recent % 8 != 0)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "n_sink=%d, n_recent=%d must be positive multiples of 8", w->n_sink,
+                    w->n_recent);
+    LQ_TRY(check_ptr(w->k_rot, "k_rot"));
+    LQ_TRY(check_ptr(w->k_pre, "k_pre"));
+    LQ_TRY(check_ptr(w->v, "v"));
+    if (!w->fill || !w->coded_end) return fail(LOOPVQ_ERR_INVALID_ARG, "fill or coded_end is NULL");
+    if ((reinterpret_cast<uintptr_t>(w->fill) & 3u) || (reinterpret_cast<uintptr_t>(w->coded_end) & 3u))
+        return fail(LOOPVQ_ERR_INVALID_ARG, "fill or coded_end not 4-byte aligned");
+    return LOOPVQ_OK;
+}
+
+int loopvq_window_slots(const loopvq_window *w) {
+    if (!w || w->n_sink <= 0 || w->n_recent <= 0 || w->n_sink % 8 || w->n_recent % 8) return 0;
+    return loopvq::window_slots(*w);
+}
+
+loopvq_status loopvq_window_advance(const loopvq_window *w, const loopvq_cache *cc, void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_window(w, cc));
+    LQ_TRY(check_ptr(cc->idx, "idx"));
+    LQ_TRY(check_ptr(cc->codebook, "codebook"));
+    cudaError_t e = loopvq::launch_window_advance(*w, *cc, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_window_advance");
+    return LOOPVQ_OK;
+}
+
+loopvq_status loopvq_window_append(const loopvq_window *w, int layer, int t, const uint16_t *k_rot,
+                                   const uint16_t *k_pre, const uint16_t *v, void *stream) {
+    g_err[0] = 0;
+    if (!w) return fail(LOOPVQ_ERR_INVALID_ARG, "window is NULL");
+    if (w->n_sink <= 0 || w->n_recent <= 0 || w->n_sink % 8 || w->n_recent % 8 || w->B <= 0 || w->Hkv <= 0 ||
+        (w->D != 64 && w->D != 128))
+        return fail(LOOPVQ_ERR_INVALID_ARG, "invalid window shape");
+    if (layer < 0 || layer >= w->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, w->L);
+    if (t < 0 || t >= w->T) return fail(LOOPVQ_ERR_INVALID_ARG, "t=%d out of [0, %d)", t, w->T);
+    LQ_TRY(check_ptr(w->k_rot, "window k_rot"));
+    LQ_TRY(check_ptr(w->k_pre, "window k_pre"));
+    LQ_TRY(check_ptr(w->v, "window v"));
+    if (!w->fill) return fail(LOOPVQ_ERR_INVALID_ARG, "fill is NULL");
+    LQ_TRY(check_ptr(k_rot, "k_rot"));
+    LQ_TRY(check_ptr(k_pre, "k_pre"));
+    LQ_TRY(check_ptr(v, "v"));
+    cudaError_t e = loopvq::launch_window_append(*w, layer, t, k_rot, k_pre, v, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_window_append");
+    return LOOPVQ_OK;
+}
+
+size_t loopvq_window_workspace_bytes(const loopvq_window *w, const loopvq_cache *cc, int max_coded) {
+    if (check_window(w, cc) != LOOPVQ_OK || max_coded < 0 || max_coded > cc->Nmax) return 0;
+    return loopvq::window_ws_bytes(*w, *cc, max_coded);
+}
+
+loopvq_status loopvq_window_decode_attn(const loopvq_window *w, const loopvq_cache *cc, int layer, int t,
+                                        const uint16_t *q, int max_coded, float scale, float *out, float *lse,
+                                        void *workspace, size_t ws_bytes, void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_window(w, cc));
+    LQ_TRY(check_ptr(cc->idx, "idx"));
+    LQ_TRY(check_ptr(cc->slices, "slices"));
+    LQ_TRY(check_ptr(cc->rope, "rope"));
+    LQ_TRY(check_ptr(q, "q"));
+    LQ_TRY(check_ptr(out, "out"));
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(LOOPVQ_ERR_INVALID_ARG, "lse not 4-byte aligned");
+    if (layer < 0 || layer >= cc->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, cc->L);
+    if (t < 0 || t >= cc->T) return fail(LOOPVQ_ERR_INVALID_ARG, "t=%d out of [0, %d)", t, cc->T);
+    if (max_coded < 0 || max_coded > cc->Nmax)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "max_coded=%d out of [0, Nmax=%d]", max_coded, cc->Nmax);
+    if (!std::isfinite(scale)) return fail(LOOPVQ_ERR_INVALID_ARG, "scale is not finite");
+    if (scale <= 0.f) scale = 1.0f / std::sqrt((float)cc->D);
+    const size_t need = loopvq::window_ws_bytes(*w, *cc, max_coded);
+    if (!workspace || ws_bytes < need)
+        return fail(LOOPVQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? ws_bytes : (size_t)0);
+    if (!aligned16(workspace)) return fail(LOOPVQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    cudaError_t e = loopvq::launch_window_decode(*w, *cc, layer, t, q, max_coded, scale, out, lse, workspace,
+                                                 (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_window_decode_attn");
     return LOOPVQ_OK;
 }
 

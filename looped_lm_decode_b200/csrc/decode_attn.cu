@@ -70,8 +70,8 @@ static cudaError_t dispatch_qpk(int qpk, const DecodeArgs &a, const DecodePlan &
 }
 
 cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
-                          const uint16_t *q, const int32_t *starts, const int32_t *lens, int max_len, float scale,
-                          float *out, float *lse, void *workspace, cudaStream_t s) {
+                          const uint16_t *q, const int32_t *starts, int start_all, const int32_t *lens, int max_len,
+                          float scale, float *out, float *lse, void *workspace, cudaStream_t s) {
     DecodeArgs a{};
     const int beta = t / cc.Tc;
     a.idx = cc.idx + idx_base(cc, layer, beta, 0, 0);
@@ -81,6 +81,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     a.q = q;
     a.lens = lens;
     a.starts = starts;
+    a.start_all = start_all;
     const size_t o_bytes = (size_t)cc.B * cc.Hq * (size_t)plan.nsplit * cc.D * sizeof(float);
     a.ws_o = reinterpret_cast<float *>(workspace);
     a.ws_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(workspace) + ((o_bytes + 255) & ~(size_t)255));

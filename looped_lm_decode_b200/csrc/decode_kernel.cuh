@@ -50,12 +50,13 @@ struct DecodeArgs {
     const float *rope;       // [Nmax][D]
     const uint16_t *q;       // [B][Hq][D] bf16
     const int32_t *lens;     // [B]
-    const int32_t *starts;   // [B] first attended token, or null for 0
+    const int32_t *starts;   // [B] first attended token, or null for start_all
     float *ws_o;             // [B][Hq][nsplit][D]  unnormalised split outputs
     float2 *ws_ml;           // [B][Hq][nsplit]     (reference max, sum) in log2 units
     float *out;              // [B][Hq][D]
     float *lse;              // [B][Hq] or null
     int B, Hkv, Hq, K, Nmax, max_len, split_len, nsplit;
+    int start_all;           // first attended token of every sequence when starts is null
     float qscale;            // scale * log2(e)
 };
 
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     const int len = min(max(__ldg(a.lens + b), 0), a.max_len);
     // tokens [st, len) are attended; splits start from st rounded down to a 4-token tile, and the
     // tokens of that tile before st are masked
-    const int st = a.starts ? min(max(__ldg(a.starts + b), 0), len) : 0;
+    const int st = min(max(a.starts ? __ldg(a.starts + b) : a.start_all, 0), len);
     const int tok_begin = (st & ~3) + split * a.split_len;
     if (tok_begin >= len) return;                          // the merge never reads this split
     const int tok_end = min(tok_begin + a.split_len, len);
@@ -466,7 +467,7 @@ __global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
     const int b = bh / a.Hq;
     const int d = threadIdx.x;
     const int len = min(max(a.lens[b], 0), a.max_len);
-    const int st = a.starts ? min(max(a.starts[b], 0), len) : 0;
+    const int st = min(max(a.starts ? a.starts[b] : a.start_all, 0), len);
     const int span = len - (st & ~3);                      // tokens covered by the splits
     const int ns = len > st ? (span + a.split_len - 1) / a.split_len : 0;
     const float2 *ml = a.ws_ml + (size_t)bh * a.nsplit;

@@ -12,7 +12,7 @@
 // the K and V codes of a channel group and of its RoPE partner group.
 #include <math_constants.h>
 
-#include "loopvq_internal.cuh"
+#include "encode_common.cuh"
 
 namespace loopvq {
 
@@ -40,12 +40,7 @@ __global__ void __launch_bounds__(128) encode_direct_kernel(const EncodeArgs a) 
     const int brel = blockIdx.z;
     const int b = a.b0 + brel;
     const int K = a.K;
-
-    for (int e = threadIdx.x; e < 2 * K * G; e += blockDim.x) {
-        const int kv = e / (K * G);
-        const int rem = e % (K * G);
-        ecb[e] = bf16_to_f32(a.cb[((size_t)kv * a.Hkv + h) * (size_t)K * G + rem]);
-    }
+    stage_codebooks<G>(ecb, a.cb, a.Hkv, h, K);
     __syncthreads();
 
     const int wl = blockIdx.x * blockDim.x + threadIdx.x;  // word within this (b, h) request
@@ -69,28 +64,7 @@ __global__ void __launch_bounds__(128) encode_direct_kernel(const EncodeArgs a) 
             z[2][i * TC + m] = ld_x(xv + off + p * C + i);
             z[3][i * TC + m] = ld_x(xv + off + (p + NP) * C + i);
         }
-
-    float best[4] = {CUDART_INF_F, CUDART_INF_F, CUDART_INF_F, CUDART_INF_F};
-    int bi[4] = {0, 0, 0, 0};
-    const float *ek = ecb;
-    const float *ev = ecb + (size_t)K * G;
-    for (int r = 0; r < K; ++r) {
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < G; ++k) {
-            const float e0 = ek[r * G + k];
-            const float e1 = ev[r * G + k];
-            float t;
-            t = __fsub_rn(z[0][k], e0); d[0] = __fadd_rn(d[0], __fmul_rn(t, t));
-            t = __fsub_rn(z[1][k], e0); d[1] = __fadd_rn(d[1], __fmul_rn(t, t));
-            t = __fsub_rn(z[2][k], e1); d[2] = __fadd_rn(d[2], __fmul_rn(t, t));
-            t = __fsub_rn(z[3][k], e1); d[3] = __fadd_rn(d[3], __fmul_rn(t, t));
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (d[u] < best[u]) { best[u] = d[u]; bi[u] = r; }
-    }
-    const uint32_t word = (uint32_t)bi[0] | ((uint32_t)bi[1] << 8) | ((uint32_t)bi[2] << 16) | ((uint32_t)bi[3] << 24);
+    const uint32_t word = nearest_word<G>(z, ecb, ecb + (size_t)K * G, K);
     a.idx[((size_t)b * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C) + idx_word(n, p, NP)] = word;
 }
 

@@ -57,13 +57,20 @@ struct DecodePlan {
 };
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len);
 cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
-                          const uint16_t *q, const int32_t *starts, const int32_t *lens, int max_len, float scale,
-                          float *out, float *lse, void *workspace, cudaStream_t s);
+                          const uint16_t *q, const int32_t *starts, int start_all, const int32_t *lens, int max_len,
+                          float scale, float *out, float *lse, void *workspace, cudaStream_t s);
 DecodePlan plan_bf16(const loopvq_bf16_cache &c, int max_len);
 cudaError_t launch_bf16_decode(const loopvq_bf16_cache &c, const DecodePlan &plan, const uint16_t *q,
                                const int32_t *starts, const int32_t *lens, int max_len, float scale, float *out,
                                float *lse, void *workspace, cudaStream_t s);
 cudaError_t launch_merge2(const float *out_a, const float *lse_a, const float *out_b, const float *lse_b, int rows,
                           int D, float *out, float *lse, cudaStream_t s);
+int window_slots(const loopvq_window &w);
+cudaError_t launch_window_advance(const loopvq_window &w, const loopvq_cache &cc, cudaStream_t s);
+cudaError_t launch_window_append(const loopvq_window &w, int layer, int t, const uint16_t *k_rot,
+                                 const uint16_t *k_pre, const uint16_t *v, cudaStream_t s);
+size_t window_ws_bytes(const loopvq_window &w, const loopvq_cache &cc, int max_coded);
+cudaError_t launch_window_decode(const loopvq_window &w, const loopvq_cache &cc, int layer, int t, const uint16_t *q,
+                                 int max_coded, float scale, float *out, float *lse, void *ws, cudaStream_t s);
 
 }  // namespace loopvq

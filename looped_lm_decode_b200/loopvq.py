@@ -22,7 +22,9 @@ EXPORTS = ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "l
            "loopvq_prepare", "loopvq_encode", "loopvq_decode_workspace_bytes", "loopvq_decode_attn",
            "loopvq_dequant_debug", "loopvq_last_error", "loopvq_abi_version",
            "loopvq_decode_attn_noalloc", "loopvq_noalloc_scratch_bytes", "loopvq_decode_attn_range",
-           "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn", "loopvq_merge2")
+           "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn", "loopvq_merge2",
+           "loopvq_window_slots", "loopvq_window_advance", "loopvq_window_append",
+           "loopvq_window_workspace_bytes", "loopvq_window_decode_attn")
 
 
 class CacheDesc(C.Structure):
@@ -37,6 +39,13 @@ class Bf16CacheDesc(C.Structure):
     """Mirror of struct loopvq_bf16_cache."""
     _fields_ = [("B", C.c_int32), ("Hkv", C.c_int32), ("Hq", C.c_int32), ("D", C.c_int32), ("Nmax", C.c_int32),
                 ("k", C.c_void_p), ("v", C.c_void_p)]
+
+
+class WindowDesc(C.Structure):
+    """Mirror of struct loopvq_window."""
+    _fields_ = [("L", C.c_int32), ("T", C.c_int32), ("B", C.c_int32), ("Hkv", C.c_int32), ("Hq", C.c_int32),
+                ("D", C.c_int32), ("n_sink", C.c_int32), ("n_recent", C.c_int32), ("k_rot", C.c_void_p),
+                ("k_pre", C.c_void_p), ("v", C.c_void_p), ("fill", C.c_void_p), ("coded_end", C.c_void_p)]
 
 
 class LoopVQError(RuntimeError):
@@ -77,6 +86,17 @@ def lib():
         L.loopvq_bf16_decode_attn.restype = i
         L.loopvq_merge2.argtypes = [vp, vp, vp, vp, i, i, vp, vp, vp]
         L.loopvq_merge2.restype = i
+        PW = C.POINTER(WindowDesc)
+        L.loopvq_window_slots.argtypes = [PW]
+        L.loopvq_window_slots.restype = i
+        L.loopvq_window_advance.argtypes = [PW, P, vp]
+        L.loopvq_window_advance.restype = i
+        L.loopvq_window_append.argtypes = [PW, i, i, vp, vp, vp, vp]
+        L.loopvq_window_append.restype = i
+        L.loopvq_window_workspace_bytes.argtypes = [PW, P, i]
+        L.loopvq_window_workspace_bytes.restype = sz
+        L.loopvq_window_decode_attn.argtypes = [PW, P, i, i, vp, i, f, vp, vp, vp, sz, vp]
+        L.loopvq_window_decode_attn.restype = i
         L.loopvq_noalloc_scratch_bytes.argtypes = []
         L.loopvq_noalloc_scratch_bytes.restype = sz
         for name in ("loopvq_prepare", "loopvq_encode", "loopvq_decode_attn", "loopvq_dequant_debug"):
@@ -257,6 +277,59 @@ def merge2(out_a, lse_a, out_b, lse_b, out=None, lse=None, stream=None):
         lse = torch.empty_like(lse_a)
     _check(lib().loopvq_merge2(_ptr(out_a), _ptr(lse_a), _ptr(out_b), _ptr(lse_b), rows, D, _ptr(out), _ptr(lse),
                                _stream(stream)))
+    return out, lse
+
+
+class Window:
+    """bf16 window of a coded cache (see include/loopvq.h): k_rot, k_pre, v bf16 [L][T][B][Hkv][W][D],
+    fill and coded_end int32 [B] (coded_end starts at n_sink, fill at 0)."""
+
+    def __init__(self, cache: Cache, n_sink: int = 8, n_recent: int = 64, device="cuda"):
+        self.L, self.T, self.B, self.Hkv, self.Hq, self.D = cache.L, cache.T, cache.B, cache.Hkv, cache.Hq, cache.D
+        self.n_sink, self.n_recent = n_sink, n_recent
+        self.W = n_sink + n_recent + 8
+        shape = (self.L, self.T, self.B, self.Hkv, self.W, self.D)
+        self.k_rot = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.k_pre = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.v = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.fill = torch.zeros(self.B, dtype=torch.int32, device=device)
+        self.coded_end = torch.full((self.B,), n_sink, dtype=torch.int32, device=device)
+        self.desc = WindowDesc(self.L, self.T, self.B, self.Hkv, self.Hq, self.D, n_sink, n_recent)
+
+    def ref(self):
+        d = self.desc
+        d.k_rot, d.k_pre, d.v = self.k_rot.data_ptr(), self.k_pre.data_ptr(), self.v.data_ptr()
+        d.fill, d.coded_end = self.fill.data_ptr(), self.coded_end.data_ptr()
+        return C.byref(d)
+
+
+def window_advance(win: Window, cache: Cache, stream=None):
+    _check(lib().loopvq_window_advance(win.ref(), cache.ref(), _stream(stream)))
+
+
+def window_append(win: Window, layer: int, t: int, k_rot, k_pre, v, stream=None):
+    """k_rot, k_pre, v: bf16 [B][Hkv][D] of the current token at (layer, loop step t)."""
+    _check(lib().loopvq_window_append(win.ref(), layer, t, _ptr(k_rot), _ptr(k_pre), _ptr(v), _stream(stream)))
+
+
+def window_workspace_bytes(win: Window, cache: Cache, max_coded: int) -> int:
+    return lib().loopvq_window_workspace_bytes(win.ref(), cache.ref(), max_coded)
+
+
+def window_decode_attn(win: Window, cache: Cache, layer: int, t: int, q, max_coded: int, scale: float = 0.0,
+                       out=None, lse=None, workspace=None, stream=None):
+    B, Hq, D = cache.B, cache.Hq, cache.D
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(window_workspace_bytes(win, cache, max_coded), 16), dtype=torch.uint8,
+                                device=dev)
+    _check(lib().loopvq_window_decode_attn(win.ref(), cache.ref(), layer, t, _ptr(q), max_coded, scale, _ptr(out),
+                                           _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                           _stream(stream)))
     return out, lse
 
 

@@ -150,3 +150,31 @@ def test_range_and_merge_validation_before_launch():
     assert lib.loopvq_merge2(fake, None, fake, fake, 4, 128, fake, fake, None) == 1
     assert lib.loopvq_merge2(fake, fake, fake, fake, 4, 128, C.c_void_p(0x20002), fake, None) == 1
     assert lib.loopvq_merge2(None, None, None, None, 0, 128, None, None, None) == 0
+
+
+def test_window_validation_before_launch():
+    lib = LQ.lib()
+    c = _cache()
+    c.desc.idx = c.desc.slices = c.desc.rope = c.desc.codebook = 0x10000
+    c.ref = lambda: C.byref(c.desc)
+    fake = C.c_void_p(0x20000)
+    w = LQ.WindowDesc(c.L, c.T, c.B, c.Hkv, c.Hq, c.D, 8, 64, 0x40000, 0x50000, 0x60000, 0x70000, 0x70100)
+    assert lib.loopvq_window_slots(C.byref(w)) == 80
+    need = lib.loopvq_window_workspace_bytes(C.byref(w), c.ref(), 1024)
+    assert need > 0
+    assert lib.loopvq_window_decode_attn(C.byref(w), c.ref(), 0, 0, fake, 1024, 0.0, fake, None, fake, need - 1,
+                                         None) == 3
+    assert lib.loopvq_window_decode_attn(C.byref(w), c.ref(), 0, 0, fake, 1025, 0.0, fake, None, fake, need,
+                                         None) == 1
+    assert lib.loopvq_window_append(C.byref(w), 2, 0, fake, fake, fake, None) == 1
+    assert lib.loopvq_window_append(C.byref(w), 0, 0, fake, C.c_void_p(0x20008), fake, None) == 1
+    w.n_recent = 60                                          # not a multiple of 8
+    assert lib.loopvq_window_slots(C.byref(w)) == 0
+    assert lib.loopvq_window_advance(C.byref(w), c.ref(), None) == 1
+    assert b"multiples of 8" in lib.loopvq_last_error()
+    w.n_recent, w.Hq = 64, 8                                 # shape differs from the cache's
+    assert lib.loopvq_window_advance(C.byref(w), c.ref(), None) == 1
+    assert b"differs" in lib.loopvq_last_error()
+    w.Hq, w.fill = c.Hq, None
+    assert lib.loopvq_window_advance(C.byref(w), c.ref(), None) == 1
+    assert lib.loopvq_window_workspace_bytes(C.byref(w), c.ref(), 1024) == 0

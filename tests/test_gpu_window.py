@@ -190,3 +190,109 @@ def test_merge2_is_attention_over_the_union():
     ok, msg = attn_tolerance_ok(out.cpu().numpy(), np.array(ref), lse.cpu().numpy(), np.array(lref), rel=1e-5,
                                 lse_tol=1e-5)
     assert ok, msg
+
+
+# ---------------------------------------------------------------- decode-time window life cycle
+
+from synth import f32_to_bf16_bits                                    # noqa: E402
+from tests.helpers import unpack_words                                 # noqa: E402
+
+LIFE = {
+    "c4tc4": WORKLOADS["ctx4k"].replace(L=2, B=2, Hkv=2, Hq=2, Nmax=128),
+    "c8tc2gqa": WORKLOADS["gqa16k"].replace(L=1, T=4, Tc=2, c=8, B=2, Hkv=1, Hq=4, Nmax=128),
+}
+
+
+def _raw(w, n):
+    """Pre-RoPE keys and values bits [T][B][n][Hkv][D] and keys rotated at their positions (fp64 RoPE of
+    the checker, stored as bf16 like a serving cache)."""
+    k = np.stack([kv_loops(w, layer, 0, 0, w.T - 1, range(w.B), range(n), range(w.Hkv)) for layer in range(w.L)])
+    v = np.stack([kv_loops(w, layer, 1, 0, w.T - 1, range(w.B), range(n), range(w.Hkv)) for layer in range(w.L)])
+    kf = bf16_bits_to_f32(k).astype(np.float64)                      # [L][T][B][n][Hkv][D]
+    kr = np.empty_like(k)
+    for idx in np.ndindex(w.L, w.T, w.B):
+        for h in range(w.Hkv):
+            kr[idx + (slice(None), h)] = f32_to_bf16_bits(O.rope(kf[idx + (slice(None), h)], w.theta, 0)
+                                                          .astype(np.float32))
+    return k, kr, v                                                   # [L][T][B][n][Hkv][D] bits
+
+
+@pytest.mark.parametrize("name", list(LIFE))
+def test_window_life_cycle(name):
+    """Prefill, then decode steps that roll the window twice: every attention call equals one softmax
+    over the bf16 window tokens and the coded tokens, and every rolled page's codes equal the checker's
+    encode of the original pre-RoPE keys and values."""
+    w = LIFE[name]
+    n_s, n_r = 8, 16
+    P0, steps = 40, 20                                                # prefill length, decode steps
+    ntot = P0 + steps
+    kp, kr, vv = _raw(w, ntot)
+    cache = make_cache(w)
+    win = LQ.Window(cache, n_sink=n_s, n_recent=n_r)
+    # ---- prefill: tokens 8 .. 23 coded, 0 .. 7 sink, 24 .. 39 recent
+    coded0 = P0 - n_r
+    for layer in range(w.L):
+        for blk in range(w.NB):
+            sl = slice(blk * w.Tc, (blk + 1) * w.Tc)
+            xk = _dev_bits(kp[layer, sl, :, n_s:coded0])
+            xv = _dev_bits(vv[layer, sl, :, n_s:coded0])
+            LQ.encode(cache, layer, blk, xk, xv, tok0=n_s)
+    order = list(range(n_s)) + list(range(coded0, P0))                # tokens in window slots 0 .. fill-1
+    for dst, src in ((win.k_rot, kr), (win.k_pre, kp), (win.v, vv)):
+        # [L][T][B][n][Hkv][D] -> [L][T][B][Hkv][slot][D]
+        dst[:, :, :, :, :len(order)] = _dev_bits(np.ascontiguousarray(src[:, :, :, order].transpose(0, 1, 2, 4, 3, 5)))
+    win.fill.fill_(len(order))
+    win.coded_end.fill_(coded0)
+    torch.cuda.synchronize()
+
+    coded_end = coded0
+    checks = [(0, 1), (w.L - 1, w.T - 1)]
+    for step in range(steps):
+        n = P0 + step                                                  # the new token
+        if n_s + (n - coded_end) > n_s + n_r + 7:                      # window full: the oldest page is coded
+            coded_end += 8
+        LQ.window_advance(win, cache)
+        for layer in range(w.L):
+            for t in range(w.T):
+                LQ.window_append(win, layer, t, _dev_bits(kr[layer, t, :, n]), _dev_bits(kp[layer, t, :, n]),
+                                 _dev_bits(vv[layer, t, :, n]))
+        for layer, t in checks:
+            qb = queries(w, layer, t, gain=1.0 + 0.25 * step)
+            out, lse = LQ.window_decode_attn(win, cache, layer, t, _dev_bits(qb), w.Nmax)
+            torch.cuda.synchronize()
+            blk, m = t // w.Tc, t % w.Tc
+            qpk = w.Hq // w.Hkv
+            ref = np.zeros((w.B, w.Hq, w.D))
+            lref = np.zeros((w.B, w.Hq))
+            wtok = list(range(n_s)) + list(range(coded_end, n + 1))
+            sl = slice(blk * w.Tc, (blk + 1) * w.Tc)
+            for b in range(w.B):
+                for h in range(w.Hkv):
+                    E_k = np_codebook_f32(w, layer, blk, 0, h)
+                    E_v = np_codebook_f32(w, layer, blk, 1, h)
+                    ik = O.encode(bf16_bits_to_f32(kp[layer, sl, b, n_s:coded_end, h]), E_k, w.c)
+                    iv = O.encode(bf16_bits_to_f32(vv[layer, sl, b, n_s:coded_end, h]), E_v, w.c)
+                    for j in range(qpk):
+                        hq = h * qpk + j
+                        ref[b, hq], lref[b, hq] = O.decode_windowed(
+                            bf16_bits_to_f32(qb[b, hq]).astype(np.float64),
+                            bf16_bits_to_f32(kr[layer, t, b, wtok, h]), bf16_bits_to_f32(vv[layer, t, b, wtok, h]),
+                            ik, iv, E_k, E_v, w.c, w.Tc, m, n_s, w.theta, 1 / math.sqrt(w.D))
+            ok, msg = attn_tolerance_ok(out.cpu().numpy(), ref, lse.cpu().numpy(), lref)
+            assert ok, f"{name} step {step} (layer {layer}, t {t}): {msg}"
+    assert int(win.coded_end[0]) == coded_end and coded_end == coded0 + 16   # two rolls
+    assert int(win.fill[0]) == n_s + (ntot - 1 - coded_end) + 1
+    # ---- the rolled pages hold the checker's codes
+    for layer in range(w.L):
+        for blk in range(w.NB):
+            sl = slice(blk * w.Tc, (blk + 1) * w.Tc)
+            for b in range(w.B):
+                for h in range(w.Hkv):
+                    words = words_view(cache, layer, blk, b, h).cpu().numpy().view(np.uint32)
+                    ck, cv = unpack_words(words, w.Nmax, cache.NP)
+                    rk = O.encode(bf16_bits_to_f32(kp[layer, sl, b, n_s:coded_end, h]),
+                                  np_codebook_f32(w, layer, blk, 0, h), w.c)
+                    rv = O.encode(bf16_bits_to_f32(vv[layer, sl, b, n_s:coded_end, h]),
+                                  np_codebook_f32(w, layer, blk, 1, h), w.c)
+                    np.testing.assert_array_equal(ck[n_s:coded_end], rk)
+                    np.testing.assert_array_equal(cv[n_s:coded_end], rv)
