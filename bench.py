@@ -143,38 +143,63 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
     bf_bytes = int(lens_np.astype(np.int64).sum()) * w.Hkv * 2 * w.D * 2 + w.B * w.Hq * (w.D * 2 + w.D * 4 + 4)
     del caches
 
+    # ---- the serving layout through the window API: a full decode step is one advance (a page roll for
+    # full windows every 8 steps), then per (loop step, layer) an append and a windowed attention call
     n_sink, n_recent = 8, 64
-    W = n_sink + n_recent
-    tmp = torch.empty((1, w.B, W, w.Hkv, w.D), dtype=torch.bfloat16, device=dev)
-    win = []
-    for k in range(2):
-        SG.fill_kv(w.replace(Nmax=W), 0, k, 0, 0, tmp)
-        win.append(tmp[0].permute(0, 2, 1, 3).contiguous())
-    wcache = LQ.Bf16Cache(win[0], win[1], w.Hq)
-    lw = torch.from_numpy(np.minimum(lens_np, W).astype(np.int32)).to(dev)
-    lo_np = np.minimum(lens_np, n_sink).astype(np.int32)
-    hi_np = np.maximum(lens_np - n_recent, lo_np).astype(np.int32)
-    lo, hi = torch.from_numpy(lo_np).to(dev), torch.from_numpy(hi_np).to(dev)
-    ws_w = torch.empty(max(LQ.bf16_decode_workspace_bytes(wcache, W), 16), dtype=torch.uint8, device=dev)
+    win = LQ.Window(cache, n_sink=n_sink, n_recent=n_recent, device=dev)
+    tmp = torch.empty((1, w.B, win.W, w.Hkv, w.D), dtype=torch.bfloat16, device=dev)
+    for dst, k in ((win.k_rot, 0), (win.k_pre, 0), (win.v, 1)):
+        SG.fill_kv(w.replace(Nmax=win.W), 0, k, 0, 0, tmp)
+        dst.copy_(tmp[0].permute(0, 2, 1, 3).reshape(1, 1, w.B, w.Hkv, win.W, w.D).expand_as(dst))
+    del tmp
+    coded = np.maximum(n_sink + ((lens_np - n_sink - n_recent) // 8) * 8, n_sink).astype(np.int32)
+    win.coded_end.copy_(torch.from_numpy(coded))
+    win.fill.copy_(torch.from_numpy((n_sink + lens_np - coded).astype(np.int32)))
+    tok = [win.k_rot[0, 0, :, :, 0].contiguous(), win.k_pre[0, 0, :, :, 0].contiguous(), win.v[0, 0, :, :, 0].contiguous()]
+    ws_w = torch.empty(max(LQ.window_workspace_bytes(win, cache, w.Nmax), 16), dtype=torch.uint8, device=dev)
     out_c = torch.empty_like(out_b)
     lse_c = torch.empty_like(lse_b)
-    hmax = int(hi_np.max())
+    call_evs = []
 
-    def windowed(i):
-        t, layer = divmod(i, w.L)
-        LQ.bf16_decode_attn(wcache, qs[i], lw, W, out=out_b, lse=lse_b, workspace=ws_w, stream=stream)
-        LQ.decode_attn_range(cache, layer, t, qs[i], lo, hi, hmax, out=out_c, lse=lse_c, workspace=ws, stream=stream)
-        LQ.merge2(out_c, lse_c, out_b, lse_b, out=out_c, lse=lse_c, stream=stream)
+    def wstep(record):
+        LQ.window_advance(win, cache, stream=stream)
+        for t in range(w.T):
+            for layer in range(w.L):
+                i = t * w.L + layer
+                LQ.window_append(win, layer, t, tok[0], tok[1], tok[2], stream=stream)
+                if record:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                LQ.window_decode_attn(win, cache, layer, t, qs[i], w.Nmax, out=out_c, lse=lse_c, workspace=ws_w,
+                                      stream=stream)
+                if record:
+                    e1.record(stream)
+                    call_evs.append((e0, e1))
 
-    win_ms = timed(windowed, w.T * w.L)
+    wstep(False)
+    torch.cuda.synchronize()
+    nsteps = 16                                       # two page rolls for every sequence
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(nsteps):
+        wstep(True)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    win_step_ms = s0.elapsed_time(s1) / nsteps
+    win_call_ms = statistics.fmean(a.elapsed_time(b) for a, b in call_evs)
+    del win
+
     peak, kind = peaks()
     return {
         "bf16_cache": {"us_per_call": bf_ms * 1e3, "gbs": bf_bytes / (bf_ms * 1e-3) / 1e9,
                        "frac": bf_bytes / (bf_ms * 1e-3) / 1e9 / peak, "peak": peak, "peak_kind": kind,
                        "bytes_per_call": bf_bytes,
                        "kernel": "loopvq_bf16_decode_attn over a bf16 cache of the same shape (keys stored rotated)"},
-        "windowed": {"us_per_call": win_ms * 1e3, "sink": n_sink, "recent": n_recent,
-                     "calls": "loopvq_bf16_decode_attn (window) + loopvq_decode_attn_range (coded) + loopvq_merge2"},
+        "windowed": {"us_per_call": win_call_ms * 1e3, "us_per_step": win_step_ms * 1e3, "steps": nsteps,
+                     "sink": n_sink, "recent": n_recent,
+                     "calls": "per step: loopvq_window_advance (page roll every 8 steps), then per (loop step, "
+                              "layer) loopvq_window_append + loopvq_window_decode_attn (bf16 window kernel + coded "
+                              "range kernel + merge2)"},
     }
 
 
