@@ -27,6 +27,10 @@
  *              through the log-sum-exp of each split (Flash-Decoding merge),
  *              which the pages state recovers the exact softmax.
  *              LoopVQ paper, Sec. 4.3 "Attention".
+ *   *_pg       the same with one codebook per channel group, E_g for group g
+ *              (the paper's notation B_{beta,l,h,g}): encode, the distance
+ *              check, reconstruction and decode.
+ *              LoopVQ paper, Sec. 2 eq. (2); Sec. 4.1 eq. (5); App. A.2.
  *   windowed   attention of one query over a cache whose sink and recent
  *              tokens are kept in bf16 (keys stored already rotated) and whose
  *              other tokens lo <= n < hi are coded: the coded keys are rebuilt
@@ -220,6 +224,69 @@ void ora_decode_windowed(const double *q, const double *kw, const double *vw, in
     ora_dequant(idx_k, NC, D, c, Tc, m, E_k, kc);
     ora_rope(kc, NC, D, theta, lo);
     ora_dequant(idx_v, NC, D, c, Tc, m, E_v, vc);
+    ora_attention(q, kh, vh, N, D, scale, out, lse);
+    free(kh);
+    free(vh);
+}
+
+/* ---- one codebook per channel group: E holds ng = D/c codebooks [ng][K][G], group g uses E_g ---- */
+
+/* Nearest entry of every coupled vector in its own group's codebook; fp32, lowest index on ties. */
+void ora_encode_pg(const float *x, int Tc, int N, int D, int c, const float *E, int K, uint8_t *idx)
+{
+    const int G = c * Tc;
+    const int ng = D / c;
+    float z[256];
+    for (int n = 0; n < N; ++n) {
+        for (int g = 0; g < ng; ++g) {
+            const float *Eg = E + (size_t)g * K * G;
+            coupled_vector(x, Tc, N, D, c, n, g, z);
+            int best = 0;
+            float best_d = INFINITY;
+            for (int r = 0; r < K; ++r) {
+                float d = 0.0f;
+                for (int k = 0; k < G; ++k) {
+                    float diff = z[k] - Eg[(size_t)r * G + k];
+                    float sq = diff * diff;
+                    d = d + sq;
+                }
+                if (d < best_d) { best_d = d; best = r; }
+            }
+            idx[(size_t)n * ng + g] = (uint8_t)best;
+        }
+    }
+}
+
+double ora_dist64_pg(const float *x, int Tc, int N, int D, int c, const float *E, int K, int n, int g, int r)
+{
+    return ora_dist64(x, Tc, N, D, c, E + (size_t)g * K * c * Tc, n, g, r);
+}
+
+/* Reconstruction of loop step m with per-group codebooks: out[n][g*c + i] = E_g[idx[n][g]][i*Tc + m]. */
+void ora_dequant_pg(const uint8_t *idx, int N, int D, int c, int Tc, int m, const float *E, int K, double *out)
+{
+    const int G = c * Tc;
+    const int ng = D / c;
+    for (int n = 0; n < N; ++n)
+        for (int g = 0; g < ng; ++g) {
+            const float *Eg = E + (size_t)g * K * G;
+            int r = idx[(size_t)n * ng + g];
+            for (int i = 0; i < c; ++i)
+                out[(size_t)n * D + (size_t)g * c + i] = (double)Eg[(size_t)r * G + i * Tc + m];
+        }
+}
+
+/* Decode attention as ora_decode, with per-group codebooks for keys and values. */
+void ora_decode_pg(const double *q, const uint8_t *idx_k, const uint8_t *idx_v, const float *E_k,
+                   const float *E_v, int K, int N, int D, int c, int Tc, int m, double theta, double scale,
+                   double *out, double *lse)
+{
+    size_t nd = (size_t)(N > 0 ? N : 1) * (size_t)D;
+    double *kh = (double *)malloc(sizeof(double) * nd);
+    double *vh = (double *)malloc(sizeof(double) * nd);
+    ora_dequant_pg(idx_k, N, D, c, Tc, m, E_k, K, kh);
+    ora_rope(kh, N, D, theta, 0);
+    ora_dequant_pg(idx_v, N, D, c, Tc, m, E_v, K, vh);
     ora_attention(q, kh, vh, N, D, scale, out, lse);
     free(kh);
     free(vh);

@@ -42,6 +42,14 @@ def lib():
         _lib.ora_decode_windowed.argtypes = [f64p, f64p, f64p, I, u8p, u8p, f32p, f32p, I, I, I, I, I, I, D_, D_,
                                              f64p, C.POINTER(D_)]
         _lib.ora_decode_windowed.restype = None
+        _lib.ora_encode_pg.argtypes = [f32p, I, I, I, I, f32p, I, u8p]
+        _lib.ora_encode_pg.restype = None
+        _lib.ora_dist64_pg.argtypes = [f32p, I, I, I, I, f32p, I, I, I, I]
+        _lib.ora_dist64_pg.restype = D_
+        _lib.ora_dequant_pg.argtypes = [u8p, I, I, I, I, I, f32p, I, f64p]
+        _lib.ora_dequant_pg.restype = None
+        _lib.ora_decode_pg.argtypes = [f64p, u8p, u8p, f32p, f32p, I, I, I, I, I, I, D_, D_, f64p, C.POINTER(D_)]
+        _lib.ora_decode_pg.restype = None
     return _lib
 
 
@@ -149,4 +157,54 @@ def decode_windowed(q, k_win, v_win, idx_k, idx_v, E_k, E_v, c: int, Tc: int, m:
     z8 = np.zeros((1, D // c), np.uint8)
     lib().ora_decode_windowed(q, kw if NW else z64, vw if NW else z64, NW, idx_k if NC else z8, idx_v if NC else z8,
                               _f32(E_k), _f32(E_v), lo, lo + NC, D, c, Tc, m, theta, scale, out, C.byref(lse))
+    return out, lse.value
+
+
+# ---- one codebook per channel group: E is [D/c][K][G]
+
+def encode_pg(x, E, c: int) -> np.ndarray:
+    x = _f32(x)
+    Tc, N, D = x.shape
+    E = _f32(E)
+    ng, K, G = E.shape
+    assert ng == D // c and G == c * Tc
+    idx = np.zeros((N, ng), dtype=np.uint8)
+    if N:
+        lib().ora_encode_pg(x, Tc, N, D, c, E, K, idx)
+    return idx
+
+
+def dist64_pg(x, E, c: int, n: int, g: int, r: int) -> float:
+    x = _f32(x)
+    Tc, N, D = x.shape
+    E = _f32(E)
+    return lib().ora_dist64_pg(x, Tc, N, D, c, E, E.shape[1], n, g, r)
+
+
+def dequant_pg(idx, E, c: int, Tc: int, m: int) -> np.ndarray:
+    idx = np.ascontiguousarray(idx, dtype=np.uint8)
+    E = _f32(E)
+    N = idx.shape[0]
+    D = idx.shape[1] * c
+    out = np.zeros((N, D), dtype=np.float64)
+    if N:
+        lib().ora_dequant_pg(idx, N, D, c, Tc, m, E, E.shape[1], out)
+    return out
+
+
+def decode_pg(q, idx_k, idx_v, E_k, E_v, c: int, Tc: int, m: int, theta: float = 1.0e4, scale: float = None):
+    """decode() with per-group codebooks E_k, E_v: [D/c][K][G]."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    D = q.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    idx_k = np.ascontiguousarray(idx_k, dtype=np.uint8).reshape(-1, D // c)
+    idx_v = np.ascontiguousarray(idx_v, dtype=np.uint8).reshape(-1, D // c)
+    N = idx_k.shape[0]
+    E_k, E_v = _f32(E_k), _f32(E_v)
+    out = np.zeros(D, dtype=np.float64)
+    lse = C.c_double(0.0)
+    z8 = np.zeros((1, D // c), np.uint8)
+    lib().ora_decode_pg(q, idx_k if N else z8, idx_v if N else z8, E_k, E_v, E_k.shape[1], N, D, c, Tc, m, theta,
+                        scale, out, C.byref(lse))
     return out, lse.value

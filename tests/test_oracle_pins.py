@@ -358,3 +358,68 @@ def test_windowed_special_cases():
     np.testing.assert_allclose(out, ro, rtol=1e-11, atol=1e-12)
     out, lse = O.decode_windowed(q, z, z, ik[:0], iv[:0], E_k, E_v, c, Tc, m, lo, 1e4, 0.3)
     assert lse == -math.inf and (out == 0).all()
+
+
+# ---------------------------------------------------------------- one codebook per channel group
+
+def test_pergroup_with_equal_codebooks_is_the_shared_case():
+    """Every group given the same codebook: per-group encode, reconstruction and decode equal the
+    shared-codebook ones (which are pinned above)."""
+    D, c, Tc, N = 64, 4, 4, 20
+    x = _rand_bf16((Tc, N, D))
+    E = _rand_bf16((256, c * Tc))
+    Eg = np.broadcast_to(E, (D // c, 256, c * Tc)).copy()
+    ik = O.encode_pg(x, Eg, c)
+    np.testing.assert_array_equal(ik, O.encode(x, E, c))
+    np.testing.assert_array_equal(O.dequant_pg(ik, Eg, c, Tc, 2), O.dequant(ik, E, c, Tc, 2))
+    q = RNG.standard_normal(D)
+    o1, l1 = O.decode_pg(q, ik, ik[::-1].copy(), Eg, Eg, c, Tc, 1, 1e4, 0.2)
+    o2, l2 = O.decode(q, ik, ik[::-1].copy(), E, E, c, Tc, 1, 1e4, 0.2)
+    np.testing.assert_array_equal(o1, o2)
+    assert l1 == l2
+
+
+def test_pergroup_encode_is_brute_force_per_group():
+    """Each group's index is the fp64 nearest entry of that group's own codebook."""
+    D, c, Tc, N, K = 32, 8, 2, 6, 40
+    x = _rand_bf16((Tc, N, D))
+    Eg = _rand_bf16((D // c, K, c * Tc))
+    idx = O.encode_pg(x, Eg, c)
+    for n in range(N):
+        for g in range(D // c):
+            z = np.array([x[m, n, g * c + i] for i in range(c) for m in range(Tc)], np.float64)
+            d = ((Eg[g].astype(np.float64) - z) ** 2).sum(1)
+            assert idx[n, g] == int(np.argmin(d)), (n, g)
+            assert abs(O.dist64_pg(x, Eg, c, n, g, int(idx[n, g])) - d.min()) < 1e-9
+
+
+def test_pergroup_reconstruction_uses_only_its_group():
+    """Changing group g's codebook changes exactly channels g*c .. g*c+c-1 of the reconstruction."""
+    D, c, Tc, N = 64, 4, 4, 8
+    Eg = _rand_bf16((D // c, 256, c * Tc))
+    idx = RNG.integers(0, 256, (N, D // c)).astype(np.uint8)
+    base = O.dequant_pg(idx, Eg, c, Tc, 3)
+    E2 = Eg.copy()
+    E2[5] += 1.0
+    diff = np.abs(O.dequant_pg(idx, E2, c, Tc, 3) - base) > 0
+    assert diff[:, 5 * c:6 * c].all() and not diff[:, :5 * c].any() and not diff[:, 6 * c:].any()
+
+
+def test_pergroup_lossless_decode_is_textbook_rope_attention():
+    """Each group's codebook holds that group's own coupled vectors: reconstruction is exact, so decode
+    equals plain RoPE attention on the original keys and values (numpy complex RoPE)."""
+    D, c, Tc, N, m = 64, 4, 4, 24, 2
+    xk, xv = _rand_bf16((Tc, N, D)), _rand_bf16((Tc, N, D))
+
+    def own(x):                                           # [D/c][K=N][G]: group g's vectors of all tokens
+        return np.ascontiguousarray(x.reshape(Tc, N, D // c, c).transpose(2, 1, 3, 0).reshape(D // c, N, c * Tc))
+
+    Ek, Ev = own(xk), own(xv)
+    ik, iv = O.encode_pg(xk, Ek, c), O.encode_pg(xv, Ev, c)
+    np.testing.assert_array_equal(ik, np.tile(np.arange(N)[:, None], (1, D // c)))
+    q = RNG.standard_normal(D)
+    out, lse = O.decode_pg(q, ik, iv, Ek, Ev, c, Tc, m, 1e4, 0.15)
+    ro, rl = _softmax_attention_np(q, _rope_complex(xk[m].astype(np.float64), np.arange(N)),
+                                   xv[m].astype(np.float64), 0.15)
+    np.testing.assert_allclose(out, ro, rtol=1e-11, atol=1e-12)
+    assert abs(lse - rl) < 1e-11
