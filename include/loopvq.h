@@ -60,12 +60,14 @@ enum { LOOPVQ_BF16 = 0, LOOPVQ_FP32 = 1 };
  *           g covers channels g*c .. g*c+c-1.  One word serves all Tc loop
  *           steps of its block (Sec. 4.3 "Cache layout": one index row per
  *           block).  2*D/c bytes per token, head and block.
- * codebook  bf16 [L][NB][2][Hkv][K][G], 2 = {K, V}; coordinate i*Tc + m of an
- *           entry belongs to channel i at loop step m of the block (eq. 4).
- *           One codebook per (layer, block, KV head, K|V), shared by all
- *           channel groups.
- * slices    bf16 [L][T][2][Hkv][K][c]: loop step t = beta*Tc + m keeps
- *           coordinates i*Tc + m, i < c, of every entry (Sec. 4.3 "Attention":
+ * codebook  bf16 [L][NB][2][Hkv][NCB][K][G], 2 = {K, V}; coordinate i*Tc + m
+ *           of an entry belongs to channel i at loop step m of the block
+ *           (eq. 4).  NCB = 1: one codebook per (layer, block, KV head, K|V),
+ *           shared by all channel groups; NCB = D/c: one per channel group g
+ *           (the paper's notation, eq. 5), set by the field ncb.
+ * slices    bf16 [L][T][2][Hkv][K][NCB*c]: loop step t = beta*Tc + m keeps
+ *           coordinates i*Tc + m, i < c, of every entry, code-major (row r
+ *           holds entry r of every group's codebook) (Sec. 4.3 "Attention":
  *           the slice B_t, cut once when the model is loaded).  Written by
  *           loopvq_prepare.
  * rope      fp32 [Nmax][D]: row p holds cos(p*w_f) in [0, D/2) and sin(p*w_f)
@@ -80,6 +82,7 @@ typedef struct loopvq_cache {
     const uint16_t *codebook;
     uint16_t *slices;
     float *rope;
+    int32_t ncb;                 /* codebooks per (layer, block, KV head, K|V): 0 or 1 = shared, D/c = per group */
 } loopvq_cache;
 
 /* Element counts of the four buffers (0 if the shape is invalid). */

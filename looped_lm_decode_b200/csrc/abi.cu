@@ -46,6 +46,8 @@ loopvq_status check_shape(const loopvq_cache *cc) {
     if (qpk != 1 && qpk != 2 && qpk != 4 && qpk != 8)
         return fail(LOOPVQ_ERR_UNSUPPORTED, "Hq/Hkv=%d (supported: 1, 2, 4, 8)", qpk);
     if (!(cc->theta > 0.f) || !std::isfinite(cc->theta)) return fail(LOOPVQ_ERR_INVALID_ARG, "theta must be positive");
+    if (cc->ncb != 0 && cc->ncb != 1 && cc->ncb != cc->D / cc->c)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "ncb=%d (1 shared, or D/c=%d per channel group)", cc->ncb, cc->D / cc->c);
     return LOOPVQ_OK;
 }
 
@@ -76,12 +78,12 @@ size_t loopvq_idx_words(const loopvq_cache *cc) {
 
 size_t loopvq_codebook_elems(const loopvq_cache *cc) {
     if (check_shape(cc) != LOOPVQ_OK) return 0;
-    return (size_t)cc->L * (cc->T / cc->Tc) * 2 * cc->Hkv * (size_t)cc->K * cc->c * cc->Tc;
+    return (size_t)cc->L * (cc->T / cc->Tc) * 2 * cc->Hkv * (size_t)cc->K * cc->c * cc->Tc * loopvq::ncb_of(*cc);
 }
 
 size_t loopvq_slice_elems(const loopvq_cache *cc) {
     if (check_shape(cc) != LOOPVQ_OK) return 0;
-    return (size_t)cc->L * cc->T * 2 * cc->Hkv * (size_t)cc->K * cc->c;
+    return (size_t)cc->L * cc->T * 2 * cc->Hkv * (size_t)cc->K * cc->c * loopvq::ncb_of(*cc);
 }
 
 size_t loopvq_rope_elems(const loopvq_cache *cc) {
@@ -243,6 +245,8 @@ loopvq_status loopvq_merge2(const float *out_a, const float *lse_a, const float 
 static loopvq_status check_window(const loopvq_window *w, const loopvq_cache *cc) {
     if (!w) return fail(LOOPVQ_ERR_INVALID_ARG, "window is NULL");
     LQ_TRY(check_shape(cc));
+    if (loopvq::ncb_of(*cc) != 1)
+        return fail(LOOPVQ_ERR_UNSUPPORTED, "the window's page encoder supports shared codebooks (ncb = 1) only");
     if (w->L != cc->L || w->T != cc->T || w->B != cc->B || w->Hkv != cc->Hkv || w->Hq != cc->Hq || w->D != cc->D)
         return fail(LOOPVQ_ERR_INVALID_ARG, "window shape (L, T, B, Hkv, Hq, D) differs from the cache's");
     if (w->n_sink <= 0 || w->n_recent <= 0 || w->n_sink % 8 != 0 || w->n_recent % 8 != 0)
@@ -348,6 +352,6 @@ loopvq_status loopvq_dequant_debug(const loopvq_cache *cc, int layer, int t, int
 
 const char *loopvq_last_error(void) { return g_err; }
 
-int loopvq_abi_version(void) { return 1; }
+int loopvq_abi_version(void) { return 2; }
 
 }  // extern "C"

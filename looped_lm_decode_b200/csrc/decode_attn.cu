@@ -18,16 +18,25 @@ static constexpr int kMinBlocks = 2;
 static constexpr int kDepth = 4;
 static constexpr int kWords = 1;                          // index words per lane per iteration (4-token tiles)
 static constexpr long kTargetCtas = 148L * 2 * 4;
+// one codebook per channel group: 128 KiB of tables, so one CTA of 16 warps per SM
+static constexpr int kPgWarps = 16;
+static constexpr int kPgMinBlocks = 1;
+static constexpr long kPgTargetCtas = 148L * 1 * 4;
 
-static size_t ring_smem_bytes() { return 65536 + (size_t)kDepth * kWarps * 32 * 16 * kWords; }
+static size_t ring_smem_bytes(bool pg) {
+    return (pg ? 131072 : 65536) + (size_t)kDepth * (pg ? kPgWarps : kWarps) * 32 * 16 * kWords;
+}
 
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len) {
     DecodePlan p{};
-    const int stride = 4 * kWords * kWarps * (32 / (cc.D / 8));   // tokens between two iterations of a slot
+    const bool pg = ncb_of(cc) > 1;
+    const int warps = pg ? kPgWarps : kWarps;
+    const long target = pg ? kPgTargetCtas : kTargetCtas;
+    const int stride = 4 * kWords * warps * (32 / (cc.D / 8));   // tokens between two iterations of a slot
     p.nbt = 1;
     p.nchunk = cc.B;
     const long units = (long)cc.Hkv * cc.B;
-    long sl = max_len > 0 ? ((long)max_len * units + kTargetCtas - 1) / kTargetCtas : stride;
+    long sl = max_len > 0 ? ((long)max_len * units + target - 1) / target : stride;
     sl = ((sl + stride - 1) / stride) * stride;
     if (sl < stride) sl = stride;
     if (sl > 8192) sl = 8192;
@@ -39,18 +48,19 @@ DecodePlan plan_decode(const loopvq_cache &cc, int max_len) {
     return p;
 }
 
-template <int D, int C, int QPK>
+template <int D, int C, int QPK, bool PG>
 static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
-    constexpr int NSLOT = kWarps * (32 / (D / 8));
+    constexpr int W = PG ? kPgWarps : kWarps;
+    constexpr int NSLOT = W * (32 / (D / 8));
     const size_t red = (size_t)NSLOT * QPK * (D + 4) * sizeof(float);
-    const size_t smem = ring_smem_bytes();
+    const size_t smem = ring_smem_bytes(PG);
     if (red > smem) return cudaErrorInvalidConfiguration;   // the slot records reuse slices and queue
-    auto kern = decode_split_kernel<D, C, QPK, kWarps, kMinBlocks, kDepth, kWords>;
+    auto kern = decode_split_kernel<D, C, QPK, W, PG ? kPgMinBlocks : kMinBlocks, kDepth, kWords, PG>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (plan.nsplit > 0) {
         dim3 grid(plan.nsplit, a.Hkv, a.B);
-        kern<<<grid, kWarps * 32, smem, s>>>(a);
+        kern<<<grid, W * 32, smem, s>>>(a);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -58,13 +68,24 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStr
     return cudaGetLastError();
 }
 
-template <int D, int C>
+template <int D, int C, bool PG>
 static cudaError_t dispatch_qpk(int qpk, const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
     switch (qpk) {
-        case 1: return launch_t<D, C, 1>(a, plan, s);
-        case 2: return launch_t<D, C, 2>(a, plan, s);
-        case 4: return launch_t<D, C, 4>(a, plan, s);
-        case 8: return launch_t<D, C, 8>(a, plan, s);
+        case 1: return launch_t<D, C, 1, PG>(a, plan, s);
+        case 2: return launch_t<D, C, 2, PG>(a, plan, s);
+        case 4: return launch_t<D, C, 4, PG>(a, plan, s);
+        case 8: return launch_t<D, C, 8, PG>(a, plan, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int D, bool PG>
+static cudaError_t dispatch_c(int c, int qpk, const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
+    switch (c) {
+        case 4: return dispatch_qpk<D, 4, PG>(qpk, a, plan, s);
+        case 8: return dispatch_qpk<D, 8, PG>(qpk, a, plan, s);
+        case 16: return dispatch_qpk<D, 16, PG>(qpk, a, plan, s);
+        case 32: return dispatch_qpk<D, 32, PG>(qpk, a, plan, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -97,14 +118,9 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     a.nsplit = plan.nsplit;
     a.qscale = scale * 1.44269504088896340736f;
     const int qpk = cc.Hq / cc.Hkv;
-    if (cc.D == 128 && cc.c == 4) return dispatch_qpk<128, 4>(qpk, a, plan, s);
-    if (cc.D == 128 && cc.c == 8) return dispatch_qpk<128, 8>(qpk, a, plan, s);
-    if (cc.D == 128 && cc.c == 16) return dispatch_qpk<128, 16>(qpk, a, plan, s);
-    if (cc.D == 128 && cc.c == 32) return dispatch_qpk<128, 32>(qpk, a, plan, s);
-    if (cc.D == 64 && cc.c == 4) return dispatch_qpk<64, 4>(qpk, a, plan, s);
-    if (cc.D == 64 && cc.c == 8) return dispatch_qpk<64, 8>(qpk, a, plan, s);
-    if (cc.D == 64 && cc.c == 16) return dispatch_qpk<64, 16>(qpk, a, plan, s);
-    if (cc.D == 64 && cc.c == 32) return dispatch_qpk<64, 32>(qpk, a, plan, s);
+    const bool pg = ncb_of(cc) > 1;
+    if (cc.D == 128) return pg ? dispatch_c<128, true>(cc.c, qpk, a, plan, s) : dispatch_c<128, false>(cc.c, qpk, a, plan, s);
+    if (cc.D == 64) return pg ? dispatch_c<64, true>(cc.c, qpk, a, plan, s) : dispatch_c<64, false>(cc.c, qpk, a, plan, s);
     return cudaErrorInvalidValue;
 }
 

@@ -144,7 +144,13 @@ __device__ __forceinline__ int tile_owner(int t) {          // a lane of the slo
     return l;
 }
 
-template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, int NW>
+// PG: one codebook per channel group.  The loop step's slice is then code-major with row r holding
+// entry r of every group's codebook (D bf16), so each lane reads its own channels of the row and the
+// 16 lanes of a token slot fall into distinct banks without replicas.  Tables: D = 128, K rows of 256 B
+// at [0, 64 KiB) and V rows at [64 KiB, 128 KiB); D = 64, rows of 256 B holding K then V, in two
+// copies whose second is rotated by 64 B within each half-row for the odd token slots of a half-warp.
+// The table choice rides in the upper bytes of the gather column, which the byte permute passes on.
+template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, int NW, bool PG = false>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const DecodeArgs a) {
     constexpr bool ROTQ = QPK == 1;                        // rotate the query, not every key
     constexpr int NP = D / (2 * C);                        // pair-groups = index words per token
@@ -158,6 +164,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     constexpr int TT = 4 * NW;                             // tokens per slot iteration
     constexpr int STRIDE = NSLOT * TT;                     // tokens between two iterations of a slot
     constexpr int QB = NT * 16 * NW;                       // bytes of one prefetch-queue stage
+    constexpr uint32_t TBL = PG ? 131072u : 65536u;        // bytes of the staged K/V tables
     static_assert(C == 4 || C == 8 || C == 16 || C == 32, "c");
     static_assert(NL >= 8 && NL <= 16, "slot width");
 
@@ -178,11 +185,28 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     const int slot = warp * SPW + lane / NL;
     const unsigned slot_mask = ((1u << NL) - 1u) << (lane & ~(NL - 1));
     const int slot_lane0 = lane & ~(NL - 1);
-    const uint32_t colk = (uint32_t)((lane % 16) * 8);     // byte 0 of every K gather address
-    const uint32_t colv = colk + 128u;                     // ... of every V gather address
+    // gather columns of the K / V entries of the lane's group (lo) and of its RoPE partner group (hi)
+    uint32_t colk_lo, colk_hi, colv_lo, colv_hi;
+    if constexpr (!PG) {
+        colk_lo = colk_hi = (uint32_t)((lane % 16) * 8);   // its own replica's 8-byte column
+        colv_lo = colv_hi = colk_lo + 128u;
+    } else if constexpr (D == 128) {
+        const uint32_t cb = (uint32_t)((gp * C + half * 4) * 2);
+        colk_lo = cb;
+        colk_hi = cb + 128u;
+        colv_lo = 0x10000u + cb;
+        colv_hi = 0x10000u + cb + 128u;
+    } else {
+        const uint32_t odd = (uint32_t)((lane >> 3) & 1);  // second token slot of the half-warp
+        const uint32_t cb = (uint32_t)((gp * C + half * 4) * 2);
+        colk_lo = (odd << 16) | ((cb + 64u * odd) & 127u);
+        colk_hi = (odd << 16) | ((cb + 64u + 64u * odd) & 127u);
+        colv_lo = colk_lo + 128u;
+        colv_hi = colk_hi + 128u;
+    }
     const int ch = gp * C + half * 4;                      // first of this lane's 4 low channels
     const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP + ((size_t)gp << 2);
-    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) + 65536u + (uint32_t)tid * 16u;
+    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) + TBL + (uint32_t)tid * 16u;
 
     // queue the first DEPTH iterations of this slot before staging the slices
     const int pfirst = tok_begin + slot * TT;
@@ -196,6 +220,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         cp_async_commit();
     }
 
+    if constexpr (!PG) {
     // stage the K and V slices as bank-private replicas (rows >= K zeroed)
     {
         const uint16_t *sk = a.slk + (size_t)h * a.K * C;
@@ -217,6 +242,26 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                     if (r < a.K) v = __ldg(reinterpret_cast<const uint4 *>(src) + u);
                     *reinterpret_cast<uint4 *>(dst + 16 * u) = v;
                 }
+            }
+        }
+    }
+
+    } else {
+        // code-major per-group tables (rows >= K zeroed): 16-byte chunks of every row
+        constexpr int CH = D / 8;                          // chunks of one K (or V) row
+        const uint4 *sk = reinterpret_cast<const uint4 *>(a.slk + (size_t)h * a.K * D);
+        const uint4 *sv = reinterpret_cast<const uint4 *>(a.slv + (size_t)h * a.K * D);
+        for (int it = tid; it < 256 * 2 * CH; it += NT) {
+            const int j = it % CH;
+            const int kv = (it / CH) & 1;
+            const int r = it / (2 * CH);
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (r < a.K) v = __ldg((kv ? sv : sk) + (size_t)r * CH + j);
+            if constexpr (D == 128) {
+                *reinterpret_cast<uint4 *>(smem + kv * 65536 + r * 256 + j * 16) = v;
+            } else {
+                *reinterpret_cast<uint4 *>(smem + r * 256 + kv * 128 + j * 16) = v;
+                *reinterpret_cast<uint4 *>(smem + 65536 + r * 256 + kv * 128 + ((j * 16 + 64) & 127)) = v;
             }
         }
     }
@@ -300,8 +345,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 #pragma unroll
             for (int k = 0; k < TT; ++k) {
                 const uint32_t w = word_k(w4[k >> 2], k & 3);
-                vraw[k][0] = lds64(smem, __byte_perm(w, colv, 0x7624));
-                vraw[k][1] = lds64(smem, __byte_perm(w, colv, 0x7634));
+                vraw[k][0] = lds64(smem, __byte_perm(w, colv_lo, 0x7624));
+                vraw[k][1] = lds64(smem, __byte_perm(w, colv_hi, 0x7634));
             }
         }
 
@@ -340,8 +385,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 }
             }
             const uint32_t w = word_k(w4[k >> 2], k & 3);
-            const uint2 elo = lds64(smem, __byte_perm(w, colk, 0x7604));
-            const uint2 ehi = lds64(smem, __byte_perm(w, colk, 0x7614));
+            const uint2 elo = lds64(smem, __byte_perm(w, colk_lo, 0x7604));
+            const uint2 ehi = lds64(smem, __byte_perm(w, colk_hi, 0x7614));
             const float2 kl[2] = {unpack2(elo.x), unpack2(elo.y)};
             const float2 kh[2] = {unpack2(ehi.x), unpack2(ehi.y)};
             if constexpr (ROTQ) {
@@ -402,8 +447,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             const int src = slot_lane0 + tile_owner<TT, NL>(k);
             if constexpr (!VEARLY) {
                 const uint32_t w = word_k(w4[k >> 2], k & 3);
-                vraw[k][0] = lds64(smem, __byte_perm(w, colv, 0x7624));
-                vraw[k][1] = lds64(smem, __byte_perm(w, colv, 0x7634));
+                vraw[k][0] = lds64(smem, __byte_perm(w, colv_lo, 0x7624));
+                vraw[k][1] = lds64(smem, __byte_perm(w, colv_hi, 0x7634));
             }
             const uint32_t vl[2] = {vraw[k][0].x, vraw[k][0].y}, vh[2] = {vraw[k][1].x, vraw[k][1].y};
 #pragma unroll

@@ -68,9 +68,59 @@ __global__ void __launch_bounds__(128) encode_direct_kernel(const EncodeArgs a) 
     a.idx[((size_t)b * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C) + idx_word(n, p, NP)] = word;
 }
 
-template <int D, int C, int TC>
-static cudaError_t launch_ct(const EncodeArgs &a, int x_dtype, int nb, cudaStream_t s) {
+// One codebook per channel group: a CTA takes one pair-group p of one head and stages the four
+// codebooks its words use (K and V of groups p and p + NP); one thread per token writes its word.
+// Grid: (ceil(ntok / 128), NP * Hkv, nb).
+template <int D, int C, int TC, typename XT>
+__global__ void __launch_bounds__(128) encode_pg_kernel(const EncodeArgs a) {
+    constexpr int G = C * TC;
     constexpr int NP = D / (2 * C);
+    constexpr int NCB = D / C;
+    extern __shared__ __align__(16) float ecb[];           // [4][K][G]: K_p, K_{p+NP}, V_p, V_{p+NP}
+    const int p = blockIdx.y % NP, h = blockIdx.y / NP;
+    const int brel = blockIdx.z;
+    const int b = a.b0 + brel;
+    const int K = a.K;
+    for (int e = threadIdx.x; e < 4 * K * G; e += blockDim.x) {
+        const int which = e / (K * G);
+        const int rem = e % (K * G);
+        const int kv = which >> 1, g = (which & 1) ? p + NP : p;
+        ecb[e] = bf16_to_f32(a.cb[(((size_t)kv * a.Hkv + h) * NCB + g) * (size_t)K * G + rem]);
+    }
+    __syncthreads();
+    const int nrel = blockIdx.x * blockDim.x + threadIdx.x;
+    if (nrel >= a.ntok) return;
+    float z[4][G];
+    const XT *xk = reinterpret_cast<const XT *>(a.xk);
+    const XT *xv = reinterpret_cast<const XT *>(a.xv);
+    const size_t base = (size_t)brel * a.s1 + (size_t)nrel * a.s2 + (size_t)h * a.s3;
+#pragma unroll
+    for (int m = 0; m < TC; ++m)
+#pragma unroll
+        for (int i = 0; i < C; ++i) {
+            const size_t off = base + (size_t)m * a.s0;
+            z[0][i * TC + m] = ld_x(xk + off + p * C + i);
+            z[1][i * TC + m] = ld_x(xk + off + (p + NP) * C + i);
+            z[2][i * TC + m] = ld_x(xv + off + p * C + i);
+            z[3][i * TC + m] = ld_x(xv + off + (p + NP) * C + i);
+        }
+    const size_t KG = (size_t)K * G;
+    const uint32_t word = nearest_word4<G>(z, ecb, ecb + KG, ecb + 2 * KG, ecb + 3 * KG, K);
+    a.idx[((size_t)b * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C) + idx_word(a.tok0 + nrel, p, NP)] = word;
+}
+
+template <int D, int C, int TC>
+static cudaError_t launch_ct(const EncodeArgs &a, int x_dtype, int nb, bool pg, cudaStream_t s) {
+    constexpr int NP = D / (2 * C);
+    if (pg) {
+        const size_t smem = 4 * (size_t)a.K * C * TC * sizeof(float);
+        dim3 grid((a.ntok + 127) / 128, NP * a.Hkv, nb);
+        auto k = x_dtype == LOOPVQ_BF16 ? encode_pg_kernel<D, C, TC, uint16_t> : encode_pg_kernel<D, C, TC, float>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k<<<grid, 128, smem, s>>>(a);
+        return cudaGetLastError();
+    }
     const size_t smem = 2 * (size_t)a.K * C * TC * sizeof(float);
     dim3 grid((a.ntok * NP + 127) / 128, a.Hkv, nb);
     if (x_dtype == LOOPVQ_BF16) {
@@ -88,20 +138,20 @@ static cudaError_t launch_ct(const EncodeArgs &a, int x_dtype, int nb, cudaStrea
 }
 
 template <int D>
-static cudaError_t dispatch_c(int c, int tc, const EncodeArgs &a, int x_dtype, int nb, cudaStream_t s) {
+static cudaError_t dispatch_c(int c, int tc, const EncodeArgs &a, int x_dtype, int nb, bool pg, cudaStream_t s) {
     if (c == 4) {
-        if (tc == 4) return launch_ct<D, 4, 4>(a, x_dtype, nb, s);
-        if (tc == 2) return launch_ct<D, 4, 2>(a, x_dtype, nb, s);
-        if (tc == 1) return launch_ct<D, 4, 1>(a, x_dtype, nb, s);
+        if (tc == 4) return launch_ct<D, 4, 4>(a, x_dtype, nb, pg, s);
+        if (tc == 2) return launch_ct<D, 4, 2>(a, x_dtype, nb, pg, s);
+        if (tc == 1) return launch_ct<D, 4, 1>(a, x_dtype, nb, pg, s);
     } else if (c == 8) {
-        if (tc == 4) return launch_ct<D, 8, 4>(a, x_dtype, nb, s);
-        if (tc == 2) return launch_ct<D, 8, 2>(a, x_dtype, nb, s);
-        if (tc == 1) return launch_ct<D, 8, 1>(a, x_dtype, nb, s);
+        if (tc == 4) return launch_ct<D, 8, 4>(a, x_dtype, nb, pg, s);
+        if (tc == 2) return launch_ct<D, 8, 2>(a, x_dtype, nb, pg, s);
+        if (tc == 1) return launch_ct<D, 8, 1>(a, x_dtype, nb, pg, s);
     } else if (c == 16) {
-        if (tc == 2) return launch_ct<D, 16, 2>(a, x_dtype, nb, s);
-        if (tc == 1) return launch_ct<D, 16, 1>(a, x_dtype, nb, s);
+        if (tc == 2) return launch_ct<D, 16, 2>(a, x_dtype, nb, pg, s);
+        if (tc == 1) return launch_ct<D, 16, 1>(a, x_dtype, nb, pg, s);
     } else if (c == 32) {
-        if (tc == 1) return launch_ct<D, 32, 1>(a, x_dtype, nb, s);
+        if (tc == 1) return launch_ct<D, 32, 1>(a, x_dtype, nb, pg, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -115,7 +165,7 @@ cudaError_t launch_encode(const loopvq_cache &cc, int layer, int block, const vo
     if (nb == 0 || ntok == 0) return cudaSuccess;
     // bf16 inputs with a tensor-core instantiation go to the tcgen05 contraction; fp32 inputs (not
     // representable as bf16 MMA operands) and other shapes use the exact CUDA-core kernel below
-    if (x_dtype == LOOPVQ_BF16) {
+    if (x_dtype == LOOPVQ_BF16 && ncb_of(cc) == 1) {
         const cudaError_t e = launch_encode_tc(cc, layer, block, xk, xv, strides, b0, nb, tok0, ntok, s);
         if (e != cudaErrorNotSupported) return e;
     }
@@ -134,8 +184,9 @@ cudaError_t launch_encode(const loopvq_cache &cc, int layer, int block, const vo
     a.b0 = b0;
     a.tok0 = tok0;
     a.ntok = ntok;
-    if (cc.D == 128) return dispatch_c<128>(cc.c, cc.Tc, a, x_dtype, nb, s);
-    if (cc.D == 64) return dispatch_c<64>(cc.c, cc.Tc, a, x_dtype, nb, s);
+    const bool pg = ncb_of(cc) > 1;
+    if (cc.D == 128) return dispatch_c<128>(cc.c, cc.Tc, a, x_dtype, nb, pg, s);
+    if (cc.D == 64) return dispatch_c<64>(cc.c, cc.Tc, a, x_dtype, nb, pg, s);
     return cudaErrorInvalidValue;
 }
 

@@ -23,13 +23,15 @@ __host__ __device__ inline size_t idx_word(int n, int p, int NP) {
     return (((size_t)(n >> 2) * NP + p) << 2) + (n & 3);
 }
 // slice base of (layer, t, kv, h): [K][c] bf16
+// codebooks per (layer, block, head, K|V): 1 (shared) or D/c (one per channel group)
+__host__ __device__ inline int ncb_of(const loopvq_cache &cc) { return cc.ncb > 1 ? cc.ncb : 1; }
 __host__ __device__ inline size_t slice_base(const loopvq_cache &cc, int layer, int t, int kv, int h) {
-    return ((((size_t)layer * cc.T + t) * 2 + kv) * cc.Hkv + h) * (size_t)cc.K * cc.c;
+    return ((((size_t)layer * cc.T + t) * 2 + kv) * cc.Hkv + h) * (size_t)cc.K * cc.c * ncb_of(cc);
 }
-// codebook base of (layer, block, kv, h): [K][G] bf16
+// codebook base of (layer, block, kv, h): [NCB][K][G] bf16
 __host__ __device__ inline size_t codebook_base(const loopvq_cache &cc, int layer, int block, int kv, int h) {
     const int NB = cc.T / cc.Tc;
-    return ((((size_t)layer * NB + block) * 2 + kv) * cc.Hkv + h) * (size_t)cc.K * (cc.c * cc.Tc);
+    return ((((size_t)layer * NB + block) * 2 + kv) * cc.Hkv + h) * (size_t)cc.K * (cc.c * cc.Tc) * ncb_of(cc);
 }
 
 // bf16 bit pattern -> fp32 (exact)

@@ -10,21 +10,22 @@
 namespace loopvq {
 
 __global__ void slice_cut_kernel(const uint16_t *__restrict__ cb, uint16_t *__restrict__ slices,
-                                 int L, int T, int Tc, int Hkv, int K, int c, size_t total) {
+                                 int L, int T, int Tc, int Hkv, int K, int c, int ncb, size_t total) {
     const int G = c * Tc;
     const int NB = T / Tc;
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
          e += (size_t)gridDim.x * blockDim.x) {
-        // e enumerates [L][T][2][Hkv][K][c]
+        // e enumerates [L][T][2][Hkv][K][ncb][c]: row r of a slice holds entry r of every codebook
         size_t r0 = e;
         const int i = (int)(r0 % c); r0 /= c;
+        const int g = (int)(r0 % ncb); r0 /= ncb;
         const int r = (int)(r0 % K); r0 /= K;
         const int h = (int)(r0 % Hkv); r0 /= Hkv;
         const int kv = (int)(r0 % 2); r0 /= 2;
         const int t = (int)(r0 % T); r0 /= T;
         const int layer = (int)r0;
         const int beta = t / Tc, m = t % Tc;
-        const size_t src = ((((size_t)layer * NB + beta) * 2 + kv) * Hkv + h) * (size_t)K * G +
+        const size_t src = (((((size_t)layer * NB + beta) * 2 + kv) * Hkv + h) * ncb + g) * (size_t)K * G +
                            (size_t)r * G + (size_t)i * Tc + m;
         slices[e] = cb[src];
     }
@@ -47,10 +48,11 @@ __global__ void rope_table_kernel(float *__restrict__ rope, int Nmax, int D, dou
 }
 
 cudaError_t launch_prepare(const loopvq_cache &cc, cudaStream_t s) {
-    const size_t ns = (size_t)cc.L * cc.T * 2 * cc.Hkv * cc.K * cc.c;
+    const size_t ns = (size_t)cc.L * cc.T * 2 * cc.Hkv * cc.K * cc.c * ncb_of(cc);
     int blocks = (int)((ns + 255) / 256);
     if (blocks > 148 * 32) blocks = 148 * 32;
-    slice_cut_kernel<<<blocks, 256, 0, s>>>(cc.codebook, cc.slices, cc.L, cc.T, cc.Tc, cc.Hkv, cc.K, cc.c, ns);
+    slice_cut_kernel<<<blocks, 256, 0, s>>>(cc.codebook, cc.slices, cc.L, cc.T, cc.Tc, cc.Hkv, cc.K, cc.c, ncb_of(cc),
+                                            ns);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t nr = (size_t)cc.Nmax * (cc.D / 2);
@@ -79,9 +81,13 @@ __global__ void dequant_kernel(loopvq_cache cc, int layer, int t, int kv, int b,
         const int r_lo = (w >> (16 * kv)) & 0xff;
         const int r_hi = (w >> (16 * kv + 8)) & 0xff;
         const uint16_t *S = cc.slices + slice_base(cc, layer, t, kv, h);
+        // row r of the slice holds entry r of every codebook: NCB * c values; a shared codebook's entry
+        // is the whole row, a per-group codebook's entry for group g sits at g * c
+        const int rs = ncb_of(cc) * c;
+        const int glo = ncb_of(cc) > 1 ? p * c : 0, ghi = ncb_of(cc) > 1 ? (p + NP) * c : 0;
         // codes outside [0, K) rebuild as zero, like the zeroed rows of the decode kernel
-        float lo = r_lo < cc.K ? bf16_to_f32(S[(size_t)r_lo * c + i]) : 0.f;
-        float hi = r_hi < cc.K ? bf16_to_f32(S[(size_t)r_hi * c + i]) : 0.f;
+        float lo = r_lo < cc.K ? bf16_to_f32(S[(size_t)r_lo * rs + glo + i]) : 0.f;
+        float hi = r_hi < cc.K ? bf16_to_f32(S[(size_t)r_hi * rs + ghi + i]) : 0.f;
         if (apply_rope && kv == 0) {
             const float cs = cc.rope[(size_t)tok * D + f];
             const float sn = cc.rope[(size_t)tok * D + h2 + f];

@@ -32,7 +32,8 @@ class CacheDesc(C.Structure):
     _fields_ = [("L", C.c_int32), ("T", C.c_int32), ("Tc", C.c_int32), ("Hkv", C.c_int32),
                 ("Hq", C.c_int32), ("D", C.c_int32), ("c", C.c_int32), ("K", C.c_int32),
                 ("B", C.c_int32), ("Nmax", C.c_int32), ("theta", C.c_float),
-                ("idx", C.c_void_p), ("codebook", C.c_void_p), ("slices", C.c_void_p), ("rope", C.c_void_p)]
+                ("idx", C.c_void_p), ("codebook", C.c_void_p), ("slices", C.c_void_p), ("rope", C.c_void_p),
+                ("ncb", C.c_int32)]
 
 
 class Bf16CacheDesc(C.Structure):
@@ -126,9 +127,11 @@ def _stream(stream):
 class Cache:
     """Shape plus the four device buffers of a coded cache (see include/loopvq.h)."""
 
-    def __init__(self, L, T, Tc, Hkv, Hq, D, c, K, B, Nmax, theta=1.0e4, device="cuda", alloc=True):
-        self.desc = CacheDesc(L, T, Tc, Hkv, Hq, D, c, K, B, Nmax, theta, None, None, None, None)
+    def __init__(self, L, T, Tc, Hkv, Hq, D, c, K, B, Nmax, theta=1.0e4, device="cuda", alloc=True, ncb=1):
+        """ncb: 1 for one codebook per (layer, block, head, K|V), D // c for one per channel group."""
+        self.desc = CacheDesc(L, T, Tc, Hkv, Hq, D, c, K, B, Nmax, theta, None, None, None, None, ncb)
         self.L, self.T, self.Tc, self.Hkv, self.Hq, self.D, self.c, self.K = L, T, Tc, Hkv, Hq, D, c, K
+        self.ncb = ncb
         self.B, self.Nmax, self.theta = B, Nmax, theta
         self.idx = self.codebook = self.slices = self.rope = None
         if alloc:

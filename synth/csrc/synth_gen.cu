@@ -69,22 +69,24 @@ __global__ void q_kernel(uint16_t *out, uint32_t seed, uint32_t tagl, int step, 
     }
 }
 
-// Codebooks of every (layer, block, kv, head) in the [L][NB][2][Hkv][K][G] order.
-__global__ void codebook_kernel(uint16_t *out, uint32_t seed, int L, int NB, int Tc, int Hkv, int K, int c, Coef cf,
-                                float ih_scale, uint32_t tag_k, uint32_t tag_v) {
+// Codebooks of every (layer, block, kv, head, group) in the [L][NB][2][Hkv][NCB][K][G] order.
+__global__ void codebook_kernel(uint16_t *out, uint32_t seed, int L, int NB, int Tc, int Hkv, int NCB, int K, int c,
+                                Coef cf, float ih_scale, uint32_t tag_k, uint32_t tag_v) {
     const int G = c * Tc;
-    const size_t total = (size_t)L * NB * 2 * Hkv * K * c;
+    const size_t total = (size_t)L * NB * 2 * Hkv * NCB * K * c;
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
         size_t r0 = e;
         const int i = (int)(r0 % c); r0 /= c;
         const int r = (int)(r0 % K); r0 /= K;
+        const int g = (int)(r0 % NCB); r0 /= NCB;
         const int h = (int)(r0 % Hkv); r0 /= Hkv;
         const int kv = (int)(r0 % 2); r0 /= 2;
         const int blk = (int)(r0 % NB); r0 /= NB;
         const int layer = (int)r0;
-        const uint64_t flat = ((uint64_t)h * K + r) * c + i;
+        const uint64_t flat = (((uint64_t)h * NCB + g) * K + r) * c + i;
         const uint32_t tagl = ((kv ? tag_v : tag_k) << 24) | (uint32_t)layer;
-        const size_t base = ((((size_t)layer * NB + blk) * 2 + kv) * Hkv + h) * (size_t)K * G + (size_t)r * G;
+        const size_t base =
+            (((((size_t)layer * NB + blk) * 2 + kv) * Hkv + h) * NCB + g) * (size_t)K * G + (size_t)r * G;
         float x = 0.f;
         for (int m = 0; m < Tc; ++m) {
             const int t = blk * Tc + m;
@@ -156,11 +158,11 @@ int synth_q(void *out, uint32_t seed, uint32_t tagl, int step, size_t n, float i
     return (int)cudaGetLastError();
 }
 
-int synth_codebook(void *out, uint32_t seed, int L, int NB, int Tc, int Hkv, int K, int c, const float *rho,
+int synth_codebook(void *out, uint32_t seed, int L, int NB, int Tc, int Hkv, int NCB, int K, int c, const float *rho,
                    const float *sig, float ih_scale, uint32_t tag_k, uint32_t tag_v, void *stream) {
     if (NB * Tc > kMaxSteps) return 1;
-    const size_t n = (size_t)L * NB * 2 * Hkv * K * c;
-    codebook_kernel<<<grid_for(n), 256, 0, (cudaStream_t)stream>>>((uint16_t *)out, seed, L, NB, Tc, Hkv, K, c,
+    const size_t n = (size_t)L * NB * 2 * Hkv * NCB * K * c;
+    codebook_kernel<<<grid_for(n), 256, 0, (cudaStream_t)stream>>>((uint16_t *)out, seed, L, NB, Tc, Hkv, NCB, K, c,
                                                                     make_coef(rho, sig, NB * Tc), ih_scale, tag_k,
                                                                     tag_v);
     return (int)cudaGetLastError();

@@ -24,7 +24,7 @@ def lib():
         fp = C.POINTER(C.c_float)
         L.synth_kv.argtypes = [vp, u32, u32, i, i, i, i, i, i, fp, fp, f, vp]
         L.synth_q.argtypes = [vp, u32, u32, i, sz, f, f, vp]
-        L.synth_codebook.argtypes = [vp, u32, i, i, i, i, i, i, fp, fp, f, u32, u32, vp]
+        L.synth_codebook.argtypes = [vp, u32, i, i, i, i, i, i, i, fp, fp, f, u32, u32, vp]
         L.synth_idx.argtypes = [vp, u32, u32, i, i, i, i, i, i, vp]
         for n in ("synth_kv", "synth_q", "synth_codebook", "synth_idx"):
             getattr(L, n).restype = i
@@ -70,9 +70,9 @@ def fill_q(w: Workload, layer: int, t: int, out: torch.Tensor, gain: float = 1.0
 
 
 def fill_codebook(w: Workload, out: torch.Tensor):
-    """out: the cache codebook buffer [L][NB][2][Hkv][K][G] (bf16 bits)."""
+    """out: the cache codebook buffer [L][NB][2][Hkv][NCB][K][G] (bf16 bits)."""
     rho, sig = _coef(w)
-    _ok(lib().synth_codebook(out.data_ptr(), w.seed, w.L, w.NB, w.Tc, w.Hkv, w.K, w.c, _fp(rho), _fp(sig),
+    _ok(lib().synth_codebook(out.data_ptr(), w.seed, w.L, w.NB, w.Tc, w.Hkv, w.ncb, w.K, w.c, _fp(rho), _fp(sig),
                              float(IH_SCALE), TAG_CBK, TAG_CBV, _stream()), "synth_codebook")
 
 

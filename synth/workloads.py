@@ -11,6 +11,8 @@ Five workload shapes (all K = 256 codes, b = 8 bits):
   ctx32k_cq  ctx32k coded per loop step (CQ: Tc = 1, c = G = 16, 0.5 bit), the
              baseline the pages compare LoopVQ against at the same bitwidth; same
              seed as ctx32k, so keys, values, queries and lengths are identical
+  ctx32k_pg  ctx32k with one codebook per channel group (32 per head and K|V),
+             the paper's notation; same seed as ctx32k
 
 The model shapes follow the pages' Ouro-1.4B description (24 layers, 16 heads of
 dimension 128, 4 loop steps) and the deep-recurrence variant follows the
@@ -65,6 +67,7 @@ class Workload:
     rho: tuple            # rho[t] for t = 1..T-1 (index 0 unused, kept 0.0)
     len_lo: int = -1      # if >= 0, lengths uniform in [len_lo, Nmax]
     theta: float = 1.0e4
+    ncb: int = 1          # codebooks per (layer, block, head, K|V): 1 shared, or D/c (one per channel group)
 
     @property
     def G(self) -> int:
@@ -102,6 +105,8 @@ WORKLOADS = {
                        rho=_rho((0.9,), 32)),
     "ctx32k_cq": Workload("ctx32k_cq", 2, L=24, T=4, Tc=1, Hkv=16, Hq=16, D=128, c=16, K=256, B=8, Nmax=32768,
                           rho=_rho((0.7, 0.8, 0.9), 4), len_lo=16384),
+    "ctx32k_pg": Workload("ctx32k_pg", 2, L=24, T=4, Tc=4, Hkv=16, Hq=16, D=128, c=4, K=256, B=8, Nmax=32768,
+                          rho=_rho((0.7, 0.8, 0.9), 4), len_lo=16384, ncb=32),
 }
 
 
@@ -159,15 +164,21 @@ def kv_loops(w: Workload, layer: int, kv: int, t_first: int, t_last: int,
     return f32_to_bf16_bits(x) if dtype == "bf16" else x
 
 
-def codebook(w: Workload, layer: int, block: int, kv: int, h: int):
-    """bf16 bits [K][G]; coordinate i*Tc + m holds 'channel' i at loop m of entry r's fresh token."""
+def codebook(w: Workload, layer: int, block: int, kv: int, h: int, g: int = 0):
+    """bf16 bits [K][G] of codebook g (0 when shared); coordinate i*Tc + m holds 'channel' i at loop m of
+    entry r's fresh token.  Codebook g of head h draws from counters ((h * ncb + g) * K + r) * c + i."""
     r = np.arange(w.K, dtype=np.uint64)[:, None]
     i = np.arange(w.c, dtype=np.uint64)[None, :]
-    flat = (np.uint64(h) * np.uint64(w.K) + r) * np.uint64(w.c) + i          # [K][c]
+    flat = ((np.uint64(h) * np.uint64(w.ncb) + np.uint64(g)) * np.uint64(w.K) + r) * np.uint64(w.c) + i   # [K][c]
     t0 = block * w.Tc
     x = _ar1(w, TAG_CBK if kv == 0 else TAG_CBV, layer, flat, t0, t0 + w.Tc - 1, t_lo_chain=t0)  # [Tc][K][c]
     x = np.transpose(x, (1, 2, 0)).reshape(w.K, w.G)                          # [K][c*Tc], coord i*Tc+m
     return f32_to_bf16_bits(x)
+
+
+def codebooks(w: Workload, layer: int, block: int, kv: int, h: int):
+    """bf16 bits [ncb][K][G]: every codebook of (layer, block, K|V, head)."""
+    return np.stack([codebook(w, layer, block, kv, h, g) for g in range(w.ncb)])
 
 
 def queries(w: Workload, layer: int, t: int, b: Sequence[int] = None, hq: Sequence[int] = None,
@@ -204,5 +215,5 @@ def random_indices(w: Workload, layer: int, block: int, kv: int, b: int, h: int,
     return (w0 % np.uint32(w.K)).astype(np.uint8)
 
 
-__all__ = ["Workload", "WORKLOADS", "kv_loops", "codebook", "queries", "lengths", "random_indices",
+__all__ = ["Workload", "WORKLOADS", "kv_loops", "codebook", "codebooks", "queries", "lengths", "random_indices",
            "rho_sigma_f32", "bf16_bits_to_f32", "f32_to_bf16_bits"]

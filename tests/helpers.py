@@ -10,7 +10,7 @@ import math
 import numpy as np
 import torch
 
-from synth import Workload, codebook, kv_loops, queries, lengths, bf16_bits_to_f32
+from synth import codebooks, Workload, codebook, kv_loops, queries, lengths, bf16_bits_to_f32
 
 
 def pack_words(idx_k: np.ndarray, idx_v: np.ndarray, NP: int) -> np.ndarray:
@@ -37,21 +37,23 @@ def words_view(cache, layer: int, block: int, b: int, h: int) -> torch.Tensor:
 
 
 def codebook_view(cache, layer: int, block: int, kv: int, h: int) -> torch.Tensor:
+    """The codebook(s) of (layer, block, K|V, head): [NCB * K * G] elements, NCB = 1 when shared."""
     G = cache.c * cache.Tc
-    base = ((((layer * cache.NB + block) * 2 + kv) * cache.Hkv + h) * cache.K) * G
-    return cache.codebook[base:base + cache.K * G]
+    n = cache.ncb * cache.K * G
+    base = (((layer * cache.NB + block) * 2 + kv) * cache.Hkv + h) * n
+    return cache.codebook[base:base + n]
 
 
 def make_cache(w: Workload, device="cuda", codebooks="numpy"):
     """Cache with the workload's shapes, numpy-generated codebooks uploaded, prepared."""
     import looped_lm_decode_b200 as LQ
-    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, device=device)
+    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, device=device, ncb=w.ncb)
     if codebooks == "numpy":
         for layer in range(w.L):
             for blk in range(w.NB):
                 for kv in range(2):
                     for h in range(w.Hkv):
-                        cb = codebook(w, layer, blk, kv, h).view(np.int16).reshape(-1)
+                        cb = np_codebook_bits(w, layer, blk, kv, h).view(np.int16).reshape(-1)
                         codebook_view(cache, layer, blk, kv, h).copy_(torch.from_numpy(cb))
     else:
         from synth import gpu as SG
@@ -60,8 +62,13 @@ def make_cache(w: Workload, device="cuda", codebooks="numpy"):
     return cache
 
 
+def np_codebook_bits(w: Workload, layer, block, kv, h):
+    """[K][G] bits when the codebook is shared, [NCB][K][G] with one per channel group."""
+    return codebook(w, layer, block, kv, h) if w.ncb == 1 else codebooks(w, layer, block, kv, h)
+
+
 def np_codebook_f32(w: Workload, layer, block, kv, h):
-    return bf16_bits_to_f32(codebook(w, layer, block, kv, h))
+    return bf16_bits_to_f32(np_codebook_bits(w, layer, block, kv, h))
 
 
 def attn_tolerance_ok(out, ref, lse=None, lse_ref=None, rel=2e-3, lse_tol=1e-3):

@@ -24,7 +24,7 @@ def test_every_declared_symbol_is_exported():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(LQ.EXPORTS)
-    assert lib.loopvq_abi_version() == 1
+    assert lib.loopvq_abi_version() == 2
 
 
 def _cache(**kw):
@@ -178,3 +178,18 @@ def test_window_validation_before_launch():
     w.Hq, w.fill = c.Hq, None
     assert lib.loopvq_window_advance(C.byref(w), c.ref(), None) == 1
     assert lib.loopvq_window_workspace_bytes(C.byref(w), c.ref(), 1024) == 0
+
+
+def test_per_group_codebook_sizes_and_validation():
+    """ncb = D/c multiplies the codebook and slice buffers; other values are refused."""
+    lib = LQ.lib()
+    c1 = _cache()
+    cg = _cache()
+    cg.desc.ncb = 128 // 4
+    assert lib.loopvq_codebook_elems(cg.ref()) == 32 * lib.loopvq_codebook_elems(c1.ref())
+    assert lib.loopvq_slice_elems(cg.ref()) == 32 * lib.loopvq_slice_elems(c1.ref())
+    assert lib.loopvq_idx_words(cg.ref()) == lib.loopvq_idx_words(c1.ref())
+    cg.desc.ncb = 7
+    assert lib.loopvq_codebook_elems(cg.ref()) == 0
+    assert lib.loopvq_prepare(cg.ref(), None) == 1
+    assert b"ncb" in lib.loopvq_last_error()

@@ -14,7 +14,7 @@ import torch
 
 import looped_lm_decode_b200 as LQ
 from oracle import oracle as O
-from synth import (WORKLOADS, kv_loops, codebook, queries, lengths, random_indices, bf16_bits_to_f32)
+from synth import (WORKLOADS, kv_loops, codebook, codebooks, queries, lengths, random_indices, bf16_bits_to_f32)
 from synth import gpu as SG
 from tests.helpers import (pack_words, unpack_words, words_view, codebook_view, make_cache, np_codebook_f32,
                            attn_tolerance_ok)
@@ -32,7 +32,29 @@ SMALL = {
     "cq16": WORKLOADS["ctx4k"].replace(L=1, B=2, Hkv=2, Hq=2, Nmax=256, c=16, Tc=1),
     "cq32g": WORKLOADS["gqa16k"].replace(L=1, B=2, Hkv=1, Hq=4, Nmax=128, c=32, Tc=1),
     "cq16d64": WORKLOADS["tiny"].replace(c=16, Tc=2, B=2, Hq=2, Hkv=2, Nmax=128),
+    # one codebook per channel group (ncb = D/c)
+    "pg4": WORKLOADS["ctx4k"].replace(L=1, B=2, Hkv=2, Hq=2, Nmax=256, ncb=32),
+    "pg8gqa": WORKLOADS["gqa16k"].replace(L=1, B=2, Hkv=1, Hq=4, Nmax=128, ncb=16),
+    "pgd64": WORKLOADS["tiny"].replace(B=2, Hq=2, Hkv=2, Nmax=128, ncb=16),
+    "pgcq16": WORKLOADS["ctx4k"].replace(L=1, B=2, Hkv=2, Hq=2, Nmax=128, c=16, Tc=1, ncb=8),
 }
+
+
+def _dec(q, ik, iv, Ek, Ev, *args):
+    """The checker's decode with a shared ([K][G]) or per-group ([NCB][K][G]) codebook."""
+    return (O.decode_pg if np.ndim(Ek) == 3 else O.decode)(q, ik, iv, Ek, Ev, *args)
+
+
+def _enc(x, E, c):
+    return (O.encode_pg if np.ndim(E) == 3 else O.encode)(x, E, c)
+
+
+def _deq(idx, E, c, Tc, m):
+    return (O.dequant_pg if np.ndim(E) == 3 else O.dequant)(idx, E, c, Tc, m)
+
+
+def _dist(x, E, c, n, g, r):
+    return (O.dist64_pg if np.ndim(E) == 3 else O.dist64)(x, E, c, n, g, r)
 
 
 def _upload_random_codes(w, cache):
@@ -59,7 +81,7 @@ def _oracle_call(w, codes, layer, t, q_bits, lens, scale):
             h = hq // qpk
             ik, iv = codes[(layer, blk, b, h)]
             n = int(lens[b])
-            o, l = O.decode(bf16_bits_to_f32(q_bits[b, hq]).astype(np.float64), ik[:n], iv[:n],
+            o, l = _dec(bf16_bits_to_f32(q_bits[b, hq]).astype(np.float64), ik[:n], iv[:n],
                             np_codebook_f32(w, layer, blk, 0, h), np_codebook_f32(w, layer, blk, 1, h),
                             w.c, w.Tc, m, w.theta, scale)
             outs[b, hq], lses[b, hq] = o, l
@@ -145,7 +167,7 @@ def test_decode_explicit_scale():
     assert ok, msg
 
 
-@pytest.mark.parametrize("name", ["tiny", "deep", "gqa"])
+@pytest.mark.parametrize("name", ["tiny", "deep", "gqa", "pg4", "pgd64", "pgcq16"])
 def test_dequant_debug_bit_exact(name):
     w = SMALL[name]
     cache = make_cache(w)
@@ -156,11 +178,11 @@ def test_dequant_debug_bit_exact(name):
         for kv in range(2):
             rec = LQ.dequant_debug(cache, 0, t, kv, b, 4, 60, apply_rope=False).cpu().numpy()
             for h in range(w.Hkv):
-                ref = O.dequant(codes[(0, blk, b, h)][kv][4:64], np_codebook_f32(w, 0, blk, kv, h), w.c, w.Tc, m)
+                ref = _deq(codes[(0, blk, b, h)][kv][4:64], np_codebook_f32(w, 0, blk, kv, h), w.c, w.Tc, m)
                 np.testing.assert_array_equal(rec[h].astype(np.float64), ref)
         rot = LQ.dequant_debug(cache, 0, t, 0, b, 100, 28, apply_rope=True).cpu().numpy()
         for h in range(w.Hkv):
-            k = O.dequant(codes[(0, blk, b, h)][0][100:128], np_codebook_f32(w, 0, blk, 0, h), w.c, w.Tc, m)
+            k = _deq(codes[(0, blk, b, h)][0][100:128], np_codebook_f32(w, 0, blk, 0, h), w.c, w.Tc, m)
             ref = O.rope(k, w.theta, 100)
             np.testing.assert_allclose(rot[h], ref, rtol=0, atol=2e-5 * np.abs(ref).max())
 
@@ -180,12 +202,12 @@ def _to_dev(x, dtype):
 def _check_codes(w, x_np, dtype, E, codes_gpu, b, h, kv):
     xf = bf16_bits_to_f32(x_np) if dtype == "bf16" else x_np
     xb = np.ascontiguousarray(xf[:, b, :, h, :])
-    ref = O.encode(xb, E, w.c)
+    ref = _enc(xb, E, w.c)
     mism = np.argwhere(codes_gpu != ref)
     ties = 0
     for n, g in mism:
-        dg = O.dist64(xb, E, w.c, n, g, int(codes_gpu[n, g]))
-        do = O.dist64(xb, E, w.c, n, g, int(ref[n, g]))
+        dg = _dist(xb, E, w.c, n, g, int(codes_gpu[n, g]))
+        do = _dist(xb, E, w.c, n, g, int(ref[n, g]))
         assert abs(dg - do) <= 1e-5 * max(dg, do), (b, h, kv, n, g, dg, do)
         ties += 1
     return ties
@@ -193,7 +215,8 @@ def _check_codes(w, x_np, dtype, E, codes_gpu, b, h, kv):
 
 @pytest.mark.parametrize("name,dtype", [("tiny", "bf16"), ("tiny", "f32"), ("ctx", "bf16"), ("gqa", "bf16"),
                                         ("deep", "bf16"), ("d64c8", "f32"), ("cq16", "bf16"), ("cq16", "f32"),
-                                        ("cq32g", "bf16"), ("cq16d64", "bf16")])
+                                        ("cq32g", "bf16"), ("cq16d64", "bf16"), ("pg4", "bf16"), ("pg8gqa", "bf16"),
+                                        ("pgd64", "f32"), ("pgcq16", "bf16")])
 def test_encode_parity(name, dtype):
     w = SMALL[name]
     if name == "ctx":
@@ -266,3 +289,13 @@ def test_generator_twins_agree():
         ck, cv = unpack_words(run, w4.Nmax, cache.NP)
         np.testing.assert_array_equal(ck, random_indices(w4, 1, 5, 0, b, h, range(w4.Nmax)))
         np.testing.assert_array_equal(cv, random_indices(w4, 1, 5, 1, b, h, range(w4.Nmax)))
+
+
+def test_generator_twins_agree_per_group_codebooks():
+    """The CUDA generator's per-group codebooks equal the numpy ones bit for bit."""
+    w = WORKLOADS["ctx4k"].replace(L=2, Hkv=2, Hq=2, B=1, Nmax=64, ncb=32)
+    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, ncb=w.ncb)
+    SG.fill_codebook(w, cache.codebook)
+    for (layer, blk, kv, h) in [(0, 0, 0, 0), (1, 0, 1, 1)]:
+        got = codebook_view(cache, layer, blk, kv, h).cpu().numpy().view(np.uint16)
+        np.testing.assert_array_equal(got, codebooks(w, layer, blk, kv, h).reshape(-1))
