@@ -35,7 +35,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import WORKLOADS, lengths, random_indices, queries, bf16_bits_to_f32, codebook  # noqa: E402
+from synth import WORKLOADS, lengths, random_indices, queries, bf16_bits_to_f32, codebook, codebooks  # noqa: E402
 
 METRIC = "LoopVQ decode-attn µs/step & GB/s at 32K ctx, 0.5 bit; % of roofline"
 SMEM_BYTES_PER_CLK_SM = 128
@@ -145,6 +145,13 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
 
     # ---- the serving layout through the window API: a full decode step is one advance (a page roll for
     # full windows every 8 steps), then per (loop step, layer) an append and a windowed attention call
+    peak, kind = peaks()
+    bf16_line = {"us_per_call": bf_ms * 1e3, "gbs": bf_bytes / (bf_ms * 1e-3) / 1e9,
+                 "frac": bf_bytes / (bf_ms * 1e-3) / 1e9 / peak, "peak": peak, "peak_kind": kind,
+                 "bytes_per_call": bf_bytes,
+                 "kernel": "loopvq_bf16_decode_attn over a bf16 cache of the same shape (keys stored rotated)"}
+    if w.ncb > 1:                                     # the window's page encoder codes shared codebooks only
+        return {"bf16_cache": bf16_line, "windowed": None}
     n_sink, n_recent = 8, 64
     win = LQ.Window(cache, n_sink=n_sink, n_recent=n_recent, device=dev)
     tmp = torch.empty((1, w.B, win.W, w.Hkv, w.D), dtype=torch.bfloat16, device=dev)
@@ -189,12 +196,8 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
     win_call_ms = statistics.fmean(a.elapsed_time(b) for a, b in call_evs)
     del win
 
-    peak, kind = peaks()
     return {
-        "bf16_cache": {"us_per_call": bf_ms * 1e3, "gbs": bf_bytes / (bf_ms * 1e-3) / 1e9,
-                       "frac": bf_bytes / (bf_ms * 1e-3) / 1e9 / peak, "peak": peak, "peak_kind": kind,
-                       "bytes_per_call": bf_bytes,
-                       "kernel": "loopvq_bf16_decode_attn over a bf16 cache of the same shape (keys stored rotated)"},
+        "bf16_cache": bf16_line,
         "windowed": {"us_per_call": win_call_ms * 1e3, "us_per_step": win_step_ms * 1e3, "steps": nsteps,
                      "sink": n_sink, "recent": n_recent,
                      "calls": "per step: loopvq_window_advance (page roll every 8 steps), then per (loop step, "
@@ -211,6 +214,7 @@ def workload_desc(w):
         "batch": w.B, "context": w.Nmax,
         "lengths": (f"uniform in [{w.len_lo}, {w.Nmax}] (seeded)" if w.len_lo >= 0 else "all full"),
         "layers": w.L, "loop_steps": w.T, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
+        "codebooks": "shared by the channel groups" if w.ncb == 1 else f"one per channel group ({w.ncb})",
         "bits_per_element": 8 / w.G,
         "l2": "inputs larger than L2: every call streams its layer's index words (> 126 MB), "
               "successive calls touch different layers",
@@ -287,8 +291,13 @@ def _cpu_inputs(w, layer, t, b, hq):
         _CPU_INPUTS[key] = (
             bf16_bits_to_f32(queries(w, layer, t, b=[b], hq=[hq])[0, 0]).astype(np.float64),
             random_indices(w, layer, blk, 0, b, h, range(n)), random_indices(w, layer, blk, 1, b, h, range(n)),
-            bf16_bits_to_f32(codebook(w, layer, blk, 0, h)), bf16_bits_to_f32(codebook(w, layer, blk, 1, h)))
+            bf16_bits_to_f32(_codebook(w, layer, blk, 0, h)), bf16_bits_to_f32(_codebook(w, layer, blk, 1, h)))
     return _CPU_INPUTS[key]
+
+
+def _codebook(w, layer, blk, kv, h):
+    """[K][G] bits of a shared codebook, [NCB][K][G] with one per channel group."""
+    return codebook(w, layer, blk, kv, h) if w.ncb == 1 else codebooks(w, layer, blk, kv, h)
 
 
 def cpu_sample(w, seconds, layer=0, t=1):
@@ -304,7 +313,7 @@ def cpu_sample(w, seconds, layer=0, t=1):
         n = int(lens[b])
         q, ik, iv, Ek, Ev = _cpu_inputs(w, layer, t, b, hq)
         t0 = time.perf_counter()
-        O.decode(q, ik, iv, Ek, Ev, w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        (O.decode_pg if w.ncb > 1 else O.decode)(q, ik, iv, Ek, Ev, w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
         total_s += time.perf_counter() - t0
         nbytes += n * 2 * (w.D // w.c)
         units += 1
@@ -365,7 +374,7 @@ def main():
         w = w.replace(B=args.batch)
 
     # ---------------- set-up: codebooks, slices, RoPE table, GPU encode of every (layer, block)
-    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, device=dev)
+    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, device=dev, ncb=w.ncb)
     SG.fill_codebook(w, cache.codebook)
     LQ.prepare(cache)
     xk = torch.empty((w.Tc, w.B, w.Nmax, w.Hkv, w.D), dtype=torch.bfloat16, device=dev)
@@ -498,12 +507,15 @@ def main():
             "encode": {"ms_per_layer_block": statistics.median(enc_ms),
                        "tokens_per_s": w.B * w.Nmax / (statistics.median(enc_ms) * 1e-3),
                        "input_gbs": 2 * w.Tc * w.B * w.Nmax * w.Hkv * w.D * 2 / (statistics.median(enc_ms) * 1e-3) / 1e9,
-                       "kernel": "encode_tc_kernel (tcgen05 bf16 distance contraction + TMEM arg-max)"},
+                       "kernel": ("encode_tc_kernel (tcgen05 bf16 distance contraction + TMEM arg-max)" if w.ncb == 1
+                                  else "encode_pg_kernel (exact fp32 distances on CUDA cores, one codebook per "
+                                       "channel group)")},
         }
         if compare is not None:
             line["bf16_cache"] = compare["bf16_cache"]
             line["bf16_cache"]["loopvq_speedup"] = compare["bf16_cache"]["us_per_call"] / (avg_call_ms * 1e3)
-            line["windowed"] = compare["windowed"]
+            if compare["windowed"] is not None:
+                line["windowed"] = compare["windowed"]
         if world == 1 and not args.no_cpu_baseline:
             s, nb, u = cpu_sample(w, args.cpu_seconds)
             line["cpu_baseline"] = {"value": nb / s / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
