@@ -31,6 +31,14 @@
  *              (the paper's notation B_{beta,l,h,g}): encode, the distance
  *              check, reconstruction and decode.
  *              LoopVQ paper, Sec. 2 eq. (2); Sec. 4.1 eq. (5); App. A.2.
+ *   tasq_*     TaSQ applied before loop-axis coupling: u = P(w (.) k / sigma),
+ *              with w a per-channel weight, sigma the root mean square of
+ *              w (.) k over all heads and channels of the token (stored in
+ *              fp16), and P a permutation that keeps every RoPE pair
+ *              {f, f + D/2} inside one code; the coupled key vectors are built
+ *              from u, reconstruction inverts the transform before RoPE.
+ *              LoopVQ paper, App. B "Formulation", "Grouping under loop
+ *              coupling", "Calibration and bitwidth".
  *   windowed   attention of one query over a cache whose sink and recent
  *              tokens are kept in bf16 (keys stored already rotated) and whose
  *              other tokens lo <= n < hi are coded: the coded keys are rebuilt
@@ -287,6 +295,131 @@ void ora_decode_pg(const double *q, const uint8_t *idx_k, const uint8_t *idx_v, 
     ora_dequant_pg(idx_k, N, D, c, Tc, m, E_k, K, kh);
     ora_rope(kh, N, D, theta, 0);
     ora_dequant_pg(idx_v, N, D, c, Tc, m, E_v, K, vh);
+    ora_attention(q, kh, vh, N, D, scale, out, lse);
+    free(kh);
+    free(vh);
+}
+
+/* ---- TaSQ before loop-axis coupling (App. B) ---- */
+
+/* Round to the nearest fp16 value, ties to even (IEEE 754 binary16: 1 sign, 5 exponent bits with
+ * bias 15, 10 fraction bits; subnormals below 2^-14; overflow to infinity), returned as a double. */
+double ora_round_fp16(double x)
+{
+    if (x != x) return x;
+    const double ax = fabs(x);
+    if (ax >= 65520.0) return x < 0 ? -INFINITY : INFINITY;     /* 65504 + half an ulp rounds up */
+    int e;
+    frexp(ax, &e);                                               /* ax = f * 2^e, f in [0.5, 1) */
+    int exp2 = e - 1;                                            /* ax in [2^exp2, 2^(exp2+1)) */
+    if (exp2 < -14) exp2 = -14;                                  /* subnormal spacing 2^-24 */
+    const double ulp = ldexp(1.0, exp2 - 10);
+    const double q = ax / ulp;                                   /* exact: a power-of-two scaling */
+    double r = floor(q);
+    const double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    const double y = r * ulp;
+    return x < 0 ? -y : y;
+}
+
+/* sigma of every token for one (loop step, layer, sequence): the root mean square of w (.) k over all
+ * Hkv heads and D channels, in fp64, rounded to fp16.  k: [Hkv][N][D], w: [Hkv][D]. */
+void ora_tasq_sigma(const float *k, const float *w, int Hkv, int N, int D, double *sigma)
+{
+    for (int n = 0; n < N; ++n) {
+        double ss = 0.0;
+        for (int h = 0; h < Hkv; ++h)
+            for (int f = 0; f < D; ++f) {
+                const double v = (double)w[(size_t)h * D + f] * (double)k[((size_t)h * N + n) * D + f];
+                ss += v * v;
+            }
+        sigma[n] = ora_round_fp16(sqrt(ss / ((double)Hkv * D)));
+    }
+}
+
+/* Channel of coordinate i < c of TaSQ group g: the group holds the c/2 RoPE pairs whose low
+ * channels are perm[g*c/2 + j], j < c/2, each pair as (low, low + D/2). */
+static int tasq_channel(const int16_t *perm, int D, int c, int g, int i)
+{
+    const int f = perm[g * (c / 2) + i / 2];
+    return (i % 2) ? f + D / 2 : f;
+}
+
+/* u = (w (.) k) / sigma of every token, in fp32 (multiply then divide, each rounded).
+ * k: [N][D] of one loop step, w: [D], sigma: [N] (fp16 values); u: [N][D]. */
+void ora_tasq_transform(const float *k, const float *w, const double *sigma, int N, int D, float *u)
+{
+    for (int n = 0; n < N; ++n)
+        for (int f = 0; f < D; ++f) {
+            const float wk = w[f] * k[(size_t)n * D + f];
+            u[(size_t)n * D + f] = wk / (float)sigma[n];
+        }
+}
+
+/* TaSQ + LoopVQ encode of one (layer, block, head) (App. B eq. 11): coupled vector of group g is
+ * z[i*Tc + m] = u^(m)[channel(g, i)]; nearest entry in fp32 as ora_encode.
+ * x: [Tc][N][D] keys, w: [Tc][D], sigma: [Tc][N], perm: [D/2]; idx: [N][D/c]. */
+void ora_tasq_encode(const float *x, const float *w, const double *sigma, const int16_t *perm, int Tc, int N, int D,
+                     int c, const float *E, int K, uint8_t *idx)
+{
+    const int G = c * Tc;
+    const int ng = D / c;
+    float *u = (float *)malloc(sizeof(float) * (size_t)Tc * (N > 0 ? N : 1) * D);
+    for (int m = 0; m < Tc; ++m)
+        ora_tasq_transform(x + (size_t)m * N * D, w + (size_t)m * D, sigma + (size_t)m * N, N, D,
+                           u + (size_t)m * N * D);
+    float z[256];
+    for (int n = 0; n < N; ++n)
+        for (int g = 0; g < ng; ++g) {
+            for (int i = 0; i < c; ++i)
+                for (int m = 0; m < Tc; ++m)
+                    z[i * Tc + m] = u[((size_t)m * N + n) * D + tasq_channel(perm, D, c, g, i)];
+            int best = 0;
+            float best_d = INFINITY;
+            for (int r = 0; r < K; ++r) {
+                float d = 0.0f;
+                for (int k = 0; k < G; ++k) {
+                    float diff = z[k] - E[(size_t)r * G + k];
+                    float sq = diff * diff;
+                    d = d + sq;
+                }
+                if (d < best_d) { best_d = d; best = r; }
+            }
+            idx[(size_t)n * ng + g] = (uint8_t)best;
+        }
+    free(u);
+}
+
+/* Reconstruction of the keys at loop step m (the transform inverted, fp64):
+ * k_hat[n][channel(g, i)] = sigma[n] * E[idx[n][g]][i*Tc + m] / w[channel(g, i)].
+ * w: [D] of that loop step, sigma: [N] of that loop step. */
+void ora_tasq_dequant(const uint8_t *idx, int N, int D, int c, int Tc, int m, const float *E, const int16_t *perm,
+                      const float *w, const double *sigma, double *out)
+{
+    const int G = c * Tc;
+    const int ng = D / c;
+    for (int n = 0; n < N; ++n)
+        for (int g = 0; g < ng; ++g) {
+            const int r = idx[(size_t)n * ng + g];
+            for (int i = 0; i < c; ++i) {
+                const int f = tasq_channel(perm, D, c, g, i);
+                out[(size_t)n * D + f] = sigma[n] * (double)E[(size_t)r * G + i * Tc + m] / (double)w[f];
+            }
+        }
+}
+
+/* Decode attention with TaSQ keys: keys rebuilt by ora_tasq_dequant and rotated at positions 0..N-1,
+ * values rebuilt as in ora_decode (values are not transformed). */
+void ora_tasq_decode(const double *q, const uint8_t *idx_k, const uint8_t *idx_v, const float *E_k, const float *E_v,
+                     const int16_t *perm, const float *w, const double *sigma, int N, int D, int c, int Tc, int m,
+                     double theta, double scale, double *out, double *lse)
+{
+    size_t nd = (size_t)(N > 0 ? N : 1) * (size_t)D;
+    double *kh = (double *)malloc(sizeof(double) * nd);
+    double *vh = (double *)malloc(sizeof(double) * nd);
+    ora_tasq_dequant(idx_k, N, D, c, Tc, m, E_k, perm, w, sigma, kh);
+    ora_rope(kh, N, D, theta, 0);
+    ora_dequant(idx_v, N, D, c, Tc, m, E_v, vh);
     ora_attention(q, kh, vh, N, D, scale, out, lse);
     free(kh);
     free(vh);

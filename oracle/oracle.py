@@ -50,6 +50,20 @@ def lib():
         _lib.ora_dequant_pg.restype = None
         _lib.ora_decode_pg.argtypes = [f64p, u8p, u8p, f32p, f32p, I, I, I, I, I, I, D_, D_, f64p, C.POINTER(D_)]
         _lib.ora_decode_pg.restype = None
+        i16p = np.ctypeslib.ndpointer(np.int16, flags="C_CONTIGUOUS")
+        _lib.ora_round_fp16.argtypes = [D_]
+        _lib.ora_round_fp16.restype = D_
+        _lib.ora_tasq_sigma.argtypes = [f32p, f32p, I, I, I, f64p]
+        _lib.ora_tasq_sigma.restype = None
+        _lib.ora_tasq_transform.argtypes = [f32p, f32p, f64p, I, I, f32p]
+        _lib.ora_tasq_transform.restype = None
+        _lib.ora_tasq_encode.argtypes = [f32p, f32p, f64p, i16p, I, I, I, I, f32p, I, u8p]
+        _lib.ora_tasq_encode.restype = None
+        _lib.ora_tasq_dequant.argtypes = [u8p, I, I, I, I, I, f32p, i16p, f32p, f64p, f64p]
+        _lib.ora_tasq_dequant.restype = None
+        _lib.ora_tasq_decode.argtypes = [f64p, u8p, u8p, f32p, f32p, i16p, f32p, f64p, I, I, I, I, I, D_, D_, f64p,
+                                         C.POINTER(D_)]
+        _lib.ora_tasq_decode.restype = None
     return _lib
 
 
@@ -207,4 +221,73 @@ def decode_pg(q, idx_k, idx_v, E_k, E_v, c: int, Tc: int, m: int, theta: float =
     z8 = np.zeros((1, D // c), np.uint8)
     lib().ora_decode_pg(q, idx_k if N else z8, idx_v if N else z8, E_k, E_v, E_k.shape[1], N, D, c, Tc, m, theta,
                         scale, out, C.byref(lse))
+    return out, lse.value
+
+
+# ---- TaSQ before loop-axis coupling (App. B)
+
+def round_fp16(x: float) -> float:
+    return lib().ora_round_fp16(float(x))
+
+
+def tasq_sigma(k, w) -> np.ndarray:
+    """k: [Hkv][N][D] keys of one (loop step, layer, sequence), w: [Hkv][D] -> sigma [N] (fp16 values)."""
+    k, w = _f32(k), _f32(w)
+    Hkv, N, D = k.shape
+    out = np.zeros(N, dtype=np.float64)
+    if N:
+        lib().ora_tasq_sigma(k, w, Hkv, N, D, out)
+    return out
+
+
+def tasq_transform(k, w, sigma) -> np.ndarray:
+    """k: [N][D], w: [D], sigma: [N] -> u [N][D] fp32."""
+    k, w = _f32(k), _f32(w)
+    N, D = k.shape
+    u = np.zeros((N, D), dtype=np.float32)
+    if N:
+        lib().ora_tasq_transform(k, w, np.ascontiguousarray(sigma, np.float64), N, D, u)
+    return u
+
+
+def tasq_encode(x, w, sigma, perm, E, c: int) -> np.ndarray:
+    """x: [Tc][N][D] keys of one (layer, block, head), w: [Tc][D], sigma: [Tc][N], perm: [D/2]."""
+    x = _f32(x)
+    Tc, N, D = x.shape
+    E = _f32(E)
+    idx = np.zeros((N, D // c), dtype=np.uint8)
+    if N:
+        lib().ora_tasq_encode(x, _f32(w), np.ascontiguousarray(sigma, np.float64),
+                              np.ascontiguousarray(perm, np.int16), Tc, N, D, c, E, E.shape[0], idx)
+    return idx
+
+
+def tasq_dequant(idx, E, c: int, Tc: int, m: int, perm, w, sigma) -> np.ndarray:
+    """Keys of loop step m rebuilt with the transform inverted; w: [D] and sigma: [N] of that step."""
+    idx = np.ascontiguousarray(idx, dtype=np.uint8)
+    N = idx.shape[0]
+    D = idx.shape[1] * c
+    out = np.zeros((N, D), dtype=np.float64)
+    if N:
+        lib().ora_tasq_dequant(idx, N, D, c, Tc, m, _f32(E), np.ascontiguousarray(perm, np.int16), _f32(w),
+                               np.ascontiguousarray(sigma, np.float64), out)
+    return out
+
+
+def tasq_decode(q, idx_k, idx_v, E_k, E_v, perm, w, sigma, c: int, Tc: int, m: int, theta: float = 1.0e4,
+                scale: float = None):
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    D = q.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    idx_k = np.ascontiguousarray(idx_k, dtype=np.uint8).reshape(-1, D // c)
+    idx_v = np.ascontiguousarray(idx_v, dtype=np.uint8).reshape(-1, D // c)
+    N = idx_k.shape[0]
+    out = np.zeros(D, dtype=np.float64)
+    lse = C.c_double(0.0)
+    z8 = np.zeros((1, D // c), np.uint8)
+    sig = np.ascontiguousarray(sigma, np.float64) if N else np.ones(1)
+    lib().ora_tasq_decode(q, idx_k if N else z8, idx_v if N else z8, _f32(E_k), _f32(E_v),
+                          np.ascontiguousarray(perm, np.int16), _f32(w), sig, N, D, c, Tc, m, theta, scale, out,
+                          C.byref(lse))
     return out, lse.value

@@ -423,3 +423,77 @@ def test_pergroup_lossless_decode_is_textbook_rope_attention():
                                    xv[m].astype(np.float64), 0.15)
     np.testing.assert_allclose(out, ro, rtol=1e-11, atol=1e-12)
     assert abs(lse - rl) < 1e-11
+
+
+# ---------------------------------------------------------------- TaSQ before loop-axis coupling
+
+def test_round_fp16_matches_the_ieee_half_conversion():
+    """The checker's fp16 rounding equals numpy's float16 cast (IEEE binary16, ties to even) across
+    normal, subnormal, tie, boundary and overflow values."""
+    vals = np.concatenate([RNG.standard_normal(20000) * 10.0 ** RNG.integers(-9, 6, 20000),
+                           np.array([0.0, 1.0, 65504.0, 65519.99, 65520.0, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -25,
+                                     2.0 ** -14, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, -6e-5])])
+    with np.errstate(over="ignore"):
+        ref = vals.astype(np.float16).astype(np.float64)
+    got = np.array([O.round_fp16(v) for v in vals])
+    np.testing.assert_array_equal(got, ref)
+
+
+def _tasq_case(Hkv=3, N=10, D=64, Tc=4, c=4, seed=5):
+    rng = np.random.default_rng(seed)
+    k = _rand_bf16((Tc, Hkv, N, D))
+    wh = np.exp(rng.uniform(-0.5, 0.5, (Tc, Hkv, D // 2))).astype(np.float32)
+    w = np.concatenate([wh, wh], axis=2)                  # a RoPE pair shares its weight
+    perm = rng.permutation(D // 2).astype(np.int16)
+    return k, w, perm
+
+
+def test_tasq_sigma_is_the_rms_over_heads_and_channels_in_fp16():
+    k, w, _ = _tasq_case()
+    for m in range(k.shape[0]):
+        sig = O.tasq_sigma(k[m], w[m])
+        wk = w[m][:, None, :].astype(np.float64) * k[m].astype(np.float64)
+        ref = np.sqrt((wk ** 2).mean(axis=(0, 2))).astype(np.float16).astype(np.float64)
+        np.testing.assert_array_equal(sig, ref)
+
+
+def test_tasq_scale_equivariance():
+    """Doubling a token's keys doubles its sigma exactly and leaves u, hence its codes, unchanged."""
+    k, w, perm = _tasq_case(Hkv=1, N=6)
+    E = _rand_bf16((256, 16))
+    sig = np.stack([O.tasq_sigma(k[m], w[m]) for m in range(4)])
+    idx = O.tasq_encode(k[:, 0], w[:, 0], sig, perm, E, 4)
+    k2 = k.copy()
+    k2[:, :, 3] *= 2.0
+    sig2 = np.stack([O.tasq_sigma(k2[m], w[m]) for m in range(4)])
+    np.testing.assert_array_equal(sig2[:, 3], 2 * sig[:, 3])
+    np.testing.assert_array_equal(O.tasq_encode(k2[:, 0], w[:, 0], sig2, perm, E, 4), idx)
+
+
+@pytest.mark.parametrize("m", [0, 3])
+def test_tasq_lossless_decode_is_textbook_rope_attention(m):
+    """Codebooks holding the exact transformed coupled vectors: reconstruction inverts the weighting,
+    the scale and the permutation, so decode equals plain RoPE attention on the original keys (numpy
+    complex RoPE) up to the fp32 rounding of u."""
+    Tc, N, D, c = 4, 16, 64, 4
+    k, w, perm = _tasq_case(Hkv=1, N=N, D=D, Tc=Tc, c=c)
+    k, w = k[:, 0], w[:, 0]                                # one head: [Tc][N][D], [Tc][D]
+    sig = np.stack([O.tasq_sigma(k[mm][None], w[mm][None]) for mm in range(Tc)])
+    u = np.stack([O.tasq_transform(k[mm], w[mm], sig[mm]) for mm in range(Tc)])   # [Tc][N][D]
+    # group g of the permutation: pairs perm[g*c/2 + j] -> channels (f, f + D/2); coordinate i*Tc + mm
+    ch = np.array([[perm[g * (c // 2) + i // 2] + (D // 2) * (i % 2) for i in range(c)] for g in range(D // c)])
+    E = np.stack([u[:, n, ch[g]].T.reshape(-1) for n in range(N) for g in range(D // c)]).astype(np.float32)
+    idx = O.tasq_encode(k, w, sig, perm, E, c)
+    np.testing.assert_array_equal(idx, np.arange(N * (D // c)).reshape(N, D // c) % 256)
+    kh = O.tasq_dequant(idx, E, c, Tc, m, perm, w[m], sig[m])
+    np.testing.assert_allclose(kh, k[m].astype(np.float64), rtol=2e-7, atol=0)
+    v = _rand_bf16((Tc, N, D))
+    Ev = np.stack([np.array([v[mm, n, g * c + i] for i in range(c) for mm in range(Tc)])
+                   for n in range(N) for g in range(D // c)]).astype(np.float32)
+    iv = O.encode(v, Ev, c)
+    q = RNG.standard_normal(D)
+    out, lse = O.tasq_decode(q, idx, iv, E, Ev, perm, w[m], sig[m], c, Tc, m, 1e4, 0.2)
+    ro, rl = _softmax_attention_np(q, _rope_complex(k[m].astype(np.float64), np.arange(N)),
+                                   v[m].astype(np.float64), 0.2)
+    np.testing.assert_allclose(out, ro, rtol=1e-6, atol=1e-7)
+    assert abs(lse - rl) < 1e-6
