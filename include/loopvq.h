@@ -216,6 +216,60 @@ loopvq_status loopvq_merge2(const float *out_a, const float *lse_a, const float 
                             void *stream);
 
 /*
+ * TaSQ applied before loop-axis coupling (App. B): keys are mapped to
+ *   u = P(w (.) k / sigma)
+ * before their coupled vectors are built, and rebuilt keys are mapped back
+ * (k_hat = sigma * P^-1(u_hat) / w) before RoPE.  Values are not transformed.
+ *   w      fp32 [L][T][Hkv][D]: channel weights of loop step t, layer and
+ *          head; the two channels of a RoPE pair {f, f + D/2} must have the
+ *          same weight (the post-RoPE query moment is pair-symmetric).
+ *   perm   int16 [L][NB][Hkv][D/2]: the permutation P of (layer, block, KV
+ *          head), as an order of the low channels 0 .. D/2-1.  Key code g
+ *          (g < D/c) holds the c/2 RoPE pairs with low channels
+ *          perm[g*c/2 + j], j < c/2, each as (f, f + D/2), at every loop step
+ *          of the block: coordinate i*Tc + m is channel f of pair i/2 (even i)
+ *          or its partner f + D/2 (odd i) at loop step m.
+ *   sigma  fp16 [L][T][B][Nmax]: per-token scale of loop step t and layer,
+ *          the root mean square of w (.) k over all KV heads and channels of
+ *          the token, rounded to fp16; written by loopvq_tasq_encode.
+ * With TaSQ the index word (token n, pair-group p) holds: byte0 = K code of
+ * TaSQ group 2p, byte1 = K code of group 2p+1, byte2/3 = V codes of channel
+ * groups p and p + NP as without TaSQ.  Caches used with TaSQ share one
+ * codebook per (layer, block, KV head, K|V) (ncb = 1) and have c in {4, 8}.
+ */
+typedef struct loopvq_tasq {
+    const float *w;
+    const int16_t *perm;
+    uint16_t *sigma;
+} loopvq_tasq;
+
+/* Elements of the three TaSQ buffers for a cache (0 if the cache cannot be used with TaSQ). */
+size_t loopvq_tasq_w_elems(const loopvq_cache *cache);
+size_t loopvq_tasq_perm_elems(const loopvq_cache *cache);
+size_t loopvq_tasq_sigma_elems(const loopvq_cache *cache);
+
+/*
+ * loopvq_encode with TaSQ (App. B, eq. 10-11): for sequences b0 .. b0+nb-1
+ * and tokens tok0 .. tok0+ntok-1 of every loop step of the block, compute
+ * sigma (fp64 root mean square, rounded to fp16) into tasq->sigma, then code
+ * the keys' coupled vectors of u and the values' coupled vectors (exact fp32
+ * nearest entries, lowest index on ties).  Arguments as for loopvq_encode;
+ * the call must cover all KV heads of the tokens (sigma spans them).
+ */
+loopvq_status loopvq_tasq_encode(const loopvq_cache *cache, const loopvq_tasq *tasq, int layer, int block,
+                                 const void *xk, const void *xv, int x_dtype, const int64_t x_strides[4],
+                                 int b0, int nb, int tok0, int ntok, void *stream);
+
+/*
+ * loopvq_decode_attn over a TaSQ-coded cache: k_n = RoPE(sigma_n *
+ * P^-1(rebuilt u) / w, position n).  Arguments and workspace as for
+ * loopvq_decode_attn.
+ */
+loopvq_status loopvq_tasq_decode_attn(const loopvq_cache *cache, const loopvq_tasq *tasq, int layer, int t,
+                                      const uint16_t *q, const int32_t *lens, int max_len, float scale,
+                                      float *out, float *lse, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * The bf16 window of a coded cache and its decode-time life cycle (Sec. 4.3
  * "Cache layout": the first n_s (sink) and the most recent n_r tokens of a
  * request stay in bf16, pages of 8 tokens; "Encoding": during decode the

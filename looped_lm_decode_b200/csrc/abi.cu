@@ -242,6 +242,84 @@ loopvq_status loopvq_merge2(const float *out_a, const float *lse_a, const float 
     return LOOPVQ_OK;
 }
 
+static loopvq_status check_tasq(const loopvq_cache *cc, const loopvq_tasq *tq) {
+    LQ_TRY(check_shape(cc));
+    if (loopvq::ncb_of(*cc) != 1) return fail(LOOPVQ_ERR_UNSUPPORTED, "TaSQ needs shared codebooks (ncb = 1)");
+    if (cc->c != 4 && cc->c != 8) return fail(LOOPVQ_ERR_UNSUPPORTED, "TaSQ supports c = 4 or 8, not %d", cc->c);
+    if (!tq) return fail(LOOPVQ_ERR_INVALID_ARG, "tasq is NULL");
+    if (!tq->w || !tq->perm || !tq->sigma) return fail(LOOPVQ_ERR_INVALID_ARG, "tasq w, perm or sigma is NULL");
+    if ((reinterpret_cast<uintptr_t>(tq->w) & 3u) || (reinterpret_cast<uintptr_t>(tq->perm) & 1u) ||
+        (reinterpret_cast<uintptr_t>(tq->sigma) & 1u))
+        return fail(LOOPVQ_ERR_INVALID_ARG, "tasq buffers misaligned");
+    return LOOPVQ_OK;
+}
+
+size_t loopvq_tasq_w_elems(const loopvq_cache *cc) {
+    if (check_shape(cc) != LOOPVQ_OK || loopvq::ncb_of(*cc) != 1 || (cc->c != 4 && cc->c != 8)) return 0;
+    return (size_t)cc->L * cc->T * cc->Hkv * cc->D;
+}
+
+size_t loopvq_tasq_perm_elems(const loopvq_cache *cc) {
+    if (check_shape(cc) != LOOPVQ_OK || loopvq::ncb_of(*cc) != 1 || (cc->c != 4 && cc->c != 8)) return 0;
+    return (size_t)cc->L * (cc->T / cc->Tc) * cc->Hkv * (cc->D / 2);
+}
+
+size_t loopvq_tasq_sigma_elems(const loopvq_cache *cc) {
+    if (check_shape(cc) != LOOPVQ_OK || loopvq::ncb_of(*cc) != 1 || (cc->c != 4 && cc->c != 8)) return 0;
+    return (size_t)cc->L * cc->T * cc->B * (size_t)cc->Nmax;
+}
+
+loopvq_status loopvq_tasq_encode(const loopvq_cache *cc, const loopvq_tasq *tq, int layer, int block, const void *xk,
+                                 const void *xv, int x_dtype, const int64_t x_strides[4], int b0, int nb, int tok0,
+                                 int ntok, void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_tasq(cc, tq));
+    LQ_TRY(check_ptr(cc->idx, "idx"));
+    LQ_TRY(check_ptr(cc->codebook, "codebook"));
+    if (!xk || !xv || !x_strides) return fail(LOOPVQ_ERR_INVALID_ARG, "xk, xv or x_strides is NULL");
+    if (x_dtype != LOOPVQ_BF16 && x_dtype != LOOPVQ_FP32) return fail(LOOPVQ_ERR_INVALID_ARG, "x_dtype=%d", x_dtype);
+    if (layer < 0 || layer >= cc->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, cc->L);
+    const int NB = cc->T / cc->Tc;
+    if (block < 0 || block >= NB) return fail(LOOPVQ_ERR_INVALID_ARG, "block=%d out of [0, %d)", block, NB);
+    if (b0 < 0 || nb < 0 || b0 + nb > cc->B) return fail(LOOPVQ_ERR_INVALID_ARG, "sequences [%d, %d) outside [0, %d)", b0, b0 + nb, cc->B);
+    if (tok0 < 0 || ntok < 0 || tok0 + ntok > cc->Nmax)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "tokens [%d, %d) outside [0, %d)", tok0, tok0 + ntok, cc->Nmax);
+    cudaError_t e = loopvq::launch_tasq_encode(*cc, *tq, layer, block, xk, xv, x_dtype, x_strides, b0, nb, tok0, ntok,
+                                               (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_tasq_encode");
+    return LOOPVQ_OK;
+}
+
+loopvq_status loopvq_tasq_decode_attn(const loopvq_cache *cc, const loopvq_tasq *tq, int layer, int t,
+                                      const uint16_t *q, const int32_t *lens, int max_len, float scale, float *out,
+                                      float *lse, void *workspace, size_t ws_bytes, void *stream) {
+    g_err[0] = 0;
+    LQ_TRY(check_tasq(cc, tq));
+    LQ_TRY(check_ptr(cc->idx, "idx"));
+    LQ_TRY(check_ptr(cc->slices, "slices"));
+    LQ_TRY(check_ptr(cc->rope, "rope"));
+    LQ_TRY(check_ptr(q, "q"));
+    LQ_TRY(check_ptr(lens, "lens"));
+    LQ_TRY(check_ptr(out, "out"));
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(LOOPVQ_ERR_INVALID_ARG, "lse not 4-byte aligned");
+    if (layer < 0 || layer >= cc->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, cc->L);
+    if (t < 0 || t >= cc->T) return fail(LOOPVQ_ERR_INVALID_ARG, "t=%d out of [0, %d)", t, cc->T);
+    if (max_len < 0 || max_len > cc->Nmax)
+        return fail(LOOPVQ_ERR_INVALID_ARG, "max_len=%d out of [0, Nmax=%d]", max_len, cc->Nmax);
+    if (!std::isfinite(scale)) return fail(LOOPVQ_ERR_INVALID_ARG, "scale is not finite");
+    if (scale <= 0.f) scale = 1.0f / std::sqrt((float)cc->D);
+    const loopvq::DecodePlan plan = loopvq::plan_decode(*cc, max_len);
+    if (plan.nsplit > 65535) return fail(LOOPVQ_ERR_UNSUPPORTED, "too many splits");
+    if (!workspace || ws_bytes < plan.ws_bytes)
+        return fail(LOOPVQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws_bytes,
+                    workspace ? ws_bytes : (size_t)0);
+    if (!aligned16(workspace)) return fail(LOOPVQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    cudaError_t e = loopvq::launch_decode(*cc, plan, layer, t, q, nullptr, 0, lens, max_len, scale, out, lse,
+                                          workspace, (cudaStream_t)stream, tq);
+    if (e != cudaSuccess) return cuda_fail(e, "loopvq_tasq_decode_attn");
+    return LOOPVQ_OK;
+}
+
 static loopvq_status check_window(const loopvq_window *w, const loopvq_cache *cc) {
     if (!w) return fail(LOOPVQ_ERR_INVALID_ARG, "window is NULL");
     LQ_TRY(check_shape(cc));

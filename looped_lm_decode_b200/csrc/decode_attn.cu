@@ -48,14 +48,14 @@ DecodePlan plan_decode(const loopvq_cache &cc, int max_len) {
     return p;
 }
 
-template <int D, int C, int QPK, bool PG>
+template <int D, int C, int QPK, bool PG, bool TQ = false>
 static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
     constexpr int W = PG ? kPgWarps : kWarps;
     constexpr int NSLOT = W * (32 / (D / 8));
     const size_t red = (size_t)NSLOT * QPK * (D + 4) * sizeof(float);
     const size_t smem = ring_smem_bytes(PG);
     if (red > smem) return cudaErrorInvalidConfiguration;   // the slot records reuse slices and queue
-    auto kern = decode_split_kernel<D, C, QPK, W, PG ? kPgMinBlocks : kMinBlocks, kDepth, kWords, PG>;
+    auto kern = decode_split_kernel<D, C, QPK, W, PG ? kPgMinBlocks : kMinBlocks, kDepth, kWords, PG, TQ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (plan.nsplit > 0) {
@@ -79,6 +79,17 @@ static cudaError_t dispatch_qpk(int qpk, const DecodeArgs &a, const DecodePlan &
     }
 }
 
+template <int D, int C>
+static cudaError_t dispatch_tq_qpk(int qpk, const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
+    switch (qpk) {
+        case 1: return launch_t<D, C, 1, false, true>(a, plan, s);
+        case 2: return launch_t<D, C, 2, false, true>(a, plan, s);
+        case 4: return launch_t<D, C, 4, false, true>(a, plan, s);
+        case 8: return launch_t<D, C, 8, false, true>(a, plan, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 template <int D, bool PG>
 static cudaError_t dispatch_c(int c, int qpk, const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
     switch (c) {
@@ -92,7 +103,8 @@ static cudaError_t dispatch_c(int c, int qpk, const DecodeArgs &a, const DecodeP
 
 cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
                           const uint16_t *q, const int32_t *starts, int start_all, const int32_t *lens, int max_len,
-                          float scale, float *out, float *lse, void *workspace, cudaStream_t s) {
+                          float scale, float *out, float *lse, void *workspace, cudaStream_t s,
+                          const loopvq_tasq *tq) {
     DecodeArgs a{};
     const int beta = t / cc.Tc;
     a.idx = cc.idx + idx_base(cc, layer, beta, 0, 0);
@@ -118,6 +130,18 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     a.nsplit = plan.nsplit;
     a.qscale = scale * 1.44269504088896340736f;
     const int qpk = cc.Hq / cc.Hkv;
+    if (tq) {
+        const int NB = cc.T / cc.Tc;
+        a.tw = tq->w + ((size_t)layer * cc.T + t) * cc.Hkv * cc.D;
+        a.tperm = tq->perm + ((size_t)layer * NB + beta) * cc.Hkv * (cc.D / 2);
+        a.tsig = tq->sigma + ((size_t)layer * cc.T + t) * cc.B * cc.Nmax;
+        if (ncb_of(cc) != 1) return cudaErrorInvalidValue;
+        if (cc.D == 128 && cc.c == 4) return dispatch_tq_qpk<128, 4>(qpk, a, plan, s);
+        if (cc.D == 128 && cc.c == 8) return dispatch_tq_qpk<128, 8>(qpk, a, plan, s);
+        if (cc.D == 64 && cc.c == 4) return dispatch_tq_qpk<64, 4>(qpk, a, plan, s);
+        if (cc.D == 64 && cc.c == 8) return dispatch_tq_qpk<64, 8>(qpk, a, plan, s);
+        return cudaErrorInvalidValue;
+    }
     const bool pg = ncb_of(cc) > 1;
     if (cc.D == 128) return pg ? dispatch_c<128, true>(cc.c, qpk, a, plan, s) : dispatch_c<128, false>(cc.c, qpk, a, plan, s);
     if (cc.D == 64) return pg ? dispatch_c<64, true>(cc.c, qpk, a, plan, s) : dispatch_c<64, false>(cc.c, qpk, a, plan, s);

@@ -37,6 +37,7 @@
 //  * Online softmax with a lazy maximum; fp32 math in packed pairs (FFMA2).
 #pragma once
 
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "loopvq_internal.cuh"
@@ -57,6 +58,9 @@ struct DecodeArgs {
     float *lse;              // [B][Hq] or null
     int B, Hkv, Hq, K, Nmax, max_len, split_len, nsplit;
     int start_all;           // first attended token of every sequence when starts is null
+    const float *tw;         // TaSQ: channel weights of (layer, t) [Hkv][D]
+    const int16_t *tperm;    // TaSQ: low-channel order of (layer, block) [Hkv][D/2]
+    const uint16_t *tsig;    // TaSQ: fp16 token scales of (layer, t) [B][Nmax]
     float qscale;            // scale * log2(e)
 };
 
@@ -150,7 +154,11 @@ __device__ __forceinline__ int tile_owner(int t) {          // a lane of the slo
 // at [0, 64 KiB) and V rows at [64 KiB, 128 KiB); D = 64, rows of 256 B holding K then V, in two
 // copies whose second is rotated by 64 B within each half-row for the odd token slots of a half-warp.
 // The table choice rides in the upper bytes of the gather column, which the byte permute passes on.
-template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, int NW, bool PG = false>
+// TQ: keys coded with TaSQ (LoopVQ paper, App. B): the lane's two key codes are TaSQ groups 2p and
+// 2p + 1, whose entries interleave complete RoPE pairs (f, f + D/2) of low channels taken from the
+// permutation; the query is gathered at those channels and divided by the channel weights, the RoPE
+// values come from those columns of the table, and each token's score is multiplied by its scale.
+template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, int NW, bool PG = false, bool TQ = false>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const DecodeArgs a) {
     constexpr bool ROTQ = QPK == 1;                        // rotate the query, not every key
     constexpr int NP = D / (2 * C);                        // pair-groups = index words per token
@@ -205,6 +213,29 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         colv_hi = colk_hi + 128u;
     }
     const int ch = gp * C + half * 4;                      // first of this lane's 4 low channels
+    // low channels of the lane's 4 RoPE pairs: ch .. ch+3, or under TaSQ the pairs 2*half, 2*half + 1
+    // of TaSQ groups 2*gp (key code lo) and 2*gp + 1 (key code hi)
+    int fq[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if constexpr (TQ) {
+            const int16_t *pm = a.tperm + (size_t)h * (D / 2);
+            fq[k] = __ldg(pm + (2 * gp + (k >> 1)) * (C / 2) + 2 * half + (k & 1)) & (D / 2 - 1);
+        } else {
+            fq[k] = ch + k;
+        }
+    }
+    // cos and sin of this lane's 4 frequencies in table row `row`
+    auto load_row4 = [&](const float *row, float4 &cv, float4 &sv) {
+        if constexpr (TQ) {
+            cv = make_float4(__ldg(row + fq[0]), __ldg(row + fq[1]), __ldg(row + fq[2]), __ldg(row + fq[3]));
+            sv = make_float4(__ldg(row + D / 2 + fq[0]), __ldg(row + D / 2 + fq[1]), __ldg(row + D / 2 + fq[2]),
+                             __ldg(row + D / 2 + fq[3]));
+        } else {
+            cv = __ldg(reinterpret_cast<const float4 *>(row + ch));
+            sv = __ldg(reinterpret_cast<const float4 *>(row + D / 2 + ch));
+        }
+    };
     const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP + ((size_t)gp << 2);
     const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) + TBL + (uint32_t)tid * 16u;
 
@@ -270,18 +301,34 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 #pragma unroll
     for (int j = 0; j < QPK; ++j) {
         const uint16_t *qp = a.q + ((size_t)b * a.Hq + h * QPK + j) * D;
-        const uint2 lo = *reinterpret_cast<const uint2 *>(qp + ch);
-        const uint2 hi = *reinterpret_cast<const uint2 *>(qp + D / 2 + ch);
-        qlo[j][0] = f2(bf16lo(lo.x) * a.qscale, bf16hi(lo.x) * a.qscale);
-        qlo[j][1] = f2(bf16lo(lo.y) * a.qscale, bf16hi(lo.y) * a.qscale);
-        qhi[j][0] = f2(bf16lo(hi.x) * a.qscale, bf16hi(hi.x) * a.qscale);
-        qhi[j][1] = f2(bf16lo(hi.y) * a.qscale, bf16hi(hi.y) * a.qscale);
+        if constexpr (TQ) {
+            // q / w at the lane's permuted pairs (a pair's two channels share their weight)
+            const float *wp = a.tw + (size_t)h * D;
+            float ql[4], qh[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float sc = a.qscale / __ldg(wp + fq[k]);
+                ql[k] = bf16_to_f32(qp[fq[k]]) * sc;
+                qh[k] = bf16_to_f32(qp[D / 2 + fq[k]]) * sc;
+            }
+            qlo[j][0] = f2(ql[0], ql[1]);
+            qlo[j][1] = f2(ql[2], ql[3]);
+            qhi[j][0] = f2(qh[0], qh[1]);
+            qhi[j][1] = f2(qh[2], qh[3]);
+        } else {
+            const uint2 lo = *reinterpret_cast<const uint2 *>(qp + ch);
+            const uint2 hi = *reinterpret_cast<const uint2 *>(qp + D / 2 + ch);
+            qlo[j][0] = f2(bf16lo(lo.x) * a.qscale, bf16hi(lo.x) * a.qscale);
+            qlo[j][1] = f2(bf16lo(lo.y) * a.qscale, bf16hi(lo.y) * a.qscale);
+            qhi[j][0] = f2(bf16lo(hi.x) * a.qscale, bf16hi(hi.x) * a.qscale);
+            qhi[j][1] = f2(bf16lo(hi.y) * a.qscale, bf16hi(hi.y) * a.qscale);
+        }
     }
     // one-position rotation of this lane's 4 frequencies (RoPE table row 1)
     float2 c1[2], s1[2];
     {
-        const float4 cv = __ldg(reinterpret_cast<const float4 *>(a.rope + D + ch));
-        const float4 sv = __ldg(reinterpret_cast<const float4 *>(a.rope + D + D / 2 + ch));
+        float4 cv, sv;
+        load_row4(a.rope + D, cv, sv);
         c1[0] = f2(cv.x, cv.y);
         c1[1] = f2(cv.z, cv.w);
         s1[0] = f2(sv.x, sv.y);
@@ -303,9 +350,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     // RoPE row of each iteration's first token, loaded one iteration ahead
     float4 ra_c, ra_s;
     {
-        const float *row = a.rope + (size_t)min(pfirst, a.Nmax - 4) * D + ch;
-        ra_c = __ldg(reinterpret_cast<const float4 *>(row));
-        ra_s = __ldg(reinterpret_cast<const float4 *>(row + D / 2));
+        load_row4(a.rope + (size_t)min(pfirst, a.Nmax - 4) * D, ra_c, ra_s);
     }
     __syncthreads();
 
@@ -332,9 +377,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         float2 cs[2] = {f2(ra_c.x, ra_c.y), f2(ra_c.z, ra_c.w)};
         float2 sn[2] = {f2(ra_s.x, ra_s.y), f2(ra_s.z, ra_s.w)};
         {
-            const float *row = a.rope + (size_t)min(p0 + STRIDE, a.Nmax - 4) * D + ch;
-            ra_c = __ldg(reinterpret_cast<const float4 *>(row));
-            ra_s = __ldg(reinterpret_cast<const float4 *>(row + D / 2));
+            load_row4(a.rope + (size_t)min(p0 + STRIDE, a.Nmax - 4) * D, ra_c, ra_s);
         }
 
         // ---- values of the tile: gathered now and used after the softmax when registers allow
@@ -353,6 +396,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         // ---- keys: rebuild, score.  ROTQ: per pair f the term is Re(Z) k_f + Im(Z) k_{f+D/2} with
         // Z = (q_f + i q_{f+D/2}) e^{-i p w_f}, advanced along the tile (see the header).  Otherwise the
         // rebuilt keys are rotated by (cos, sin), advanced the same way, and shared by the query heads.
+        float sig = 1.f;                                   // TaSQ scale of the token this lane finishes
+        if constexpr (TQ) {
+            const int n = p0 + tk;
+            if (n < tok_end) sig = __half2float(__ushort_as_half(__ldg(a.tsig + (size_t)b * a.Nmax + n)));
+        }
         float ps[QPK][TT];
         float2 zu[2], zw[2], xu[2], xw[2];                // X_k and X_{k-1} of the advanced pair
         if constexpr (ROTQ) {
@@ -387,8 +435,20 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             const uint32_t w = word_k(w4[k >> 2], k & 3);
             const uint2 elo = lds64(smem, __byte_perm(w, colk_lo, 0x7604));
             const uint2 ehi = lds64(smem, __byte_perm(w, colk_hi, 0x7614));
-            const float2 kl[2] = {unpack2(elo.x), unpack2(elo.y)};
-            const float2 kh[2] = {unpack2(ehi.x), unpack2(ehi.y)};
+            // kl: low channels (real parts) of the lane's pairs, kh: their partners (imaginary parts)
+            float2 kl[2], kh[2];
+            if constexpr (TQ) {
+                // a TaSQ entry interleaves each pair's two channels: (f, f + D/2, f', f' + D/2)
+                kl[0] = f2(bf16lo(elo.x), bf16lo(elo.y));
+                kh[0] = f2(bf16hi(elo.x), bf16hi(elo.y));
+                kl[1] = f2(bf16lo(ehi.x), bf16lo(ehi.y));
+                kh[1] = f2(bf16hi(ehi.x), bf16hi(ehi.y));
+            } else {
+                kl[0] = unpack2(elo.x);
+                kl[1] = unpack2(elo.y);
+                kh[0] = unpack2(ehi.x);
+                kh[1] = unpack2(ehi.y);
+            }
             if constexpr (ROTQ) {
                 float2 acc = __fmul2_rn(zu[0], kl[0]);
                 acc = __ffma2_rn(zw[0], kh[0], acc);
@@ -417,7 +477,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         float pe[QPK];
 #pragma unroll
         for (int j = 0; j < QPK; ++j) {
-            const float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
+            float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
+            if constexpr (TQ) keep *= sig;
             const float s = (p0 + tk < tok_end && p0 + tk >= st) ? keep : -CUDART_INF_F;
             // Lazy maximum: the reference only has to stay within 2^8 of the running maximum for
             // the weights to stay finite, so it moves (with an exact rescale) only when a score of

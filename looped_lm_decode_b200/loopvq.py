@@ -24,7 +24,8 @@ EXPORTS = ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "l
            "loopvq_decode_attn_noalloc", "loopvq_noalloc_scratch_bytes", "loopvq_decode_attn_range",
            "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn", "loopvq_merge2",
            "loopvq_window_slots", "loopvq_window_advance", "loopvq_window_append",
-           "loopvq_window_workspace_bytes", "loopvq_window_decode_attn")
+           "loopvq_window_workspace_bytes", "loopvq_window_decode_attn", "loopvq_tasq_w_elems",
+           "loopvq_tasq_perm_elems", "loopvq_tasq_sigma_elems", "loopvq_tasq_encode", "loopvq_tasq_decode_attn")
 
 
 class CacheDesc(C.Structure):
@@ -47,6 +48,11 @@ class WindowDesc(C.Structure):
     _fields_ = [("L", C.c_int32), ("T", C.c_int32), ("B", C.c_int32), ("Hkv", C.c_int32), ("Hq", C.c_int32),
                 ("D", C.c_int32), ("n_sink", C.c_int32), ("n_recent", C.c_int32), ("k_rot", C.c_void_p),
                 ("k_pre", C.c_void_p), ("v", C.c_void_p), ("fill", C.c_void_p), ("coded_end", C.c_void_p)]
+
+
+class TasqDesc(C.Structure):
+    """Mirror of struct loopvq_tasq."""
+    _fields_ = [("w", C.c_void_p), ("perm", C.c_void_p), ("sigma", C.c_void_p)]
 
 
 class LoopVQError(RuntimeError):
@@ -98,6 +104,14 @@ def lib():
         L.loopvq_window_workspace_bytes.restype = sz
         L.loopvq_window_decode_attn.argtypes = [PW, P, i, i, vp, i, f, vp, vp, vp, sz, vp]
         L.loopvq_window_decode_attn.restype = i
+        PT = C.POINTER(TasqDesc)
+        for name in ("loopvq_tasq_w_elems", "loopvq_tasq_perm_elems", "loopvq_tasq_sigma_elems"):
+            getattr(L, name).argtypes = [P]
+            getattr(L, name).restype = sz
+        L.loopvq_tasq_encode.argtypes = [P, PT, i, i, vp, vp, i, C.POINTER(C.c_int64), i, i, i, i, vp]
+        L.loopvq_tasq_encode.restype = i
+        L.loopvq_tasq_decode_attn.argtypes = [P, PT, i, i, vp, vp, i, f, vp, vp, vp, sz, vp]
+        L.loopvq_tasq_decode_attn.restype = i
         L.loopvq_noalloc_scratch_bytes.argtypes = []
         L.loopvq_noalloc_scratch_bytes.restype = sz
         for name in ("loopvq_prepare", "loopvq_encode", "loopvq_decode_attn", "loopvq_dequant_debug"):
@@ -280,6 +294,55 @@ def merge2(out_a, lse_a, out_b, lse_b, out=None, lse=None, stream=None):
         lse = torch.empty_like(lse_a)
     _check(lib().loopvq_merge2(_ptr(out_a), _ptr(lse_a), _ptr(out_b), _ptr(lse_b), rows, D, _ptr(out), _ptr(lse),
                                _stream(stream)))
+    return out, lse
+
+
+class Tasq:
+    """TaSQ buffers of a cache (see include/loopvq.h): w fp32 [L][T][Hkv][D], perm int16 [L][NB][Hkv][D/2],
+    sigma fp16 [L][T][B][Nmax] (written by tasq_encode)."""
+
+    def __init__(self, cache: Cache, w=None, perm=None, device="cuda"):
+        L = lib()
+        nw, npm, ns = (L.loopvq_tasq_w_elems(cache.ref()), L.loopvq_tasq_perm_elems(cache.ref()),
+                       L.loopvq_tasq_sigma_elems(cache.ref()))
+        if nw == 0:
+            raise LoopVQError(LOOPVQ_ERR_UNSUPPORTED, "this cache cannot be used with TaSQ (ncb = 1, c in {4, 8})")
+        self.w = torch.ones(nw, dtype=torch.float32, device=device) if w is None else w.reshape(-1)
+        self.perm = (torch.arange(cache.D // 2, dtype=torch.int16, device=device).repeat(npm // (cache.D // 2))
+                     if perm is None else perm.reshape(-1))
+        self.sigma = torch.ones(ns, dtype=torch.float16, device=device)
+        self.desc = TasqDesc()
+
+    def ref(self):
+        self.desc.w, self.desc.perm, self.desc.sigma = self.w.data_ptr(), self.perm.data_ptr(), self.sigma.data_ptr()
+        return C.byref(self.desc)
+
+
+def tasq_encode(cache: Cache, tasq: Tasq, layer: int, block: int, xk, xv, b0: int = 0, tok0: int = 0, stream=None):
+    """encode() with TaSQ; xk, xv as for encode()."""
+    assert xk.shape == xv.shape and xk.stride() == xv.stride() and xk.dtype == xv.dtype
+    Tc, nb, ntok, Hkv, D = xk.shape
+    assert xk.stride(4) == 1
+    dt = {torch.bfloat16: LOOPVQ_BF16, torch.float32: LOOPVQ_FP32}[xk.dtype]
+    strides = (C.c_int64 * 4)(*xk.stride()[:4])
+    _check(lib().loopvq_tasq_encode(cache.ref(), tasq.ref(), layer, block, _ptr(xk), _ptr(xv), dt, strides, b0, nb,
+                                    tok0, ntok, _stream(stream)))
+
+
+def tasq_decode_attn(cache: Cache, tasq: Tasq, layer: int, t: int, q, lens, max_len: int, scale: float = 0.0,
+                     out=None, lse=None, workspace=None, stream=None):
+    B, Hq, D = cache.B, cache.Hq, cache.D
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    need = decode_workspace_bytes(cache, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().loopvq_tasq_decode_attn(cache.ref(), tasq.ref(), layer, t, _ptr(q), _ptr(lens), max_len, scale,
+                                         _ptr(out), _ptr(lse), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
 
 

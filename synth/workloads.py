@@ -47,7 +47,7 @@ from .philox import philox4x32, approx_normal_from_words, f32_to_bf16_bits, bf16
 SEED_BASE = 20261102
 KEY1 = 0x4C565142          # second key word, fixed
 
-TAG_K, TAG_V, TAG_Q, TAG_CBK, TAG_CBV, TAG_LEN, TAG_IDX = 1, 2, 3, 4, 5, 6, 7
+TAG_K, TAG_V, TAG_Q, TAG_CBK, TAG_CBV, TAG_LEN, TAG_IDX, TAG_TW, TAG_TP = 1, 2, 3, 4, 5, 6, 7, 8, 9
 
 
 @dataclasses.dataclass(frozen=True)
@@ -204,6 +204,35 @@ def lengths(w: Workload) -> np.ndarray:
     return (w.len_lo + (w0.astype(np.int64) % span)).astype(np.int32)
 
 
+def tasq_weights(w: Workload) -> np.ndarray:
+    """TaSQ channel weights fp32 [L][T][Hkv][D]: exp(0.25 n) for the low channel of each RoPE pair,
+    the same weight for its partner (a stand-in for calibrated query moments, which need a model)."""
+    L, T, H, h2 = w.L, w.T, w.Hkv, w.D // 2
+    out = np.empty((L, T, H, w.D), np.float32)
+    flat = np.arange(H * h2, dtype=np.uint64)
+    for layer in range(L):
+        for t in range(T):
+            n = _normal(w.seed, TAG_TW, layer, t, flat).reshape(H, h2)
+            half = np.exp(np.float32(0.25) * n.astype(np.float32)).astype(np.float32)
+            out[layer, t] = np.concatenate([half, half], axis=1)
+    return out
+
+
+def tasq_perm(w: Workload) -> np.ndarray:
+    """TaSQ low-channel orders int16 [L][NB][Hkv][D/2]: a seeded permutation per (layer, block, head)
+    (a stand-in for the covariance grouping, which needs real caches)."""
+    L, NB, H, h2 = w.L, w.NB, w.Hkv, w.D // 2
+    out = np.empty((L, NB, H, h2), np.int16)
+    for layer in range(L):
+        for blk in range(NB):
+            flat = np.arange(H * h2, dtype=np.uint64)
+            k0, _, _, _ = philox4x32(flat & np.uint64(0xFFFFFFFF), flat >> np.uint64(32), np.uint64(blk),
+                                     np.uint64((TAG_TP << 24) | layer), w.seed, KEY1)
+            keys = k0.reshape(H, h2).astype(np.uint64) * np.uint64(h2) + np.arange(h2, dtype=np.uint64)[None, :]
+            out[layer, blk] = np.argsort(keys, axis=1).astype(np.int16)
+    return out
+
+
 def random_indices(w: Workload, layer: int, block: int, kv: int, b: int, h: int, tok: Sequence[int]):
     """uint8 [len(tok)][D/c] code indices drawn uniformly in [0, K): decode input independent of any encoder."""
     ng = w.D // w.c
@@ -215,5 +244,5 @@ def random_indices(w: Workload, layer: int, block: int, kv: int, b: int, h: int,
     return (w0 % np.uint32(w.K)).astype(np.uint8)
 
 
-__all__ = ["Workload", "WORKLOADS", "kv_loops", "codebook", "codebooks", "queries", "lengths", "random_indices",
+__all__ = ["Workload", "WORKLOADS", "kv_loops", "codebook", "codebooks", "tasq_weights", "tasq_perm", "queries", "lengths", "random_indices",
            "rho_sigma_f32", "bf16_bits_to_f32", "f32_to_bf16_bits"]

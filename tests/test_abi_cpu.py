@@ -193,3 +193,33 @@ def test_per_group_codebook_sizes_and_validation():
     assert lib.loopvq_codebook_elems(cg.ref()) == 0
     assert lib.loopvq_prepare(cg.ref(), None) == 1
     assert b"ncb" in lib.loopvq_last_error()
+
+
+def test_tasq_sizes_and_validation_before_launch():
+    lib = LQ.lib()
+    c = _cache()
+    c.desc.idx = c.desc.slices = c.desc.rope = c.desc.codebook = 0x10000
+    c.ref = lambda: C.byref(c.desc)
+    assert lib.loopvq_tasq_w_elems(c.ref()) == 2 * 4 * 16 * 128
+    assert lib.loopvq_tasq_perm_elems(c.ref()) == 2 * 1 * 16 * 64
+    assert lib.loopvq_tasq_sigma_elems(c.ref()) == 2 * 4 * 8 * 1024
+    fake = C.c_void_p(0x20000)
+    t = LQ.TasqDesc(0x30000, 0x40000, 0x50000)
+    need = lib.loopvq_decode_workspace_bytes(c.ref(), 1024)
+    assert lib.loopvq_tasq_decode_attn(c.ref(), C.byref(t), 0, 4, fake, fake, 1024, 0.0, fake, None, fake, need,
+                                       None) == 1
+    assert lib.loopvq_tasq_decode_attn(c.ref(), None, 0, 0, fake, fake, 1024, 0.0, fake, None, fake, need, None) == 1
+    t.perm = 0x40001                                                       # misaligned int16 array
+    assert lib.loopvq_tasq_decode_attn(c.ref(), C.byref(t), 0, 0, fake, fake, 1024, 0.0, fake, None, fake, need,
+                                       None) == 1
+    assert b"misaligned" in lib.loopvq_last_error()
+    t.perm = 0x40000
+    strides = (C.c_int64 * 4)(1, 1, 1, 1)
+    assert lib.loopvq_tasq_encode(c.ref(), C.byref(t), 0, 1, fake, fake, 0, strides, 0, 1, 0, 4, None) == 1
+    assert b"block" in lib.loopvq_last_error()
+    c16 = _cache(c=16, Tc=1)
+    assert lib.loopvq_tasq_w_elems(c16.ref()) == 0
+    c16.desc.idx = c16.desc.slices = c16.desc.rope = c16.desc.codebook = 0x10000
+    c16.ref = lambda: C.byref(c16.desc)
+    assert lib.loopvq_tasq_decode_attn(c16.ref(), C.byref(t), 0, 0, fake, fake, 1024, 0.0, fake, None, fake, need,
+                                       None) == 2
