@@ -35,7 +35,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import WORKLOADS, lengths, random_indices, queries, bf16_bits_to_f32, codebook, codebooks  # noqa: E402
+from synth import (WORKLOADS, lengths, random_indices, queries, bf16_bits_to_f32, codebook, codebooks,  # noqa: E402
+                   tasq_weights, tasq_perm)
 
 METRIC = "LoopVQ decode-attn µs/step & GB/s at 32K ctx, 0.5 bit; % of roofline"
 SMEM_BYTES_PER_CLK_SM = 128
@@ -150,7 +151,7 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
                  "frac": bf_bytes / (bf_ms * 1e-3) / 1e9 / peak, "peak": peak, "peak_kind": kind,
                  "bytes_per_call": bf_bytes,
                  "kernel": "loopvq_bf16_decode_attn over a bf16 cache of the same shape (keys stored rotated)"}
-    if w.ncb > 1:                                     # the window's page encoder codes shared codebooks only
+    if w.ncb > 1 or w.tasq:                           # the window's page encoder codes plain, shared-codebook keys
         return {"bf16_cache": bf16_line, "windowed": None}
     n_sink, n_recent = 8, 64
     win = LQ.Window(cache, n_sink=n_sink, n_recent=n_recent, device=dev)
@@ -215,6 +216,7 @@ def workload_desc(w):
         "lengths": (f"uniform in [{w.len_lo}, {w.Nmax}] (seeded)" if w.len_lo >= 0 else "all full"),
         "layers": w.L, "loop_steps": w.T, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
         "codebooks": "shared by the channel groups" if w.ncb == 1 else f"one per channel group ({w.ncb})",
+        "keys": "TaSQ transform before coupling (seeded weights and pair orders)" if w.tasq else "plain",
         "bits_per_element": 8 / w.G,
         "l2": "inputs larger than L2: every call streams its layer's index words (> 126 MB), "
               "successive calls touch different layers",
@@ -295,6 +297,16 @@ def _cpu_inputs(w, layer, t, b, hq):
     return _CPU_INPUTS[key]
 
 
+_TASQ = {}
+
+
+def _tasq_params(w):
+    """Seeded TaSQ weights and pair orders of a workload (host copies)."""
+    if w.name not in _TASQ:
+        _TASQ[w.name] = (tasq_weights(w), tasq_perm(w))
+    return _TASQ[w.name]
+
+
 def _codebook(w, layer, blk, kv, h):
     """[K][G] bits of a shared codebook, [NCB][K][G] with one per channel group."""
     return codebook(w, layer, blk, kv, h) if w.ncb == 1 else codebooks(w, layer, blk, kv, h)
@@ -313,7 +325,12 @@ def cpu_sample(w, seconds, layer=0, t=1):
         n = int(lens[b])
         q, ik, iv, Ek, Ev = _cpu_inputs(w, layer, t, b, hq)
         t0 = time.perf_counter()
-        (O.decode_pg if w.ncb > 1 else O.decode)(q, ik, iv, Ek, Ev, w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        if w.tasq:
+            h = hq // (w.Hq // w.Hkv)
+            O.tasq_decode(q, ik, iv, Ek, Ev, _tasq_params(w)[1][layer, t // w.Tc, h], _tasq_params(w)[0][layer, t, h],
+                          np.ones(n), w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        else:
+            (O.decode_pg if w.ncb > 1 else O.decode)(q, ik, iv, Ek, Ev, w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
         total_s += time.perf_counter() - t0
         nbytes += n * 2 * (w.D // w.c)
         units += 1
@@ -377,6 +394,10 @@ def main():
     cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, device=dev, ncb=w.ncb)
     SG.fill_codebook(w, cache.codebook)
     LQ.prepare(cache)
+    tq = None
+    if w.tasq:
+        tw, tp = _tasq_params(w)
+        tq = LQ.Tasq(cache, w=torch.from_numpy(tw).to(dev), perm=torch.from_numpy(tp).to(dev), device=dev)
     xk = torch.empty((w.Tc, w.B, w.Nmax, w.Hkv, w.D), dtype=torch.bfloat16, device=dev)
     xv = torch.empty_like(xk)
     enc_ms = []
@@ -386,7 +407,10 @@ def main():
             SG.fill_kv(w, layer, 1, blk * w.Tc, blk * w.Tc + w.Tc - 1, xv)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            LQ.encode(cache, layer, blk, xk, xv)
+            if tq is not None:
+                LQ.tasq_encode(cache, tq, layer, blk, xk, xv)
+            else:
+                LQ.encode(cache, layer, blk, xk, xv)
             e1.record()
             torch.cuda.synchronize()
             enc_ms.append(e0.elapsed_time(e1))
@@ -412,8 +436,12 @@ def main():
                 i = t * w.L + layer
                 if evs is not None:
                     evs[2 * i].record(stream)
-                LQ.decode_attn(cache, layer, t, qs[i], lens, max_len, 0.0, out=out[i], lse=lse[i], workspace=ws,
-                               stream=stream)
+                if tq is not None:
+                    LQ.tasq_decode_attn(cache, tq, layer, t, qs[i], lens, max_len, 0.0, out=out[i], lse=lse[i],
+                                        workspace=ws, stream=stream)
+                else:
+                    LQ.decode_attn(cache, layer, t, qs[i], lens, max_len, 0.0, out=out[i], lse=lse[i], workspace=ws,
+                                   stream=stream)
                 if evs is not None:
                     evs[2 * i + 1].record(stream)
 
@@ -507,7 +535,9 @@ def main():
             "encode": {"ms_per_layer_block": statistics.median(enc_ms),
                        "tokens_per_s": w.B * w.Nmax / (statistics.median(enc_ms) * 1e-3),
                        "input_gbs": 2 * w.Tc * w.B * w.Nmax * w.Hkv * w.D * 2 / (statistics.median(enc_ms) * 1e-3) / 1e9,
-                       "kernel": ("encode_tc_kernel (tcgen05 bf16 distance contraction + TMEM arg-max)" if w.ncb == 1
+                       "kernel": ("tasq_sigma_kernel + tasq_encode_kernel (exact fp32 distances on CUDA cores)"
+                                  if w.tasq else
+                                  "encode_tc_kernel (tcgen05 bf16 distance contraction + TMEM arg-max)" if w.ncb == 1
                                   else "encode_pg_kernel (exact fp32 distances on CUDA cores, one codebook per "
                                        "channel group)")},
         }

@@ -13,6 +13,8 @@ Five workload shapes (all K = 256 codes, b = 8 bits):
              seed as ctx32k, so keys, values, queries and lengths are identical
   ctx32k_pg  ctx32k with one codebook per channel group (32 per head and K|V),
              the paper's notation; same seed as ctx32k
+  ctx32k_tasq  ctx32k with keys coded after the TaSQ transform (seeded weights
+             and pair permutations); same seed as ctx32k
 
 The model shapes follow the pages' Ouro-1.4B description (24 layers, 16 heads of
 dimension 128, 4 loop steps) and the deep-recurrence variant follows the
@@ -68,6 +70,7 @@ class Workload:
     len_lo: int = -1      # if >= 0, lengths uniform in [len_lo, Nmax]
     theta: float = 1.0e4
     ncb: int = 1          # codebooks per (layer, block, head, K|V): 1 shared, or D/c (one per channel group)
+    tasq: bool = False    # keys coded after the TaSQ transform (LoopVQ paper, App. B)
 
     @property
     def G(self) -> int:
@@ -107,6 +110,8 @@ WORKLOADS = {
                           rho=_rho((0.7, 0.8, 0.9), 4), len_lo=16384),
     "ctx32k_pg": Workload("ctx32k_pg", 2, L=24, T=4, Tc=4, Hkv=16, Hq=16, D=128, c=4, K=256, B=8, Nmax=32768,
                           rho=_rho((0.7, 0.8, 0.9), 4), len_lo=16384, ncb=32),
+    "ctx32k_tasq": Workload("ctx32k_tasq", 2, L=24, T=4, Tc=4, Hkv=16, Hq=16, D=128, c=4, K=256, B=8, Nmax=32768,
+                            rho=_rho((0.7, 0.8, 0.9), 4), len_lo=16384, tasq=True),
 }
 
 
