@@ -101,10 +101,43 @@ def profiled_traffic(workload_name):
     return prof["dram_bytes_read_per_launch"] + prof["dram_bytes_write_per_launch"]
 
 
+def graph_of(fn):
+    """A CUDA graph of fn(stream): one eager run first (so every kernel's attributes are set), then a
+    capture on a side stream.  Replaying it re-issues the same launches with no host work per call, as a
+    serving loop replays its decode step."""
+    import torch
+    cur = torch.cuda.current_stream()
+    fn(cur)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(cur)
+    with torch.cuda.graph(g, stream=cap):
+        fn(cap)
+    cur.wait_stream(cap)
+    torch.cuda.synchronize()
+    return g
+
+
+def replay_ms(g, reps, stream):
+    """Mean device time of one replay of g over reps back-to-back replays (CUDA events on `stream`)."""
+    import torch
+    g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
 def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
     """Same decode calls on a cache held entirely in bf16 (the pages' comparison, LoopVQ paper Sec. 5.3),
     and on the pages' serving layout: 8 sink + 64 recent tokens in a bf16 window, the rest coded, merged
-    through the log-sum-exps (Sec. 4.3 "Cache layout", "Attention").  Timed per call with CUDA events."""
+    through the log-sum-exps (Sec. 4.3 "Cache layout", "Attention").  Timed as CUDA graph replays with CUDA
+    events, like the coded calls."""
     import torch
     import looped_lm_decode_b200 as LQ
     from synth import gpu as SG
@@ -124,23 +157,14 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
     lse_b = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
 
     def timed(fn, calls):
-        for i in range(calls):
-            fn(i)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(reps * calls)]
-        torch.cuda.synchronize()
-        for r in range(reps):
+        def seq(st):
             for i in range(calls):
-                e0, e1 = evs[r * calls + i]
-                e0.record(stream)
-                fn(i)
-                e1.record(stream)
-        torch.cuda.synchronize()
-        return statistics.fmean(a.elapsed_time(b) for a, b in evs)
+                fn(i, st)
+        return replay_ms(graph_of(seq), reps, stream) / calls
 
     calls = w.T * nl
-    bf_ms = timed(lambda i: LQ.bf16_decode_attn(caches[i % nl], qs[i], lens, max_len, out=out_b, lse=lse_b,
-                                                workspace=ws_b, stream=stream), calls)
+    bf_ms = timed(lambda i, st: LQ.bf16_decode_attn(caches[i % nl], qs[i], lens, max_len, out=out_b, lse=lse_b,
+                                                    workspace=ws_b, stream=st), calls)
     bf_bytes = int(lens_np.astype(np.int64).sum()) * w.Hkv * 2 * w.D * 2 + w.B * w.Hq * (w.D * 2 + w.D * 4 + 4)
     del caches
 
@@ -167,34 +191,24 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
     ws_w = torch.empty(max(LQ.window_workspace_bytes(win, cache, w.Nmax), 16), dtype=torch.uint8, device=dev)
     out_c = torch.empty_like(out_b)
     lse_c = torch.empty_like(lse_b)
-    call_evs = []
-
-    def wstep(record):
-        LQ.window_advance(win, cache, stream=stream)
+    def wstep(st):
+        LQ.window_advance(win, cache, stream=st)
         for t in range(w.T):
             for layer in range(w.L):
                 i = t * w.L + layer
-                LQ.window_append(win, layer, t, tok[0], tok[1], tok[2], stream=stream)
-                if record:
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
+                LQ.window_append(win, layer, t, tok[0], tok[1], tok[2], stream=st)
                 LQ.window_decode_attn(win, cache, layer, t, qs[i], w.Nmax, out=out_c, lse=lse_c, workspace=ws_w,
-                                      stream=stream)
-                if record:
-                    e1.record(stream)
-                    call_evs.append((e0, e1))
+                                      stream=st)
 
-    wstep(False)
-    torch.cuda.synchronize()
+    def wcalls(st):                                   # the attention calls of a step alone
+        for t in range(w.T):
+            for layer in range(w.L):
+                LQ.window_decode_attn(win, cache, layer, t, qs[t * w.L + layer], w.Nmax, out=out_c, lse=lse_c,
+                                      workspace=ws_w, stream=st)
+
     nsteps = 16                                       # two page rolls for every sequence
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record(stream)
-    for _ in range(nsteps):
-        wstep(True)
-    s1.record(stream)
-    torch.cuda.synchronize()
-    win_step_ms = s0.elapsed_time(s1) / nsteps
-    win_call_ms = statistics.fmean(a.elapsed_time(b) for a, b in call_evs)
+    win_step_ms = replay_ms(graph_of(wstep), nsteps, stream)      # the window state lives on the device
+    win_call_ms = replay_ms(graph_of(wcalls), 2, stream) / (w.T * w.L)
     del win
 
     return {
@@ -430,20 +444,17 @@ def main():
     ws = torch.empty(LQ.decode_workspace_bytes(cache, max_len), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(evs=None):
+    def step(st=None):
+        st = stream if st is None else st
         for t in range(w.T):
             for layer in range(w.L):
                 i = t * w.L + layer
-                if evs is not None:
-                    evs[2 * i].record(stream)
                 if tq is not None:
                     LQ.tasq_decode_attn(cache, tq, layer, t, qs[i], lens, max_len, 0.0, out=out[i], lse=lse[i],
-                                        workspace=ws, stream=stream)
+                                        workspace=ws, stream=st)
                 else:
                     LQ.decode_attn(cache, layer, t, qs[i], lens, max_len, 0.0, out=out[i], lse=lse[i], workspace=ws,
-                                   stream=stream)
-                if evs is not None:
-                    evs[2 * i + 1].record(stream)
+                                   stream=st)
 
     def barrier():
         torch.cuda.synchronize()
@@ -453,7 +464,9 @@ def main():
 
     for _ in range(max(args.warmup, 3)):
         step()
-    call_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * ncall)] for _ in range(args.steps)]
+    graph = graph_of(step)                # the step's L x T calls as one CUDA graph
+    for _ in range(max(args.warmup, 3)):
+        graph.replay()
     clocks = Clocks(local)
     barrier()
     clocks.start()
@@ -461,14 +474,13 @@ def main():
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for k in range(args.steps):
-        step(call_evs[k])
+        graph.replay()
     t1.record(stream)
     barrier()
     clk = clocks.stop()
     ms_total = t0.elapsed_time(t1)
-    call_ms = [call_evs[k][2 * i].elapsed_time(call_evs[k][2 * i + 1])
-               for k in range(args.steps) for i in range(ncall)]
     ms_step_local = ms_total / args.steps
+    call_ms_local = ms_step_local / ncall  # one call = split kernel + merge kernel
 
     # ---------------- end to end through the public API with host buffers
     q_host = torch.empty(qs.shape, dtype=qs.dtype, pin_memory=True)
@@ -503,7 +515,7 @@ def main():
 
     ms_step = max_over_ranks(ms_step_local, dist, dev)
     e2e_ms = max_over_ranks(e2e_ms_local, dist, dev)
-    avg_call_ms = max_over_ranks(statistics.fmean(call_ms), dist, dev)
+    avg_call_ms = max_over_ranks(call_ms_local, dist, dev)
 
     if rank == 0:
         cb = call_bytes(w, lens_np)

@@ -2,6 +2,9 @@
 // Every entry point checks its arguments before launching anything and never
 // allocates or synchronises.
 #include <cmath>
+#include <map>
+#include <mutex>
+#include <utility>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -67,6 +70,21 @@ loopvq_status check_ptr(const void *p, const char *name) {
 
 namespace loopvq {
 void set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
+cudaError_t ensure_dynamic_smem(const void *kern, size_t bytes) {
+    if (bytes <= 48u * 1024u) return cudaSuccess;          // within the default limit
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> done;
+    std::lock_guard<std::mutex> lock(mu);
+    size_t &cur = done[{kern, dev}];
+    if (cur >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) cur = bytes;
+    return e;
+}
 }  // namespace loopvq
 
 extern "C" {

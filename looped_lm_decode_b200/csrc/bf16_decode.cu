@@ -251,6 +251,33 @@ __global__ void __launch_bounds__(D) merge2_kernel(const float *out_a, const flo
 
 // ------------------------------------------------------------------ host side
 
+// Log-sum-exp merge of the splits of every (sequence, query head).
+template <int D>
+__global__ void __launch_bounds__(D) bf16_merge_kernel(const Bf16Args a, float *out, float *lse) {
+    const int bh = blockIdx.x;
+    const int b = bh / a.Hq;
+    const int d = threadIdx.x;
+    const int len = min(max(a.lens[b], 0), a.max_len);
+    const int st = min(max(a.starts ? a.starts[b] : 0, 0), len);
+    const int span = len - (st & ~3);                      // tokens covered by the splits
+    const int ns = len > st ? (span + a.split_len - 1) / a.split_len : 0;
+    const float2 *ml = a.ws_ml + (size_t)bh * a.nsplit;
+    float mx = -CUDART_INF_F;
+    for (int sp = 0; sp < ns; ++sp) mx = fmaxf(mx, ml[sp].x);
+    float acc = 0.f, lsum = 0.f;
+    if (mx != -CUDART_INF_F) {
+        const float *o = a.ws_o + (size_t)bh * a.nsplit * D + d;
+        for (int sp = 0; sp < ns; ++sp) {
+            const float wgt = ex2(ml[sp].x - mx);
+            acc += o[(size_t)sp * D] * wgt;
+            lsum += ml[sp].y * wgt;
+        }
+    }
+    const bool any = (mx != -CUDART_INF_F) && lsum > 0.f;
+    out[(size_t)bh * D + d] = any ? acc / lsum : 0.f;
+    if (lse != nullptr && d == 0) lse[bh] = any ? (mx + log2f(lsum)) * 0.69314718055994530942f : -CUDART_INF_F;
+}
+
 static constexpr int kBfWarps = 8;
 static constexpr int kBfMinBlocks = 2;
 static constexpr int kBfDepth = 3;
@@ -277,29 +304,29 @@ DecodePlan plan_bf16(const loopvq_bf16_cache &c, int max_len) {
 }
 
 template <int D, int QPK>
-static cudaError_t launch_bf16_t(const Bf16Args &a, const DecodeArgs &m, cudaStream_t s) {
+static cudaError_t launch_bf16_t(const Bf16Args &a, float *out, float *lse, cudaStream_t s) {
     constexpr int NSLOT = kBfWarps * (32 / (D / 8));
     const size_t smem = bf16_smem_bytes();
     if ((size_t)NSLOT * QPK * (D + 4) * sizeof(float) > smem) return cudaErrorInvalidConfiguration;
     auto kern = bf16_split_kernel<D, QPK, kBfWarps, kBfMinBlocks, kBfDepth>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_dynamic_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     if (a.nsplit > 0) {
         kern<<<dim3(a.nsplit, a.Hkv, a.B), kBfWarps * 32, smem, s>>>(a);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    merge_kernel<D><<<a.B * a.Hq, D, 0, s>>>(m);
+    bf16_merge_kernel<D><<<a.B * a.Hq, D, 0, s>>>(a, out, lse);
     return cudaGetLastError();
 }
 
 template <int D>
-static cudaError_t dispatch_bf16(int qpk, const Bf16Args &a, const DecodeArgs &m, cudaStream_t s) {
+static cudaError_t dispatch_bf16(int qpk, const Bf16Args &a, float *out, float *lse, cudaStream_t s) {
     switch (qpk) {
-        case 1: return launch_bf16_t<D, 1>(a, m, s);
-        case 2: return launch_bf16_t<D, 2>(a, m, s);
-        case 4: return launch_bf16_t<D, 4>(a, m, s);
-        case 8: return launch_bf16_t<D, 8>(a, m, s);
+        case 1: return launch_bf16_t<D, 1>(a, out, lse, s);
+        case 2: return launch_bf16_t<D, 2>(a, out, lse, s);
+        case 4: return launch_bf16_t<D, 4>(a, out, lse, s);
+        case 8: return launch_bf16_t<D, 8>(a, out, lse, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -324,23 +351,9 @@ cudaError_t launch_bf16_decode(const loopvq_bf16_cache &c, const DecodePlan &pla
     a.split_len = plan.split_len;
     a.nsplit = plan.nsplit;
     a.qscale = scale * 1.44269504088896340736f;
-    // the merge reads the split partials through the coded path's argument block
-    DecodeArgs m{};
-    m.lens = lens;
-    m.starts = starts;
-    m.ws_o = a.ws_o;
-    m.ws_ml = a.ws_ml;
-    m.out = out;
-    m.lse = lse;
-    m.B = c.B;
-    m.Hkv = c.Hkv;
-    m.Hq = c.Hq;
-    m.max_len = max_len;
-    m.split_len = plan.split_len;
-    m.nsplit = plan.nsplit;
     const int qpk = c.Hq / c.Hkv;
-    if (c.D == 128) return dispatch_bf16<128>(qpk, a, m, s);
-    if (c.D == 64) return dispatch_bf16<64>(qpk, a, m, s);
+    if (c.D == 128) return dispatch_bf16<128>(qpk, a, out, lse, s);
+    if (c.D == 64) return dispatch_bf16<64>(qpk, a, out, lse, s);
     return cudaErrorInvalidValue;
 }
 

@@ -10,57 +10,62 @@ namespace loopvq {
 
 // ------------------------------------------------------------------ host side
 //
-// One CTA per (token split, KV head, sequence): 8 warps, two CTAs per SM (64 KB of codebook-slice
-// replicas plus a 16 KB prefetch queue each), splits sized for about six waves of resident CTAs.
+// Exactly one wave of resident CTAs shares the tile space evenly (decode_kernel.cuh): with a shared
+// codebook, two CTAs of 8 warps per SM (64 KiB of slice replicas plus a 2-deep prefetch queue each;
+// the shared memory left over serves as L1 for the RoPE rows); with one codebook per channel group,
+// one CTA of 16 warps per SM (128 KiB of tables).  Measured at ctx32k: a second wave, or three CTAs
+// per SM at 80 registers, is 3 to 10 % slower.
 
-static constexpr int kWarps = 8;
-static constexpr int kMinBlocks = 2;
-static constexpr int kDepth = 4;
-static constexpr int kWords = 1;                          // index words per lane per iteration (4-token tiles)
-static constexpr long kTargetCtas = 148L * 2 * 4;
-// one codebook per channel group: 128 KiB of tables, so one CTA of 16 warps per SM
-static constexpr int kPgWarps = 16;
-static constexpr int kPgMinBlocks = 1;
-static constexpr long kPgTargetCtas = 148L * 1 * 4;
+static constexpr int kSms = 148;                           // B200; more CTAs than fit only add a wave
+static constexpr int kWords = 1;                           // index words per lane per iteration (4-token tiles)
+static constexpr long kMinTiles = 128;                     // tiles per CTA below which fewer CTAs are used
 
-static size_t ring_smem_bytes(bool pg) {
-    return (pg ? 131072 : 65536) + (size_t)kDepth * (pg ? kPgWarps : kWarps) * 32 * 16 * kWords;
+struct KernelShape {
+    int warps, min_blocks, depth;
+};
+static constexpr KernelShape kernel_shape(bool pg, int qpk) {
+    return pg ? KernelShape{16, 1, 4} : KernelShape{8, 2, 2};
+}
+
+static size_t ring_smem_bytes(bool pg, int qpk) {
+    const KernelShape k = kernel_shape(pg, qpk);
+    return (pg ? 131072 : 65536) + (size_t)k.depth * k.warps * 32 * 16 * kWords;
 }
 
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len) {
     DecodePlan p{};
     const bool pg = ncb_of(cc) > 1;
-    const int warps = pg ? kPgWarps : kWarps;
-    const long target = pg ? kPgTargetCtas : kTargetCtas;
-    const int stride = 4 * kWords * warps * (32 / (cc.D / 8));   // tokens between two iterations of a slot
+    const int qpk = cc.Hq / cc.Hkv;
+    const KernelShape k = kernel_shape(pg, qpk);
     p.nbt = 1;
     p.nchunk = cc.B;
-    const long units = (long)cc.Hkv * cc.B;
-    long sl = max_len > 0 ? ((long)max_len * units + target - 1) / target : stride;
-    sl = ((sl + stride - 1) / stride) * stride;
-    if (sl < stride) sl = stride;
-    if (sl > 8192) sl = 8192;
-    p.split_len = (int)sl;
-    p.nsplit = max_len > 0 ? (int)((max_len + sl - 1) / sl) : 0;
-    const size_t o_bytes = (size_t)cc.B * cc.Hq * (size_t)p.nsplit * cc.D * sizeof(float);
-    const size_t ml_bytes = (size_t)cc.B * cc.Hq * (size_t)p.nsplit * sizeof(float2);
+    // an upper bound of the tiles: every sequence at max_len
+    const long tiles = (long)cc.B * cc.Hkv * ((max_len + 3) / 4);
+    long g = (tiles + kMinTiles - 1) / kMinTiles;
+    const long cap = (long)kSms * k.min_blocks;
+    if (g > cap) g = cap;
+    p.ncta = max_len > 0 ? (int)g : 0;
+    p.npiece = cc.B * cc.Hkv + p.ncta;
+    p.split_len = 0;
+    p.nsplit = p.ncta;
+    const size_t o_bytes = (size_t)p.npiece * qpk * cc.D * sizeof(float);
+    const size_t ml_bytes = (size_t)p.npiece * qpk * sizeof(float2);
     p.ws_bytes = ((o_bytes + 255) & ~(size_t)255) + ml_bytes;
     return p;
 }
 
 template <int D, int C, int QPK, bool PG, bool TQ = false>
 static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
-    constexpr int W = PG ? kPgWarps : kWarps;
-    constexpr int NSLOT = W * (32 / (D / 8));
+    constexpr KernelShape K = kernel_shape(PG, QPK);
+    constexpr int NSLOT = K.warps * (32 / (D / 8));
     const size_t red = (size_t)NSLOT * QPK * (D + 4) * sizeof(float);
-    const size_t smem = ring_smem_bytes(PG);
+    const size_t smem = ring_smem_bytes(PG, QPK);
     if (red > smem) return cudaErrorInvalidConfiguration;   // the slot records reuse slices and queue
-    auto kern = decode_split_kernel<D, C, QPK, W, PG ? kPgMinBlocks : kMinBlocks, kDepth, kWords, PG, TQ>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = decode_split_kernel<D, C, QPK, K.warps, K.min_blocks, K.depth, kWords, PG, TQ>;
+    cudaError_t e = ensure_dynamic_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
-    if (plan.nsplit > 0) {
-        dim3 grid(plan.nsplit, a.Hkv, a.B);
-        kern<<<grid, W * 32, smem, s>>>(a);
+    if (plan.ncta > 0) {
+        kern<<<plan.ncta, K.warps * 32, smem, s>>>(a);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -115,7 +120,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     a.lens = lens;
     a.starts = starts;
     a.start_all = start_all;
-    const size_t o_bytes = (size_t)cc.B * cc.Hq * (size_t)plan.nsplit * cc.D * sizeof(float);
+    const size_t o_bytes = (size_t)plan.npiece * (cc.Hq / cc.Hkv) * cc.D * sizeof(float);
     a.ws_o = reinterpret_cast<float *>(workspace);
     a.ws_ml = reinterpret_cast<float2 *>(reinterpret_cast<char *>(workspace) + ((o_bytes + 255) & ~(size_t)255));
     a.out = out;
@@ -126,8 +131,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     a.K = cc.K;
     a.Nmax = cc.Nmax;
     a.max_len = max_len;
-    a.split_len = plan.split_len;
-    a.nsplit = plan.nsplit;
+    a.ncta = plan.ncta;
     a.qscale = scale * 1.44269504088896340736f;
     const int qpk = cc.Hq / cc.Hkv;
     if (tq) {

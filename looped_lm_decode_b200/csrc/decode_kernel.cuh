@@ -52,11 +52,12 @@ struct DecodeArgs {
     const uint16_t *q;       // [B][Hq][D] bf16
     const int32_t *lens;     // [B]
     const int32_t *starts;   // [B] first attended token, or null for start_all
-    float *ws_o;             // [B][Hq][nsplit][D]  unnormalised split outputs
-    float2 *ws_ml;           // [B][Hq][nsplit]     (reference max, sum) in log2 units
+    float *ws_o;             // [piece][QPK][D]  unnormalised partial outputs, piece = segment + CTA
+    float2 *ws_ml;           // [piece][QPK]     (reference max, sum) in log2 units
     float *out;              // [B][Hq][D]
     float *lse;              // [B][Hq] or null
-    int B, Hkv, Hq, K, Nmax, max_len, split_len, nsplit;
+    int B, Hkv, Hq, K, Nmax, max_len;
+    int ncta;                // CTAs of the split kernel (its grid); the tile space is shared out evenly
     int start_all;           // first attended token of every sequence when starts is null
     const float *tw;         // TaSQ: channel weights of (layer, t) [Hkv][D]
     const int16_t *tperm;    // TaSQ: low-channel order of (layer, block) [Hkv][D/2]
@@ -148,6 +149,89 @@ __device__ __forceinline__ int tile_owner(int t) {          // a lane of the slo
     return l;
 }
 
+// ---- the tile space.  Sequence b attends tokens [st_b, len_b); they are covered by 4-token tiles
+// from st_b rounded down to a tile (the tile's earlier tokens are masked), so index-word loads stay
+// 16-byte aligned.  A segment is one (KV head h, sequence b), numbered s = h * B + b, and the tiles of
+// all segments are laid end to end in that order: T = Hkv * Tb tiles, Tb = sum over b of the tiles of
+// b.  CTA c of the G = ncta CTAs takes tiles [c T / G, (c + 1) T / G), so every CTA gets the same
+// number of tiles whatever the lengths.  The part of segment s inside CTA c is a piece; pieces follow
+// a staircase in which s and c never decrease, so s + c numbers them without collision, and the
+// pieces of segment s are those of the CTAs that hold its first through its last tile.
+__device__ __forceinline__ int seq_tiles(const DecodeArgs &a, int b, int &base, int &st, int &len) {
+    len = min(max(__ldg(a.lens + b), 0), a.max_len);
+    st = min(max(a.starts ? __ldg(a.starts + b) : a.start_all, 0), len);
+    base = st & ~3;
+    return len > st ? (len - base + 3) >> 2 : 0;
+}
+
+__device__ __forceinline__ long long warp_sum64(long long v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Tiles per KV head, Tb, and the tiles of the sequences before b, Pb(b) (one warp).
+__device__ __forceinline__ void head_tiles(const DecodeArgs &a, int lane, int b, long long &Tb, long long &Pb) {
+    Tb = 0;
+    Pb = 0;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+        const int bb = b0 + lane;
+        int base, st, len;
+        const long long t = bb < a.B ? seq_tiles(a, bb, base, st, len) : 0;
+        Tb += warp_sum64(t);
+        Pb += warp_sum64(bb < b ? t : 0);
+    }
+}
+
+// First tile of CTA c among T tiles shared by G CTAs.
+__device__ __forceinline__ long long cta_first_tile(long long c, long long T, long long G) { return c * T / G; }
+
+// The CTA that holds tile x: the largest c with floor(c T / G) <= x.
+__device__ __forceinline__ long long cta_of_tile(long long x, long long T, long long G) {
+    return ((x + 1) * G + T - 1) / T - 1;
+}
+
+// This CTA's tile range and the segment holding its first tile (one warp; lane 0 writes info):
+// info = {first tile, end tile, first tile of that segment, (h << 32) | b}.
+__device__ __forceinline__ void cta_range(const DecodeArgs &a, int lane, long long *info) {
+    long long Tb, unused;
+    head_tiles(a, lane, 0, Tb, unused);
+    const long long T = Tb * a.Hkv, G = a.ncta;
+    const long long x0 = cta_first_tile(blockIdx.x, T, G), x1 = cta_first_tile(blockIdx.x + 1, T, G);
+    long long seg0 = 0, hb = 0;
+    if (x0 < x1) {
+        const long long h0 = x0 / Tb, r = x0 - h0 * Tb;
+        long long carry = 0;
+        for (int b0 = 0; b0 < a.B; b0 += 32) {
+            const int bb = b0 + lane;
+            int base, st, len;
+            const long long t = bb < a.B ? seq_tiles(a, bb, base, st, len) : 0;
+            long long inc = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            inc += carry;
+            const unsigned hit = __ballot_sync(0xffffffffu, bb < a.B && inc > r);
+            if (hit) {
+                const int l = __ffs(hit) - 1;
+                const long long incl = __shfl_sync(0xffffffffu, inc, l), tl = __shfl_sync(0xffffffffu, t, l);
+                seg0 = h0 * Tb + incl - tl;
+                hb = (h0 << 32) | (long long)(b0 + l);
+                break;
+            }
+            carry = __shfl_sync(0xffffffffu, inc, 31);
+        }
+    }
+    if (lane == 0) {
+        info[0] = x0;
+        info[1] = x0 < x1 ? x1 : x0;
+        info[2] = seg0;
+        info[3] = hb;
+    }
+}
+
 // PG: one codebook per channel group.  The loop step's slice is then code-major with row r holding
 // entry r of every group's codebook (D bf16), so each lane reads its own channels of the row and the
 // 16 lanes of a token slot fall into distinct banks without replicas.  Tables: D = 128, K rows of 256 B
@@ -177,15 +261,14 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     static_assert(NL >= 8 && NL <= 16, "slot width");
 
     extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ long long range_info[4];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int len = min(max(__ldg(a.lens + b), 0), a.max_len);
-    // tokens [st, len) are attended; splits start from st rounded down to a 4-token tile, and the
-    // tokens of that tile before st are masked
-    const int st = min(max(a.starts ? __ldg(a.starts + b) : a.start_all, 0), len);
-    const int tok_begin = (st & ~3) + split * a.split_len;
-    if (tok_begin >= len) return;                          // the merge never reads this split
-    const int tok_end = min(tok_begin + a.split_len, len);
+    if (warp == 0) cta_range(a, lane, range_info);
+    __syncthreads();
+    long long pos = range_info[0];                         // next tile of this CTA
+    const long long x_end = range_info[1];
+    long long seg0 = range_info[2];                        // first tile of segment (h, b)
+    int h = (int)(range_info[3] >> 32), b = (int)(range_info[3] & 0xffffffffLL);
 
     const int ls = lane % NL;                              // lane within the slot
     const int gp = ls / HALVES;                            // pair-group
@@ -213,379 +296,420 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
         colv_hi = colk_hi + 128u;
     }
     const int ch = gp * C + half * 4;                      // first of this lane's 4 low channels
-    // low channels of the lane's 4 RoPE pairs: ch .. ch+3, or under TaSQ the pairs 2*half, 2*half + 1
-    // of TaSQ groups 2*gp (key code lo) and 2*gp + 1 (key code hi)
-    int fq[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        if constexpr (TQ) {
-            const int16_t *pm = a.tperm + (size_t)h * (D / 2);
-            fq[k] = __ldg(pm + (2 * gp + (k >> 1)) * (C / 2) + 2 * half + (k & 1)) & (D / 2 - 1);
-        } else {
-            fq[k] = ch + k;
-        }
-    }
-    // cos and sin of this lane's 4 frequencies in table row `row`
-    auto load_row4 = [&](const float *row, float4 &cv, float4 &sv) {
-        if constexpr (TQ) {
-            cv = make_float4(__ldg(row + fq[0]), __ldg(row + fq[1]), __ldg(row + fq[2]), __ldg(row + fq[3]));
-            sv = make_float4(__ldg(row + D / 2 + fq[0]), __ldg(row + D / 2 + fq[1]), __ldg(row + D / 2 + fq[2]),
-                             __ldg(row + D / 2 + fq[3]));
-        } else {
-            cv = __ldg(reinterpret_cast<const float4 *>(row + ch));
-            sv = __ldg(reinterpret_cast<const float4 *>(row + D / 2 + ch));
-        }
-    };
-    const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP + ((size_t)gp << 2);
-    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) + TBL + (uint32_t)tid * 16u;
 
-    // queue the first DEPTH iterations of this slot before staging the slices
-    const int pfirst = tok_begin + slot * TT;
-#pragma unroll
-    for (int d = 0; d < DEPTH; ++d) {
-        const int p = pfirst + d * STRIDE;
-#pragma unroll
-        for (int u = 0; u < NW; ++u)
-            if (p + 4 * u < tok_end)
-                cp_async16(ring + (uint32_t)(d * QB + u * NT * 16), idx_b + (size_t)((p >> 2) + u) * NP * 4);
-        cp_async_commit();
-    }
+    // the pieces of this CTA, segment by segment
+    while (pos < x_end && h < a.Hkv) {
+        int len, st, base;
+        const long long seg_end = seg0 + seq_tiles(a, b, base, st, len);
+        const long long pend = seg_end < x_end ? seg_end : x_end;
+        if (pend > pos) {
+            const int piece = h * a.B + b + (int)blockIdx.x;
+            // tokens [st, len) are attended; this piece covers the tiles [pos, pend) of the segment
+            const int tok_begin = base + 4 * (int)(pos - seg0);
+            const int tok_end = min(base + 4 * (int)(pend - seg0), len);
+            __syncthreads();                               // the previous piece's slot records have been read
 
-    if constexpr (!PG) {
-    // stage the K and V slices as bank-private replicas (rows >= K zeroed)
-    {
-        const uint16_t *sk = a.slk + (size_t)h * a.K * C;
-        const uint16_t *sv = a.slv + (size_t)h * a.K * C;
-        for (int it = tid; it < 256 * 2 * REPL; it += NT) {
-            const int rep = it % REPL;
-            const int kv = (it / REPL) & 1;
-            const int r = it / (2 * REPL);
-            unsigned char *dst = smem + r * 256 + kv * 128 + rep * EB;
-            const uint16_t *src = (kv ? sv : sk) + (size_t)r * C;
-            if constexpr (C == 4) {
-                uint2 v = make_uint2(0u, 0u);
-                if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(src));
-                *reinterpret_cast<uint2 *>(dst) = v;
-            } else {
-#pragma unroll
-                for (int u = 0; u < EB / 16; ++u) {
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (r < a.K) v = __ldg(reinterpret_cast<const uint4 *>(src) + u);
-                    *reinterpret_cast<uint4 *>(dst + 16 * u) = v;
-                }
-            }
-        }
-    }
-
-    } else {
-        // code-major per-group tables (rows >= K zeroed): 16-byte chunks of every row
-        constexpr int CH = D / 8;                          // chunks of one K (or V) row
-        const uint4 *sk = reinterpret_cast<const uint4 *>(a.slk + (size_t)h * a.K * D);
-        const uint4 *sv = reinterpret_cast<const uint4 *>(a.slv + (size_t)h * a.K * D);
-        for (int it = tid; it < 256 * 2 * CH; it += NT) {
-            const int j = it % CH;
-            const int kv = (it / CH) & 1;
-            const int r = it / (2 * CH);
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (r < a.K) v = __ldg((kv ? sv : sk) + (size_t)r * CH + j);
-            if constexpr (D == 128) {
-                *reinterpret_cast<uint4 *>(smem + kv * 65536 + r * 256 + j * 16) = v;
-            } else {
-                *reinterpret_cast<uint4 *>(smem + r * 256 + kv * 128 + j * 16) = v;
-                *reinterpret_cast<uint4 *>(smem + 65536 + r * 256 + kv * 128 + ((j * 16 + 64) & 127)) = v;
-            }
-        }
-    }
-
-    float2 qlo[QPK][2], qhi[QPK][2];
-#pragma unroll
-    for (int j = 0; j < QPK; ++j) {
-        const uint16_t *qp = a.q + ((size_t)b * a.Hq + h * QPK + j) * D;
-        if constexpr (TQ) {
-            // q / w at the lane's permuted pairs (a pair's two channels share their weight)
-            const float *wp = a.tw + (size_t)h * D;
-            float ql[4], qh[4];
-#pragma unroll
+            // low channels of the lane's 4 RoPE pairs: ch .. ch+3, or under TaSQ the pairs 2*half, 2*half + 1
+            // of TaSQ groups 2*gp (key code lo) and 2*gp + 1 (key code hi)
+            int fq[4];
+        #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const float sc = a.qscale / __ldg(wp + fq[k]);
-                ql[k] = bf16_to_f32(qp[fq[k]]) * sc;
-                qh[k] = bf16_to_f32(qp[D / 2 + fq[k]]) * sc;
+                if constexpr (TQ) {
+                    const int16_t *pm = a.tperm + (size_t)h * (D / 2);
+                    fq[k] = __ldg(pm + (2 * gp + (k >> 1)) * (C / 2) + 2 * half + (k & 1)) & (D / 2 - 1);
+                } else {
+                    fq[k] = ch + k;
+                }
             }
-            qlo[j][0] = f2(ql[0], ql[1]);
-            qlo[j][1] = f2(ql[2], ql[3]);
-            qhi[j][0] = f2(qh[0], qh[1]);
-            qhi[j][1] = f2(qh[2], qh[3]);
-        } else {
-            const uint2 lo = *reinterpret_cast<const uint2 *>(qp + ch);
-            const uint2 hi = *reinterpret_cast<const uint2 *>(qp + D / 2 + ch);
-            qlo[j][0] = f2(bf16lo(lo.x) * a.qscale, bf16hi(lo.x) * a.qscale);
-            qlo[j][1] = f2(bf16lo(lo.y) * a.qscale, bf16hi(lo.y) * a.qscale);
-            qhi[j][0] = f2(bf16lo(hi.x) * a.qscale, bf16hi(hi.x) * a.qscale);
-            qhi[j][1] = f2(bf16lo(hi.y) * a.qscale, bf16hi(hi.y) * a.qscale);
-        }
-    }
-    // one-position rotation of this lane's 4 frequencies (RoPE table row 1)
-    float2 c1[2], s1[2];
-    {
-        float4 cv, sv;
-        load_row4(a.rope + D, cv, sv);
-        c1[0] = f2(cv.x, cv.y);
-        c1[1] = f2(cv.z, cv.w);
-        s1[0] = f2(sv.x, sv.y);
-        s1[1] = f2(sv.z, sv.w);
-    }
-    const float2 ns1[2] = {neg2(s1[0]), neg2(s1[1])};
-    const float2 tc1[2] = {f2(2.f * c1[0].x, 2.f * c1[0].y), f2(2.f * c1[1].x, 2.f * c1[1].y)};   // 2 cos(w)
-    const float2 nqlo[2] = {neg2(qlo[0][0]), neg2(qlo[0][1])};
-    float m_[QPK], l_[QPK];
-    float2 olo[QPK][2], ohi[QPK][2];
-#pragma unroll
-    for (int j = 0; j < QPK; ++j) {
-        m_[j] = -CUDART_INF_F;
-        l_[j] = 0.f;
-        olo[j][0] = olo[j][1] = ohi[j][0] = ohi[j][1] = f2(0.f, 0.f);
-    }
-    const int tk = tile_token<TT, NL>(ls);                 // token of the iteration this lane finishes
+            // cos and sin of this lane's 4 frequencies in table row `row`
+            auto load_row4 = [&](const float *row, float4 &cv, float4 &sv) {
+                if constexpr (TQ) {
+                    cv = make_float4(__ldg(row + fq[0]), __ldg(row + fq[1]), __ldg(row + fq[2]), __ldg(row + fq[3]));
+                    sv = make_float4(__ldg(row + D / 2 + fq[0]), __ldg(row + D / 2 + fq[1]), __ldg(row + D / 2 + fq[2]),
+                                     __ldg(row + D / 2 + fq[3]));
+                } else {
+                    cv = __ldg(reinterpret_cast<const float4 *>(row + ch));
+                    sv = __ldg(reinterpret_cast<const float4 *>(row + D / 2 + ch));
+                }
+            };
+            const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP + ((size_t)gp << 2);
+            const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) + TBL + (uint32_t)tid * 16u;
 
-    // RoPE row of each iteration's first token, loaded one iteration ahead
-    float4 ra_c, ra_s;
-    {
-        load_row4(a.rope + (size_t)min(pfirst, a.Nmax - 4) * D, ra_c, ra_s);
-    }
-    __syncthreads();
-
-    int stage = 0;
-    for (int p0 = pfirst; p0 < tok_end; p0 += STRIDE) {
-        cp_async_wait<DEPTH - 1>();                        // this thread's oldest queued stage has landed
-        uint4 w4[NW];
-#pragma unroll
-        for (int u = 0; u < NW; ++u) {
-            const uint32_t addr = ring + (uint32_t)(stage * QB + u * NT * 16);
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w4[u].x), "=r"(w4[u].y), "=r"(w4[u].z), "=r"(w4[u].w) : "r"(addr) : "memory");
-        }
-        // the stage has been read into registers: queue the iteration DEPTH steps ahead into it
-        {
-            const int pq = p0 + DEPTH * STRIDE;
-#pragma unroll
-            for (int u = 0; u < NW; ++u)
-                if (pq + 4 * u < tok_end)
-                    cp_async16(ring + (uint32_t)(stage * QB + u * NT * 16), idx_b + (size_t)((pq >> 2) + u) * NP * 4);
-            cp_async_commit();
-            stage = stage + 1 == DEPTH ? 0 : stage + 1;
-        }
-        float2 cs[2] = {f2(ra_c.x, ra_c.y), f2(ra_c.z, ra_c.w)};
-        float2 sn[2] = {f2(ra_s.x, ra_s.y), f2(ra_s.z, ra_s.w)};
-        {
-            load_row4(a.rope + (size_t)min(p0 + STRIDE, a.Nmax - 4) * D, ra_c, ra_s);
-        }
-
-        // ---- values of the tile: gathered now and used after the softmax when registers allow
-        // (one or two query heads per KV head); otherwise gathered in the value loop
-        constexpr bool VEARLY = QPK <= 2;
-        uint2 vraw[TT][2];
-        if constexpr (VEARLY) {
-#pragma unroll
-            for (int k = 0; k < TT; ++k) {
-                const uint32_t w = word_k(w4[k >> 2], k & 3);
-                vraw[k][0] = lds64(smem, __byte_perm(w, colv_lo, 0x7624));
-                vraw[k][1] = lds64(smem, __byte_perm(w, colv_hi, 0x7634));
+            // queue the first DEPTH iterations of this slot before staging the slices
+            const int pfirst = tok_begin + slot * TT;
+        #pragma unroll
+            for (int d = 0; d < DEPTH; ++d) {
+                const int p = pfirst + d * STRIDE;
+        #pragma unroll
+                for (int u = 0; u < NW; ++u)
+                    if (p + 4 * u < tok_end)
+                        cp_async16(ring + (uint32_t)(d * QB + u * NT * 16), idx_b + (size_t)((p >> 2) + u) * NP * 4);
+                cp_async_commit();
             }
-        }
 
-        // ---- keys: rebuild, score.  ROTQ: per pair f the term is Re(Z) k_f + Im(Z) k_{f+D/2} with
-        // Z = (q_f + i q_{f+D/2}) e^{-i p w_f}, advanced along the tile (see the header).  Otherwise the
-        // rebuilt keys are rotated by (cos, sin), advanced the same way, and shared by the query heads.
-        float sig = 1.f;                                   // TaSQ scale of the token this lane finishes
-        if constexpr (TQ) {
-            const int n = p0 + tk;
-            if (n < tok_end) sig = __half2float(__ushort_as_half(__ldg(a.tsig + (size_t)b * a.Nmax + n)));
-        }
-        float ps[QPK][TT];
-        float2 zu[2], zw[2], xu[2], xw[2];                // X_k and X_{k-1} of the advanced pair
-        if constexpr (ROTQ) {
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                zu[i] = __ffma2_rn(qlo[0][i], cs[i], __fmul2_rn(qhi[0][i], sn[i]));
-                zw[i] = __ffma2_rn(qhi[0][i], cs[i], __fmul2_rn(nqlo[i], sn[i]));
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < TT; ++k) {
-            if (k > 0) {
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    // the pair (re, im) advanced by one position: ROTQ by e^{-iw}, else by e^{+iw}
-                    float2 &re = ROTQ ? zu[i] : cs[i];
-                    float2 &im = ROTQ ? zw[i] : sn[i];
-                    float2 nre, nim;
-                    if (k == 1) {
-                        nre = ROTQ ? __ffma2_rn(re, c1[i], __fmul2_rn(im, s1[i])) : __ffma2_rn(re, c1[i], __fmul2_rn(im, ns1[i]));
-                        nim = ROTQ ? __ffma2_rn(im, c1[i], __fmul2_rn(re, ns1[i])) : __ffma2_rn(im, c1[i], __fmul2_rn(re, s1[i]));
+            if constexpr (!PG) {
+            // stage the K and V slices as bank-private replicas (rows >= K zeroed)
+            {
+                const uint16_t *sk = a.slk + (size_t)h * a.K * C;
+                const uint16_t *sv = a.slv + (size_t)h * a.K * C;
+                for (int it = tid; it < 256 * 2 * REPL; it += NT) {
+                    const int rep = it % REPL;
+                    const int kv = (it / REPL) & 1;
+                    const int r = it / (2 * REPL);
+                    unsigned char *dst = smem + r * 256 + kv * 128 + rep * EB;
+                    const uint16_t *src = (kv ? sv : sk) + (size_t)r * C;
+                    if constexpr (C == 4) {
+                        uint2 v = make_uint2(0u, 0u);
+                        if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(src));
+                        *reinterpret_cast<uint2 *>(dst) = v;
                     } else {
-                        nre = __ffma2_rn(tc1[i], re, neg2(xu[i]));
-                        nim = __ffma2_rn(tc1[i], im, neg2(xw[i]));
+        #pragma unroll
+                        for (int u = 0; u < EB / 16; ++u) {
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (r < a.K) v = __ldg(reinterpret_cast<const uint4 *>(src) + u);
+                            *reinterpret_cast<uint4 *>(dst + 16 * u) = v;
+                        }
                     }
-                    xu[i] = re;
-                    xw[i] = im;
-                    re = nre;
-                    im = nim;
                 }
             }
-            const uint32_t w = word_k(w4[k >> 2], k & 3);
-            const uint2 elo = lds64(smem, __byte_perm(w, colk_lo, 0x7604));
-            const uint2 ehi = lds64(smem, __byte_perm(w, colk_hi, 0x7614));
-            // kl: low channels (real parts) of the lane's pairs, kh: their partners (imaginary parts)
-            float2 kl[2], kh[2];
-            if constexpr (TQ) {
-                // a TaSQ entry interleaves each pair's two channels: (f, f + D/2, f', f' + D/2)
-                kl[0] = f2(bf16lo(elo.x), bf16lo(elo.y));
-                kh[0] = f2(bf16hi(elo.x), bf16hi(elo.y));
-                kl[1] = f2(bf16lo(ehi.x), bf16lo(ehi.y));
-                kh[1] = f2(bf16hi(ehi.x), bf16hi(ehi.y));
-            } else {
-                kl[0] = unpack2(elo.x);
-                kl[1] = unpack2(elo.y);
-                kh[0] = unpack2(ehi.x);
-                kh[1] = unpack2(ehi.y);
-            }
-            if constexpr (ROTQ) {
-                float2 acc = __fmul2_rn(zu[0], kl[0]);
-                acc = __ffma2_rn(zw[0], kh[0], acc);
-                acc = __ffma2_rn(zu[1], kl[1], acc);
-                acc = __ffma2_rn(zw[1], kh[1], acc);
-                ps[0][k] = acc.x + acc.y;
-            } else {
-                float2 rlo[2], rhi[2];
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    rlo[i] = __ffma2_rn(kl[i], cs[i], __fmul2_rn(kh[i], neg2(sn[i])));   // kl*cos - kh*sin
-                    rhi[i] = __ffma2_rn(kh[i], cs[i], __fmul2_rn(kl[i], sn[i]));         // kh*cos + kl*sin
-                }
-#pragma unroll
-                for (int j = 0; j < QPK; ++j) {
-                    float2 acc = __fmul2_rn(qlo[j][0], rlo[0]);
-                    acc = __ffma2_rn(qhi[j][0], rhi[0], acc);
-                    acc = __ffma2_rn(qlo[j][1], rlo[1], acc);
-                    acc = __ffma2_rn(qhi[j][1], rhi[1], acc);
-                    ps[j][k] = acc.x + acc.y;
-                }
-            }
-        }
 
-        // ---- reduce-scatter the scores over the slot, online-softmax update
-        float pe[QPK];
-#pragma unroll
-        for (int j = 0; j < QPK; ++j) {
-            float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
-            if constexpr (TQ) keep *= sig;
-            const float s = (p0 + tk < tok_end && p0 + tk >= st) ? keep : -CUDART_INF_F;
-            // Lazy maximum: the reference only has to stay within 2^8 of the running maximum for
-            // the weights to stay finite, so it moves (with an exact rescale) only when a score of
-            // the iteration exceeds it by more than 8 in log2 units.
-            if (__any_sync(slot_mask, s > m_[j] + 8.f)) {
-                float tmax = s;
-#pragma unroll
-                for (int o = NL / 2; o >= NL / TT; o >>= 1)
-                    tmax = fmaxf(tmax, __shfl_xor_sync(slot_mask, tmax, o));
-                const float corr = ex2(m_[j] - tmax);
-                l_[j] *= corr;
-                const float2 c2 = f2(corr, corr);
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    olo[j][i] = __fmul2_rn(olo[j][i], c2);
-                    ohi[j][i] = __fmul2_rn(ohi[j][i], c2);
+            } else {
+                // code-major per-group tables (rows >= K zeroed): 16-byte chunks of every row
+                constexpr int CH = D / 8;                          // chunks of one K (or V) row
+                const uint4 *sk = reinterpret_cast<const uint4 *>(a.slk + (size_t)h * a.K * D);
+                const uint4 *sv = reinterpret_cast<const uint4 *>(a.slv + (size_t)h * a.K * D);
+                for (int it = tid; it < 256 * 2 * CH; it += NT) {
+                    const int j = it % CH;
+                    const int kv = (it / CH) & 1;
+                    const int r = it / (2 * CH);
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < a.K) v = __ldg((kv ? sv : sk) + (size_t)r * CH + j);
+                    if constexpr (D == 128) {
+                        *reinterpret_cast<uint4 *>(smem + kv * 65536 + r * 256 + j * 16) = v;
+                    } else {
+                        *reinterpret_cast<uint4 *>(smem + r * 256 + kv * 128 + j * 16) = v;
+                        *reinterpret_cast<uint4 *>(smem + 65536 + r * 256 + kv * 128 + ((j * 16 + 64) & 127)) = v;
+                    }
                 }
-                m_[j] = tmax;
             }
-            pe[j] = ex2(s - m_[j]);
-            l_[j] += pe[j];
-        }
 
-        // ---- values: rebuild and accumulate with each token's weight
-#pragma unroll
-        for (int k = 0; k < TT; ++k) {
-            const int src = slot_lane0 + tile_owner<TT, NL>(k);
-            if constexpr (!VEARLY) {
-                const uint32_t w = word_k(w4[k >> 2], k & 3);
-                vraw[k][0] = lds64(smem, __byte_perm(w, colv_lo, 0x7624));
-                vraw[k][1] = lds64(smem, __byte_perm(w, colv_hi, 0x7634));
-            }
-            const uint32_t vl[2] = {vraw[k][0].x, vraw[k][0].y}, vh[2] = {vraw[k][1].x, vraw[k][1].y};
-#pragma unroll
+            float2 qlo[QPK][2], qhi[QPK][2];
+        #pragma unroll
             for (int j = 0; j < QPK; ++j) {
-                const float pk = __shfl_sync(slot_mask, pe[j], src);
-                const float2 p2 = f2(pk, pk);
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    olo[j][i] = __ffma2_rn(p2, unpack2(vl[i]), olo[j][i]);
-                    ohi[j][i] = __ffma2_rn(p2, unpack2(vh[i]), ohi[j][i]);
+                const uint16_t *qp = a.q + ((size_t)b * a.Hq + h * QPK + j) * D;
+                if constexpr (TQ) {
+                    // q / w at the lane's permuted pairs (a pair's two channels share their weight)
+                    const float *wp = a.tw + (size_t)h * D;
+                    float ql[4], qh[4];
+        #pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float sc = a.qscale / __ldg(wp + fq[k]);
+                        ql[k] = bf16_to_f32(qp[fq[k]]) * sc;
+                        qh[k] = bf16_to_f32(qp[D / 2 + fq[k]]) * sc;
+                    }
+                    qlo[j][0] = f2(ql[0], ql[1]);
+                    qlo[j][1] = f2(ql[2], ql[3]);
+                    qhi[j][0] = f2(qh[0], qh[1]);
+                    qhi[j][1] = f2(qh[2], qh[3]);
+                } else {
+                    const uint2 lo = *reinterpret_cast<const uint2 *>(qp + ch);
+                    const uint2 hi = *reinterpret_cast<const uint2 *>(qp + D / 2 + ch);
+                    qlo[j][0] = f2(bf16lo(lo.x) * a.qscale, bf16hi(lo.x) * a.qscale);
+                    qlo[j][1] = f2(bf16lo(lo.y) * a.qscale, bf16hi(lo.y) * a.qscale);
+                    qhi[j][0] = f2(bf16lo(hi.x) * a.qscale, bf16hi(hi.x) * a.qscale);
+                    qhi[j][1] = f2(bf16lo(hi.y) * a.qscale, bf16hi(hi.y) * a.qscale);
                 }
             }
-        }
-    }
-    cp_async_wait<0>();
-
-    // ---- combine the slots of this CTA, write the split's partial result
-    __syncthreads();                                       // slices and queue no longer needed
-    constexpr int RS = D + 4;                              // floats per (slot, query head) record
-    // l_ sums the weights of the tokens this lane finished: add the other token positions of the slot
-    constexpr int TOKBITS = (TT == 8) ? 3 : 2;
-    float *red = reinterpret_cast<float *>(smem);
-#pragma unroll
-    for (int j = 0; j < QPK; ++j) {
-        float lsum = l_[j];
-#pragma unroll
-        for (int sb = 0; sb < TOKBITS; ++sb) lsum += __shfl_xor_sync(slot_mask, lsum, NL >> (1 + sb));
-        float *rec = red + ((size_t)slot * QPK + j) * RS;
-        *reinterpret_cast<float4 *>(rec + ch) = make_float4(olo[j][0].x, olo[j][0].y, olo[j][1].x, olo[j][1].y);
-        *reinterpret_cast<float4 *>(rec + D / 2 + ch) = make_float4(ohi[j][0].x, ohi[j][0].y, ohi[j][1].x, ohi[j][1].y);
-        if (ls == 0) {
-            rec[D] = m_[j];
-            rec[D + 1] = lsum;
-        }
-    }
-    __syncthreads();
-    for (int it = tid; it < QPK * D; it += NT) {
-        const int d = it % D;
-        const int j = it / D;
-        float mx = -CUDART_INF_F;
-        for (int s2 = 0; s2 < NSLOT; ++s2) mx = fmaxf(mx, red[((size_t)s2 * QPK + j) * RS + D]);
-        float acc = 0.f, lsum = 0.f;
-        if (mx != -CUDART_INF_F) {
-            for (int s2 = 0; s2 < NSLOT; ++s2) {
-                const float *rec = red + ((size_t)s2 * QPK + j) * RS;
-                const float wgt = ex2(rec[D] - mx);
-                acc += rec[d] * wgt;
-                lsum += rec[D + 1] * wgt;
+            // one-position rotation of this lane's 4 frequencies (RoPE table row 1)
+            float2 c1[2], s1[2];
+            {
+                float4 cv, sv;
+                load_row4(a.rope + D, cv, sv);
+                c1[0] = f2(cv.x, cv.y);
+                c1[1] = f2(cv.z, cv.w);
+                s1[0] = f2(sv.x, sv.y);
+                s1[1] = f2(sv.z, sv.w);
             }
+            const float2 ns1[2] = {neg2(s1[0]), neg2(s1[1])};
+            const float2 tc1[2] = {f2(2.f * c1[0].x, 2.f * c1[0].y), f2(2.f * c1[1].x, 2.f * c1[1].y)};   // 2 cos(w)
+            const float2 nqlo[2] = {neg2(qlo[0][0]), neg2(qlo[0][1])};
+            float m_[QPK], l_[QPK];
+            float2 olo[QPK][2], ohi[QPK][2];
+        #pragma unroll
+            for (int j = 0; j < QPK; ++j) {
+                m_[j] = -CUDART_INF_F;
+                l_[j] = 0.f;
+                olo[j][0] = olo[j][1] = ohi[j][0] = ohi[j][1] = f2(0.f, 0.f);
+            }
+            const int tk = tile_token<TT, NL>(ls);                 // token of the iteration this lane finishes
+
+            // RoPE row of each iteration's first token, loaded one iteration ahead
+            float4 ra_c, ra_s;
+            {
+                load_row4(a.rope + (size_t)min(pfirst, a.Nmax - 4) * D, ra_c, ra_s);
+            }
+            __syncthreads();
+
+            int stage = 0;
+            for (int p0 = pfirst; p0 < tok_end; p0 += STRIDE) {
+                cp_async_wait<DEPTH - 1>();                        // this thread's oldest queued stage has landed
+                uint4 w4[NW];
+        #pragma unroll
+                for (int u = 0; u < NW; ++u) {
+                    const uint32_t addr = ring + (uint32_t)(stage * QB + u * NT * 16);
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w4[u].x), "=r"(w4[u].y), "=r"(w4[u].z), "=r"(w4[u].w) : "r"(addr) : "memory");
+                }
+                // the stage has been read into registers: queue the iteration DEPTH steps ahead into it
+                {
+                    const int pq = p0 + DEPTH * STRIDE;
+        #pragma unroll
+                    for (int u = 0; u < NW; ++u)
+                        if (pq + 4 * u < tok_end)
+                            cp_async16(ring + (uint32_t)(stage * QB + u * NT * 16), idx_b + (size_t)((pq >> 2) + u) * NP * 4);
+                    cp_async_commit();
+                    stage = stage + 1 == DEPTH ? 0 : stage + 1;
+                }
+                float2 cs[2] = {f2(ra_c.x, ra_c.y), f2(ra_c.z, ra_c.w)};
+                float2 sn[2] = {f2(ra_s.x, ra_s.y), f2(ra_s.z, ra_s.w)};
+                {
+                    load_row4(a.rope + (size_t)min(p0 + STRIDE, a.Nmax - 4) * D, ra_c, ra_s);
+                }
+
+                // ---- values of the tile: gathered now and used after the softmax when registers allow
+                // (one or two query heads per KV head); otherwise gathered in the value loop
+                constexpr bool VEARLY = QPK <= 2;
+                uint2 vraw[TT][2];
+                if constexpr (VEARLY) {
+        #pragma unroll
+                    for (int k = 0; k < TT; ++k) {
+                        const uint32_t w = word_k(w4[k >> 2], k & 3);
+                        vraw[k][0] = lds64(smem, __byte_perm(w, colv_lo, 0x7624));
+                        vraw[k][1] = lds64(smem, __byte_perm(w, colv_hi, 0x7634));
+                    }
+                }
+
+                // ---- keys: rebuild, score.  ROTQ: per pair f the term is Re(Z) k_f + Im(Z) k_{f+D/2} with
+                // Z = (q_f + i q_{f+D/2}) e^{-i p w_f}, advanced along the tile (see the header).  Otherwise the
+                // rebuilt keys are rotated by (cos, sin), advanced the same way, and shared by the query heads.
+                float sig = 1.f;                                   // TaSQ scale of the token this lane finishes
+                if constexpr (TQ) {
+                    const int n = p0 + tk;
+                    if (n < tok_end) sig = __half2float(__ushort_as_half(__ldg(a.tsig + (size_t)b * a.Nmax + n)));
+                }
+                float ps[QPK][TT];
+                float2 zu[2], zw[2], xu[2], xw[2];                // X_k and X_{k-1} of the advanced pair
+                if constexpr (ROTQ) {
+        #pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        zu[i] = __ffma2_rn(qlo[0][i], cs[i], __fmul2_rn(qhi[0][i], sn[i]));
+                        zw[i] = __ffma2_rn(qhi[0][i], cs[i], __fmul2_rn(nqlo[i], sn[i]));
+                    }
+                }
+        #pragma unroll
+                for (int k = 0; k < TT; ++k) {
+                    if (k > 0) {
+        #pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            // the pair (re, im) advanced by one position: ROTQ by e^{-iw}, else by e^{+iw}
+                            float2 &re = ROTQ ? zu[i] : cs[i];
+                            float2 &im = ROTQ ? zw[i] : sn[i];
+                            float2 nre, nim;
+                            if (k == 1) {
+                                nre = ROTQ ? __ffma2_rn(re, c1[i], __fmul2_rn(im, s1[i])) : __ffma2_rn(re, c1[i], __fmul2_rn(im, ns1[i]));
+                                nim = ROTQ ? __ffma2_rn(im, c1[i], __fmul2_rn(re, ns1[i])) : __ffma2_rn(im, c1[i], __fmul2_rn(re, s1[i]));
+                            } else {
+                                nre = __ffma2_rn(tc1[i], re, neg2(xu[i]));
+                                nim = __ffma2_rn(tc1[i], im, neg2(xw[i]));
+                            }
+                            xu[i] = re;
+                            xw[i] = im;
+                            re = nre;
+                            im = nim;
+                        }
+                    }
+                    const uint32_t w = word_k(w4[k >> 2], k & 3);
+                    const uint2 elo = lds64(smem, __byte_perm(w, colk_lo, 0x7604));
+                    const uint2 ehi = lds64(smem, __byte_perm(w, colk_hi, 0x7614));
+                    // kl: low channels (real parts) of the lane's pairs, kh: their partners (imaginary parts)
+                    float2 kl[2], kh[2];
+                    if constexpr (TQ) {
+                        // a TaSQ entry interleaves each pair's two channels: (f, f + D/2, f', f' + D/2)
+                        kl[0] = f2(bf16lo(elo.x), bf16lo(elo.y));
+                        kh[0] = f2(bf16hi(elo.x), bf16hi(elo.y));
+                        kl[1] = f2(bf16lo(ehi.x), bf16lo(ehi.y));
+                        kh[1] = f2(bf16hi(ehi.x), bf16hi(ehi.y));
+                    } else {
+                        kl[0] = unpack2(elo.x);
+                        kl[1] = unpack2(elo.y);
+                        kh[0] = unpack2(ehi.x);
+                        kh[1] = unpack2(ehi.y);
+                    }
+                    if constexpr (ROTQ) {
+                        float2 acc = __fmul2_rn(zu[0], kl[0]);
+                        acc = __ffma2_rn(zw[0], kh[0], acc);
+                        acc = __ffma2_rn(zu[1], kl[1], acc);
+                        acc = __ffma2_rn(zw[1], kh[1], acc);
+                        ps[0][k] = acc.x + acc.y;
+                    } else {
+                        float2 rlo[2], rhi[2];
+        #pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            rlo[i] = __ffma2_rn(kl[i], cs[i], __fmul2_rn(kh[i], neg2(sn[i])));   // kl*cos - kh*sin
+                            rhi[i] = __ffma2_rn(kh[i], cs[i], __fmul2_rn(kl[i], sn[i]));         // kh*cos + kl*sin
+                        }
+        #pragma unroll
+                        for (int j = 0; j < QPK; ++j) {
+                            float2 acc = __fmul2_rn(qlo[j][0], rlo[0]);
+                            acc = __ffma2_rn(qhi[j][0], rhi[0], acc);
+                            acc = __ffma2_rn(qlo[j][1], rlo[1], acc);
+                            acc = __ffma2_rn(qhi[j][1], rhi[1], acc);
+                            ps[j][k] = acc.x + acc.y;
+                        }
+                    }
+                }
+
+                // ---- reduce-scatter the scores over the slot, online-softmax update
+                float pe[QPK];
+        #pragma unroll
+                for (int j = 0; j < QPK; ++j) {
+                    float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
+                    if constexpr (TQ) keep *= sig;
+                    const float s = (p0 + tk < tok_end && p0 + tk >= st) ? keep : -CUDART_INF_F;
+                    // Lazy maximum: the reference only has to stay within 2^8 of the running maximum for
+                    // the weights to stay finite, so it moves (with an exact rescale) only when a score of
+                    // the iteration exceeds it by more than 8 in log2 units.
+                    if (__any_sync(slot_mask, s > m_[j] + 8.f)) {
+                        float tmax = s;
+        #pragma unroll
+                        for (int o = NL / 2; o >= NL / TT; o >>= 1)
+                            tmax = fmaxf(tmax, __shfl_xor_sync(slot_mask, tmax, o));
+                        const float corr = ex2(m_[j] - tmax);
+                        l_[j] *= corr;
+                        const float2 c2 = f2(corr, corr);
+        #pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            olo[j][i] = __fmul2_rn(olo[j][i], c2);
+                            ohi[j][i] = __fmul2_rn(ohi[j][i], c2);
+                        }
+                        m_[j] = tmax;
+                    }
+                    pe[j] = ex2(s - m_[j]);
+                    l_[j] += pe[j];
+                }
+
+                // ---- values: rebuild and accumulate with each token's weight
+        #pragma unroll
+                for (int k = 0; k < TT; ++k) {
+                    const int src = slot_lane0 + tile_owner<TT, NL>(k);
+                    if constexpr (!VEARLY) {
+                        const uint32_t w = word_k(w4[k >> 2], k & 3);
+                        vraw[k][0] = lds64(smem, __byte_perm(w, colv_lo, 0x7624));
+                        vraw[k][1] = lds64(smem, __byte_perm(w, colv_hi, 0x7634));
+                    }
+                    const uint32_t vl[2] = {vraw[k][0].x, vraw[k][0].y}, vh[2] = {vraw[k][1].x, vraw[k][1].y};
+        #pragma unroll
+                    for (int j = 0; j < QPK; ++j) {
+                        const float pk = __shfl_sync(slot_mask, pe[j], src);
+                        const float2 p2 = f2(pk, pk);
+        #pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            olo[j][i] = __ffma2_rn(p2, unpack2(vl[i]), olo[j][i]);
+                            ohi[j][i] = __ffma2_rn(p2, unpack2(vh[i]), ohi[j][i]);
+                        }
+                    }
+                }
+            }
+            cp_async_wait<0>();
+
+            // ---- combine the slots of this CTA, write the split's partial result
+            __syncthreads();                                       // slices and queue no longer needed
+            constexpr int RS = D + 4;                              // floats per (slot, query head) record
+            // l_ sums the weights of the tokens this lane finished: add the other token positions of the slot
+            constexpr int TOKBITS = (TT == 8) ? 3 : 2;
+            float *red = reinterpret_cast<float *>(smem);
+        #pragma unroll
+            for (int j = 0; j < QPK; ++j) {
+                float lsum = l_[j];
+        #pragma unroll
+                for (int sb = 0; sb < TOKBITS; ++sb) lsum += __shfl_xor_sync(slot_mask, lsum, NL >> (1 + sb));
+                float *rec = red + ((size_t)slot * QPK + j) * RS;
+                *reinterpret_cast<float4 *>(rec + ch) = make_float4(olo[j][0].x, olo[j][0].y, olo[j][1].x, olo[j][1].y);
+                *reinterpret_cast<float4 *>(rec + D / 2 + ch) = make_float4(ohi[j][0].x, ohi[j][0].y, ohi[j][1].x, ohi[j][1].y);
+                if (ls == 0) {
+                    rec[D] = m_[j];
+                    rec[D + 1] = lsum;
+                }
+            }
+            __syncthreads();
+            for (int it = tid; it < QPK * D; it += NT) {
+                const int d = it % D;
+                const int j = it / D;
+                float mx = -CUDART_INF_F;
+                for (int s2 = 0; s2 < NSLOT; ++s2) mx = fmaxf(mx, red[((size_t)s2 * QPK + j) * RS + D]);
+                float acc = 0.f, lsum = 0.f;
+                if (mx != -CUDART_INF_F) {
+                    for (int s2 = 0; s2 < NSLOT; ++s2) {
+                        const float *rec = red + ((size_t)s2 * QPK + j) * RS;
+                        const float wgt = ex2(rec[D] - mx);
+                        acc += rec[d] * wgt;
+                        lsum += rec[D + 1] * wgt;
+                    }
+                }
+                const size_t rec = (size_t)piece * QPK + j;
+                a.ws_o[rec * D + d] = acc;
+                if (d == 0) a.ws_ml[rec] = f2(mx, lsum);
+            }
+            pos = pend;
         }
-        const size_t bh = (size_t)b * a.Hq + h * QPK + j;
-        a.ws_o[(bh * a.nsplit + split) * D + d] = acc;
-        if (d == 0) a.ws_ml[bh * a.nsplit + split] = f2(mx, lsum);
+        seg0 = seg_end;
+        if (++b == a.B) {
+            b = 0;
+            ++h;
+        }
     }
 }
 
-// Log-sum-exp merge of the splits of every (sequence, query head).
+// Log-sum-exp merge of the pieces of every (sequence, query head).
 template <int D>
 __global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
+    __shared__ long long info[3];                          // Tb, Pb(b), tiles of b
     const int bh = blockIdx.x;
-    const int b = bh / a.Hq;
+    const int b = bh / a.Hq, hq = bh % a.Hq;
+    const int qpk = a.Hq / a.Hkv, h = hq / qpk, j = hq % qpk;
     const int d = threadIdx.x;
-    const int len = min(max(a.lens[b], 0), a.max_len);
-    const int st = min(max(a.starts ? a.starts[b] : a.start_all, 0), len);
-    const int span = len - (st & ~3);                      // tokens covered by the splits
-    const int ns = len > st ? (span + a.split_len - 1) / a.split_len : 0;
-    const float2 *ml = a.ws_ml + (size_t)bh * a.nsplit;
+    if (d < 32) {
+        long long Tb, Pb;
+        head_tiles(a, d, b, Tb, Pb);
+        int base, st, len;
+        const int nt = seq_tiles(a, b, base, st, len);
+        if (d == 0) {
+            info[0] = Tb;
+            info[1] = Pb;
+            info[2] = nt;
+        }
+    }
+    __syncthreads();
+    const long long Tb = info[0], T = Tb * a.Hkv, G = a.ncta;
+    const long long P = h * Tb + info[1], E = P + info[2];  // tiles [P, E) of segment s
+    const long long s = (long long)h * a.B + b;
+    long long c0 = 0, c1 = -1;
+    if (E > P) {
+        c0 = cta_of_tile(P, T, G);
+        c1 = cta_of_tile(E - 1, T, G);
+    }
     float mx = -CUDART_INF_F;
-    for (int s = 0; s < ns; ++s) mx = fmaxf(mx, ml[s].x);
+    for (long long c = c0; c <= c1; ++c)
+        if (cta_first_tile(c, T, G) < cta_first_tile(c + 1, T, G)) mx = fmaxf(mx, a.ws_ml[(s + c) * qpk + j].x);
     float acc = 0.f, lsum = 0.f;
     if (mx != -CUDART_INF_F) {
-        const float *o = a.ws_o + (size_t)bh * a.nsplit * D + d;
-        for (int s = 0; s < ns; ++s) {
-            const float wgt = ex2(ml[s].x - mx);
-            acc += o[(size_t)s * D] * wgt;
-            lsum += ml[s].y * wgt;
+        for (long long c = c0; c <= c1; ++c) {
+            if (cta_first_tile(c, T, G) == cta_first_tile(c + 1, T, G)) continue;   // a CTA without tiles
+            const size_t rec = (size_t)(s + c) * qpk + j;
+            const float2 ml = a.ws_ml[rec];
+            const float wgt = ex2(ml.x - mx);
+            acc += a.ws_o[rec * D + d] * wgt;
+            lsum += ml.y * wgt;
         }
     }
     const bool any = (mx != -CUDART_INF_F) && lsum > 0.f;

@@ -116,7 +116,7 @@ static cudaError_t launch_ct(const EncodeArgs &a, int x_dtype, int nb, bool pg, 
         const size_t smem = 4 * (size_t)a.K * C * TC * sizeof(float);
         dim3 grid((a.ntok + 127) / 128, NP * a.Hkv, nb);
         auto k = x_dtype == LOOPVQ_BF16 ? encode_pg_kernel<D, C, TC, uint16_t> : encode_pg_kernel<D, C, TC, float>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = ensure_dynamic_smem((const void *)k, smem);
         if (e != cudaSuccess) return e;
         k<<<grid, 128, smem, s>>>(a);
         return cudaGetLastError();
@@ -125,12 +125,12 @@ static cudaError_t launch_ct(const EncodeArgs &a, int x_dtype, int nb, bool pg, 
     dim3 grid((a.ntok * NP + 127) / 128, a.Hkv, nb);
     if (x_dtype == LOOPVQ_BF16) {
         auto k = encode_direct_kernel<D, C, TC, uint16_t>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = ensure_dynamic_smem((const void *)k, smem);
         if (e != cudaSuccess) return e;
         k<<<grid, 128, smem, s>>>(a);
     } else {
         auto k = encode_direct_kernel<D, C, TC, float>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = ensure_dynamic_smem((const void *)k, smem);
         if (e != cudaSuccess) return e;
         k<<<grid, 128, smem, s>>>(a);
     }

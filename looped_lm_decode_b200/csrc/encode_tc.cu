@@ -438,7 +438,7 @@ static cudaError_t launch_tc_ct(const EncodeTcArgs &a0, cudaStream_t s) {
     constexpr int KD = ((C * TC + 3 + 15) / 16) * 16;
     EncodeTcArgs a = a0;
     auto k = encode_tc_kernel<D, C, TC>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSmem<KD>::kAlloc);
+    cudaError_t e = ensure_dynamic_smem((const void *)k, TcSmem<KD>::kAlloc);
     if (e != cudaSuccess) return e;
     // CTAs resident per SM, from the limits that bind here: shared memory, registers and tensor memory
     // (each CTA allocates 256 of the SM's 512 TMEM columns)

@@ -42,6 +42,12 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_floa
 // Sets the thread-local message returned by loopvq_last_error().
 void set_last_error(const char *msg);
 
+// Raises a kernel's dynamic shared-memory limit on the current device to at least `bytes`.  The
+// attribute is set on the first such request (or a larger one) per kernel and device only, so steady
+// launches make no attribute call: less host time per call, and nothing but launches inside a CUDA
+// graph capture.
+cudaError_t ensure_dynamic_smem(const void *kern, size_t bytes);
+
 // Launchers (host); each returns a cudaError_t from the launch.
 cudaError_t launch_prepare(const loopvq_cache &cc, cudaStream_t s);
 cudaError_t launch_encode(const loopvq_cache &cc, int layer, int block, const void *xk, const void *xv,
@@ -51,8 +57,10 @@ cudaError_t launch_dequant(const loopvq_cache &cc, int layer, int t, int kv, int
                            int apply_rope, float *out, cudaStream_t s);
 
 struct DecodePlan {
-    int split_len;      // tokens per split (multiple of 4)
-    int nsplit;         // splits covering max_len
+    int split_len;      // bf16 kernel: tokens per split (multiple of 4)
+    int nsplit;         // bf16 kernel: splits covering max_len; coded kernel: its CTAs
+    int ncta;           // coded kernel: CTAs sharing the tile space
+    int npiece;         // coded kernel: partial records (segments + CTAs)
     int nbt;            // sequences per thread block
     int nchunk;         // ceil(B / nbt)
     size_t ws_bytes;    // workspace needed

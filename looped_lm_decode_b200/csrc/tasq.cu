@@ -113,7 +113,7 @@ static cudaError_t launch_tasq_t(const TasqArgs &a, int nb, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const size_t smem = 2 * (size_t)a.K * C * TC * sizeof(float) + (D / 2) * sizeof(int16_t);
     auto k = tasq_encode_kernel<D, C, TC, XT>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    if ((e = ensure_dynamic_smem((const void *)k, smem)) != cudaSuccess) return e;
     k<<<dim3((a.ntok * NP + 127) / 128, a.Hkv, nb), 128, smem, s>>>(a);
     return cudaGetLastError();
 }

@@ -128,7 +128,7 @@ static cudaError_t launch_page_encode(const WinEncArgs &a, cudaStream_t s) {
     constexpr int NP = D / (2 * C);
     const size_t smem = 2 * (size_t)a.K * C * TC * sizeof(float);
     auto k = window_page_encode_kernel<D, C, TC>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_dynamic_smem((const void *)k, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((8 * NP + 127) / 128, a.L * a.NB * a.Hkv, a.B);
     k<<<grid, 128, smem, s>>>(a);
@@ -171,7 +171,7 @@ cudaError_t launch_window_advance(const loopvq_window &w, const loopvq_cache &cc
                                 : dispatch_page_encode<64>(cc.c, cc.Tc, a, s);
     if (e != cudaSuccess) return e;
     const size_t smem = (size_t)w.n_recent * w.D * 2;
-    e = cudaFuncSetAttribute(window_shift_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = ensure_dynamic_smem((const void *)window_shift_kernel, smem);
     if (e != cudaSuccess) return e;
     window_shift_kernel<<<dim3(w.L * w.T * w.Hkv, w.B), 256, smem, s>>>(w.k_rot, w.k_pre, w.v, w.fill, w.B, w.Hkv,
                                                                          w.D, W, w.n_sink, w.n_recent);

@@ -133,6 +133,41 @@ def test_decode_range_parity(w):
     assert ok, msg
 
 
+MANY = WORKLOADS["ctx4k"].replace(L=1, B=24, Hkv=2, Hq=2, Nmax=512)
+MANY_GQA = WORKLOADS["gqa16k"].replace(L=1, B=20, Hkv=2, Hq=8, Nmax=256)
+
+
+@pytest.mark.parametrize("w", [MANY, MANY_GQA], ids=["mha", "gqa"])
+@pytest.mark.parametrize("kind", ["short", "tiny"])
+def test_decode_pieces_many_segments(w, kind):
+    """The split kernel shares the tiles of all (KV head, sequence) segments evenly among its CTAs: here
+    CTAs run across many short segments ("short"), or outnumber the tiles so that some hold none
+    ("tiny"); empty sequences, empty ranges and starts inside a tile included."""
+    cache, codes = _coded_cache(w)
+    rng = np.random.default_rng(23 if kind == "short" else 29)
+    if kind == "short":
+        lens = rng.choice([0, 1, 3, 4, 9, 37, 100, w.Nmax // 2, w.Nmax], w.B).astype(np.int32)
+    else:
+        lens = rng.choice([0, 1, 2, 4, 5], w.B).astype(np.int32)
+    starts = np.array([rng.integers(0, int(l) + 1) for l in lens], np.int32)
+    starts[:3] = 0
+    t = 1
+    qb = queries(w, 0, t)
+    for with_starts in (False, True):
+        st = starts if with_starts else np.zeros(w.B, np.int32)
+        if with_starts:
+            out, lse = LQ.decode_attn_range(cache, 0, t, _dev_bits(qb), _dev_i32(st), _dev_i32(lens), w.Nmax)
+        else:
+            out, lse = LQ.decode_attn(cache, 0, t, _dev_bits(qb), _dev_i32(lens), w.Nmax)
+        torch.cuda.synchronize()
+        ref, lref = _oracle_windowed(w, codes, t, qb, None, None, [0] * w.B, st, lens, 1 / math.sqrt(w.D))
+        out, lse = out.cpu().numpy(), lse.cpu().numpy()
+        ok, msg = attn_tolerance_ok(out, ref, lse, lref)
+        assert ok, f"{kind} starts={with_starts}: {msg}"
+        empty = st >= lens
+        assert (out[empty] == 0).all() and np.isneginf(lse[empty]).all()
+
+
 @pytest.mark.parametrize("w", [CODED, CODED_GQA], ids=["mha", "gqa"])
 @pytest.mark.parametrize("t", [0, 3])
 def test_windowed_cache_parity(w, t):

@@ -57,7 +57,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 
 
 def test_noalloc_rejects_calls_larger_than_its_scratch():
-    c = LQ.Cache(1, 4, 4, 16, 16, 128, 4, 256, 256, 32768, alloc=False)
+    # the partial records scale with (sequences x KV heads + CTAs) x query heads per KV head
+    c = LQ.Cache(1, 4, 4, 16, 32, 128, 4, 256, 1024, 32768, alloc=False)
     need = LQ.lib().loopvq_decode_workspace_bytes(c.ref(), 32768)
     assert need > LQ.lib().loopvq_noalloc_scratch_bytes()
     # aligned addresses that are never dereferenced: the call must be refused before any launch
