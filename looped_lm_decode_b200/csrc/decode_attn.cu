@@ -69,8 +69,18 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStr
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    merge_kernel<D><<<a.B * a.Hq, D, 0, s>>>(a);
-    return cudaGetLastError();
+    // the merge as a programmatic dependent launch: it overlaps the split kernel's last CTAs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B * a.Hq);
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, merge_kernel<D>, a);
 }
 
 template <int D, int C, bool PG>

@@ -7,8 +7,12 @@
 // partial outputs are merged through their log-sum-exp (exact softmax).
 //
 // B200 design (not the pages' kernel):
-//  * One CTA per (token split, KV head, sequence).  The head's K and V slices are
-//    staged as bank-private replicas: row r (256 bytes) holds entry r of the K
+//  * Exactly one wave of resident CTAs, sharing the 4-token tiles of all (KV head,
+//    sequence) segments evenly whatever the sequence lengths (see the tile-space
+//    helpers below): a CTA walks its tile range segment by segment, and each part
+//    of a segment it covers (a piece) is one split of that segment, with its own
+//    partial record for the log-sum-exp merge.
+//  * For each piece the head's K and V slices are staged as bank-private replicas: row r (256 bytes) holds entry r of the K
 //    slice in bytes [0,128) and of the V slice in [128,256), replicated so that
 //    the 8-byte piece a lane reads sits in its own bank pair: lane l reads bytes
 //    (l % 16) * 8 of the half-row.  For c = 4 that is replica l % 16 of the
@@ -263,6 +267,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ long long range_info[4];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // the merge kernel may be scheduled now; it waits for this grid before reading any record
+    asm volatile("griddepcontrol.launch_dependents;");
     if (warp == 0) cta_range(a, lane, range_info);
     __syncthreads();
     long long pos = range_info[0];                         // next tile of this CTA
@@ -670,9 +676,14 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     }
 }
 
-// Log-sum-exp merge of the pieces of every (sequence, query head).
+// Log-sum-exp merge of the pieces of every (sequence, query head).  Launched as a programmatic
+// dependent of the split kernel: it finds its segment's records while the split kernel finishes, then
+// waits for that grid (griddepcontrol.wait returns once the split kernel has completed and its writes
+// are visible) before reading them.  The records' (max, sum) pairs, then their outputs, are read in
+// batches of independent loads.
 template <int D>
 __global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
+    constexpr int RB = 8;                                  // records read per batch
     __shared__ long long info[3];                          // Tb, Pb(b), tiles of b
     const int bh = blockIdx.x;
     const int b = bh / a.Hq, hq = bh % a.Hq;
@@ -698,19 +709,33 @@ __global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
         c0 = cta_of_tile(P, T, G);
         c1 = cta_of_tile(E - 1, T, G);
     }
-    float mx = -CUDART_INF_F;
-    for (long long c = c0; c <= c1; ++c)
-        if (cta_first_tile(c, T, G) < cta_first_tile(c + 1, T, G)) mx = fmaxf(mx, a.ws_ml[(s + c) * qpk + j].x);
-    float acc = 0.f, lsum = 0.f;
-    if (mx != -CUDART_INF_F) {
-        for (long long c = c0; c <= c1; ++c) {
-            if (cta_first_tile(c, T, G) == cta_first_tile(c + 1, T, G)) continue;   // a CTA without tiles
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    float mx = -CUDART_INF_F, acc = 0.f, lsum = 0.f;
+    for (long long cb = c0; cb <= c1; cb += RB) {
+        float2 ml[RB];
+        float o[RB];
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+            const long long c = cb + r;
+            const bool live = c <= c1 && cta_first_tile(c, T, G) < cta_first_tile(c + 1, T, G);
             const size_t rec = (size_t)(s + c) * qpk + j;
-            const float2 ml = a.ws_ml[rec];
-            const float wgt = ex2(ml.x - mx);
-            acc += a.ws_o[rec * D + d] * wgt;
-            lsum += ml.y * wgt;
+            ml[r] = live ? __ldcg(a.ws_ml + rec) : make_float2(-CUDART_INF_F, 0.f);
+            o[r] = live ? __ldcg(a.ws_o + rec * D + d) : 0.f;
         }
+        float bm = mx;
+#pragma unroll
+        for (int r = 0; r < RB; ++r) bm = fmaxf(bm, ml[r].x);
+        if (bm == -CUDART_INF_F) continue;
+        const float corr = ex2(mx - bm);                   // 0 while mx is still -inf
+        acc *= corr;
+        lsum *= corr;
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+            const float wgt = ex2(ml[r].x - bm);           // 0 for absent records
+            acc += o[r] * wgt;
+            lsum += ml[r].y * wgt;
+        }
+        mx = bm;
     }
     const bool any = (mx != -CUDART_INF_F) && lsum > 0.f;
     a.out[(size_t)bh * D + d] = any ? acc / lsum : 0.f;
