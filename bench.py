@@ -135,7 +135,7 @@ def replay_ms(g, reps, stream):
 
 def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
     """Same decode calls on a cache held entirely in bf16 (the pages' comparison, LoopVQ paper Sec. 5.3),
-    and on the pages' serving layout: 8 sink + 64 recent tokens in a bf16 window, the rest coded, merged
+    and on the pages' serving layout: 8 sink + 64 recent tokens in a bf16 window, the rest coded, combined
     through the log-sum-exps (Sec. 4.3 "Cache layout", "Attention").  Timed as CUDA graph replays with CUDA
     events, like the coded calls."""
     import torch
@@ -216,8 +216,8 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
         "windowed": {"us_per_call": win_call_ms * 1e3, "us_per_step": win_step_ms * 1e3, "steps": nsteps,
                      "sink": n_sink, "recent": n_recent,
                      "calls": "per step: loopvq_window_advance (page roll every 8 steps), then per (loop step, "
-                              "layer) loopvq_window_append + loopvq_window_decode_attn (bf16 window kernel + coded "
-                              "range kernel + merge2)"},
+                              "layer) loopvq_window_append + loopvq_window_decode_attn (coded split kernel + merge "
+                              "kernel, which also attends to the window slots)"},
     }
 
 

@@ -328,10 +328,12 @@ loopvq_status loopvq_window_append(const loopvq_window *w, int layer, int t, con
 size_t loopvq_window_workspace_bytes(const loopvq_window *w, const loopvq_cache *cache, int max_coded);
 
 /*
- * Decode attention of (layer, t) over the window and the coded cache: the
- * bf16 kernel over window slots 0 .. fill_b-1, the coded kernel over tokens
- * n_sink <= n < coded_end_b, merged through their log-sum-exps (Sec. 4.3
- * "Attention").  max_coded is a host upper bound of coded_end (<= Nmax).
+ * Decode attention of (layer, t) over the window and the coded cache: window
+ * slots 0 .. fill_b-1 (keys stored rotated) and the coded tokens
+ * n_sink <= n < coded_end_b, combined through their log-sum-exps (Sec. 4.3
+ * "Attention").  Two launches: the coded split kernel, and its merge kernel,
+ * which attends to the window slots while the split kernel finishes.
+ * max_coded is a host upper bound of coded_end (<= Nmax).
  * q, scale, out, lse as for loopvq_decode_attn; workspace of at least
  * loopvq_window_workspace_bytes(w, cache, max_coded) bytes.
  */

@@ -61,7 +61,11 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStr
     const size_t red = (size_t)NSLOT * QPK * (D + 4) * sizeof(float);
     const size_t smem = ring_smem_bytes(PG, QPK);
     if (red > smem) return cudaErrorInvalidConfiguration;   // the slot records reuse slices and queue
-    auto kern = decode_split_kernel<D, C, QPK, K.warps, K.min_blocks, K.depth, kWords, PG, TQ>;
+    // TaSQ with one query head per KV head carries the rotated query from tile to tile (XR): its
+    // table values sit at permuted columns, 8 scalar loads per tile.  The plain kernels load the
+    // table row one iteration ahead, which measured faster for them (143 vs 150 us at ctx32k).
+    constexpr bool XR = TQ && QPK == 1;
+    auto kern = decode_split_kernel<D, C, QPK, K.warps, K.min_blocks, K.depth, kWords, PG, TQ, XR>;
     cudaError_t e = ensure_dynamic_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     if (plan.ncta > 0) {
@@ -119,7 +123,8 @@ static cudaError_t dispatch_c(int c, int qpk, const DecodeArgs &a, const DecodeP
 cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
                           const uint16_t *q, const int32_t *starts, int start_all, const int32_t *lens, int max_len,
                           float scale, float *out, float *lse, void *workspace, cudaStream_t s,
-                          const loopvq_tasq *tq) {
+                          const loopvq_tasq *tq, const uint16_t *wk, const uint16_t *wv, const int32_t *wfill,
+                          int W) {
     DecodeArgs a{};
     const int beta = t / cc.Tc;
     a.idx = cc.idx + idx_base(cc, layer, beta, 0, 0);
@@ -143,6 +148,10 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     a.max_len = max_len;
     a.ncta = plan.ncta;
     a.qscale = scale * 1.44269504088896340736f;
+    a.wk = wk;
+    a.wv = wv;
+    a.wfill = wfill;
+    a.W = W;
     const int qpk = cc.Hq / cc.Hkv;
     if (tq) {
         const int NB = cc.T / cc.Tc;

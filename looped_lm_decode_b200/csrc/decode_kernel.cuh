@@ -66,6 +66,10 @@ struct DecodeArgs {
     const float *tw;         // TaSQ: channel weights of (layer, t) [Hkv][D]
     const int16_t *tperm;    // TaSQ: low-channel order of (layer, block) [Hkv][D/2]
     const uint16_t *tsig;    // TaSQ: fp16 token scales of (layer, t) [B][Nmax]
+    const uint16_t *wk;      // bf16 window of (layer, t), or null: rotated keys [B][Hkv][W][D]
+    const uint16_t *wv;      //   values [B][Hkv][W][D]
+    const int32_t *wfill;    //   [B] slots in use
+    int W;                   //   slots per (sequence, KV head)
     float qscale;            // scale * log2(e)
 };
 
@@ -246,7 +250,11 @@ __device__ __forceinline__ void cta_range(const DecodeArgs &a, int lane, long lo
 // 2p + 1, whose entries interleave complete RoPE pairs (f, f + D/2) of low channels taken from the
 // permutation; the query is gathered at those channels and divided by the channel weights, the RoPE
 // values come from those columns of the table, and each token's score is multiplied by its scale.
-template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, int NW, bool PG = false, bool TQ = false>
+// XR: the RoPE values at each iteration's first token are carried from the previous iteration (one
+// complex multiply by e^{-+i STRIDE w}) and set from the table every 16 iterations, instead of loading
+// the table row one iteration ahead.
+template <int D, int C, int QPK, int WARPS, int MINB, int DEPTH, int NW, bool PG = false, bool TQ = false,
+          bool XR = false>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const DecodeArgs a) {
     constexpr bool ROTQ = QPK == 1;                        // rotate the query, not every key
     constexpr int NP = D / (2 * C);                        // pair-groups = index words per token
@@ -318,7 +326,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             // low channels of the lane's 4 RoPE pairs: ch .. ch+3, or under TaSQ the pairs 2*half, 2*half + 1
             // of TaSQ groups 2*gp (key code lo) and 2*gp + 1 (key code hi)
             int fq[4];
-        #pragma unroll
+#pragma unroll
             for (int k = 0; k < 4; ++k) {
                 if constexpr (TQ) {
                     const int16_t *pm = a.tperm + (size_t)h * (D / 2);
@@ -343,10 +351,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 
             // queue the first DEPTH iterations of this slot before staging the slices
             const int pfirst = tok_begin + slot * TT;
-        #pragma unroll
+#pragma unroll
             for (int d = 0; d < DEPTH; ++d) {
                 const int p = pfirst + d * STRIDE;
-        #pragma unroll
+#pragma unroll
                 for (int u = 0; u < NW; ++u)
                     if (p + 4 * u < tok_end)
                         cp_async16(ring + (uint32_t)(d * QB + u * NT * 16), idx_b + (size_t)((p >> 2) + u) * NP * 4);
@@ -369,7 +377,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                         if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(src));
                         *reinterpret_cast<uint2 *>(dst) = v;
                     } else {
-        #pragma unroll
+#pragma unroll
                         for (int u = 0; u < EB / 16; ++u) {
                             uint4 v = make_uint4(0u, 0u, 0u, 0u);
                             if (r < a.K) v = __ldg(reinterpret_cast<const uint4 *>(src) + u);
@@ -400,14 +408,14 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             }
 
             float2 qlo[QPK][2], qhi[QPK][2];
-        #pragma unroll
+#pragma unroll
             for (int j = 0; j < QPK; ++j) {
                 const uint16_t *qp = a.q + ((size_t)b * a.Hq + h * QPK + j) * D;
                 if constexpr (TQ) {
                     // q / w at the lane's permuted pairs (a pair's two channels share their weight)
                     const float *wp = a.tw + (size_t)h * D;
                     float ql[4], qh[4];
-        #pragma unroll
+#pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const float sc = a.qscale / __ldg(wp + fq[k]);
                         ql[k] = bf16_to_f32(qp[fq[k]]) * sc;
@@ -441,7 +449,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             const float2 nqlo[2] = {neg2(qlo[0][0]), neg2(qlo[0][1])};
             float m_[QPK], l_[QPK];
             float2 olo[QPK][2], ohi[QPK][2];
-        #pragma unroll
+#pragma unroll
             for (int j = 0; j < QPK; ++j) {
                 m_[j] = -CUDART_INF_F;
                 l_[j] = 0.f;
@@ -449,18 +457,32 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             }
             const int tk = tile_token<TT, NL>(ls);                 // token of the iteration this lane finishes
 
-            // RoPE row of each iteration's first token, loaded one iteration ahead
+            // RoPE values at each iteration's first token p0.  XR: carried from the previous iteration
+            // by one complex multiply with e^{-+i STRIDE w} (ROTQ: the rotated query itself), and set
+            // from the table row every 16 iterations so that rounding stays within 16 products;
+            // otherwise the table row is loaded one iteration ahead.
             float4 ra_c, ra_s;
-            {
+            float2 xa_c[2], xa_s[2], sc[2], ssn[2];
+            if constexpr (XR) {
+                sc[0] = sc[1] = ssn[0] = ssn[1] = f2(0.f, 0.f);
+                if (STRIDE < a.Nmax) {                       // else no slot runs a second iteration
+                    float4 c4, s4;
+                    load_row4(a.rope + (size_t)STRIDE * D, c4, s4);
+                    sc[0] = f2(c4.x, c4.y);
+                    sc[1] = f2(c4.z, c4.w);
+                    ssn[0] = f2(s4.x, s4.y);
+                    ssn[1] = f2(s4.z, s4.w);
+                }
+            } else {
                 load_row4(a.rope + (size_t)min(pfirst, a.Nmax - 4) * D, ra_c, ra_s);
             }
             __syncthreads();
 
-            int stage = 0;
-            for (int p0 = pfirst; p0 < tok_end; p0 += STRIDE) {
+            int stage = 0, iter = 0;
+            for (int p0 = pfirst; p0 < tok_end; p0 += STRIDE, ++iter) {
                 cp_async_wait<DEPTH - 1>();                        // this thread's oldest queued stage has landed
                 uint4 w4[NW];
-        #pragma unroll
+#pragma unroll
                 for (int u = 0; u < NW; ++u) {
                     const uint32_t addr = ring + (uint32_t)(stage * QB + u * NT * 16);
                     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -469,16 +491,55 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 // the stage has been read into registers: queue the iteration DEPTH steps ahead into it
                 {
                     const int pq = p0 + DEPTH * STRIDE;
-        #pragma unroll
+#pragma unroll
                     for (int u = 0; u < NW; ++u)
                         if (pq + 4 * u < tok_end)
                             cp_async16(ring + (uint32_t)(stage * QB + u * NT * 16), idx_b + (size_t)((pq >> 2) + u) * NP * 4);
                     cp_async_commit();
                     stage = stage + 1 == DEPTH ? 0 : stage + 1;
                 }
-                float2 cs[2] = {f2(ra_c.x, ra_c.y), f2(ra_c.z, ra_c.w)};
-                float2 sn[2] = {f2(ra_s.x, ra_s.y), f2(ra_s.z, ra_s.w)};
-                {
+                float2 cs[2], sn[2];
+                if constexpr (XR) {
+                    if ((iter & 15) == 0) {
+                        float4 c4, s4;
+                        load_row4(a.rope + (size_t)min(p0, a.Nmax - 4) * D, c4, s4);
+                        cs[0] = f2(c4.x, c4.y);
+                        cs[1] = f2(c4.z, c4.w);
+                        sn[0] = f2(s4.x, s4.y);
+                        sn[1] = f2(s4.z, s4.w);
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            if constexpr (ROTQ) {
+                                xa_c[i] = __ffma2_rn(qlo[0][i], cs[i], __fmul2_rn(qhi[0][i], sn[i]));
+                                xa_s[i] = __ffma2_rn(qhi[0][i], cs[i], __fmul2_rn(nqlo[i], sn[i]));
+                            } else {
+                                xa_c[i] = cs[i];
+                                xa_s[i] = sn[i];
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const float2 re = xa_c[i], im = xa_s[i];
+                            if constexpr (ROTQ) {                 // times e^{-i STRIDE w}
+                                xa_c[i] = __ffma2_rn(re, sc[i], __fmul2_rn(im, ssn[i]));
+                                xa_s[i] = __ffma2_rn(im, sc[i], __fmul2_rn(re, neg2(ssn[i])));
+                            } else {                              // times e^{+i STRIDE w}
+                                xa_c[i] = __ffma2_rn(re, sc[i], __fmul2_rn(im, neg2(ssn[i])));
+                                xa_s[i] = __ffma2_rn(im, sc[i], __fmul2_rn(re, ssn[i]));
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        cs[i] = xa_c[i];
+                        sn[i] = xa_s[i];
+                    }
+                } else {
+                    cs[0] = f2(ra_c.x, ra_c.y);
+                    cs[1] = f2(ra_c.z, ra_c.w);
+                    sn[0] = f2(ra_s.x, ra_s.y);
+                    sn[1] = f2(ra_s.z, ra_s.w);
                     load_row4(a.rope + (size_t)min(p0 + STRIDE, a.Nmax - 4) * D, ra_c, ra_s);
                 }
 
@@ -487,7 +548,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 constexpr bool VEARLY = QPK <= 2;
                 uint2 vraw[TT][2];
                 if constexpr (VEARLY) {
-        #pragma unroll
+#pragma unroll
                     for (int k = 0; k < TT; ++k) {
                         const uint32_t w = word_k(w4[k >> 2], k & 3);
                         vraw[k][0] = lds64(smem, __byte_perm(w, colv_lo, 0x7624));
@@ -506,16 +567,21 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 float ps[QPK][TT];
                 float2 zu[2], zw[2], xu[2], xw[2];                // X_k and X_{k-1} of the advanced pair
                 if constexpr (ROTQ) {
-        #pragma unroll
+#pragma unroll
                     for (int i = 0; i < 2; ++i) {
-                        zu[i] = __ffma2_rn(qlo[0][i], cs[i], __fmul2_rn(qhi[0][i], sn[i]));
-                        zw[i] = __ffma2_rn(qhi[0][i], cs[i], __fmul2_rn(nqlo[i], sn[i]));
+                        if constexpr (XR) {                   // cs, sn already hold Z
+                            zu[i] = cs[i];
+                            zw[i] = sn[i];
+                        } else {
+                            zu[i] = __ffma2_rn(qlo[0][i], cs[i], __fmul2_rn(qhi[0][i], sn[i]));
+                            zw[i] = __ffma2_rn(qhi[0][i], cs[i], __fmul2_rn(nqlo[i], sn[i]));
+                        }
                     }
                 }
-        #pragma unroll
+#pragma unroll
                 for (int k = 0; k < TT; ++k) {
                     if (k > 0) {
-        #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 2; ++i) {
                             // the pair (re, im) advanced by one position: ROTQ by e^{-iw}, else by e^{+iw}
                             float2 &re = ROTQ ? zu[i] : cs[i];
@@ -559,12 +625,12 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                         ps[0][k] = acc.x + acc.y;
                     } else {
                         float2 rlo[2], rhi[2];
-        #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 2; ++i) {
                             rlo[i] = __ffma2_rn(kl[i], cs[i], __fmul2_rn(kh[i], neg2(sn[i])));   // kl*cos - kh*sin
                             rhi[i] = __ffma2_rn(kh[i], cs[i], __fmul2_rn(kl[i], sn[i]));         // kh*cos + kl*sin
                         }
-        #pragma unroll
+#pragma unroll
                         for (int j = 0; j < QPK; ++j) {
                             float2 acc = __fmul2_rn(qlo[j][0], rlo[0]);
                             acc = __ffma2_rn(qhi[j][0], rhi[0], acc);
@@ -577,7 +643,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 
                 // ---- reduce-scatter the scores over the slot, online-softmax update
                 float pe[QPK];
-        #pragma unroll
+#pragma unroll
                 for (int j = 0; j < QPK; ++j) {
                     float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
                     if constexpr (TQ) keep *= sig;
@@ -587,13 +653,13 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                     // the iteration exceeds it by more than 8 in log2 units.
                     if (__any_sync(slot_mask, s > m_[j] + 8.f)) {
                         float tmax = s;
-        #pragma unroll
+#pragma unroll
                         for (int o = NL / 2; o >= NL / TT; o >>= 1)
                             tmax = fmaxf(tmax, __shfl_xor_sync(slot_mask, tmax, o));
                         const float corr = ex2(m_[j] - tmax);
                         l_[j] *= corr;
                         const float2 c2 = f2(corr, corr);
-        #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 2; ++i) {
                             olo[j][i] = __fmul2_rn(olo[j][i], c2);
                             ohi[j][i] = __fmul2_rn(ohi[j][i], c2);
@@ -605,7 +671,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 }
 
                 // ---- values: rebuild and accumulate with each token's weight
-        #pragma unroll
+#pragma unroll
                 for (int k = 0; k < TT; ++k) {
                     const int src = slot_lane0 + tile_owner<TT, NL>(k);
                     if constexpr (!VEARLY) {
@@ -614,11 +680,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                         vraw[k][1] = lds64(smem, __byte_perm(w, colv_hi, 0x7634));
                     }
                     const uint32_t vl[2] = {vraw[k][0].x, vraw[k][0].y}, vh[2] = {vraw[k][1].x, vraw[k][1].y};
-        #pragma unroll
+#pragma unroll
                     for (int j = 0; j < QPK; ++j) {
                         const float pk = __shfl_sync(slot_mask, pe[j], src);
                         const float2 p2 = f2(pk, pk);
-        #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 2; ++i) {
                             olo[j][i] = __ffma2_rn(p2, unpack2(vl[i]), olo[j][i]);
                             ohi[j][i] = __ffma2_rn(p2, unpack2(vh[i]), ohi[j][i]);
@@ -634,10 +700,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             // l_ sums the weights of the tokens this lane finished: add the other token positions of the slot
             constexpr int TOKBITS = (TT == 8) ? 3 : 2;
             float *red = reinterpret_cast<float *>(smem);
-        #pragma unroll
+#pragma unroll
             for (int j = 0; j < QPK; ++j) {
                 float lsum = l_[j];
-        #pragma unroll
+#pragma unroll
                 for (int sb = 0; sb < TOKBITS; ++sb) lsum += __shfl_xor_sync(slot_mask, lsum, NL >> (1 + sb));
                 float *rec = red + ((size_t)slot * QPK + j) * RS;
                 *reinterpret_cast<float4 *>(rec + ch) = make_float4(olo[j][0].x, olo[j][0].y, olo[j][1].x, olo[j][1].y);
@@ -681,14 +747,73 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
 // waits for that grid (griddepcontrol.wait returns once the split kernel has completed and its writes
 // are visible) before reading them.  The records' (max, sum) pairs, then their outputs, are read in
 // batches of independent loads.
+//
+// With a bf16 window (LoopVQ paper, Sec. 4.3 "Cache layout" and "Attention": the sink and recent tokens
+// stay in bf16 and their attention is combined with the coded tokens' through the log-sum-exp), the
+// merge first attends to the window slots [0, fill_b) itself, before the wait, so that this work
+// overlaps the split kernel: warp w takes slots w, w + D/32, ..., each lane D/32 channels of a slot,
+// an online softmax per warp, and the warps' results are combined in shared memory.  Window keys are
+// stored rotated, so no RoPE is applied to them.
 template <int D>
 __global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
     constexpr int RB = 8;                                  // records read per batch
+    constexpr int NWARP = D / 32, CPL = D / 32;            // warps; window channels per lane
     __shared__ long long info[3];                          // Tb, Pb(b), tiles of b
+    __shared__ float wrec[NWARP][D + 2];                   // window: per-warp (o, max, sum)
     const int bh = blockIdx.x;
     const int b = bh / a.Hq, hq = bh % a.Hq;
     const int qpk = a.Hq / a.Hkv, h = hq / qpk, j = hq % qpk;
     const int d = threadIdx.x;
+    float mw = -CUDART_INF_F, lw = 0.f, ow = 0.f;          // the window's part for channel d
+    if (a.wk != nullptr) {
+        const int lane = d & 31, warp = d >> 5;
+        const int n = min(max(__ldg(a.wfill + b), 0), a.W);
+        float qv[CPL];
+        const uint16_t *qp = a.q + (size_t)bh * D + lane * CPL;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) qv[c] = bf16_to_f32(__ldg(qp + c)) * a.qscale;
+        const size_t row0 = ((size_t)b * a.Hkv + h) * (size_t)a.W * D + lane * CPL;
+        float m = -CUDART_INF_F, l = 0.f, o[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) o[c] = 0.f;
+        for (int t = warp; t < n; t += NWARP) {
+            float kv[CPL], vv[CPL];
+            const uint16_t *kp = a.wk + row0 + (size_t)t * D, *vp = a.wv + row0 + (size_t)t * D;
+            if constexpr (CPL == 4) {
+                const uint2 k4 = __ldg(reinterpret_cast<const uint2 *>(kp));
+                const uint2 v4 = __ldg(reinterpret_cast<const uint2 *>(vp));
+                kv[0] = bf16lo(k4.x); kv[1] = bf16hi(k4.x); kv[2] = bf16lo(k4.y); kv[3] = bf16hi(k4.y);
+                vv[0] = bf16lo(v4.x); vv[1] = bf16hi(v4.x); vv[2] = bf16lo(v4.y); vv[3] = bf16hi(v4.y);
+            } else {
+                const uint32_t k2 = __ldg(reinterpret_cast<const uint32_t *>(kp));
+                const uint32_t v2 = __ldg(reinterpret_cast<const uint32_t *>(vp));
+                kv[0] = bf16lo(k2); kv[1] = bf16hi(k2);
+                vv[0] = bf16lo(v2); vv[1] = bf16hi(v2);
+            }
+            float sc = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) sc = fmaf(qv[c], kv[c], sc);
+#pragma unroll
+            for (int o2 = 16; o2 >= 1; o2 >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o2);
+            if (sc > m) {
+                const float corr = ex2(m - sc);
+                l *= corr;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) o[c] *= corr;
+                m = sc;
+            }
+            const float pw = ex2(sc - m);
+            l += pw;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) o[c] = fmaf(pw, vv[c], o[c]);
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) wrec[warp][lane * CPL + c] = o[c];
+        if (lane == 0) {
+            wrec[warp][D] = m;
+            wrec[warp][D + 1] = l;
+        }
+    }
     if (d < 32) {
         long long Tb, Pb;
         head_tiles(a, d, b, Tb, Pb);
@@ -701,6 +826,18 @@ __global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
         }
     }
     __syncthreads();
+    if (a.wk != nullptr) {
+#pragma unroll
+        for (int w = 0; w < NWARP; ++w) mw = fmaxf(mw, wrec[w][D]);
+        if (mw != -CUDART_INF_F) {
+#pragma unroll
+            for (int w = 0; w < NWARP; ++w) {
+                const float wgt = ex2(wrec[w][D] - mw);
+                ow += wrec[w][d] * wgt;
+                lw += wrec[w][D + 1] * wgt;
+            }
+        }
+    }
     const long long Tb = info[0], T = Tb * a.Hkv, G = a.ncta;
     const long long P = h * Tb + info[1], E = P + info[2];  // tiles [P, E) of segment s
     const long long s = (long long)h * a.B + b;
@@ -735,6 +872,13 @@ __global__ void __launch_bounds__(D) merge_kernel(const DecodeArgs a) {
             acc += o[r] * wgt;
             lsum += ml[r].y * wgt;
         }
+        mx = bm;
+    }
+    if (mw != -CUDART_INF_F) {                             // fold in the window's part
+        const float bm = fmaxf(mx, mw);
+        const float cc = ex2(mx - bm), cw = ex2(mw - bm);
+        acc = acc * cc + ow * cw;
+        lsum = lsum * cc + lw * cw;
         mx = bm;
     }
     const bool any = (mx != -CUDART_INF_F) && lsum > 0.f;

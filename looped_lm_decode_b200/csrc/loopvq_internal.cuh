@@ -69,7 +69,8 @@ DecodePlan plan_decode(const loopvq_cache &cc, int max_len);
 cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
                           const uint16_t *q, const int32_t *starts, int start_all, const int32_t *lens, int max_len,
                           float scale, float *out, float *lse, void *workspace, cudaStream_t s,
-                          const loopvq_tasq *tq = nullptr);
+                          const loopvq_tasq *tq = nullptr, const uint16_t *wk = nullptr,
+                          const uint16_t *wv = nullptr, const int32_t *wfill = nullptr, int W = 0);
 cudaError_t launch_tasq_encode(const loopvq_cache &cc, const loopvq_tasq &tq, int layer, int block, const void *xk,
                                const void *xv, int x_dtype, const int64_t *strides, int b0, int nb, int tok0, int ntok,
                                cudaStream_t s);

@@ -14,7 +14,8 @@
 //            one launch), move the recent slots down by 8 (one launch) and update the counters;
 //            then every sequence reserves the new token's slot.
 //   append:  the new token's K (rotated and not) and V of one (layer, loop step) go to slot fill-1.
-//   attend:  bf16 kernel over the window + coded kernel over [n_s, coded_end) + merge2.
+//   attend:  the coded kernel over [n_s, coded_end), whose merge kernel also attends to the window
+//            slots and combines both parts through their log-sum-exps (two launches in all).
 #include "encode_common.cuh"
 
 namespace loopvq {
@@ -189,52 +190,22 @@ cudaError_t launch_window_append(const loopvq_window &w, int layer, int t, const
     return cudaGetLastError();
 }
 
-// Workspace: [bf16 split partials][coded split partials][window out][window lse][coded lse]
-static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-static loopvq_bf16_cache window_view(const loopvq_window &w, int layer, int t) {
-    const int W = window_slots(w);
-    const size_t off = ((size_t)layer * w.T + t) * w.B * w.Hkv * W * w.D;
-    loopvq_bf16_cache c{};
-    c.B = w.B;
-    c.Hkv = w.Hkv;
-    c.Hq = w.Hq;
-    c.D = w.D;
-    c.Nmax = W;
-    c.k = w.k_rot + off;
-    c.v = w.v + off;
-    return c;
-}
+// Workspace: the coded kernel's partial records.
 
 size_t window_ws_bytes(const loopvq_window &w, const loopvq_cache &cc, int max_coded) {
-    const loopvq_bf16_cache view = window_view(w, 0, 0);
-    const size_t rows = (size_t)w.B * w.Hq;
-    return align256(plan_bf16(view, window_slots(w)).ws_bytes) + align256(plan_decode(cc, max_coded).ws_bytes) +
-           align256(rows * w.D * 4) + align256(rows * 4) + align256(rows * 4);
+    (void)w;
+    return plan_decode(cc, max_coded).ws_bytes;
 }
 
+// The coded kernel over tokens [n_sink, coded_end_b); its merge kernel attends to the window slots
+// [0, fill_b) of (layer, t) itself and folds them into the log-sum-exp merge (decode_kernel.cuh).
 cudaError_t launch_window_decode(const loopvq_window &w, const loopvq_cache &cc, int layer, int t, const uint16_t *q,
                                  int max_coded, float scale, float *out, float *lse, void *ws, cudaStream_t s) {
     const int W = window_slots(w);
-    const loopvq_bf16_cache view = window_view(w, layer, t);
-    const DecodePlan pb = plan_bf16(view, W);
+    const size_t off = ((size_t)layer * w.T + t) * w.B * w.Hkv * W * w.D;
     const DecodePlan pc = plan_decode(cc, max_coded);
-    const size_t rows = (size_t)w.B * w.Hq;
-    char *p = reinterpret_cast<char *>(ws);
-    void *ws_b = p;
-    p += align256(pb.ws_bytes);
-    void *ws_c = p;
-    p += align256(pc.ws_bytes);
-    float *out_w = reinterpret_cast<float *>(p);
-    p += align256(rows * w.D * 4);
-    float *lse_w = reinterpret_cast<float *>(p);
-    p += align256(rows * 4);
-    float *lse_c = lse ? lse : reinterpret_cast<float *>(p);
-    cudaError_t e = launch_bf16_decode(view, pb, q, nullptr, w.fill, W, scale, out_w, lse_w, ws_b, s);
-    if (e != cudaSuccess) return e;
-    e = launch_decode(cc, pc, layer, t, q, nullptr, w.n_sink, w.coded_end, max_coded, scale, out, lse_c, ws_c, s);
-    if (e != cudaSuccess) return e;
-    return launch_merge2(out, lse_c, out_w, lse_w, (int)rows, w.D, out, lse_c, s);
+    return launch_decode(cc, pc, layer, t, q, nullptr, w.n_sink, w.coded_end, max_coded, scale, out, lse, ws, s,
+                         nullptr, w.k_rot + off, w.v + off, w.fill, W);
 }
 
 }  // namespace loopvq

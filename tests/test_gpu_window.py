@@ -235,6 +235,7 @@ from tests.helpers import unpack_words                                 # noqa: E
 LIFE = {
     "c4tc4": WORKLOADS["ctx4k"].replace(L=2, B=2, Hkv=2, Hq=2, Nmax=128),
     "c8tc2gqa": WORKLOADS["gqa16k"].replace(L=1, T=4, Tc=2, c=8, B=2, Hkv=1, Hq=4, Nmax=128),
+    "d64qpk2": WORKLOADS["tiny"].replace(B=3, Hkv=2, Hq=4, Nmax=128),
 }
 
 
