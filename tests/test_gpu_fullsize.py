@@ -21,11 +21,11 @@ from tests.helpers import unpack_words, words_view, np_codebook_f32, attn_tolera
 pytestmark = pytest.mark.gpu
 
 SAMPLES = {"ctx32k": [(0, 0), (3, 7), (7, 15)], "ctx4k": [(0, 0), (31, 15)], "gqa16k": [(0, 0), (63, 13)],
-           "deep32": [(1, 39), (0, 17)]}
+           "deep32": [(1, 39), (0, 17)], "ctx32k_cq": [(0, 0), (6, 11)], "ctx32k_pg": [(2, 3), (7, 15)]}
 
 
 def _full_cache(w):
-    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta)
+    cache = LQ.Cache(w.L, w.T, w.Tc, w.Hkv, w.Hq, w.D, w.c, w.K, w.B, w.Nmax, w.theta, ncb=w.ncb)
     SG.fill_codebook(w, cache.codebook)
     LQ.prepare(cache)
     return cache
@@ -52,8 +52,9 @@ def test_decode_full_size_sampled(name):
         ik = random_indices(w, 0, blk, 0, b, h, range(n))
         iv = random_indices(w, 0, blk, 1, b, h, range(n))
         qb = queries(w, 0, t, b=[b], hq=[hq])[0, 0]
-        ref, lref = O.decode(bf16_bits_to_f32(qb).astype(np.float64), ik, iv, np_codebook_f32(w, 0, blk, 0, h),
-                             np_codebook_f32(w, 0, blk, 1, h), w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        dec = O.decode_pg if w.ncb > 1 else O.decode
+        ref, lref = dec(bf16_bits_to_f32(qb).astype(np.float64), ik, iv, np_codebook_f32(w, 0, blk, 0, h),
+                        np_codebook_f32(w, 0, blk, 1, h), w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
         ok, msg = attn_tolerance_ok(out[b, hq], ref, lse[b, hq:hq + 1], np.array([lref]))
         assert ok, f"{name} (b={b}, hq={hq}): {msg}"
 
