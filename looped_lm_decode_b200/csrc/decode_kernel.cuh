@@ -642,31 +642,50 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 }
 
                 // ---- reduce-scatter the scores over the slot, online-softmax update
-                float pe[QPK];
+                // Lazy maximum: the reference only has to stay within 2^8 of the running maximum for the
+                // weights to stay finite, so it moves (with an exact rescale) only when a score of the
+                // iteration exceeds it by more than 8 in log2 units.
+                float pe[QPK], sc[QPK];
+                auto lazy_max = [&](int j) {
+                    float tmax = sc[j];
+#pragma unroll
+                    for (int o = NL / 2; o >= NL / TT; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(slot_mask, tmax, o));
+                    const float corr = ex2(m_[j] - tmax);
+                    l_[j] *= corr;
+                    const float2 c2 = f2(corr, corr);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        olo[j][i] = __fmul2_rn(olo[j][i], c2);
+                        ohi[j][i] = __fmul2_rn(ohi[j][i], c2);
+                    }
+                    m_[j] = tmax;
+                };
+                if constexpr (QPK == 1) {
+                    float keep = reduce_scatter<TT, NL>(ps[0], ls, slot_mask);
+                    if constexpr (TQ) keep *= sig;
+                    sc[0] = (p0 + tk < tok_end && p0 + tk >= st) ? keep : -CUDART_INF_F;
+                    if (__any_sync(slot_mask, sc[0] > m_[0] + 8.f)) lazy_max(0);
+                } else {
+                    // one vote covers every query head (measured 15 % faster than a vote per head at 4
+                    // query heads); the rare update then checks each head
+                    bool over = false;
+                    const bool live = p0 + tk < tok_end && p0 + tk >= st;
+#pragma unroll
+                    for (int j = 0; j < QPK; ++j) {
+                        float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
+                        if constexpr (TQ) keep *= sig;
+                        sc[j] = live ? keep : -CUDART_INF_F;
+                        over |= sc[j] > m_[j] + 8.f;
+                    }
+                    if (__any_sync(slot_mask, over)) {
+#pragma unroll
+                        for (int j = 0; j < QPK; ++j)
+                            if (__any_sync(slot_mask, sc[j] > m_[j] + 8.f)) lazy_max(j);
+                    }
+                }
 #pragma unroll
                 for (int j = 0; j < QPK; ++j) {
-                    float keep = reduce_scatter<TT, NL>(ps[j], ls, slot_mask);
-                    if constexpr (TQ) keep *= sig;
-                    const float s = (p0 + tk < tok_end && p0 + tk >= st) ? keep : -CUDART_INF_F;
-                    // Lazy maximum: the reference only has to stay within 2^8 of the running maximum for
-                    // the weights to stay finite, so it moves (with an exact rescale) only when a score of
-                    // the iteration exceeds it by more than 8 in log2 units.
-                    if (__any_sync(slot_mask, s > m_[j] + 8.f)) {
-                        float tmax = s;
-#pragma unroll
-                        for (int o = NL / 2; o >= NL / TT; o >>= 1)
-                            tmax = fmaxf(tmax, __shfl_xor_sync(slot_mask, tmax, o));
-                        const float corr = ex2(m_[j] - tmax);
-                        l_[j] *= corr;
-                        const float2 c2 = f2(corr, corr);
-#pragma unroll
-                        for (int i = 0; i < 2; ++i) {
-                            olo[j][i] = __fmul2_rn(olo[j][i], c2);
-                            ohi[j][i] = __fmul2_rn(ohi[j][i], c2);
-                        }
-                        m_[j] = tmax;
-                    }
-                    pe[j] = ex2(s - m_[j]);
+                    pe[j] = ex2(sc[j] - m_[j]);
                     l_[j] += pe[j];
                 }
 
