@@ -4,7 +4,10 @@
 // LoopVQ paper, Sec. 4.3 "Attention": the quantized tokens are divided into
 // splits processed by separate thread blocks, and the partial outputs of all
 // splits are combined using the log-sum-exp of their scores.
+#include <math.h>
+
 #include "decode_kernel.cuh"
+#include "decode_mha.cuh"
 
 namespace loopvq {
 
@@ -32,6 +35,37 @@ static size_t ring_smem_bytes(bool pg, int qpk) {
     return (pg ? 131072 : 65536) + (size_t)k.depth * k.warps * 32 * 16 * kWords;
 }
 
+// decode_mha_kernel (one query head per KV head, D = 128, groups of 4 channels, one shared codebook)
+// runs the step-4 RoPE recurrence in plain form on the frequencies f < D/4 and in difference form on
+// f >= D/4; it needs |sin 4w_f| >= 0.04 on the first (the recurrence's rounding grows as 1/|sin 4w|),
+// 4w_f <= 1 on the second, and table rows 2 and 4.  With the base 1e4: min |sin 4w| = 0.046 (f = 31).
+static constexpr int kMhaWarps = 8, kMhaMinBlocks = 2, kMhaDepth = 3;
+
+static bool mha_applies(const loopvq_cache &cc) {
+    if (cc.D != 128 || cc.c != 4 || cc.Hq != cc.Hkv || ncb_of(cc) != 1 || cc.Nmax < 8) return false;
+    for (int f = 0; f < 64; ++f) {
+        const double w = pow((double)cc.theta, -2.0 * f / 128.0);
+        if (f < 32 ? fabs(sin(4.0 * w)) < 0.04 : 4.0 * w > 1.0) return false;
+    }
+    return true;
+}
+
+template <int D>
+static cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s);
+
+static cudaError_t launch_mha(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
+    using S = MhaSmem<kMhaWarps, kMhaDepth>;
+    auto kern = decode_mha_kernel<kMhaWarps, kMhaMinBlocks, kMhaDepth>;
+    cudaError_t e = ensure_dynamic_smem((const void *)kern, S::kBytes);
+    if (e != cudaSuccess) return e;
+    if (plan.ncta > 0) {
+        kern<<<plan.ncta, kMhaWarps * 32, S::kBytes, s>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return launch_merge<128>(a, s);
+}
+
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len) {
     DecodePlan p{};
     const bool pg = ncb_of(cc) > 1;
@@ -48,6 +82,7 @@ DecodePlan plan_decode(const loopvq_cache &cc, int max_len) {
     p.npiece = cc.B * cc.Hkv + p.ncta;
     p.split_len = 0;
     p.nsplit = p.ncta;
+    p.mha = mha_applies(cc);
     const size_t o_bytes = (size_t)p.npiece * qpk * cc.D * sizeof(float);
     const size_t ml_bytes = (size_t)p.npiece * qpk * sizeof(float2);
     p.ws_bytes = ((o_bytes + 255) & ~(size_t)255) + ml_bytes;
@@ -73,7 +108,12 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStr
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    // the merge as a programmatic dependent launch: it overlaps the split kernel's last CTAs
+    return launch_merge<D>(a, s);
+}
+
+// the merge as a programmatic dependent launch: it overlaps the split kernel's last CTAs
+template <int D>
+static cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.Hq);
     cfg.blockDim = dim3(D);
@@ -166,6 +206,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
         return cudaErrorInvalidValue;
     }
     const bool pg = ncb_of(cc) > 1;
+    if (plan.mha) return launch_mha(a, plan, s);
     if (cc.D == 128) return pg ? dispatch_c<128, true>(cc.c, qpk, a, plan, s) : dispatch_c<128, false>(cc.c, qpk, a, plan, s);
     if (cc.D == 64) return pg ? dispatch_c<64, true>(cc.c, qpk, a, plan, s) : dispatch_c<64, false>(cc.c, qpk, a, plan, s);
     return cudaErrorInvalidValue;

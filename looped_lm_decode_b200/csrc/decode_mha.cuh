@@ -1,0 +1,386 @@
+// Split-K decode attention over the loop-axis coded cache, one query head per KV head, D = 128,
+// channel groups of 4 (the looped-decoder workloads): a kernel with 8 RoPE pairs per lane and the
+// value accumulation on the tensor cores.
+//
+// LoopVQ paper, Sec. 4.3 "Attention" and App. C: every index is looked up in the loop step's
+// codebook slice held in shared memory, keys are rebuilt before RoPE and rotated at their positions,
+// and the tokens are cut into splits whose partial outputs are merged through their log-sum-exp.
+//
+// Design (B200, sm_100a):
+//  * The tile space, pieces, slice staging (bank-private replicas) and partial records are those of
+//    decode_split_kernel (decode_kernel.cuh), and its merge kernel combines the records.
+//  * A warp takes a contiguous run of 16-token tiles of the piece.  Lane (g, t) = (lane / 4, lane % 4)
+//    owns the tokens t, t + 4, t + 8, t + 12 of each tile and the two pair-groups g and g + 8: the
+//    channel groups g, g + 8 (low channels) and g + 16, g + 24 (their RoPE partners), 8 RoPE pairs.
+//    Its positions advance by 4 from token to token and from tile to tile.
+//  * Keys: the query is rotated instead of the keys, Z_f(n) = (q_f + i q_{f+D/2}) e^{-i n w_f}, and the
+//    score is the sum over pairs of Re(Z_f) k_f + Im(Z_f) k_{f+D/2}.  Along a lane's positions Z follows
+//    X_{j+1} = 2 cos(4w) X_j - X_{j-1}.  For the 4 high-frequency pairs (|sin 4w| bounded away from 0)
+//    that is one fused multiply-add per component and step.  For the 4 low-frequency pairs the same
+//    recurrence is run in the difference form D_{j+1} = D_j - 4 sin^2(2w) X_j, X_{j+1} = X_j + D_{j+1}
+//    (Reinsch), whose coefficient keeps full relative precision as w -> 0.  Both are set from the
+//    table every 16 tiles, which bounds the rounding drift to 64 steps.
+//  * The lane's 4 partial scores are reduce-scattered over the 8 lanes of its t (3 exchanges); each
+//    lane finishes one token.  The softmax maximum is one value per warp, lazy (it moves, with an exact
+//    rescale, only when a score exceeds it by more than 8 in log2 units).
+//  * Values: out^T += Vhat^T P^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate).  A fragments are
+//    the gathered bf16 value entries, re-paired across two tokens by one byte permute per register (no
+//    conversion to fp32).  The B fragment holds each weight split into bf16 hi + lo parts (column 0:
+//    the hi parts, column 1: the lo parts), which represents the fp32 weight to about 2^-16 relative;
+//    the two accumulator columns are added at the end.
+//  * Index words arrive through a per-warp ring of 1 KiB stages in shared memory filled with 16-byte
+//    cp.async copies (lane L copies chunks L and L + 32 of the tile); each lane reads its 8 words with
+//    conflict-free 4-byte loads.
+#pragma once
+
+#include "decode_kernel.cuh"
+
+namespace loopvq {
+
+__device__ __forceinline__ uint32_t cvt_bf16x2(float hi_elem, float lo_elem) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi_elem), "f"(lo_elem));
+    return r;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float4 &d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d.x), "+f"(d.y), "+f"(d.z), "+f"(d.w)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst_smem, const void *src, bool full) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(full ? 16 : 0)
+                 : "memory");
+}
+
+// Shared memory of the kernel: K/V replicas, then the index ring, then the warp records.
+template <int WARPS, int DEPTH>
+struct MhaSmem {
+    static constexpr uint32_t kTables = 65536u;
+    static constexpr uint32_t kRing = kTables;
+    static constexpr uint32_t kRingBytes = (uint32_t)WARPS * DEPTH * 1024u;
+    static constexpr uint32_t kRec = kRing + kRingBytes;
+    static constexpr uint32_t kRecFloats = 128 + 4;
+    static constexpr uint32_t kBytes = kRec + (uint32_t)WARPS * kRecFloats * 4u;
+};
+
+template <int WARPS, int MINB, int DEPTH>
+__global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const DecodeArgs a) {
+    constexpr int D = 128, NP = 16;                        // pair-groups = index words per token
+    constexpr int NT = WARPS * 32;
+    constexpr int ANCHOR = 16;                             // tiles between two settings from the table
+    using S = MhaSmem<WARPS, DEPTH>;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ long long range_info[4];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    asm volatile("griddepcontrol.launch_dependents;");
+    if (warp == 0) cta_range(a, lane, range_info);
+    __syncthreads();
+    long long pos = range_info[0];
+    const long long x_end = range_info[1];
+    long long seg0 = range_info[2];
+    int h = (int)(range_info[3] >> 32), b = (int)(range_info[3] & 0xffffffffLL);
+
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t colk = (uint32_t)((lane & 15) * 8);      // the lane's replica column (K half-row)
+    const uint32_t colv = colk + 128u;                      // and in the V half-row
+    const uint32_t smem_base = (uint32_t)__cvta_generic_to_shared(smem);
+    const uint32_t ring = smem_base + S::kRing + (uint32_t)warp * DEPTH * 1024u;
+    float *rec = reinterpret_cast<float *>(smem + S::kRec) + warp * S::kRecFloats;
+
+    // recurrence coefficients of the lane's pairs: high pairs f = 4g + e (2 cos 4w), low pairs
+    // f = 32 + 4g + e (-4 sin^2 2w); from table rows 4 and 2
+    float2 tcA[2], nlB[2];
+    {
+        const float4 c4 = __ldg(reinterpret_cast<const float4 *>(a.rope + 4 * D + 4 * g));
+        const float4 s2 = __ldg(reinterpret_cast<const float4 *>(a.rope + 2 * D + D / 2 + 32 + 4 * g));
+        tcA[0] = f2(2.f * c4.x, 2.f * c4.y);
+        tcA[1] = f2(2.f * c4.z, 2.f * c4.w);
+        nlB[0] = f2(-4.f * s2.x * s2.x, -4.f * s2.y * s2.y);
+        nlB[1] = f2(-4.f * s2.z * s2.z, -4.f * s2.w * s2.w);
+    }
+
+    while (pos < x_end && h < a.Hkv) {
+        int len, st, base;
+        const long long seg_end = seg0 + seq_tiles(a, b, base, st, len);
+        const long long pend = seg_end < x_end ? seg_end : x_end;
+        if (pend > pos) {
+            const int piece = h * a.B + b + (int)blockIdx.x;
+            const int tok_begin = base + 4 * (int)(pos - seg0);
+            const int tok_end = min(base + 4 * (int)(pend - seg0), len);
+            const int n4 = (int)(pend - pos);              // four-token tiles of the piece
+            const int n16 = (n4 + 3) >> 2;
+            __syncthreads();                               // the previous piece's tables and records are done
+
+            // stage the K and V slices of head h as bank-private replicas (rows >= K zeroed)
+            {
+                const uint16_t *sk = a.slk + (size_t)h * a.K * 4;
+                const uint16_t *sv = a.slv + (size_t)h * a.K * 4;
+                for (int it = tid; it < 256 * 2 * 16; it += NT) {
+                    const int rep = it & 15;
+                    const int kv = (it >> 4) & 1;
+                    const int r = it >> 5;
+                    uint2 v = make_uint2(0u, 0u);
+                    if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>((kv ? sv : sk) + (size_t)r * 4));
+                    *reinterpret_cast<uint2 *>(smem + r * 256 + kv * 128 + rep * 8) = v;
+                }
+            }
+
+            // this warp's run of 16-token tiles [i0, i1) of the piece
+            const int i0 = (int)((long long)warp * n16 / WARPS), i1 = (int)((long long)(warp + 1) * n16 / WARPS);
+            const int kown = 2 * (g & 1) + ((g >> 1) & 1);  // the token (0..3) this lane finishes
+            // index copies: lane L takes chunks L (four-tile L / 16) and L + 32 (four-tile L / 16 + 2)
+            const int kc = lane >> 4;
+            const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP;
+            const char *src = reinterpret_cast<const char *>(idx_b + ((size_t)((tok_begin >> 2) + 4 * i0 + kc) * NP + (lane & 15)) * 4);
+            const uint32_t dst = ring + (uint32_t)lane * 16u;
+            int crem = n4 - 4 * i0, ctl = i1 - i0;         // four-tiles of the piece / tiles of the warp, from the copy on
+            auto copy_tile = [&](uint32_t soff) {
+                const bool f0 = ctl > 0 && crem > kc, f1 = ctl > 0 && crem > kc + 2;
+                // a chunk outside the piece reads nothing (source size 0) from a valid address
+                cp_async16_zfill(dst + soff, f0 ? src : reinterpret_cast<const char *>(a.idx), f0);
+                cp_async16_zfill(dst + soff + 512u, f1 ? src + 512 : reinterpret_cast<const char *>(a.idx), f1);
+                cp_async_commit();
+                src += 1024;
+                crem -= 4;
+                --ctl;
+            };
+#pragma unroll
+            for (int d = 0; d < DEPTH; ++d) copy_tile((uint32_t)d * 1024u);
+
+            float4 acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            float m = -1e30f, l = 0.f;
+            float2 zar[2], zai[2], par[2], pai[2];         // high pairs: X_j and X_{j-1} (re, im)
+            float2 zbr[2], zbi[2], dbr[2], dbi[2];         // low pairs: X_j and D_j = X_j - X_{j-1}
+            // the lane's finished token n is attended iff 0 <= n - st < tok_end - st
+            int nrel = tok_begin + 16 * i0 + t + 4 * kown - st;
+            const unsigned span = (unsigned)(tok_end - st);
+            const unsigned char *wrd = smem + S::kRing + (uint32_t)warp * DEPTH * 1024u + 4u * (4 * g + t);
+            uint32_t soff = 0;
+            __syncthreads();                               // tables staged
+
+            for (int ib = i0; ib < i1; ib += ANCHOR) {
+                {
+                    // X at the lane's first position n0 from the table and the query; the second state from
+                    // X(n0 - 4) = X(n0) e^{+4iw}
+                    const int n0 = tok_begin + 16 * ib + t;
+                    const float *row = a.rope + (size_t)min(n0, a.Nmax - 1) * D;
+                    const uint16_t *qp = a.q + ((size_t)b * a.Hq + h) * D;
+                    const float4 cA = __ldg(reinterpret_cast<const float4 *>(row + 4 * g));
+                    const float4 sA = __ldg(reinterpret_cast<const float4 *>(row + D / 2 + 4 * g));
+                    const float4 cB = __ldg(reinterpret_cast<const float4 *>(row + 32 + 4 * g));
+                    const float4 sB = __ldg(reinterpret_cast<const float4 *>(row + D / 2 + 32 + 4 * g));
+                    const uint2 qal = __ldg(reinterpret_cast<const uint2 *>(qp + 4 * g));
+                    const uint2 qah = __ldg(reinterpret_cast<const uint2 *>(qp + D / 2 + 4 * g));
+                    const uint2 qbl = __ldg(reinterpret_cast<const uint2 *>(qp + 32 + 4 * g));
+                    const uint2 qbh = __ldg(reinterpret_cast<const uint2 *>(qp + D / 2 + 32 + 4 * g));
+                    const float4 c4A = __ldg(reinterpret_cast<const float4 *>(a.rope + 4 * D + 4 * g));
+                    const float4 s4A = __ldg(reinterpret_cast<const float4 *>(a.rope + 4 * D + D / 2 + 4 * g));
+                    const float4 s4B = __ldg(reinterpret_cast<const float4 *>(a.rope + 4 * D + D / 2 + 32 + 4 * g));
+                    const float4 s2B = __ldg(reinterpret_cast<const float4 *>(a.rope + 2 * D + D / 2 + 32 + 4 * g));
+                    const float qs = a.qscale;
+                    const float2 ql[2][2] = {{f2(bf16lo(qal.x) * qs, bf16hi(qal.x) * qs), f2(bf16lo(qal.y) * qs, bf16hi(qal.y) * qs)},
+                                             {f2(bf16lo(qbl.x) * qs, bf16hi(qbl.x) * qs), f2(bf16lo(qbl.y) * qs, bf16hi(qbl.y) * qs)}};
+                    const float2 qh[2][2] = {{f2(bf16lo(qah.x) * qs, bf16hi(qah.x) * qs), f2(bf16lo(qah.y) * qs, bf16hi(qah.y) * qs)},
+                                             {f2(bf16lo(qbh.x) * qs, bf16hi(qbh.x) * qs), f2(bf16lo(qbh.y) * qs, bf16hi(qbh.y) * qs)}};
+                    const float2 cs[2][2] = {{f2(cA.x, cA.y), f2(cA.z, cA.w)}, {f2(cB.x, cB.y), f2(cB.z, cB.w)}};
+                    const float2 sn[2][2] = {{f2(sA.x, sA.y), f2(sA.z, sA.w)}, {f2(sB.x, sB.y), f2(sB.z, sB.w)}};
+                    float2 zr[2][2], zi[2][2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            // Z = (ql + i qh)(cos - i sin)
+                            zr[u][e] = __ffma2_rn(ql[u][e], cs[u][e], __fmul2_rn(qh[u][e], sn[u][e]));
+                            zi[u][e] = __ffma2_rn(qh[u][e], cs[u][e], __fmul2_rn(neg2(ql[u][e]), sn[u][e]));
+                        }
+                    const float2 c4[2] = {f2(c4A.x, c4A.y), f2(c4A.z, c4A.w)};
+                    const float2 s4[2] = {f2(s4A.x, s4A.y), f2(s4A.z, s4A.w)};
+                    const float2 sb4[2] = {f2(s4B.x, s4B.y), f2(s4B.z, s4B.w)};
+                    const float2 al[2] = {f2(2.f * s2B.x * s2B.x, 2.f * s2B.y * s2B.y),
+                                          f2(2.f * s2B.z * s2B.z, 2.f * s2B.w * s2B.w)};
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        zar[e] = zr[0][e];
+                        zai[e] = zi[0][e];
+                        // X(n0 - 4) = X (cos 4w + i sin 4w)
+                        par[e] = __ffma2_rn(zr[0][e], c4[e], __fmul2_rn(neg2(zi[0][e]), s4[e]));
+                        pai[e] = __ffma2_rn(zi[0][e], c4[e], __fmul2_rn(zr[0][e], s4[e]));
+                        zbr[e] = zr[1][e];
+                        zbi[e] = zi[1][e];
+                        // D = X (1 - e^{4iw}) = X (2 sin^2 2w - i sin 4w)
+                        dbr[e] = __ffma2_rn(zr[1][e], al[e], __fmul2_rn(zi[1][e], sb4[e]));
+                        dbi[e] = __ffma2_rn(zi[1][e], al[e], __fmul2_rn(neg2(zr[1][e]), sb4[e]));
+                    }
+                }
+
+                const int ie = min(ib + ANCHOR, i1);
+                for (int i = ib; i < ie; ++i) {
+                    cp_async_wait<DEPTH - 1>();
+                    __syncwarp();
+                    const uint32_t *wp = reinterpret_cast<const uint32_t *>(wrd + soff);
+                    uint32_t wa[4], wb[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        wa[k] = wp[64 * k];                // four-tile k, pair-group g, token t
+                        wb[k] = wp[64 * k + 32];           // pair-group g + 8
+                    }
+
+                    // ---- keys: gather, rebuild, score the lane's 4 tokens over its 8 pairs
+                    float s[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint2 e0 = lds64(smem, __byte_perm(wa[k], colk, 0x7604));   // group g
+                        const uint2 e1 = lds64(smem, __byte_perm(wa[k], colk, 0x7614));   // group g + 16
+                        const uint2 e2 = lds64(smem, __byte_perm(wb[k], colk, 0x7604));   // group g + 8
+                        const uint2 e3 = lds64(smem, __byte_perm(wb[k], colk, 0x7614));   // group g + 24
+                        float2 sc2 = __fmul2_rn(zar[0], unpack2(e0.x));
+                        sc2 = __ffma2_rn(zar[1], unpack2(e0.y), sc2);
+                        sc2 = __ffma2_rn(zai[0], unpack2(e1.x), sc2);
+                        sc2 = __ffma2_rn(zai[1], unpack2(e1.y), sc2);
+                        sc2 = __ffma2_rn(zbr[0], unpack2(e2.x), sc2);
+                        sc2 = __ffma2_rn(zbr[1], unpack2(e2.y), sc2);
+                        sc2 = __ffma2_rn(zbi[0], unpack2(e3.x), sc2);
+                        sc2 = __ffma2_rn(zbi[1], unpack2(e3.y), sc2);
+                        s[k] = sc2.x + sc2.y;
+                        // advance every pair by 4 positions
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float2 nr = __ffma2_rn(tcA[e], zar[e], neg2(par[e]));
+                            const float2 ni = __ffma2_rn(tcA[e], zai[e], neg2(pai[e]));
+                            par[e] = zar[e];
+                            pai[e] = zai[e];
+                            zar[e] = nr;
+                            zai[e] = ni;
+                            dbr[e] = __ffma2_rn(nlB[e], zbr[e], dbr[e]);
+                            dbi[e] = __ffma2_rn(nlB[e], zbi[e], dbi[e]);
+                            zbr[e] = __fadd2_rn(zbr[e], dbr[e]);
+                            zbi[e] = __fadd2_rn(zbi[e], dbi[e]);
+                        }
+                    }
+                    // the stage's words are in registers: refill it with the tile DEPTH ahead
+                    __syncwarp();
+                    copy_tile(soff);
+                    soff = soff + 1024u == DEPTH * 1024u ? 0u : soff + 1024u;
+
+                    // ---- reduce-scatter over the 8 lanes of this t: lane (g, t) ends with token kown
+                    float sk;
+                    {
+                        const bool b1 = (g & 1) != 0, b2 = (g & 2) != 0;
+                        const float k0 = b1 ? s[2] : s[0], k1 = b1 ? s[3] : s[1];
+                        const float o0 = b1 ? s[0] : s[2], o1 = b1 ? s[1] : s[3];
+                        const float a0 = k0 + __shfl_xor_sync(0xffffffffu, o0, 4);
+                        const float a1 = k1 + __shfl_xor_sync(0xffffffffu, o1, 4);
+                        const float kk = b2 ? a1 : a0, oo = b2 ? a0 : a1;
+                        sk = kk + __shfl_xor_sync(0xffffffffu, oo, 8);
+                        sk += __shfl_xor_sync(0xffffffffu, sk, 16);
+                    }
+                    sk = (unsigned)nrel < span ? sk : -CUDART_INF_F;
+                    nrel += 16;
+
+                    // ---- online softmax, one lazy maximum per warp
+                    if (__any_sync(0xffffffffu, sk > m + 8.f)) {
+                        float tmax = sk;
+#pragma unroll
+                        for (int o = 16; o >= 1; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+                        const float corr = ex2(m - tmax);
+                        l *= corr;
+                        const float2 c2 = f2(corr, corr);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float2 lo2 = __fmul2_rn(f2(acc[j].x, acc[j].y), c2), hi2 = __fmul2_rn(f2(acc[j].z, acc[j].w), c2);
+                            acc[j] = make_float4(lo2.x, lo2.y, hi2.x, hi2.y);
+                        }
+                        m = tmax;
+                    }
+                    const float p = ex2(sk - m);
+                    l += p;
+
+                    // ---- weights to the B fragment: {bf16 hi part, bf16 lo part} per token, routed to the
+                    // lanes of columns 0 (hi) and 1 (lo); other columns carry unused values
+                    uint32_t bq0, bq1;
+                    {
+                        const float hv = __uint_as_float(__float_as_uint(p) & 0xffff0000u);
+                        const uint32_t x = cvt_bf16x2(p - hv, hv);        // upper: lo part, lower: hi part
+                        // token k is finished by lane 4 g'(k) + t, g'(k) = (k >> 1) | ((k & 1) << 1)
+                        const uint32_t x0 = __shfl_sync(0xffffffffu, x, t);
+                        const uint32_t x1 = __shfl_sync(0xffffffffu, x, 8 + t);
+                        const uint32_t x2 = __shfl_sync(0xffffffffu, x, 4 + t);
+                        const uint32_t x3 = __shfl_sync(0xffffffffu, x, 12 + t);
+                        const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;
+                        bq0 = __byte_perm(x0, x1, sel);    // k-slots 2t, 2t + 1: tokens k = 0, 1
+                        bq1 = __byte_perm(x2, x3, sel);    // k-slots 2t + 8, 2t + 9: tokens k = 2, 3
+                    }
+
+                    // ---- values: group 8u + g, m-tiles 2u (channels e = 0, 1) and 2u + 1 (e = 2, 3)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t sel = (u < 2) ? 0x7624u : 0x7634u;
+                        uint2 v[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) v[k] = lds64(smem, __byte_perm((u & 1) ? wb[k] : wa[k], colv, sel));
+                        mma_bf16_16816(acc[2 * u], __byte_perm(v[0].x, v[1].x, 0x5410), __byte_perm(v[0].x, v[1].x, 0x7632),
+                                       __byte_perm(v[2].x, v[3].x, 0x5410), __byte_perm(v[2].x, v[3].x, 0x7632), bq0, bq1);
+                        mma_bf16_16816(acc[2 * u + 1], __byte_perm(v[0].y, v[1].y, 0x5410), __byte_perm(v[0].y, v[1].y, 0x7632),
+                                       __byte_perm(v[2].y, v[3].y, 0x5410), __byte_perm(v[2].y, v[3].y, 0x7632), bq0, bq1);
+                    }
+                }
+            }
+            cp_async_wait<0>();
+
+            // ---- the warp's record: lanes t = 0 hold columns 0 (hi) and 1 (lo) of every m-tile
+            {
+                float lsum = l;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+                lsum *= 0.5f;                              // every token is finished by two lanes
+                if (t == 0) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int ch = 4 * (8 * (j >> 1) + g) + 2 * (j & 1);
+                        rec[ch] = acc[j].x + acc[j].y;
+                        rec[ch + 1] = acc[j].z + acc[j].w;
+                    }
+                }
+                if (lane == 0) {
+                    rec[D] = lsum > 0.f ? m : -CUDART_INF_F;
+                    rec[D + 1] = lsum;
+                }
+            }
+            __syncthreads();
+            // ---- combine the warps, write the piece's partial record
+            {
+                const float *recs = reinterpret_cast<const float *>(smem + S::kRec);
+                for (int d = tid; d < D; d += NT) {
+                    float mx = -CUDART_INF_F;
+                    for (int w = 0; w < WARPS; ++w) mx = fmaxf(mx, recs[w * S::kRecFloats + D]);
+                    float o = 0.f, lsum = 0.f;
+                    if (mx != -CUDART_INF_F) {
+                        for (int w = 0; w < WARPS; ++w) {
+                            const float *r = recs + w * S::kRecFloats;
+                            const float wgt = ex2(r[D] - mx);
+                            o += r[d] * wgt;
+                            lsum += r[D + 1] * wgt;
+                        }
+                    }
+                    a.ws_o[(size_t)piece * D + d] = o;
+                    if (d == 0) a.ws_ml[piece] = f2(mx, lsum);
+                }
+            }
+            pos = pend;
+        }
+        seg0 = seg_end;
+        if (++b == a.B) {
+            b = 0;
+            ++h;
+        }
+    }
+}
+
+}  // namespace loopvq

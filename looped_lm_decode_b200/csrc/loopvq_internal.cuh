@@ -63,6 +63,7 @@ struct DecodePlan {
     int npiece;         // coded kernel: partial records (segments + CTAs)
     int nbt;            // sequences per thread block
     int nchunk;         // ceil(B / nbt)
+    bool mha;           // coded kernel: decode_mha_kernel applies (one query head per KV head, D 128, c 4)
     size_t ws_bytes;    // workspace needed
 };
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len);
