@@ -83,17 +83,27 @@ def job_throughput(world, bytes_per_step_per_rank, ms_per_step_max):
     return world * bytes_per_step_per_rank / (ms_per_step_max * 1e-3) / 1e9
 
 
-def profiled_traffic(workload_name):
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if that summary was
-    taken from the kernel sources as they are now (else None)."""
+def decode_kernel_name(w):
+    """The split kernel a plain decode call of workload w runs: decode_mha_kernel for one query head per
+    KV head at D = 128 with groups of 4 channels and a shared codebook, decode_split_kernel otherwise."""
+    mha = w.D == 128 and w.c == 4 and w.Hq == w.Hkv and w.ncb == 1 and not w.tasq
+    return "decode_mha" if mha else "decode_split"
+
+
+def profiled_traffic(w):
+    """DRAM bytes per launch of the decode split kernel from the committed ncu summary, if that summary
+    was taken from the kernel sources as they are now (else None)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"decode_split_{workload_name}.json")
+    kern = decode_kernel_name(w)
+    path = os.path.join(ROOT, "profiles", f"{kern}_{w.name}.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         prof = json.load(f)
     h = hashlib.sha256()
-    for src in ("decode_kernel.cuh", "decode_attn.cu"):
+    srcs = ("decode_mha.cuh", "decode_kernel.cuh", "decode_attn.cu") if kern == "decode_mha" else \
+        ("decode_kernel.cuh", "decode_attn.cu")
+    for src in srcs:
         with open(os.path.join(ROOT, "looped_lm_decode_b200", "csrc", src), "rb") as f:
             h.update(f.read())
     if h.hexdigest()[:16] != prof.get("kernel_sources_sha256_16"):
@@ -534,8 +544,8 @@ def main():
             "config": dict(workload_desc(w), parallelism=("replicas" if world > 1 else "single GPU")),
             "us_per_step": ms_step * 1e3, "us_per_call": avg_call_ms * 1e3, "calls_per_step": ncall,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": profiled_traffic(w.name), "peak_kind": peak_kind,
-                         "kernel": "one loopvq_decode_attn call (split kernel + merge kernel)",
+                         "frac": achieved / hbm_peak, "traffic": profiled_traffic(w), "peak_kind": peak_kind,
+                         "kernel": f"one loopvq_decode_attn call ({decode_kernel_name(w)}_kernel + merge_kernel)",
                          "bytes_per_launch": cb},
             "smem_gather": {"achieved": smem_achieved, "peak": smem_peak, "unit": "GB/s",
                             "frac": smem_achieved / smem_peak, "bytes_per_launch": gb,

@@ -326,7 +326,7 @@ loopvq_status loopvq_tasq_decode_attn(const loopvq_cache *cc, const loopvq_tasq 
         return fail(LOOPVQ_ERR_INVALID_ARG, "max_len=%d out of [0, Nmax=%d]", max_len, cc->Nmax);
     if (!std::isfinite(scale)) return fail(LOOPVQ_ERR_INVALID_ARG, "scale is not finite");
     if (scale <= 0.f) scale = 1.0f / std::sqrt((float)cc->D);
-    const loopvq::DecodePlan plan = loopvq::plan_decode(*cc, max_len);
+    const loopvq::DecodePlan plan = loopvq::plan_decode(*cc, max_len, true);
     if (plan.nsplit > 65535) return fail(LOOPVQ_ERR_UNSUPPORTED, "too many splits");
     if (!workspace || ws_bytes < plan.ws_bytes)
         return fail(LOOPVQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws_bytes,

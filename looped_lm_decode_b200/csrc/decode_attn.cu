@@ -17,7 +17,9 @@ namespace loopvq {
 // codebook, two CTAs of 8 warps per SM (64 KiB of slice replicas plus a 2-deep prefetch queue each;
 // the shared memory left over serves as L1 for the RoPE rows); with one codebook per channel group,
 // one CTA of 16 warps per SM (128 KiB of tables).  Measured at ctx32k: a second wave, or three CTAs
-// per SM at 80 registers, is 3 to 10 % slower.
+// per SM at 80 registers, is 3 to 10 % slower.  decode_mha_kernel runs one CTA of 16 warps per SM
+// (one copy of the tables per SM, 2-deep index ring per warp): 124 us per ctx32k call, against 129 us
+// for two CTAs of 8 warps and 126 us with a 3-deep ring.
 
 static constexpr int kSms = 148;                           // B200; more CTAs than fit only add a wave
 static constexpr int kWords = 1;                           // index words per lane per iteration (4-token tiles)
@@ -39,7 +41,7 @@ static size_t ring_smem_bytes(bool pg, int qpk) {
 // runs the step-4 RoPE recurrence in plain form on the frequencies f < D/4 and in difference form on
 // f >= D/4; it needs |sin 4w_f| >= 0.04 on the first (the recurrence's rounding grows as 1/|sin 4w|),
 // 4w_f <= 1 on the second, and table rows 2 and 4.  With the base 1e4: min |sin 4w| = 0.046 (f = 31).
-static constexpr int kMhaWarps = 8, kMhaMinBlocks = 2, kMhaDepth = 3;
+static constexpr int kMhaWarps = 16, kMhaMinBlocks = 1, kMhaDepth = 2;
 
 static bool mha_applies(const loopvq_cache &cc) {
     if (cc.D != 128 || cc.c != 4 || cc.Hq != cc.Hkv || ncb_of(cc) != 1 || cc.Nmax < 8) return false;
@@ -66,25 +68,27 @@ static cudaError_t launch_mha(const DecodeArgs &a, const DecodePlan &plan, cudaS
     return launch_merge<128>(a, s);
 }
 
-DecodePlan plan_decode(const loopvq_cache &cc, int max_len) {
+DecodePlan plan_decode(const loopvq_cache &cc, int max_len, bool tasq) {
     DecodePlan p{};
     const bool pg = ncb_of(cc) > 1;
     const int qpk = cc.Hq / cc.Hkv;
     const KernelShape k = kernel_shape(pg, qpk);
     p.nbt = 1;
     p.nchunk = cc.B;
+    p.mha = !tasq && mha_applies(cc);
     // an upper bound of the tiles: every sequence at max_len
     const long tiles = (long)cc.B * cc.Hkv * ((max_len + 3) / 4);
-    long g = (tiles + kMinTiles - 1) / kMinTiles;
-    const long cap = (long)kSms * k.min_blocks;
-    if (g > cap) g = cap;
-    p.ncta = max_len > 0 ? (int)g : 0;
+    const long g = (tiles + kMinTiles - 1) / kMinTiles;
+    const long cap = (long)kSms * (p.mha ? kMhaMinBlocks : k.min_blocks);
+    p.ncta = max_len > 0 ? (int)(g < cap ? g : cap) : 0;
     p.npiece = cc.B * cc.Hkv + p.ncta;
     p.split_len = 0;
     p.nsplit = p.ncta;
-    p.mha = mha_applies(cc);
-    const size_t o_bytes = (size_t)p.npiece * qpk * cc.D * sizeof(float);
-    const size_t ml_bytes = (size_t)p.npiece * qpk * sizeof(float2);
+    // the workspace covers either kernel's records, so one size serves plain and TaSQ calls
+    const long cap_ws = (long)kSms * (k.min_blocks > kMhaMinBlocks ? k.min_blocks : kMhaMinBlocks);
+    const long npiece_ws = (long)cc.B * cc.Hkv + (max_len > 0 ? (g < cap_ws ? g : cap_ws) : 0);
+    const size_t o_bytes = (size_t)npiece_ws * qpk * cc.D * sizeof(float);
+    const size_t ml_bytes = (size_t)npiece_ws * qpk * sizeof(float2);
     p.ws_bytes = ((o_bytes + 255) & ~(size_t)255) + ml_bytes;
     return p;
 }

@@ -66,7 +66,7 @@ struct DecodePlan {
     bool mha;           // coded kernel: decode_mha_kernel applies (one query head per KV head, D 128, c 4)
     size_t ws_bytes;    // workspace needed
 };
-DecodePlan plan_decode(const loopvq_cache &cc, int max_len);
+DecodePlan plan_decode(const loopvq_cache &cc, int max_len, bool tasq = false);
 cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
                           const uint16_t *q, const int32_t *starts, int start_all, const int32_t *lens, int max_len,
                           float scale, float *out, float *lse, void *workspace, cudaStream_t s,
