@@ -7,6 +7,7 @@
 #include <math.h>
 
 #include "decode_kernel.cuh"
+#include "decode_gqa.cuh"
 #include "decode_mha.cuh"
 
 namespace loopvq {
@@ -55,6 +56,27 @@ static bool mha_applies(const loopvq_cache &cc) {
 template <int D>
 static cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s);
 
+// decode_gqa_kernel (4 query heads per KV head, D = 128, groups of 8 channels, one shared codebook):
+// one CTA of 8 warps per SM (251 registers per thread), 2-stage index ring per warp.
+static constexpr int kGqaWarps = 8, kGqaMinBlocks = 1, kGqaDepth = 2;
+
+static bool gqa_applies(const loopvq_cache &cc) {
+    return cc.D == 128 && cc.c == 8 && cc.Hq == 4 * cc.Hkv && ncb_of(cc) == 1 && cc.Nmax >= 8;
+}
+
+static cudaError_t launch_gqa(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
+    using S = GqaSmem<kGqaWarps, kGqaDepth>;
+    auto kern = decode_gqa_kernel<kGqaWarps, kGqaMinBlocks, kGqaDepth>;
+    cudaError_t e = ensure_dynamic_smem((const void *)kern, S::kBytes);
+    if (e != cudaSuccess) return e;
+    if (plan.ncta > 0) {
+        kern<<<plan.ncta, kGqaWarps * 32, S::kBytes, s>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return launch_merge<128>(a, s);
+}
+
 static cudaError_t launch_mha(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
     using S = MhaSmem<kMhaWarps, kMhaDepth>;
     auto kern = decode_mha_kernel<kMhaWarps, kMhaMinBlocks, kMhaDepth>;
@@ -76,10 +98,11 @@ DecodePlan plan_decode(const loopvq_cache &cc, int max_len, bool tasq) {
     p.nbt = 1;
     p.nchunk = cc.B;
     p.mha = !tasq && mha_applies(cc);
+    p.gqa = !tasq && gqa_applies(cc);
     // an upper bound of the tiles: every sequence at max_len
     const long tiles = (long)cc.B * cc.Hkv * ((max_len + 3) / 4);
     const long g = (tiles + kMinTiles - 1) / kMinTiles;
-    const long cap = (long)kSms * (p.mha ? kMhaMinBlocks : k.min_blocks);
+    const long cap = (long)kSms * (p.mha ? kMhaMinBlocks : p.gqa ? kGqaMinBlocks : k.min_blocks);
     p.ncta = max_len > 0 ? (int)(g < cap ? g : cap) : 0;
     p.npiece = cc.B * cc.Hkv + p.ncta;
     p.split_len = 0;
@@ -211,6 +234,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     }
     const bool pg = ncb_of(cc) > 1;
     if (plan.mha) return launch_mha(a, plan, s);
+    if (plan.gqa) return launch_gqa(a, plan, s);
     if (cc.D == 128) return pg ? dispatch_c<128, true>(cc.c, qpk, a, plan, s) : dispatch_c<128, false>(cc.c, qpk, a, plan, s);
     if (cc.D == 64) return pg ? dispatch_c<64, true>(cc.c, qpk, a, plan, s) : dispatch_c<64, false>(cc.c, qpk, a, plan, s);
     return cudaErrorInvalidValue;

@@ -64,6 +64,7 @@ struct DecodePlan {
     int nbt;            // sequences per thread block
     int nchunk;         // ceil(B / nbt)
     bool mha;           // coded kernel: decode_mha_kernel applies (one query head per KV head, D 128, c 4)
+    bool gqa;           // coded kernel: decode_gqa_kernel applies (4 query heads per KV head, D 128, c 8)
     size_t ws_bytes;    // workspace needed
 };
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len, bool tasq = false);
