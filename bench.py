@@ -85,28 +85,44 @@ def job_throughput(world, bytes_per_step_per_rank, ms_per_step_max):
 
 def decode_kernel_name(w):
     """The split kernel a plain decode call of workload w runs: decode_mha_kernel for one query head per
-    KV head at D = 128 with groups of 4 channels and a shared codebook, decode_split_kernel otherwise."""
-    mha = w.D == 128 and w.c == 4 and w.Hq == w.Hkv and w.ncb == 1 and not w.tasq
-    return "decode_mha" if mha else "decode_split"
+    KV head at D = 128 with groups of 4 channels, decode_gqa_kernel for 4 query heads per KV head at
+    D = 128 with groups of 8 (both with a shared codebook), decode_split_kernel otherwise."""
+    if w.D == 128 and w.ncb == 1 and not w.tasq:
+        if w.c == 4 and w.Hq == w.Hkv:
+            return "decode_mha"
+        if w.c == 8 and w.Hq == 4 * w.Hkv:
+            return "decode_gqa"
+    return "decode_split"
+
+
+def kernel_sources_hash(kern):
+    """Hash of what decides a decode split kernel's code and launch: its headers, and for the MHA and GQA
+    kernels the line of decode_attn.cu that fixes their launch shape (the whole file otherwise)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "looped_lm_decode_b200", "csrc")
+    h = hashlib.sha256()
+    heads = {"decode_mha": ("decode_mha.cuh", "decode_kernel.cuh"),
+             "decode_gqa": ("decode_gqa.cuh", "decode_mha.cuh", "decode_kernel.cuh")}.get(kern, ("decode_kernel.cuh",))
+    for src in heads:
+        with open(os.path.join(csrc, src), "rb") as f:
+            h.update(f.read())
+    with open(os.path.join(csrc, "decode_attn.cu"), "rb") as f:
+        attn = f.read()
+    tag = {"decode_mha": b"static constexpr int kMhaWarps", "decode_gqa": b"static constexpr int kGqaWarps"}.get(kern)
+    h.update(attn if tag is None else next(ln for ln in attn.splitlines() if ln.startswith(tag)))
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(w):
     """DRAM bytes per launch of the decode split kernel from the committed ncu summary, if that summary
     was taken from the kernel sources as they are now (else None)."""
-    import hashlib
     kern = decode_kernel_name(w)
     path = os.path.join(ROOT, "profiles", f"{kern}_{w.name}.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         prof = json.load(f)
-    h = hashlib.sha256()
-    srcs = ("decode_mha.cuh", "decode_kernel.cuh", "decode_attn.cu") if kern == "decode_mha" else \
-        ("decode_kernel.cuh", "decode_attn.cu")
-    for src in srcs:
-        with open(os.path.join(ROOT, "looped_lm_decode_b200", "csrc", src), "rb") as f:
-            h.update(f.read())
-    if h.hexdigest()[:16] != prof.get("kernel_sources_sha256_16"):
+    if kernel_sources_hash(kern) != prof.get("kernel_sources_sha256_16"):
         return None
     return prof["dram_bytes_read_per_launch"] + prof["dram_bytes_write_per_launch"]
 

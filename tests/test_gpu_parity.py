@@ -120,34 +120,40 @@ def test_decode_parity_small(name, lens_kind):
             assert ok, f"{name} layer {layer} t {t}: {msg}"
 
 
+@pytest.mark.parametrize("name", ["ctx", "gqa"])
 @pytest.mark.parametrize("gain", [8.0, 0.0])
-def test_decode_peaky_and_flat_queries(gain):
-    """q x 8 makes the softmax peaky (large max-rescale traffic); q = 0 gives the mean of values."""
-    w = SMALL["ctx"]
+def test_decode_peaky_and_flat_queries(name, gain):
+    """q x 8 makes the softmax peaky (large max-rescale traffic); q = 0 gives the mean of values.  "ctx"
+    runs the one-head-per-KV-head kernel, "gqa" the 4-heads-per-KV-head kernel."""
+    w = SMALL[name]
     cache = make_cache(w)
     codes = _upload_random_codes(w, cache)
     lens = _lens(w, "ragged")
-    qb = queries(w, 1, 2, gain=gain)
-    out, lse = _gpu_call(cache, 1, 2, qb, lens, int(lens.max()))
-    ref, lref = _oracle_call(w, codes, 1, 2, qb, lens, 1 / math.sqrt(w.D))
+    layer = min(1, w.L - 1)
+    qb = queries(w, layer, 2, gain=gain)
+    out, lse = _gpu_call(cache, layer, 2, qb, lens, int(lens.max()))
+    ref, lref = _oracle_call(w, codes, layer, 2, qb, lens, 1 / math.sqrt(w.D))
     ok, msg = attn_tolerance_ok(out, ref, lse, lref)
     assert ok, msg
 
 
-def test_decode_edge_lengths():
-    w = SMALL["ctx"].replace(B=8)
+@pytest.mark.parametrize("name", ["ctx", "gqa"])
+def test_decode_edge_lengths(name):
+    w = SMALL[name].replace(B=8)
+    N = w.Nmax
     cache = make_cache(w)
     codes = _upload_random_codes(w, cache)
-    lens = np.array([0, 1, 3, 4, 5, 511, 1023, 1024], np.int32)
+    lens = np.array([0, 1, 3, 4, 5, N // 2 - 1, N - 1, N], np.int32)
     qb = queries(w, 0, 3)
-    out, lse = _gpu_call(cache, 0, 3, qb, lens, 1024)
+    out, lse = _gpu_call(cache, 0, 3, qb, lens, N)
     ref, lref = _oracle_call(w, codes, 0, 3, qb, lens, 1 / math.sqrt(w.D))
     ok, msg = attn_tolerance_ok(out, ref, lse, lref)
     assert ok, msg
     assert (out[0] == 0).all() and np.isneginf(lse[0]).all()
     # lengths above max_len are clamped to it
-    out2, lse2 = _gpu_call(cache, 0, 3, qb, np.full(8, 1024, np.int32), 600)
-    ref2, lref2 = _oracle_call(w, codes, 0, 3, qb, np.full(8, 600, np.int32), 1 / math.sqrt(w.D))
+    cut = N * 3 // 5
+    out2, lse2 = _gpu_call(cache, 0, 3, qb, np.full(8, N, np.int32), cut)
+    ref2, lref2 = _oracle_call(w, codes, 0, 3, qb, np.full(8, cut, np.int32), 1 / math.sqrt(w.D))
     ok, msg = attn_tolerance_ok(out2, ref2, lse2, lref2)
     assert ok, msg
     # max_len = 0: nothing to attend
@@ -155,13 +161,14 @@ def test_decode_edge_lengths():
     assert (out3 == 0).all() and np.isneginf(lse3).all()
 
 
-def test_decode_explicit_scale():
-    w = SMALL["tiny"]
+@pytest.mark.parametrize("name", ["tiny", "ctx", "gqa"])
+def test_decode_explicit_scale(name):
+    w = SMALL[name]
     cache = make_cache(w)
     codes = _upload_random_codes(w, cache)
-    lens = np.array([200], np.int32)
+    lens = np.array([200, w.Nmax, 77][:w.B], np.int32)
     qb = queries(w, 0, 1)
-    out, lse = _gpu_call(cache, 0, 1, qb, lens, 256, scale=0.3)
+    out, lse = _gpu_call(cache, 0, 1, qb, lens, w.Nmax, scale=0.3)
     ref, lref = _oracle_call(w, codes, 0, 1, qb, lens, 0.3)
     ok, msg = attn_tolerance_ok(out, ref, lse, lref)
     assert ok, msg
