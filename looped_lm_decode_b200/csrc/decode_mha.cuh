@@ -23,11 +23,13 @@
 //  * The lane's 4 partial scores are reduce-scattered over the 8 lanes of its t (3 exchanges); each
 //    lane finishes one token.  The softmax maximum is one value per warp, lazy (it moves, with an exact
 //    rescale, only when a score exceeds it by more than 8 in log2 units).
-//  * Values: out^T += Vhat^T P^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate).  A fragments are
-//    the gathered bf16 value entries, re-paired across two tokens by one byte permute per register (no
-//    conversion to fp32).  The B fragment holds each weight split into bf16 hi + lo parts (column 0:
-//    the hi parts, column 1: the lo parts), which represents the fp32 weight to about 2^-16 relative;
-//    the two accumulator columns are added at the end.
+//  * Values on the tensor cores, one mma.sync m16n8k16 (bf16 in, fp32 accumulate) per (token, group
+//    quad): the k dimension is (token slot t, channel e) of one token per lane group, so a lane's B
+//    fragment is exactly its gathered 8-byte value entry (channels 0-1 and 2-3 of group 8u + g, no
+//    conversion or re-pairing).  A row g holds, at channel g % 4, the token's weight split into a bf16
+//    hi part (rows 0-3) or lo part (rows 4-7), which represents the fp32 weight to about 2^-16
+//    relative; the two rows are added at the end.  The 16 MMAs of a tile are issued token-major, so
+//    consecutive ones write different accumulators.
 //  * Index words arrive through a per-warp ring of 1 KiB stages in shared memory filled with 16-byte
 //    cp.async copies (lane L copies chunks L and L + 32 of the tile); each lane reads its 8 words with
 //    conflict-free 4-byte loads.
@@ -133,6 +135,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             // this warp's run of 16-token tiles [i0, i1) of the piece
             const int i0 = (int)((long long)warp * n16 / WARPS), i1 = (int)((long long)(warp + 1) * n16 / WARPS);
             const int kown = 2 * (g & 1) + ((g >> 1) & 1);  // the token (0..3) this lane finishes
+            // A row g: part g >> 2 (0: bytes 0-1 of x, 1: bytes 2-3) at channel e = g & 3
+            const uint32_t part_lo = (g & 4) ? 0x4432u : 0x4410u, part_hi = (g & 4) ? 0x3244u : 0x1044u;
+            const uint32_t sel0 = (g & 2) ? 0x4444u : ((g & 1) ? part_hi : part_lo);
+            const uint32_t sel2 = (g & 2) ? ((g & 1) ? part_hi : part_lo) : 0x4444u;
             // index copies: lane L takes chunks L (four-tile L / 16) and L + 32 (four-tile L / 16 + 2)
             const int kc = lane >> 4;
             const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP;
@@ -152,9 +158,9 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
 #pragma unroll
             for (int d = 0; d < DEPTH; ++d) copy_tile((uint32_t)d * 1024u);
 
-            float4 acc[8];
+            float4 acc[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
             float m = -1e30f, l = 0.f;
             float2 zar[2], zai[2], par[2], pai[2];         // high pairs: X_j and X_{j-1} (re, im)
             float2 zbr[2], zbi[2], dbr[2], dbi[2];         // low pairs: X_j and D_j = X_j - X_{j-1}
@@ -293,43 +299,43 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                         l *= corr;
                         const float2 c2 = f2(corr, corr);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float2 lo2 = __fmul2_rn(f2(acc[j].x, acc[j].y), c2), hi2 = __fmul2_rn(f2(acc[j].z, acc[j].w), c2);
-                            acc[j] = make_float4(lo2.x, lo2.y, hi2.x, hi2.y);
+                        for (int j = 0; j < 4; ++j) {              // rows 8..15 (z, w) stay zero
+                            const float2 lo2 = __fmul2_rn(f2(acc[j].x, acc[j].y), c2);
+                            acc[j].x = lo2.x;
+                            acc[j].y = lo2.y;
                         }
                         m = tmax;
                     }
                     const float p = ex2(sk - m);
                     l += p;
 
-                    // ---- weights to the B fragment: {bf16 hi part, bf16 lo part} per token, routed to the
-                    // lanes of columns 0 (hi) and 1 (lo); other columns carry unused values
-                    uint32_t bq0, bq1;
+                    // ---- weights: token k's {bf16 hi, bf16 lo} from lane 4 g'(k) + t; A row g = (part g >> 2,
+                    // channel g & 3): a0 holds the part at channel 0 or 1, a2 at channel 2 or 3, else zero
+                    uint32_t ak0[4], ak2[4];
                     {
                         const float hv = __uint_as_float(__float_as_uint(p) & 0xffff0000u);
                         const uint32_t x = cvt_bf16x2(p - hv, hv);        // upper: lo part, lower: hi part
-                        // token k is finished by lane 4 g'(k) + t, g'(k) = (k >> 1) | ((k & 1) << 1)
-                        const uint32_t x0 = __shfl_sync(0xffffffffu, x, t);
-                        const uint32_t x1 = __shfl_sync(0xffffffffu, x, 8 + t);
-                        const uint32_t x2 = __shfl_sync(0xffffffffu, x, 4 + t);
-                        const uint32_t x3 = __shfl_sync(0xffffffffu, x, 12 + t);
-                        const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;
-                        bq0 = __byte_perm(x0, x1, sel);    // k-slots 2t, 2t + 1: tokens k = 0, 1
-                        bq1 = __byte_perm(x2, x3, sel);    // k-slots 2t + 8, 2t + 9: tokens k = 2, 3
+                        const uint32_t xk[4] = {__shfl_sync(0xffffffffu, x, t), __shfl_sync(0xffffffffu, x, 8 + t),
+                                                __shfl_sync(0xffffffffu, x, 4 + t), __shfl_sync(0xffffffffu, x, 12 + t)};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            ak0[k] = __byte_perm(xk[k], 0u, sel0);
+                            ak2[k] = __byte_perm(xk[k], 0u, sel2);
+                        }
                     }
 
-                    // ---- values: group 8u + g, m-tiles 2u (channels e = 0, 1) and 2u + 1 (e = 2, 3)
+                    // ---- values: k-slot 2t + e (e < 2: word .x, channel e) and 2t + 8 + e (word .y, channel
+                    // 2 + e) of the lane's token; column g = group 8u + g
+                    uint2 v[4][4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t sel = (u < 2) ? 0x7624u : 0x7634u;
-                        uint2 v[4];
+                    for (int k = 0; k < 4; ++k)
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) v[k] = lds64(smem, __byte_perm((u & 1) ? wb[k] : wa[k], colv, sel));
-                        mma_bf16_16816(acc[2 * u], __byte_perm(v[0].x, v[1].x, 0x5410), __byte_perm(v[0].x, v[1].x, 0x7632),
-                                       __byte_perm(v[2].x, v[3].x, 0x5410), __byte_perm(v[2].x, v[3].x, 0x7632), bq0, bq1);
-                        mma_bf16_16816(acc[2 * u + 1], __byte_perm(v[0].y, v[1].y, 0x5410), __byte_perm(v[0].y, v[1].y, 0x7632),
-                                       __byte_perm(v[2].y, v[3].y, 0x5410), __byte_perm(v[2].y, v[3].y, 0x7632), bq0, bq1);
-                    }
+                        for (int u = 0; u < 4; ++u)
+                            v[k][u] = lds64(smem, __byte_perm((u & 1) ? wb[k] : wa[k], colv, (u < 2) ? 0x7624u : 0x7634u));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) mma_bf16_16816(acc[u], ak0[k], 0u, ak2[k], 0u, v[k][u].x, v[k][u].y);
                 }
             }
             cp_async_wait<0>();
@@ -340,12 +346,13 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
                 lsum *= 0.5f;                              // every token is finished by two lanes
-                if (t == 0) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int ch = 4 * (8 * (j >> 1) + g) + 2 * (j & 1);
-                        rec[ch] = acc[j].x + acc[j].y;
-                        rec[ch + 1] = acc[j].z + acc[j].w;
+                for (int u = 0; u < 4; ++u) {              // rows g + 4 (lo parts) to lanes g < 4
+                    const float vx = acc[u].x + __shfl_xor_sync(0xffffffffu, acc[u].x, 16);
+                    const float vy = acc[u].y + __shfl_xor_sync(0xffffffffu, acc[u].y, 16);
+                    if (g < 4) {
+                        rec[4 * (8 * u + 2 * t) + g] = vx;
+                        rec[4 * (8 * u + 2 * t + 1) + g] = vy;
                     }
                 }
                 if (lane == 0) {
