@@ -340,7 +340,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             }
             cp_async_wait<0>();
 
-            // ---- the warp's record: lanes t = 0 hold columns 0 (hi) and 1 (lo) of every m-tile
+            // ---- the warp's record: lane (g < 4, t) holds channel g of groups 8u + 2t, 8u + 2t + 1 (hi
+            // parts; the lo parts come from lane + 16)
             {
                 float lsum = l;
 #pragma unroll
