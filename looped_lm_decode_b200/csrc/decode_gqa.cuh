@@ -16,7 +16,7 @@
 //    t, t + 4, t + 8, t + 12 of each tile and pair-group g: channel group g (8 low channels) and its RoPE
 //    partner group g + 8.  Its positions advance by 4 from token to token and from tile to tile, and
 //    the rotation e^{i n w} of its 8 pairs follows the step-4 recurrence in difference form
-//    (D_{j+1} = D_j - 4 sin^2(2w) X_j, X_{j+1} = X_j + D_{j+1}), set from the table every 16 tiles.
+//    (D_{j+1} = D_j - 4 sin^2(2w) X_j, X_{j+1} = X_j + D_{j+1}), set from the table every 32 tiles.
 //  * Scores: the lane keeps the 4 query heads in the order h ^ hl, hl = 2 (g & 1) + ((g >> 1) & 1), so the
 //    reduce-scatter over the 8 lanes of its t sends fixed registers: after exchanges over lane bits 2
 //    and 3 the lane holds head hl of its 4 tokens, after bit 4 tokens 2 b, 2 b + 1 (b = g >> 2).
@@ -51,7 +51,7 @@ template <int WARPS, int MINB, int DEPTH>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_gqa_kernel(const DecodeArgs a) {
     constexpr int D = 128, NP = 8, QPK = 4;                // pair-groups = index words per token
     constexpr int NT = WARPS * 32;
-    constexpr int ANCHOR = 16;                             // tiles between two settings from the table
+    constexpr int ANCHOR = 32;                             // tiles between two settings from the table
     using S = GqaSmem<WARPS, DEPTH>;
 
     extern __shared__ __align__(128) unsigned char smem[];

@@ -19,7 +19,7 @@
 //    that is one fused multiply-add per component and step.  For the 4 low-frequency pairs the same
 //    recurrence is run in the difference form D_{j+1} = D_j - 4 sin^2(2w) X_j, X_{j+1} = X_j + D_{j+1}
 //    (Reinsch), whose coefficient keeps full relative precision as w -> 0.  Both are set from the
-//    table every 16 tiles, which bounds the rounding drift to 64 steps.
+//    table every 32 tiles, which bounds the rounding drift to 128 steps.
 //  * The lane's 4 partial scores are reduce-scattered over the 8 lanes of its t (3 exchanges); each
 //    lane finishes one token.  The softmax maximum is one value per warp, lazy (it moves, with an exact
 //    rescale, only when a score exceeds it by more than 8 in log2 units).
@@ -73,7 +73,7 @@ template <int WARPS, int MINB, int DEPTH>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const DecodeArgs a) {
     constexpr int D = 128, NP = 16;                        // pair-groups = index words per token
     constexpr int NT = WARPS * 32;
-    constexpr int ANCHOR = 16;                             // tiles between two settings from the table
+    constexpr int ANCHOR = 32;                             // tiles between two settings from the table
     using S = MhaSmem<WARPS, DEPTH>;
 
     extern __shared__ __align__(128) unsigned char smem[];

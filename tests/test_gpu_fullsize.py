@@ -56,6 +56,7 @@ def test_decode_full_size_sampled(name):
         ref, lref = dec(bf16_bits_to_f32(qb).astype(np.float64), ik, iv, np_codebook_f32(w, 0, blk, 0, h),
                         np_codebook_f32(w, 0, blk, 1, h), w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
         ok, msg = attn_tolerance_ok(out[b, hq], ref, lse[b, hq:hq + 1], np.array([lref]))
+        print(f"{name} (b={b}, hq={hq}, {n} tokens): {msg}")
         assert ok, f"{name} (b={b}, hq={hq}): {msg}"
 
 
