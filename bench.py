@@ -576,8 +576,8 @@ def main():
                        "kernel": ("tasq_sigma_kernel + tasq_encode_kernel (exact fp32 distances on CUDA cores)"
                                   if w.tasq else
                                   "encode_tc_kernel (tcgen05 bf16 distance contraction + TMEM arg-max)" if w.ncb == 1
-                                  else "encode_pg_kernel (exact fp32 distances on CUDA cores, one codebook per "
-                                       "channel group)")},
+                                  else "encode_tc_kernel, one codebook per channel group (tiles of 128 tokens of "
+                                       "one group, that group's codebook as the B operand)")},
         }
         if compare is not None:
             line["bf16_cache"] = compare["bf16_cache"]

@@ -163,9 +163,10 @@ cudaError_t launch_encode(const loopvq_cache &cc, int layer, int block, const vo
                           int x_dtype, const int64_t *strides, int b0, int nb, int tok0, int ntok,
                           cudaStream_t s) {
     if (nb == 0 || ntok == 0) return cudaSuccess;
-    // bf16 inputs with a tensor-core instantiation go to the tcgen05 contraction; fp32 inputs (not
-    // representable as bf16 MMA operands) and other shapes use the exact CUDA-core kernel below
-    if (x_dtype == LOOPVQ_BF16 && ncb_of(cc) == 1) {
+    // bf16 inputs with a tensor-core instantiation (shared or per-group codebooks) go to the tcgen05
+    // contraction; fp32 inputs (not representable as bf16 MMA operands) and other shapes use the exact
+    // CUDA-core kernels below
+    if (x_dtype == LOOPVQ_BF16) {
         const cudaError_t e = launch_encode_tc(cc, layer, block, xk, xv, strides, b0, nb, tok0, ntok, s);
         if (e != cudaErrorNotSupported) return e;
     }

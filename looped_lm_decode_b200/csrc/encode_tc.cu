@@ -11,7 +11,9 @@
 // epilogue is a plain arg-max (first maximum, i.e. lowest index on ties) per TMEM lane.
 //
 // Tile: M = 128 coupled vectors (TOKS tokens x D/c channel groups of one sequence and KV head) by
-// N = 256 entries; keys and values are two MMAs into the same 256 TMEM columns in turn.  Operands are
+// N = 256 entries; keys and values are two MMAs into the same 256 TMEM columns in turn.  With one
+// codebook per channel group (PG) a tile is 128 tokens of one channel group, whose codebook is the B
+// operand, and each tile writes its group's bytes of the index words.  Operands are
 // staged in shared memory in the canonical K-major layout without swizzle: 8-row x 16-byte core
 // matrices, the K-direction neighbour 128 bytes on (leading byte offset), the next 8 rows KB*128
 // bytes on (stride byte offset).  One thread issues the MMAs and commits to an mbarrier; every wait
@@ -195,7 +197,7 @@ struct EncodeTcArgs {
     uint32_t *idx;            // words of (layer, block, b = 0, h = 0)
     const uint16_t *cb;       // codebook of (layer, block, kv = 0, h = 0): [2][Hkv][K][G]
     int Hkv, K, Nmax, b0, nb, tok0, ntok;
-    long long units_per_cta;  // flattened (head, sequence, tile) units, head-major, per CTA
+    long long units_per_cta;  // flattened (head, [group,] sequence, tile) units, head-major, per CTA
 };
 
 // Shared-memory plan (bytes): B operands for K and V (256 x KD bf16 each), A operands for K and V
@@ -219,14 +221,15 @@ struct TcSmem {
 // Threads: 256.  Thread (half, row) owns tile row `row` (= its TMEM lane, row = tid % 128): it stages
 // the row's key (half 0) or value (half 1) coupled vector, and takes the arg-max over TMEM columns
 // [128 * half, 128 * half + 128); the two halves combine through shared memory.
-template <int D, int C, int TC>
+template <int D, int C, int TC, bool PG>
 __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a) {
     constexpr int G = C * TC;
     constexpr int KD = ((G + 3 + 15) / 16) * 16;      // contraction length: coordinates + 3, padded
     constexpr int KB = KD / 8;                          // 16-byte k-blocks per row
     constexpr int NG = D / C;                           // channel groups per token
     constexpr int NP = NG / 2;
-    constexpr int TOKS = 128 / NG;                      // tokens per 128-row tile
+    constexpr int TOKS = PG ? 128 : 128 / NG;           // tokens per 128-row tile
+    constexpr int NGU = PG ? NG : 1;                    // channel groups in the unit space
     using S = TcSmem<KD>;
     static_assert(128 % NG == 0, "tile rows");
     static_assert(S::kUsed <= S::kAlloc, "shared memory plan");
@@ -251,15 +254,16 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
 
-    // ---- B operands of head h: entry r -> [e_r (G coords), -h_hi, -h_mid, -h_lo, 0 ...], h_r = ||e_r||^2 / 2
-    auto build_b = [&](int h) {
+    // ---- B operands of head h (and group gq with PG): entry r -> [e_r (G coords), -h_hi, -h_mid, -h_lo,
+    // 0 ...], h_r = ||e_r||^2 / 2
+    auto build_b = [&](int h, int gq) {
         for (int it = tid; it < 2 * 256; it += 256) {
             const int kv = it >> 8, r = it & 255;
             uint16_t rw[KD];
 #pragma unroll
             for (int k = 0; k < KD; ++k) rw[k] = 0;
             if (r < a.K) {
-                const uint16_t *e = a.cb + ((size_t)kv * a.Hkv + h) * (size_t)a.K * G + (size_t)r * G;
+                const uint16_t *e = a.cb + (((size_t)kv * a.Hkv + h) * NGU + gq) * (size_t)a.K * G + (size_t)r * G;
                 double hh = 0.0;
 #pragma unroll
                 for (int k = 0; k < G; ++k) {
@@ -295,40 +299,45 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
         tc::tc_fence_after();
     };
 
-    // ---- this CTA's run of units u = (h * nb + brel) * ntiles + tile, walked without divisions
+    // ---- this CTA's run of units u = ((h * NGU + gq) * nb + brel) * ntiles + tile, walked without divisions
     const long long ntiles = (a.ntok + TOKS - 1) / TOKS;
-    const long long total = ntiles * a.nb * a.Hkv;
+    const long long total = ntiles * a.nb * a.Hkv * NGU;
     const long long u_begin = (long long)blockIdx.x * a.units_per_cta;
     const long long u_end = u_begin + a.units_per_cta < total ? u_begin + a.units_per_cta : total;
     struct Pos {
-        int h, brel, tile;
+        int h, gq, brel, tile;
     };
     Pos cur;
     {
         const long long hb = u_begin / ntiles;
         cur.tile = (int)(u_begin - hb * ntiles);
-        cur.h = (int)(hb / a.nb);
-        cur.brel = (int)(hb - (long long)cur.h * a.nb);
+        const long long hg = hb / a.nb;
+        cur.brel = (int)(hb - hg * a.nb);
+        cur.h = (int)(hg / NGU);
+        cur.gq = (int)(hg - (long long)cur.h * NGU);
     }
     auto advance = [&](Pos &p) {
         if (++p.tile == (int)ntiles) {
             p.tile = 0;
             if (++p.brel == a.nb) {
                 p.brel = 0;
-                ++p.h;
+                if (++p.gq == NGU) {
+                    p.gq = 0;
+                    ++p.h;
+                }
             }
         }
     };
 
-    int cur_h = cur.h;
-    build_b(cur_h);                                        // also publishes the TMEM address
+    int cur_h = cur.h, cur_g = cur.gq;
+    build_b(cur_h, cur_g);                                 // also publishes the TMEM address
     const uint32_t tmem = *tmem_slot;
 
     const uint32_t idesc = tc::idesc_bf16(128, 256);
     const uint32_t bkaddr = tc::smem_u32(smem + S::offBK), bvaddr = tc::smem_u32(smem + S::offBV);
     uint32_t phase = 0;
     bool ok = true;
-    const int rtok = row / NG, rg = row % NG;
+    const int rtok = PG ? row : row / NG, rg = PG ? 0 : row % NG;
 
     // this thread's coupled vector (key for half 0, value for half 1) of the next unit, one unit ahead
     uint16_t zn[G];
@@ -338,7 +347,7 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
         for (int k = 0; k < G; ++k) z[k] = 0;
         if (valid && nrel < a.ntok) {
             const uint16_t *x = (half ? a.xv : a.xk) + (size_t)p.brel * a.s1 + (size_t)nrel * a.s2 +
-                                (size_t)p.h * a.s3 + rg * C;
+                                (size_t)p.h * a.s3 + (PG ? p.gq : rg) * C;
 #pragma unroll
             for (int m = 0; m < TC; ++m)
 #pragma unroll
@@ -348,11 +357,12 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
     load_row(u_begin < u_end, cur, zn);
 
     for (long long u = u_begin; u < u_end; ++u) {
-        const int tile = cur.tile, brel = cur.brel, h = cur.h;
+        const int tile = cur.tile, brel = cur.brel, h = cur.h, gq = cur.gq;
         advance(cur);
-        if (h != cur_h) {                                  // previous MMAs have completed: B may be rewritten
-            build_b(h);
+        if (h != cur_h || gq != cur_g) {                   // previous MMAs have completed: B may be rewritten
+            build_b(h, gq);
             cur_h = h;
+            cur_g = gq;
         }
         // ---- A operand of this thread's half: the coupled vector extended by three ones
         {
@@ -410,8 +420,16 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
             }
         }
         __syncthreads();
-        // ---- pack {K p, K p+NP, V p, V p+NP} words and store them (sentinel words after a timeout)
-        if (tid < TOKS * NP) {
+        if constexpr (PG) {
+            // ---- group gq's bytes of the index words: K code at byte gq / NP, V code at byte 2 + gq / NP
+            const int nr = tile * TOKS + row;
+            if (nr < a.ntok) {
+                uint32_t *idx_bh = a.idx + ((size_t)(a.b0 + brel) * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C);
+                uint8_t *wb = reinterpret_cast<uint8_t *>(idx_bh + idx_word(a.tok0 + nr, gq % NP, NP));
+                wb[2 * half + gq / NP] = ok ? codes[half * 128 + row] : (uint8_t)0xFF;
+            }
+        } else if (tid < TOKS * NP) {
+            // ---- pack {K p, K p+NP, V p, V p+NP} words and store them (sentinel words after a timeout)
             const int t = tid / NP, p = tid % NP;
             const int nr = tile * TOKS + t;
             if (nr < a.ntok) {
@@ -431,13 +449,13 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
     if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
 }
 
-template <int D, int C, int TC>
+template <int D, int C, int TC, bool PG>
 static cudaError_t launch_tc_ct(const EncodeTcArgs &a0, cudaStream_t s) {
     constexpr int NG = D / C;
-    constexpr int TOKS = 128 / NG;
+    constexpr int TOKS = PG ? 128 : 128 / NG;
     constexpr int KD = ((C * TC + 3 + 15) / 16) * 16;
     EncodeTcArgs a = a0;
-    auto k = encode_tc_kernel<D, C, TC>;
+    auto k = encode_tc_kernel<D, C, TC, PG>;
     cudaError_t e = ensure_dynamic_smem((const void *)k, TcSmem<KD>::kAlloc);
     if (e != cudaSuccess) return e;
     // CTAs resident per SM, from the limits that bind here: shared memory, registers and tensor memory
@@ -457,7 +475,7 @@ static cudaError_t launch_tc_ct(const EncodeTcArgs &a0, cudaStream_t s) {
     if (per_sm < 1) return cudaErrorNotSupported;
     // persistent grid: one wave of CTAs, each taking an equal run of the head-major units
     const long long ntiles = (a.ntok + TOKS - 1) / TOKS;
-    const long long total = ntiles * a.nb * a.Hkv;
+    const long long total = ntiles * a.nb * a.Hkv * (PG ? NG : 1);
     long long ctas = (long long)sms * per_sm;
     if (ctas > total) ctas = total;
     a.units_per_cta = (total + ctas - 1) / ctas;
@@ -485,16 +503,22 @@ cudaError_t launch_encode_tc(const loopvq_cache &cc, int layer, int block, const
     a.nb = nb;
     a.tok0 = tok0;
     a.ntok = ntok;
-    const int G = cc.c * cc.Tc;
-    if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4>(a, s);
-    if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4>(a, s);
-    if (cc.D == 128 && cc.c == 16 && cc.Tc == 1) return launch_tc_ct<128, 16, 1>(a, s);
-    if (cc.D == 128 && cc.c == 32 && cc.Tc == 1) return launch_tc_ct<128, 32, 1>(a, s);
-    if (cc.D == 64 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<64, 4, 4>(a, s);
-    if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4>(a, s);
-    if (cc.D == 64 && cc.c == 16 && cc.Tc == 1) return launch_tc_ct<64, 16, 1>(a, s);
-    if (cc.D == 64 && cc.c == 32 && cc.Tc == 1) return launch_tc_ct<64, 32, 1>(a, s);
-    (void)G;
+    if (ncb_of(cc) == 1) {
+        if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4, false>(a, s);
+        if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4, false>(a, s);
+        if (cc.D == 128 && cc.c == 16 && cc.Tc == 1) return launch_tc_ct<128, 16, 1, false>(a, s);
+        if (cc.D == 128 && cc.c == 32 && cc.Tc == 1) return launch_tc_ct<128, 32, 1, false>(a, s);
+        if (cc.D == 64 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<64, 4, 4, false>(a, s);
+        if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4, false>(a, s);
+        if (cc.D == 64 && cc.c == 16 && cc.Tc == 1) return launch_tc_ct<64, 16, 1, false>(a, s);
+        if (cc.D == 64 && cc.c == 32 && cc.Tc == 1) return launch_tc_ct<64, 32, 1, false>(a, s);
+    } else if (ncb_of(cc) == cc.D / cc.c) {
+        if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4, true>(a, s);
+        if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4, true>(a, s);
+        if (cc.D == 128 && cc.c == 16 && cc.Tc == 1) return launch_tc_ct<128, 16, 1, true>(a, s);
+        if (cc.D == 64 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<64, 4, 4, true>(a, s);
+        if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4, true>(a, s);
+    }
     return cudaErrorNotSupported;
 }
 

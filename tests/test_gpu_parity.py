@@ -245,9 +245,11 @@ def test_encode_parity(name, dtype):
     print(f"near-ties: {ties}")
 
 
-def test_encode_partial_ranges_and_strides():
-    """Encoding sub-ranges (b0, tok0 offsets, ragged token counts, strided input) writes exactly those words."""
-    w = SMALL["ctx"].replace(Nmax=128, L=1)
+@pytest.mark.parametrize("name", ["ctx", "pg4"])
+def test_encode_partial_ranges_and_strides(name):
+    """Encoding sub-ranges (b0, tok0 offsets, ragged token counts, strided input) writes exactly those words.
+    "pg4" has one codebook per channel group: the tensor-core encoder writes each group's bytes."""
+    w = SMALL[name].replace(Nmax=128, L=1, B=3)
     cache = make_cache(w)
     sentinel = torch.full_like(cache.idx, -1)
     cache.idx.copy_(sentinel)
@@ -267,9 +269,12 @@ def test_encode_partial_ranges_and_strides():
             untouched = words.reshape(w.Nmax // 4, cache.NP, 4).transpose(0, 2, 1).reshape(w.Nmax, cache.NP)
             assert (untouched[~wr] == 0xFFFFFFFF).all()
             if wr.any():
-                ref_k = O.encode(np.ascontiguousarray(bf16_bits_to_f32(xk)[:, b, 37:87, h, :]),
-                                 np_codebook_f32(w, 0, 0, 0, h), w.c)
+                ref_k = _enc(np.ascontiguousarray(bf16_bits_to_f32(xk)[:, b, 37:87, h, :]),
+                             np_codebook_f32(w, 0, 0, 0, h), w.c)
+                ref_v = _enc(np.ascontiguousarray(bf16_bits_to_f32(xv)[:, b, 37:87, h, :]),
+                             np_codebook_f32(w, 0, 0, 1, h), w.c)
                 np.testing.assert_array_equal(ck[37:87], ref_k)
+                np.testing.assert_array_equal(cv[37:87], ref_v)
 
 
 def test_generator_twins_agree():
