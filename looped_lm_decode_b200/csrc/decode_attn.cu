@@ -18,9 +18,9 @@ namespace loopvq {
 // codebook, two CTAs of 8 warps per SM (64 KiB of slice replicas plus a 2-deep prefetch queue each;
 // the shared memory left over serves as L1 for the RoPE rows); with one codebook per channel group,
 // one CTA of 16 warps per SM (128 KiB of tables).  Measured at ctx32k: a second wave, or three CTAs
-// per SM at 80 registers, is 3 to 10 % slower.  decode_mha_kernel runs one CTA of 16 warps per SM
-// (one copy of the tables per SM, 2-deep index ring per warp): one CTA of 16 warps measured 3% faster
-// than two CTAs of 8 warps, and a 2-deep ring 2% faster than a 3-deep one.
+// per SM at 80 registers, is 3 to 10 % slower.  decode_mha_kernel runs two CTAs of 8 warps per SM
+// (2-deep index ring per warp): with fp32 key tables this is as fast as one CTA of 16 warps at ctx32k
+// and 4% faster on the short deep32 calls; a 3-deep ring is 2% slower.
 
 static constexpr int kSms = 148;                           // B200; more CTAs than fit only add a wave
 static constexpr int kWords = 1;                           // index words per lane per iteration (4-token tiles)
@@ -42,7 +42,7 @@ static size_t ring_smem_bytes(bool pg, int qpk) {
 // runs the step-4 RoPE recurrence in plain form on the frequencies f < D/4 and in difference form on
 // f >= D/4; it needs |sin 4w_f| >= 0.04 on the first (the recurrence's rounding grows as 1/|sin 4w|),
 // 4w_f <= 1 on the second, and table rows 2 and 4.  With the base 1e4: min |sin 4w| = 0.046 (f = 31).
-static constexpr int kMhaWarps = 16, kMhaMinBlocks = 1, kMhaDepth = 2;
+static constexpr int kMhaWarps = 8, kMhaMinBlocks = 2, kMhaDepth = 2;
 
 static bool mha_applies(const loopvq_cache &cc) {
     if (cc.D != 128 || cc.c != 4 || cc.Hq != cc.Hkv || ncb_of(cc) != 1 || cc.Nmax < 8) return false;
