@@ -161,6 +161,24 @@ def test_decode_edge_lengths(name):
     assert (out3 == 0).all() and np.isneginf(lse3).all()
 
 
+@pytest.mark.parametrize("w", [WORKLOADS["ctx4k"].replace(L=1, B=3, Hkv=2, Hq=2, Nmax=20),
+                               WORKLOADS["gqa16k"].replace(L=1, B=3, Hkv=1, Hq=4, Nmax=12),
+                               WORKLOADS["ctx4k"].replace(L=1, B=2, Hkv=1, Hq=1, Nmax=4)],
+                         ids=["mha-nmax20", "gqa-nmax12", "mha-nmax4"])
+def test_decode_short_caches(w):
+    """Caches shorter than a 16-token tile (and one below the 8 positions the one- and four-head kernels
+    need, which takes the general kernel): partial tiles, zero-filled index copies, RoPE rows near Nmax."""
+    cache = make_cache(w)
+    codes = _upload_random_codes(w, cache)
+    lens = np.array([w.Nmax, 7, 3][:w.B], np.int32)
+    for t in (0, 3):
+        qb = queries(w, 0, t)
+        out, lse = _gpu_call(cache, 0, t, qb, lens, w.Nmax)
+        ref, lref = _oracle_call(w, codes, 0, t, qb, lens, 1 / math.sqrt(w.D))
+        ok, msg = attn_tolerance_ok(out, ref, lse, lref)
+        assert ok, f"t {t}: {msg}"
+
+
 @pytest.mark.parametrize("name", ["tiny", "ctx", "gqa"])
 def test_decode_explicit_scale(name):
     w = SMALL[name]
