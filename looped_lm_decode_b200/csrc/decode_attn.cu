@@ -78,9 +78,10 @@ static cudaError_t launch_gqa(const DecodeArgs &a, const DecodePlan &plan, cudaS
     return launch_merge<128>(a, s);
 }
 
+template <bool TQ>
 static cudaError_t launch_mha(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
     using S = MhaSmem<kMhaWarps, kMhaDepth>;
-    auto kern = decode_mha_kernel<kMhaWarps, kMhaMinBlocks, kMhaDepth>;
+    auto kern = decode_mha_kernel<kMhaWarps, kMhaMinBlocks, kMhaDepth, TQ>;
     cudaError_t e = ensure_dynamic_smem((const void *)kern, S::kBytes);
     if (e != cudaSuccess) return e;
     if (plan.ncta > 0) {
@@ -98,7 +99,7 @@ DecodePlan plan_decode(const loopvq_cache &cc, int max_len, bool tasq) {
     const KernelShape k = kernel_shape(pg, qpk);
     p.nbt = 1;
     p.nchunk = cc.B;
-    p.mha = !tasq && mha_applies(cc);
+    p.mha = mha_applies(cc);                               // plain or TaSQ keys
     p.gqa = !tasq && gqa_applies(cc);
     // an upper bound of the tiles: every sequence at max_len
     const long tiles = (long)cc.B * cc.Hkv * ((max_len + 3) / 4);
@@ -227,6 +228,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
         a.tperm = tq->perm + ((size_t)layer * NB + beta) * cc.Hkv * (cc.D / 2);
         a.tsig = tq->sigma + ((size_t)layer * cc.T + t) * cc.B * cc.Nmax;
         if (ncb_of(cc) != 1) return cudaErrorInvalidValue;
+        if (plan.mha) return launch_mha<true>(a, plan, s);
         if (cc.D == 128 && cc.c == 4) return dispatch_tq_qpk<128, 4>(qpk, a, plan, s);
         if (cc.D == 128 && cc.c == 8) return dispatch_tq_qpk<128, 8>(qpk, a, plan, s);
         if (cc.D == 64 && cc.c == 4) return dispatch_tq_qpk<64, 4>(qpk, a, plan, s);
@@ -234,7 +236,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
         return cudaErrorInvalidValue;
     }
     const bool pg = ncb_of(cc) > 1;
-    if (plan.mha) return launch_mha(a, plan, s);
+    if (plan.mha) return launch_mha<false>(a, plan, s);
     if (plan.gqa) return launch_gqa(a, plan, s);
     if (cc.D == 128) return pg ? dispatch_c<128, true>(cc.c, qpk, a, plan, s) : dispatch_c<128, false>(cc.c, qpk, a, plan, s);
     if (cc.D == 64) return pg ? dispatch_c<64, true>(cc.c, qpk, a, plan, s) : dispatch_c<64, false>(cc.c, qpk, a, plan, s);

@@ -73,7 +73,12 @@ struct MhaSmem {
     static constexpr uint32_t kBytes = kRec + (uint32_t)WARPS * kRecFloats * 4u;
 };
 
-template <int WARPS, int MINB, int DEPTH>
+// TQ: keys coded after the TaSQ transform (LoopVQ paper, App. B).  Word p's key codes are TaSQ groups 2p
+// and 2p + 1, whose entries hold complete RoPE pairs (f, f + D/2) of the low channels perm[4p .. 4p + 3]
+// interleaved; the lane keeps one rotated query pair (re, im) per pair, divided by the channel weight,
+// runs the difference-form recurrence on every pair, and multiplies each finished score by its token's
+// scale sigma.
+template <int WARPS, int MINB, int DEPTH, bool TQ = false>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const DecodeArgs a) {
     constexpr int D = 128, NP = 16;                        // pair-groups = index words per token
     constexpr int NT = WARPS * 32;
@@ -173,6 +178,16 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             float m = -1e30f, l = 0.f;
             float2 zar[2], zai[2], par[2], pai[2];         // high pairs: X_j and X_{j-1} (re, im)
             float2 zbr[2], zbi[2], dbr[2], dbi[2];         // low pairs: X_j and D_j = X_j - X_{j-1}
+            float2 xq[8], dq[8], nq[8];                    // TQ: per pair (re, im) of X_j and D_j, -4 sin^2 2w
+            if constexpr (TQ) {
+                const int16_t *pm = a.tperm + (size_t)h * (D / 2);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int f = __ldg(pm + (j < 4 ? 4 * g + j : 32 + 4 * g + j - 4)) & (D / 2 - 1);
+                    const float s2 = __ldg(a.rope + 2 * D + D / 2 + f);
+                    nq[j] = f2(-4.f * s2 * s2, -4.f * s2 * s2);
+                }
+            }
             // the lane's finished token n is attended iff 0 <= n - st < tok_end - st
             int nrel = tok_begin + 16 * i0 + t + 4 * kown - st;
             const unsigned span = (unsigned)(tok_end - st);
@@ -181,7 +196,27 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             __syncthreads();                               // tables staged
 
             for (int ib = i0; ib < i1; ib += ANCHOR) {
-                {
+                if constexpr (TQ) {
+                    // X = (q_f + i q_{f+D/2}) / w_f e^{-i n0 w_f} at the lane's permuted pairs, D = X (2 sin^2 2w
+                    // - i sin 4w)
+                    const int n0 = tok_begin + 16 * ib + t;
+                    const float *row = a.rope + (size_t)min(n0, a.Nmax - 1) * D;
+                    const uint16_t *qp = a.q + ((size_t)b * a.Hq + h) * D;
+                    const int16_t *pm = a.tperm + (size_t)h * (D / 2);
+                    const float *wp = a.tw + (size_t)h * D;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int f = __ldg(pm + (j < 4 ? 4 * g + j : 32 + 4 * g + j - 4)) & (D / 2 - 1);
+                        const float sc = a.qscale / __ldg(wp + f);
+                        const float qf = bf16_to_f32(__ldg(qp + f)) * sc, qh = bf16_to_f32(__ldg(qp + D / 2 + f)) * sc;
+                        const float c = __ldg(row + f), sn = __ldg(row + D / 2 + f);
+                        const float s2 = __ldg(a.rope + 2 * D + D / 2 + f), s4 = __ldg(a.rope + 4 * D + D / 2 + f);
+                        const float al = 2.f * s2 * s2;
+                        const float zr = fmaf(qf, c, qh * sn), zi = fmaf(qh, c, -(qf * sn));
+                        xq[j] = f2(zr, zi);
+                        dq[j] = f2(fmaf(zr, al, zi * s4), fmaf(zi, al, -(zr * s4)));
+                    }
+                } else {
                     // X at the lane's first position n0 from the table and the query; the second state from
                     // X(n0 - 4) = X(n0) e^{+4iw}
                     const int n0 = tok_begin + 16 * ib + t;
@@ -255,6 +290,24 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                         const float4 e1 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wa[k], colk, 0x7614));
                         const float4 e2 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wb[k], colk, 0x7604));
                         const float4 e3 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wb[k], colk, 0x7614));
+                        if constexpr (TQ) {
+                            // entries (u_f, u_{f+D/2}, u_f', u_{f'+D/2}): one packed FMA per pair
+                            float2 sc2 = __fmul2_rn(xq[0], f2(e0.x, e0.y));
+                            sc2 = __ffma2_rn(xq[1], f2(e0.z, e0.w), sc2);
+                            sc2 = __ffma2_rn(xq[2], f2(e1.x, e1.y), sc2);
+                            sc2 = __ffma2_rn(xq[3], f2(e1.z, e1.w), sc2);
+                            sc2 = __ffma2_rn(xq[4], f2(e2.x, e2.y), sc2);
+                            sc2 = __ffma2_rn(xq[5], f2(e2.z, e2.w), sc2);
+                            sc2 = __ffma2_rn(xq[6], f2(e3.x, e3.y), sc2);
+                            sc2 = __ffma2_rn(xq[7], f2(e3.z, e3.w), sc2);
+                            s[k] = sc2.x + sc2.y;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                dq[j] = __ffma2_rn(nq[j], xq[j], dq[j]);
+                                xq[j] = __fadd2_rn(xq[j], dq[j]);
+                            }
+                            continue;
+                        }
                         float2 sc2 = __fmul2_rn(zar[0], f2(e0.x, e0.y));
                         sc2 = __ffma2_rn(zar[1], f2(e0.z, e0.w), sc2);
                         sc2 = __ffma2_rn(zai[0], f2(e1.x, e1.y), sc2);
@@ -295,6 +348,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                         const float kk = b2 ? a1 : a0, oo = b2 ? a0 : a1;
                         sk = kk + __shfl_xor_sync(0xffffffffu, oo, 8);
                         sk += __shfl_xor_sync(0xffffffffu, sk, 16);
+                    }
+                    if constexpr (TQ) {                    // the finished token's TaSQ scale
+                        if ((unsigned)nrel < span)
+                            sk *= __half2float(__ushort_as_half(__ldg(a.tsig + (size_t)b * a.Nmax + st + nrel)));
                     }
                     sk = (unsigned)nrel < span ? sk : -CUDART_INF_F;
                     nrel += 16;

@@ -120,3 +120,42 @@ def test_bf16_cache_full_size_sampled(name):
         ref, lref = O.attention(bf16_bits_to_f32(qb).astype(np.float64), kb, vb, 1 / math.sqrt(w.D))
         ok, msg = attn_tolerance_ok(out[b, hq], ref, lse[b, hq:hq + 1], np.array([lref]))
         assert ok, f"{name} (b={b}, hq={hq}): {msg}"
+
+
+def test_tasq_decode_full_size_sampled():
+    """TaSQ keys at the full ctx32k shape in the launch configuration the benchmark times (long per-warp
+    runs, so the rotation recurrence is set from the table several times); uniform random codes, seeded
+    token scales, sampled (sequence, query head) outputs against the checker."""
+    from synth import tasq_weights, tasq_perm
+    w = WORKLOADS["ctx32k_tasq"].replace(L=1)
+    cache = _full_cache(w)
+    tw, tp = tasq_weights(w), tasq_perm(w)
+    tq = LQ.Tasq(cache, w=torch.from_numpy(tw).cuda(), perm=torch.from_numpy(tp).cuda())
+    t = 1
+    blk, m = t // w.Tc, t % w.Tc
+    per_lb = w.B * w.Hkv * w.Nmax * cache.NP
+    SG.fill_idx(w, 0, blk, cache.idx[blk * per_lb:(blk + 1) * per_lb])
+    sig = np.random.default_rng(41).uniform(0.25, 4.0, (w.L, w.T, w.B, w.Nmax)).astype(np.float16)
+    tq.sigma.copy_(torch.from_numpy(sig.reshape(-1)).cuda())
+    lens = lengths(w)
+    qd = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    SG.fill_q(w, 0, t, qd)
+    out, lse = LQ.tasq_decode_attn(cache, tq, 0, t, qd.view(torch.int16), torch.from_numpy(lens).cuda(),
+                                   int(lens.max()))
+    torch.cuda.synchronize()
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for b, hq in [(0, 0), (5, 9)]:
+        h = hq
+        n = int(lens[b])
+        ik = random_indices(w, 0, blk, 0, b, h, range(n))
+        it = np.empty_like(ik)                       # word bytes 0/1 of pair-group p: TaSQ groups 2p, 2p+1
+        it[:, 0::2] = ik[:, :cache.NP]
+        it[:, 1::2] = ik[:, cache.NP:]
+        iv = random_indices(w, 0, blk, 1, b, h, range(n))
+        qb = queries(w, 0, t, b=[b], hq=[hq])[0, 0]
+        ref, lref = O.tasq_decode(bf16_bits_to_f32(qb).astype(np.float64), it, iv, np_codebook_f32(w, 0, blk, 0, h),
+                                  np_codebook_f32(w, 0, blk, 1, h), tp[0, blk, h], tw[0, t, h],
+                                  sig[0, t, b, :n].astype(np.float64), w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        ok, msg = attn_tolerance_ok(out[b, hq], ref, lse[b, hq:hq + 1], np.array([lref]))
+        print(f"ctx32k_tasq (b={b}, hq={hq}, {n} tokens): {msg}")
+        assert ok, f"ctx32k_tasq (b={b}, hq={hq}): {msg}"
