@@ -574,8 +574,8 @@ def main():
             "encode": {"ms_per_layer_block": statistics.median(enc_ms),
                        "tokens_per_s": w.B * w.Nmax / (statistics.median(enc_ms) * 1e-3),
                        "input_gbs": 2 * w.Tc * w.B * w.Nmax * w.Hkv * w.D * 2 / (statistics.median(enc_ms) * 1e-3) / 1e9,
-                       "kernel": ("tasq_sigma_kernel + tasq_encode_kernel (exact fp32 distances on CUDA cores)"
-                                  if w.tasq else
+                       "kernel": ("tasq_sigma_kernel + encode_tc_kernel with TaSQ keys (u split into three "
+                                  "bf16 parts along the contraction)" if w.tasq else
                                   "encode_tc_kernel (tcgen05 bf16 distance contraction + TMEM arg-max)" if w.ncb == 1
                                   else "encode_tc_kernel, one codebook per channel group (tiles of 128 tokens of "
                                        "one group, that group's codebook as the B operand)")},

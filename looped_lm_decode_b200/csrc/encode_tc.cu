@@ -198,6 +198,12 @@ struct EncodeTcArgs {
     const uint16_t *cb;       // codebook of (layer, block, kv = 0, h = 0): [2][Hkv][K][G]
     int Hkv, K, Nmax, b0, nb, tok0, ntok;
     long long units_per_cta;  // flattened (head, [group,] sequence, tile) units, head-major, per CTA
+    // TaSQ keys (TQ): weights of (layer, t = block Tc) [Tc][Hkv][D], order of (layer, block) [Hkv][D/2],
+    // fp16 scales of (layer, t = block Tc) [Tc][B][Nmax]
+    const float *tw;
+    const int16_t *tperm;
+    const uint16_t *tsig;
+    int B;
 };
 
 // Shared-memory plan (bytes): B operands for K and V (256 x KD bf16 each), A operands for K and V
@@ -215,16 +221,21 @@ struct TcSmem {
     static constexpr int offMbar = offRed + 2048;
     static constexpr int offTmem = offMbar + 8;
     static constexpr int kUsed = offTmem + 8;
-    static constexpr int kAlloc = 80 * 1024;            // keeps at most two CTAs per SM: 2 x 256 TMEM columns
+    // at least 80 KiB keeps at most two CTAs per SM: 2 x 256 TMEM columns
+    static constexpr int kAlloc = kUsed <= 80 * 1024 ? 80 * 1024 : ((kUsed + 1023) / 1024) * 1024;
 };
 
 // Threads: 256.  Thread (half, row) owns tile row `row` (= its TMEM lane, row = tid % 128): it stages
 // the row's key (half 0) or value (half 1) coupled vector, and takes the arg-max over TMEM columns
 // [128 * half, 128 * half + 128); the two halves combine through shared memory.
-template <int D, int C, int TC, bool PG>
+// TQ: keys coded after the TaSQ transform (LoopVQ paper, App. B): the key rows are the coupled vectors of
+// TaSQ groups, u = fl(fl(w k) / sigma) in fp32 at the permuted channels, each split exactly into three
+// bf16 parts (hi, mid, lo) along the contraction, against the entry repeated three times; values are
+// coded plainly.  Key codes of TaSQ groups 2p and 2p + 1 go to bytes 0 and 1 of word p.
+template <int D, int C, int TC, bool PG, bool TQ = false>
 __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a) {
     constexpr int G = C * TC;
-    constexpr int KD = ((G + 3 + 15) / 16) * 16;      // contraction length: coordinates + 3, padded
+    constexpr int KD = (((TQ ? 3 * G : G) + 3 + 15) / 16) * 16;   // contraction length: coordinates + 3, padded
     constexpr int KB = KD / 8;                          // 16-byte k-blocks per row
     constexpr int NG = D / C;                           // channel groups per token
     constexpr int NP = NG / 2;
@@ -262,12 +273,19 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
             uint16_t rw[KD];
 #pragma unroll
             for (int k = 0; k < KD; ++k) rw[k] = 0;
+            const int rep = (TQ && kv == 0) ? 3 : 1;       // TaSQ key rows: the entry against hi, mid, lo
             if (r < a.K) {
                 const uint16_t *e = a.cb + (((size_t)kv * a.Hkv + h) * NGU + gq) * (size_t)a.K * G + (size_t)r * G;
                 double hh = 0.0;
 #pragma unroll
                 for (int k = 0; k < G; ++k) {
                     rw[k] = e[k];
+                    if constexpr (TQ) {
+                        if (rep == 3) {
+                            rw[G + k] = e[k];
+                            rw[2 * G + k] = e[k];
+                        }
+                    }
                     const double v = (double)bf16_to_f32(e[k]);
                     hh += v * v;
                 }
@@ -276,11 +294,11 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
                 const double r1 = hh - (double)p1;
                 const float p2 = __bfloat162float(__float2bfloat16_rn((float)r1));
                 const double r2 = r1 - (double)p2;
-                rw[G] = tc::bf16_bits_rn(-p1);
-                rw[G + 1] = tc::bf16_bits_rn(-p2);
-                rw[G + 2] = tc::bf16_bits_rn((float)-r2);
+                rw[rep * G] = tc::bf16_bits_rn(-p1);
+                rw[rep * G + 1] = tc::bf16_bits_rn(-p2);
+                rw[rep * G + 2] = tc::bf16_bits_rn((float)-r2);
             } else {
-                rw[G] = tc::bf16_bits_rn(-1.0e30f);        // entries past K never win
+                rw[rep * G] = tc::bf16_bits_rn(-1.0e30f);  // entries past K never win
             }
             unsigned char *base = smem + (kv ? S::offBV : S::offBK) + ((r >> 3) * KB) * 128 + (r & 7) * 16;
 #pragma unroll
@@ -339,19 +357,39 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
     bool ok = true;
     const int rtok = PG ? row : row / NG, rg = PG ? 0 : row % NG;
 
-    // this thread's coupled vector (key for half 0, value for half 1) of the next unit, one unit ahead
-    uint16_t zn[G];
-    auto load_row = [&](bool valid, const Pos &p, uint16_t (&z)[G]) {
+    // this thread's coupled vector (key for half 0, value for half 1) of the next unit, one unit ahead:
+    // bf16 bits, or with TaSQ keys the fp32 bits of u
+    uint32_t zn[G];
+    auto load_row = [&](bool valid, const Pos &p, uint32_t (&z)[G]) {
         const int nrel = p.tile * TOKS + rtok;
 #pragma unroll
         for (int k = 0; k < G; ++k) z[k] = 0;
         if (valid && nrel < a.ntok) {
-            const uint16_t *x = (half ? a.xv : a.xk) + (size_t)p.brel * a.s1 + (size_t)nrel * a.s2 +
-                                (size_t)p.h * a.s3 + (PG ? p.gq : rg) * C;
+            if (TQ && half == 0) {
+                // TaSQ group rg: channel i is the low (i even) or high (i odd) channel of pair perm[rg C/2 + i/2]
+                const uint16_t *x = a.xk + (size_t)p.brel * a.s1 + (size_t)nrel * a.s2 + (size_t)p.h * a.s3;
+                const int16_t *pm = a.tperm + (size_t)p.h * (D / 2) + rg * (C / 2);
 #pragma unroll
-            for (int m = 0; m < TC; ++m)
+                for (int i = 0; i < C; ++i) {
+                    const int lowf = __ldg(pm + i / 2) & (D / 2 - 1);
+                    const int f = (i & 1) ? lowf + D / 2 : lowf;
 #pragma unroll
-                for (int i = 0; i < C; ++i) z[i * TC + m] = __ldg(x + (size_t)m * a.s0 + i);
+                    for (int m = 0; m < TC; ++m) {
+                        const float wt = __ldg(a.tw + ((size_t)m * a.Hkv + p.h) * D + f);
+                        const float sg = __half2float(__ushort_as_half(
+                            __ldg(a.tsig + ((size_t)m * a.B + a.b0 + p.brel) * a.Nmax + a.tok0 + nrel)));
+                        const float k = bf16_to_f32(__ldg(x + (size_t)m * a.s0 + f));
+                        z[i * TC + m] = __float_as_uint(__fdiv_rn(__fmul_rn(wt, k), sg));
+                    }
+                }
+            } else {
+                const uint16_t *x = (half ? a.xv : a.xk) + (size_t)p.brel * a.s1 + (size_t)nrel * a.s2 +
+                                    (size_t)p.h * a.s3 + (PG ? p.gq : rg) * C;
+#pragma unroll
+                for (int m = 0; m < TC; ++m)
+#pragma unroll
+                    for (int i = 0; i < C; ++i) z[i * TC + m] = __ldg(x + (size_t)m * a.s0 + i);
+            }
         }
     };
     load_row(u_begin < u_end, cur, zn);
@@ -367,9 +405,27 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
         // ---- A operand of this thread's half: the coupled vector extended by three ones
         {
             uint16_t zr[KD];
+            if (TQ && half == 0) {
+                // u = hi + mid + lo exactly (three round-to-nearest bf16 parts of an fp32 value)
 #pragma unroll
-            for (int k = 0; k < KD; ++k) zr[k] = k < G ? zn[k] : 0;
-            zr[G] = zr[G + 1] = zr[G + 2] = 0x3F80;           // bf16 1.0
+                for (int k = 0; k < KD; ++k) zr[k] = 0;
+#pragma unroll
+                for (int k = 0; k < G; ++k) {
+                    const float u = __uint_as_float(zn[k]);
+                    const uint16_t p1 = tc::bf16_bits_rn(u);
+                    const float r1 = u - bf16_to_f32(p1);
+                    const uint16_t p2 = tc::bf16_bits_rn(r1);
+                    const float r2 = r1 - bf16_to_f32(p2);
+                    zr[k] = p1;
+                    zr[G + k] = p2;
+                    zr[2 * G + k] = tc::bf16_bits_rn(r2);
+                }
+                zr[3 * G] = zr[3 * G + 1] = zr[3 * G + 2] = 0x3F80;   // bf16 1.0
+            } else {
+#pragma unroll
+                for (int k = 0; k < KD; ++k) zr[k] = k < G ? (uint16_t)zn[k] : 0;
+                zr[G] = zr[G + 1] = zr[G + 2] = 0x3F80;           // bf16 1.0
+            }
             unsigned char *base = smem + (half ? S::offA2 : S::offA) + ((row >> 3) * KB) * 128 + (row & 7) * 16;
 #pragma unroll
             for (int kb = 0; kb < KB; ++kb) {
@@ -433,7 +489,9 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
             const int t = tid / NP, p = tid % NP;
             const int nr = tile * TOKS + t;
             if (nr < a.ntok) {
-                const uint32_t w = ok ? ((uint32_t)codes[t * NG + p] | ((uint32_t)codes[t * NG + p + NP] << 8) |
+                // key bytes: groups p and p + NP, or with TaSQ keys TaSQ groups 2p and 2p + 1
+                const int k0 = TQ ? 2 * p : p, k1 = TQ ? 2 * p + 1 : p + NP;
+                const uint32_t w = ok ? ((uint32_t)codes[t * NG + k0] | ((uint32_t)codes[t * NG + k1] << 8) |
                                          ((uint32_t)codes[128 + t * NG + p] << 16) |
                                          ((uint32_t)codes[128 + t * NG + p + NP] << 24))
                                       : 0xFFFFFFFFu;
@@ -449,13 +507,13 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
     if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
 }
 
-template <int D, int C, int TC, bool PG>
+template <int D, int C, int TC, bool PG, bool TQ = false>
 static cudaError_t launch_tc_ct(const EncodeTcArgs &a0, cudaStream_t s) {
     constexpr int NG = D / C;
     constexpr int TOKS = PG ? 128 : 128 / NG;
-    constexpr int KD = ((C * TC + 3 + 15) / 16) * 16;
+    constexpr int KD = (((TQ ? 3 : 1) * C * TC + 3 + 15) / 16) * 16;
     EncodeTcArgs a = a0;
-    auto k = encode_tc_kernel<D, C, TC, PG>;
+    auto k = encode_tc_kernel<D, C, TC, PG, TQ>;
     cudaError_t e = ensure_dynamic_smem((const void *)k, TcSmem<KD>::kAlloc);
     if (e != cudaSuccess) return e;
     // CTAs resident per SM, from the limits that bind here: shared memory, registers and tensor memory
@@ -519,6 +577,41 @@ cudaError_t launch_encode_tc(const loopvq_cache &cc, int layer, int block, const
         if (cc.D == 64 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<64, 4, 4, true>(a, s);
         if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4, true>(a, s);
     }
+    return cudaErrorNotSupported;
+}
+
+// TaSQ keys (the scales must already be written): returns cudaErrorNotSupported when the shape has no
+// tensor-core instantiation.
+cudaError_t launch_tasq_encode_tc(const loopvq_cache &cc, const loopvq_tasq &tq, int layer, int block, const void *xk,
+                                  const void *xv, const int64_t *strides, int b0, int nb, int tok0, int ntok,
+                                  cudaStream_t s) {
+    if (ncb_of(cc) != 1) return cudaErrorNotSupported;
+    const int NB = cc.T / cc.Tc;
+    const int t0 = block * cc.Tc;
+    EncodeTcArgs a{};
+    a.xk = reinterpret_cast<const uint16_t *>(xk);
+    a.xv = reinterpret_cast<const uint16_t *>(xv);
+    a.s0 = strides[0];
+    a.s1 = strides[1];
+    a.s2 = strides[2];
+    a.s3 = strides[3];
+    a.idx = cc.idx + idx_base(cc, layer, block, 0, 0);
+    a.cb = cc.codebook + codebook_base(cc, layer, block, 0, 0);
+    a.Hkv = cc.Hkv;
+    a.K = cc.K;
+    a.Nmax = cc.Nmax;
+    a.b0 = b0;
+    a.nb = nb;
+    a.tok0 = tok0;
+    a.ntok = ntok;
+    a.tw = tq.w + ((size_t)layer * cc.T + t0) * cc.Hkv * cc.D;
+    a.tperm = tq.perm + ((size_t)layer * NB + block) * cc.Hkv * (cc.D / 2);
+    a.tsig = tq.sigma + ((size_t)layer * cc.T + t0) * cc.B * cc.Nmax;
+    a.B = cc.B;
+    if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4, false, true>(a, s);
+    if (cc.D == 128 && cc.c == 4 && cc.Tc == 2) return launch_tc_ct<128, 4, 2, false, true>(a, s);
+    if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4, false, true>(a, s);
+    if (cc.D == 64 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<64, 8, 4, false, true>(a, s);
     return cudaErrorNotSupported;
 }
 

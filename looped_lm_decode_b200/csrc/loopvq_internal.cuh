@@ -76,6 +76,9 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
 cudaError_t launch_tasq_encode(const loopvq_cache &cc, const loopvq_tasq &tq, int layer, int block, const void *xk,
                                const void *xv, int x_dtype, const int64_t *strides, int b0, int nb, int tok0, int ntok,
                                cudaStream_t s);
+cudaError_t launch_tasq_encode_tc(const loopvq_cache &cc, const loopvq_tasq &tq, int layer, int block, const void *xk,
+                                  const void *xv, const int64_t *strides, int b0, int nb, int tok0, int ntok,
+                                  cudaStream_t s);
 DecodePlan plan_bf16(const loopvq_bf16_cache &c, int max_len);
 cudaError_t launch_bf16_decode(const loopvq_bf16_cache &c, const DecodePlan &plan, const uint16_t *q,
                                const int32_t *starts, const int32_t *lens, int max_len, float scale, float *out,

@@ -105,12 +105,17 @@ __global__ void __launch_bounds__(128) tasq_encode_kernel(const TasqArgs a) {
     a.idx[((size_t)b * a.Hkv + h) * idx_words_per_bh(a.Nmax, D, C) + idx_word(a.tok0 + nrel, p, NP)] = word;
 }
 
+// parts: 1 = the scales, 2 = the CUDA-core encode, 3 = both
 template <int D, int C, int TC, typename XT>
-static cudaError_t launch_tasq_t(const TasqArgs &a, int nb, cudaStream_t s) {
+static cudaError_t launch_tasq_t(const TasqArgs &a, int nb, int parts, cudaStream_t s) {
     constexpr int NP = D / (2 * C);
-    tasq_sigma_kernel<D, XT><<<dim3(a.ntok, TC, nb), 32, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (parts & 1) {
+        tasq_sigma_kernel<D, XT><<<dim3(a.ntok, TC, nb), 32, 0, s>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (!(parts & 2)) return cudaSuccess;
     const size_t smem = 2 * (size_t)a.K * C * TC * sizeof(float) + (D / 2) * sizeof(int16_t);
     auto k = tasq_encode_kernel<D, C, TC, XT>;
     if ((e = ensure_dynamic_smem((const void *)k, smem)) != cudaSuccess) return e;
@@ -119,13 +124,13 @@ static cudaError_t launch_tasq_t(const TasqArgs &a, int nb, cudaStream_t s) {
 }
 
 template <int D, typename XT>
-static cudaError_t dispatch_tasq(int c, int tc, const TasqArgs &a, int nb, cudaStream_t s) {
-    if (c == 4 && tc == 4) return launch_tasq_t<D, 4, 4, XT>(a, nb, s);
-    if (c == 4 && tc == 2) return launch_tasq_t<D, 4, 2, XT>(a, nb, s);
-    if (c == 4 && tc == 1) return launch_tasq_t<D, 4, 1, XT>(a, nb, s);
-    if (c == 8 && tc == 4) return launch_tasq_t<D, 8, 4, XT>(a, nb, s);
-    if (c == 8 && tc == 2) return launch_tasq_t<D, 8, 2, XT>(a, nb, s);
-    if (c == 8 && tc == 1) return launch_tasq_t<D, 8, 1, XT>(a, nb, s);
+static cudaError_t dispatch_tasq(int c, int tc, const TasqArgs &a, int nb, int parts, cudaStream_t s) {
+    if (c == 4 && tc == 4) return launch_tasq_t<D, 4, 4, XT>(a, nb, parts, s);
+    if (c == 4 && tc == 2) return launch_tasq_t<D, 4, 2, XT>(a, nb, parts, s);
+    if (c == 4 && tc == 1) return launch_tasq_t<D, 4, 1, XT>(a, nb, parts, s);
+    if (c == 8 && tc == 4) return launch_tasq_t<D, 8, 4, XT>(a, nb, parts, s);
+    if (c == 8 && tc == 2) return launch_tasq_t<D, 8, 2, XT>(a, nb, parts, s);
+    if (c == 8 && tc == 1) return launch_tasq_t<D, 8, 1, XT>(a, nb, parts, s);
     return cudaErrorInvalidValue;
 }
 
@@ -155,11 +160,22 @@ cudaError_t launch_tasq_encode(const loopvq_cache &cc, const loopvq_tasq &tq, in
     a.tok0 = tok0;
     a.ntok = ntok;
     const bool bf = x_dtype == LOOPVQ_BF16;
-    if (cc.D == 128)
-        return bf ? dispatch_tasq<128, uint16_t>(cc.c, cc.Tc, a, nb, s) : dispatch_tasq<128, float>(cc.c, cc.Tc, a, nb, s);
-    if (cc.D == 64)
-        return bf ? dispatch_tasq<64, uint16_t>(cc.c, cc.Tc, a, nb, s) : dispatch_tasq<64, float>(cc.c, cc.Tc, a, nb, s);
-    return cudaErrorInvalidValue;
+    auto run = [&](int parts) -> cudaError_t {
+        if (cc.D == 128)
+            return bf ? dispatch_tasq<128, uint16_t>(cc.c, cc.Tc, a, nb, parts, s)
+                      : dispatch_tasq<128, float>(cc.c, cc.Tc, a, nb, parts, s);
+        if (cc.D == 64)
+            return bf ? dispatch_tasq<64, uint16_t>(cc.c, cc.Tc, a, nb, parts, s)
+                      : dispatch_tasq<64, float>(cc.c, cc.Tc, a, nb, parts, s);
+        return cudaErrorInvalidValue;
+    };
+    if (!bf) return run(3);
+    // bf16 keys and values: the scales, then the tensor-core encode where the shape has one
+    cudaError_t e = run(1);
+    if (e != cudaSuccess) return e;
+    e = launch_tasq_encode_tc(cc, tq, layer, block, xk, xv, strides, b0, nb, tok0, ntok, s);
+    if (e != cudaErrorNotSupported) return e;
+    return run(2);
 }
 
 }  // namespace loopvq

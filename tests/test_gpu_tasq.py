@@ -45,10 +45,13 @@ def _tasq_codes(ck, NP):
 
 @pytest.mark.parametrize("name", list(SHAPES))
 def test_tasq_encode_parity(name):
+    """Codes bit-exact except near-ties (fp64 distances within 1e-5 relative, counted); scales bit-exact.
+    bf16 input at these shapes runs the tensor-core encode with the three-part split of u."""
     w = SHAPES[name]
     cache = make_cache(w)
     tq, tw, tp = _tasq(w, cache)
     NP = cache.NP
+    ties = 0
     for blk in range(w.NB):
         x = [kv_loops(w, 0, kv, blk * w.Tc, blk * w.Tc + w.Tc - 1, range(w.B), range(w.Nmax), range(w.Hkv))
              for kv in range(2)]                                          # [Tc][B][N][Hkv][D] bits
@@ -62,11 +65,30 @@ def test_tasq_encode_parity(name):
             for h in range(w.Hkv):
                 words = words_view(cache, 0, blk, b, h).cpu().numpy().view(np.uint32)
                 ck, cv = unpack_words(words, w.Nmax, NP)
-                rk = O.tasq_encode(xk[:, b, :, h, :], tw[0, blk * w.Tc:(blk + 1) * w.Tc, h], sig, tp[0, blk, h],
-                                   np_codebook_f32(w, 0, blk, 0, h), w.c)
-                np.testing.assert_array_equal(_tasq_codes(ck, NP), rk)
-                rv = O.encode(xv[:, b, :, h, :], np_codebook_f32(w, 0, blk, 1, h), w.c)
-                np.testing.assert_array_equal(cv, rv)
+                Ek, Ev = np_codebook_f32(w, 0, blk, 0, h), np_codebook_f32(w, 0, blk, 1, h)
+                rk = O.tasq_encode(xk[:, b, :, h, :], tw[0, blk * w.Tc:(blk + 1) * w.Tc, h], sig, tp[0, blk, h], Ek,
+                                   w.c)
+                gk = _tasq_codes(ck, NP)
+                mism = np.argwhere(gk != rk)
+                if len(mism):
+                    # the coupled vectors of TaSQ groups: u at the permuted channels, group g = channels g c ..
+                    u = np.stack([O.tasq_transform(xk[m, b, :, h, :], tw[0, blk * w.Tc + m, h], sig[m])
+                                  for m in range(w.Tc)])
+                    pairs = tp[0, blk, h].astype(np.int64) & (w.D // 2 - 1)
+                    chans = np.stack([pairs, pairs + w.D // 2], axis=1).reshape(-1)     # (f, f + D/2) per pair
+                    ut = np.ascontiguousarray(u[:, :, chans])
+                    for n, g in mism:
+                        dg = O.dist64(ut, Ek, w.c, n, g, int(gk[n, g]))
+                        do = O.dist64(ut, Ek, w.c, n, g, int(rk[n, g]))
+                        assert abs(dg - do) <= 1e-5 * max(dg, do), (b, h, n, g, dg, do)
+                    ties += len(mism)
+                rv = O.encode(xv[:, b, :, h, :], Ev, w.c)
+                for n, g in np.argwhere(cv != rv):
+                    dg = O.dist64(xv[:, b, :, h, :], Ev, w.c, n, g, int(cv[n, g]))
+                    do = O.dist64(xv[:, b, :, h, :], Ev, w.c, n, g, int(rv[n, g]))
+                    assert abs(dg - do) <= 1e-5 * max(dg, do), (b, h, n, g, dg, do)
+                    ties += 1
+    print(f"{name}: near-ties {ties}")
 
 
 @pytest.mark.parametrize("name", list(SHAPES))
