@@ -265,12 +265,15 @@ def workload_desc(w):
 
 
 def call_bytes(w, lens):
-    """Algorithmic bytes of one decode call: index words, codebook slices, query, output, lse."""
+    """Algorithmic bytes of one decode call: index words, codebook slices, query, output, lse; with TaSQ
+    keys also the fp16 token scales (one per token, shared by the heads) and each head's channel weights
+    (fp32) and pair order (int16)."""
     idx = int(np.sum(lens)) * w.Hkv * 2 * (w.D // w.c)
     slices = 2 * w.Hkv * w.K * w.c * 2
     q = w.B * w.Hq * w.D * 2
     out = w.B * w.Hq * w.D * 4 + w.B * w.Hq * 4
-    return idx + slices + q + out
+    tasq = int(np.sum(lens)) * 2 + w.Hkv * (w.D * 4 + (w.D // 2) * 2) if w.tasq else 0
+    return idx + slices + q + out + tasq
 
 
 def gather_bytes(w, lens):

@@ -191,6 +191,14 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             // the lane's finished token n is attended iff 0 <= n - st < tok_end - st
             int nrel = tok_begin + 16 * i0 + t + 4 * kown - st;
             const unsigned span = (unsigned)(tok_end - st);
+            // TQ: the TaSQ scale of the token a lane finishes, loaded one tile ahead (0 outside the span,
+            // where the score is masked anyway)
+            const uint16_t *sig_b = TQ ? a.tsig + (size_t)b * a.Nmax + st : nullptr;
+            auto load_sig = [&](int nr) {
+                return (unsigned)nr < span ? __half2float(__ushort_as_half(__ldg(sig_b + nr))) : 0.f;
+            };
+            float sig_next = 0.f;
+            if constexpr (TQ) sig_next = load_sig(nrel);
             const unsigned char *wrd = smem + S::kRing + (uint32_t)warp * DEPTH * 1024u + 4u * (4 * g + t);
             uint32_t soff = 0;
             __syncthreads();                               // tables staged
@@ -274,6 +282,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                 for (int i = ib; i < ie; ++i) {
                     cp_async_wait<DEPTH - 1>();
                     __syncwarp();
+                    float sig = 0.f;
+                    if constexpr (TQ) {
+                        sig = sig_next;
+                        sig_next = load_sig(nrel + 16);
+                    }
                     const uint32_t *wp = reinterpret_cast<const uint32_t *>(wrd + soff);
                     uint32_t wa[4], wb[4];
 #pragma unroll
@@ -349,10 +362,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                         sk = kk + __shfl_xor_sync(0xffffffffu, oo, 8);
                         sk += __shfl_xor_sync(0xffffffffu, sk, 16);
                     }
-                    if constexpr (TQ) {                    // the finished token's TaSQ scale
-                        if ((unsigned)nrel < span)
-                            sk *= __half2float(__ushort_as_half(__ldg(a.tsig + (size_t)b * a.Nmax + st + nrel)));
-                    }
+                    if constexpr (TQ) sk *= sig;          // the finished token's TaSQ scale
                     sk = (unsigned)nrel < span ? sk : -CUDART_INF_F;
                     nrel += 16;
 
