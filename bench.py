@@ -96,9 +96,19 @@ def decode_kernel_name(w):
     return "decode_split"
 
 
+def _code_only(src: bytes) -> bytes:
+    """C++ source without its comments and with whitespace runs collapsed, so that editing a comment
+    does not mark a profile as stale."""
+    import re
+    src = re.sub(rb"/\*.*?\*/", b" ", src, flags=re.S)
+    src = re.sub(rb"//[^\n]*", b" ", src)
+    return re.sub(rb"\s+", b" ", src).strip()
+
+
 def kernel_sources_hash(kern):
     """Hash of what decides a decode split kernel's code and launch: its headers, and for the MHA and GQA
-    kernels the line of decode_attn.cu that fixes their launch shape (the whole file otherwise)."""
+    kernels the line of decode_attn.cu that fixes their launch shape (the whole file otherwise), each
+    without comments."""
     import hashlib
     csrc = os.path.join(ROOT, "looped_lm_decode_b200", "csrc")
     h = hashlib.sha256()
@@ -106,11 +116,11 @@ def kernel_sources_hash(kern):
              "decode_gqa": ("decode_gqa.cuh", "decode_mha.cuh", "decode_kernel.cuh")}.get(kern, ("decode_kernel.cuh",))
     for src in heads:
         with open(os.path.join(csrc, src), "rb") as f:
-            h.update(f.read())
+            h.update(_code_only(f.read()))
     with open(os.path.join(csrc, "decode_attn.cu"), "rb") as f:
         attn = f.read()
     tag = {"decode_mha": b"static constexpr int kMhaWarps", "decode_gqa": b"static constexpr int kGqaWarps"}.get(kern)
-    h.update(attn if tag is None else next(ln for ln in attn.splitlines() if ln.startswith(tag)))
+    h.update(_code_only(attn if tag is None else next(ln for ln in attn.splitlines() if ln.startswith(tag))))
     return h.hexdigest()[:16]
 
 

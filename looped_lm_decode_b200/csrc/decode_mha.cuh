@@ -37,6 +37,10 @@
 //  * Index words arrive through a per-warp ring of 1 KiB stages in shared memory filled with 16-byte
 //    cp.async copies (lane L copies chunks L and L + 32 of the tile); each lane reads its 8 words with
 //    conflict-free 4-byte loads.
+//  * TaSQ keys (TQ, LoopVQ paper App. B): word p's key codes are TaSQ groups 2p and 2p + 1, whose fp32
+//    entries hold the RoPE pairs of the head's pair order interleaved.  The lane's 8 pairs come from
+//    that order, so all of them run the difference form; their rotated query is divided by the channel
+//    weight, and the finished score is multiplied by the token's scale, read one tile ahead.
 #pragma once
 
 #include "decode_kernel.cuh"

@@ -48,3 +48,12 @@ def test_single_process_helpers():
     import bench
     assert bench.max_over_ranks(3.5) == 3.5
     assert abs(bench.job_throughput(1, 193257984 * 96, 15.6) - 1189.3) < 1.0
+
+
+def test_profile_hash_ignores_comments_only():
+    """A committed ncu summary stays valid across comment edits of the kernel sources, not code edits."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = b"int x = 1; // old note\n/* block\n comment */ float y;\n"
+    assert bench._code_only(a) == bench._code_only(b"int x = 1;   // new note\nfloat y;")
+    assert bench._code_only(a) != bench._code_only(b"int x = 2; float y;")
