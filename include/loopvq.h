@@ -252,9 +252,11 @@ size_t loopvq_tasq_sigma_elems(const loopvq_cache *cache);
  * loopvq_encode with TaSQ (App. B, eq. 10-11): for sequences b0 .. b0+nb-1
  * and tokens tok0 .. tok0+ntok-1 of every loop step of the block, compute
  * sigma (fp64 root mean square, rounded to fp16) into tasq->sigma, then code
- * the keys' coupled vectors of u and the values' coupled vectors (exact fp32
- * nearest entries, lowest index on ties).  Arguments as for loopvq_encode;
- * the call must cover all KV heads of the tokens (sigma spans them).
+ * the keys' coupled vectors of u and the values' coupled vectors (nearest
+ * entries as in loopvq_encode, lowest index on ties; for bf16 input the fp32
+ * u is split exactly into three bf16 parts, so the tensor-core products stay
+ * exact).  Arguments as for loopvq_encode; the call must cover all KV heads
+ * of the tokens (sigma spans them).
  */
 loopvq_status loopvq_tasq_encode(const loopvq_cache *cache, const loopvq_tasq *tasq, int layer, int block,
                                  const void *xk, const void *xv, int x_dtype, const int64_t x_strides[4],
