@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_gqa_kernel(const Deco
         nl[3] = f2(-4.f * s2b.z * s2b.z, -4.f * s2b.w * s2b.w);
     }
 
+    int staged_h = -1;                                     // the KV head whose slices the tables hold
     while (pos < x_end && h < a.Hkv) {
         int len, st, base;
         const long long seg_end = seg0 + seq_tiles(a, b, base, st, len);
@@ -105,23 +106,32 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_gqa_kernel(const Deco
 
             // stage the slices of head h: K entry r in fp32 (32 bytes) at row r of [0, 64 KiB), its first
             // half in 8 replicas at bytes [0, 128), its second half in 8 replicas at [128, 256); V entry r
-            // in bf16 (16 bytes) in 16 replicas at row r of [64 KiB, 128 KiB)
-            {
+            // in bf16 (16 bytes) in 16 replicas at row r of [64 KiB, 128 KiB).  The slices depend on the KV
+            // head only, so a piece of the head already staged keeps them.  Thread r reads entry r once and
+            // writes its replicas starting at replica r mod 8 (16), so the 8 lanes of each quarter-warp
+            // store write distinct banks.
+            const bool restage = h != staged_h;
+            if (restage) {
                 const uint4 *sk = reinterpret_cast<const uint4 *>(a.slk + (size_t)h * a.K * 8);
                 const uint4 *sv = reinterpret_cast<const uint4 *>(a.slv + (size_t)h * a.K * 8);
-                for (int it = tid; it < 256 * 8; it += NT) {
-                    const int rep = it & 7, r = it >> 3;
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (r < a.K) v = __ldg(sk + r);
-                    *reinterpret_cast<float4 *>(smem + r * 256 + rep * 16) = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-                    *reinterpret_cast<float4 *>(smem + r * 256 + 128 + rep * 16) = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
+                for (int r = tid; r < 256; r += NT) {
+                    uint4 ek = make_uint4(0u, 0u, 0u, 0u), ev = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < a.K) {
+                        ek = __ldg(sk + r);
+                        ev = __ldg(sv + r);
+                    }
+                    const float4 k0 = make_float4(bf16lo(ek.x), bf16hi(ek.x), bf16lo(ek.y), bf16hi(ek.y));
+                    const float4 k1 = make_float4(bf16lo(ek.z), bf16hi(ek.z), bf16lo(ek.w), bf16hi(ek.w));
+                    unsigned char *row = smem + r * 256;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        *reinterpret_cast<float4 *>(row + ((k + r) & 7) * 16) = k0;
+                        *reinterpret_cast<float4 *>(row + 128 + ((k + r) & 7) * 16) = k1;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) *reinterpret_cast<uint4 *>(row + 65536 + ((k + r) & 15) * 16) = ev;
                 }
-                for (int it = tid; it < 256 * 16; it += NT) {
-                    const int rep = it & 15, r = it >> 4;
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (r < a.K) v = __ldg(sv + r);
-                    *reinterpret_cast<uint4 *>(smem + 65536 + r * 256 + rep * 16) = v;
-                }
+                staged_h = h;
             }
 
             // the query heads in slot order s -> head s ^ hl, scaled, at the lane's channels
@@ -169,7 +179,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_gqa_kernel(const Deco
             const unsigned span = (unsigned)(tok_end - st);
             const unsigned char *wrd = smem + S::kRing + (uint32_t)warp * DEPTH * 512u + 4u * (4 * g + t);
             uint32_t soff = 0;
-            __syncthreads();                               // tables staged
+            if (restage) __syncthreads();                  // tables staged (the condition is CTA-uniform)
 
             for (int ib = i0; ib < i1; ib += ANCHOR) {
                 {

@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
         nlB[1] = f2(-4.f * s2.z * s2.z, -4.f * s2.w * s2.w);
     }
 
+    int staged_h = -1;                                     // the KV head whose slices the tables hold
     while (pos < x_end && h < a.Hkv) {
         int len, st, base;
         const long long seg_end = seg0 + seq_tiles(a, b, base, st, len);
@@ -132,22 +133,28 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             __syncthreads();                               // the previous piece's tables and records are done
 
             // stage: row r = K entry r in fp32, 8 replicas of 16 bytes at [0, 128); V entry r in bf16,
-            // 16 replicas of 8 bytes at [128, 256)
-            {
+            // 16 replicas of 8 bytes at [128, 256).  The slices depend on the KV head only, so a piece of
+            // the head already staged (the next sequence of the same head) keeps them.  Thread r reads
+            // entry r once and writes its replicas starting at replica r mod 8 (16), so the lanes of each
+            // quarter-warp (half-warp) store write distinct banks.
+            const bool restage = h != staged_h;
+            if (restage) {
                 const uint16_t *sk = a.slk + (size_t)h * a.K * 4;
                 const uint16_t *sv = a.slv + (size_t)h * a.K * 4;
-                for (int it = tid; it < 256 * 8; it += NT) {
-                    const int rep = it & 7, r = it >> 3;
-                    uint2 v = make_uint2(0u, 0u);
-                    if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(sk + (size_t)r * 4));
-                    *reinterpret_cast<float4 *>(smem + r * 256 + rep * 16) = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+                for (int r = tid; r < 256; r += NT) {
+                    uint2 ek = make_uint2(0u, 0u), ev = make_uint2(0u, 0u);
+                    if (r < a.K) {
+                        ek = __ldg(reinterpret_cast<const uint2 *>(sk + (size_t)r * 4));
+                        ev = __ldg(reinterpret_cast<const uint2 *>(sv + (size_t)r * 4));
+                    }
+                    const float4 kf = make_float4(bf16lo(ek.x), bf16hi(ek.x), bf16lo(ek.y), bf16hi(ek.y));
+                    unsigned char *row = smem + r * 256;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) *reinterpret_cast<float4 *>(row + ((k + r) & 7) * 16) = kf;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + 128 + ((k + r) & 15) * 8) = ev;
                 }
-                for (int it = tid; it < 256 * 16; it += NT) {
-                    const int rep = it & 15, r = it >> 4;
-                    uint2 v = make_uint2(0u, 0u);
-                    if (r < a.K) v = __ldg(reinterpret_cast<const uint2 *>(sv + (size_t)r * 4));
-                    *reinterpret_cast<uint2 *>(smem + r * 256 + 128 + rep * 8) = v;
-                }
+                staged_h = h;
             }
 
             // this warp's run of 16-token tiles [i0, i1) of the piece
@@ -205,7 +212,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             if constexpr (TQ) sig_next = load_sig(nrel);
             const unsigned char *wrd = smem + S::kRing + (uint32_t)warp * DEPTH * 1024u + 4u * (4 * g + t);
             uint32_t soff = 0;
-            __syncthreads();                               // tables staged
+            if (restage) __syncthreads();                  // tables staged (the condition is CTA-uniform)
 
             for (int ib = i0; ib < i1; ib += ANCHOR) {
                 if constexpr (TQ) {
