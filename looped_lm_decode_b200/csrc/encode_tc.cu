@@ -358,12 +358,21 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
     const int rtok = PG ? row : row / NG, rg = PG ? 0 : row % NG;
 
     // this thread's coupled vector (key for half 0, value for half 1) of the next unit, one unit ahead:
-    // bf16 bits, or with TaSQ keys the fp32 bits of u
+    // bf16 bits, or with TaSQ keys the fp32 bits of u.  With TaSQ keys and G <= 16 (DEFER) the row holds
+    // the raw key channels at the permuted positions and sgn the token's sigma of each loop step instead;
+    // u is formed when the A operand is built, so the loads stay in flight across the current unit's
+    // arg-max rather than stalling on the division here (at G = 32 the registers are not there).
+    constexpr bool DEFER = TQ && G <= 16;
     uint32_t zn[G];
+    float sgn[DEFER ? TC : 1];
     auto load_row = [&](bool valid, const Pos &p, uint32_t (&z)[G]) {
         const int nrel = p.tile * TOKS + rtok;
 #pragma unroll
         for (int k = 0; k < G; ++k) z[k] = 0;
+        if constexpr (DEFER) {
+#pragma unroll
+            for (int m = 0; m < TC; ++m) sgn[m] = 1.f;     // rows past the range: u = 0, no 0/0
+        }
         if (valid && nrel < a.ntok) {
             if (TQ && half == 0) {
                 // TaSQ group rg: channel i is the low (i even) or high (i odd) channel of pair perm[rg C/2 + i/2]
@@ -375,12 +384,22 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
                     const int f = (i & 1) ? lowf + D / 2 : lowf;
 #pragma unroll
                     for (int m = 0; m < TC; ++m) {
-                        const float wt = __ldg(a.tw + ((size_t)m * a.Hkv + p.h) * D + f);
-                        const float sg = __half2float(__ushort_as_half(
-                            __ldg(a.tsig + ((size_t)m * a.B + a.b0 + p.brel) * a.Nmax + a.tok0 + nrel)));
-                        const float k = bf16_to_f32(__ldg(x + (size_t)m * a.s0 + f));
-                        z[i * TC + m] = __float_as_uint(__fdiv_rn(__fmul_rn(wt, k), sg));
+                        if constexpr (DEFER) {
+                            z[i * TC + m] = __ldg(x + (size_t)m * a.s0 + f);
+                        } else {
+                            const float wt = __ldg(a.tw + ((size_t)m * a.Hkv + p.h) * D + f);
+                            const float sg = __half2float(__ushort_as_half(
+                                __ldg(a.tsig + ((size_t)m * a.B + a.b0 + p.brel) * a.Nmax + a.tok0 + nrel)));
+                            const float k = bf16_to_f32(__ldg(x + (size_t)m * a.s0 + f));
+                            z[i * TC + m] = __float_as_uint(__fdiv_rn(__fmul_rn(wt, k), sg));
+                        }
                     }
+                }
+                if constexpr (DEFER) {
+#pragma unroll
+                    for (int m = 0; m < TC; ++m)
+                        sgn[m] = __half2float(__ushort_as_half(
+                            __ldg(a.tsig + ((size_t)m * a.B + a.b0 + p.brel) * a.Nmax + a.tok0 + nrel)));
                 }
             } else {
                 const uint16_t *x = (half ? a.xv : a.xk) + (size_t)p.brel * a.s1 + (size_t)nrel * a.s2 +
@@ -406,19 +425,36 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
         {
             uint16_t zr[KD];
             if (TQ && half == 0) {
+                // u = fl(fl(w k) / sigma) at the permuted channels (DEFER: formed here), then
                 // u = hi + mid + lo exactly (three round-to-nearest bf16 parts of an fp32 value)
+                const int16_t *pm = a.tperm + (size_t)h * (D / 2) + rg * (C / 2);
 #pragma unroll
                 for (int k = 0; k < KD; ++k) zr[k] = 0;
 #pragma unroll
-                for (int k = 0; k < G; ++k) {
-                    const float u = __uint_as_float(zn[k]);
-                    const uint16_t p1 = tc::bf16_bits_rn(u);
-                    const float r1 = u - bf16_to_f32(p1);
-                    const uint16_t p2 = tc::bf16_bits_rn(r1);
-                    const float r2 = r1 - bf16_to_f32(p2);
-                    zr[k] = p1;
-                    zr[G + k] = p2;
-                    zr[2 * G + k] = tc::bf16_bits_rn(r2);
+                for (int i = 0; i < C; ++i) {
+                    int f = 0;
+                    if constexpr (DEFER) {
+                        const int lowf = __ldg(pm + i / 2) & (D / 2 - 1);
+                        f = (i & 1) ? lowf + D / 2 : lowf;
+                    }
+#pragma unroll
+                    for (int m = 0; m < TC; ++m) {
+                        const int k = i * TC + m;
+                        float u;
+                        if constexpr (DEFER) {
+                            const float wt = __ldg(a.tw + ((size_t)m * a.Hkv + h) * D + f);
+                            u = __fdiv_rn(__fmul_rn(wt, bf16_to_f32((uint16_t)zn[k])), sgn[m]);
+                        } else {
+                            u = __uint_as_float(zn[k]);
+                        }
+                        const uint16_t p1 = tc::bf16_bits_rn(u);
+                        const float r1 = u - bf16_to_f32(p1);
+                        const uint16_t p2 = tc::bf16_bits_rn(r1);
+                        const float r2 = r1 - bf16_to_f32(p2);
+                        zr[k] = p1;
+                        zr[G + k] = p2;
+                        zr[2 * G + k] = tc::bf16_bits_rn(r2);
+                    }
                 }
                 zr[3 * G] = zr[3 * G + 1] = zr[3 * G + 2] = 0x3F80;   // bf16 1.0
             } else {
