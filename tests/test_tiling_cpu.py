@@ -90,3 +90,37 @@ def test_shares_are_even():
     for s, c, n in recs.values():
         per_cta[c] = per_cta.get(c, 0) + n
     assert max(per_cta.values()) - min(per_cta.values()) <= 1
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_a_cta_never_returns_to_a_kv_head(seed):
+    """The one-head and four-head decode kernels keep their staged codebook tables while a CTA's next
+    piece has the same KV head.  That is sound because a CTA walks its pieces in segment order, s = h B + b,
+    so its heads never decrease: once it leaves a head it does not come back to it."""
+    rng = np.random.default_rng(100 + seed)
+    B = int(rng.integers(1, 30))
+    Hkv = int(rng.integers(1, 9))
+    lens = rng.integers(0, int(rng.choice([8, 300, 4096])) + 1, B)
+    starts = np.array([rng.integers(0, int(l) + 1) for l in lens])
+    G = int(rng.integers(1, 600))
+    recs, _, _ = written_records(lens, starts, Hkv, G)
+    walks = {}
+    for r in sorted(recs):                               # record index s + c grows along a CTA's walk
+        s, c, _ = recs[r]
+        walks.setdefault(c, []).append(s // B)
+    for c, heads in walks.items():
+        assert heads == sorted(heads), (c, heads)
+
+
+def test_ctx32k_ctas_restage_rarely():
+    """At ctx32k (296 CTAs, 8 sequences, 16 KV heads) most CTAs touch one or two pieces of one head; the
+    tables are staged once per head a CTA visits."""
+    lens = np.array([18460, 28363, 24578, 16564, 31514, 21536, 21419, 26134])
+    recs, _, _ = written_records(lens, np.zeros(8, int), 16, 296)
+    pieces, heads = {}, {}
+    for s, c, _ in recs.values():
+        pieces[c] = pieces.get(c, 0) + 1
+        heads.setdefault(c, set()).add(s // 8)
+    stagings = sum(len(v) for v in heads.values())
+    assert stagings < sum(pieces.values())
+    assert max(len(v) for v in heads.values()) <= 2
