@@ -43,7 +43,9 @@ typedef enum {
     LOOPVQ_ERR_INVALID_ARG = 1,   /* null pointer, out-of-range index or size */
     LOOPVQ_ERR_UNSUPPORTED = 2,   /* valid but not built: D, c, Tc, Hq/Hkv outside the supported set */
     LOOPVQ_ERR_WORKSPACE = 3,     /* workspace missing or smaller than loopvq_decode_workspace_bytes */
-    LOOPVQ_ERR_CUDA = 4           /* a launch failed; loopvq_last_error() holds the CUDA message */
+    LOOPVQ_ERR_CUDA = 4,          /* a launch failed; loopvq_last_error() holds the CUDA message */
+    LOOPVQ_ERR_TIMEOUT = 5,       /* reported by loopvq_fault_check: an encode's bounded wait ran out */
+    LOOPVQ_ERR_OVERFLOW = 6       /* reported by loopvq_fault_check: a window roll found the coded cache full */
 } loopvq_status;
 
 enum { LOOPVQ_BF16 = 0, LOOPVQ_FP32 = 1 };
@@ -392,6 +394,36 @@ loopvq_status loopvq_decode_attn_noalloc(const loopvq_cache *cache, int layer, i
 
 /* Message of the last failed call on this thread ("" if none). */
 const char *loopvq_last_error(void);
+
+/*
+ * Faults found on the device.  Calls are asynchronous, so a kernel that cannot
+ * finish its job cannot return an error from the call that launched it;
+ * instead it sets a bit in a fault word that the library keeps on each GPU:
+ *   - the tensor-core encoder (loopvq_encode and loopvq_tasq_encode with bf16
+ *     input) bounds each wait for its own contraction; when the bound runs
+ *     out it stops, waits (bounded by 2 s) for the work it already issued,
+ *     releases its tensor memory, writes 0xFF code bytes for the tokens it
+ *     had not finished and sets the fault;
+ *   - loopvq_window_advance does not roll a sequence whose coded cache has no
+ *     room for the page (coded_end + 8 > Nmax) and sets the fault; that
+ *     sequence's window stays full, so its next append overwrites the newest
+ *     slot.
+ * loopvq_fault_check synchronises `stream` (the one call that does), reads
+ * and clears the current GPU's fault word and returns LOOPVQ_ERR_TIMEOUT or
+ * LOOPVQ_ERR_OVERFLOW (message in loopvq_last_error) or LOOPVQ_OK.  The word
+ * is shared by every stream and thread of the process on that GPU; its first
+ * use on a device looks up the word's address (make that first call before
+ * any stream capture).
+ *
+ * loopvq_set_wait_limit_ns sets, for the whole process, the bound in
+ * nanoseconds on each such wait of the encoder (default 2e9); 0 tests the
+ * wait once without blocking and gives up if the work is not finished,
+ * which tests use to exercise this path.
+ * No page of the paper corresponds; it is the library's error channel.
+ */
+loopvq_status loopvq_fault_check(void *stream);
+void loopvq_set_wait_limit_ns(uint64_t ns);
+uint64_t loopvq_wait_limit_ns(void);
 
 /* ABI version, bumped on any incompatible change. */
 int loopvq_abi_version(void);

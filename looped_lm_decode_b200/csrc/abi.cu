@@ -15,6 +15,9 @@ namespace {
 
 thread_local char g_err[512] = "";
 
+// Opt-in shared memory per CTA on B200 (227 KiB).
+constexpr size_t kMaxOptinSmem = 232448;
+
 loopvq_status fail(loopvq_status st, const char *fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
@@ -348,6 +351,11 @@ static loopvq_status check_window(const loopvq_window *w, const loopvq_cache *cc
     if (w->n_sink <= 0 || w->n_recent <= 0 || w->n_sink % 8 != 0 || w->n_recent % 8 != 0)
         return fail(LOOPVQ_ERR_INVALID_ARG, "n_sink=%d, n_recent=%d must be positive multiples of 8", w->n_sink,
                     w->n_recent);
+    // the page roll stages a (layer, loop step, sequence, head)'s n_recent recent slots in shared memory
+    if ((size_t)w->n_recent * (size_t)w->D * 2 > kMaxOptinSmem)
+        return fail(LOOPVQ_ERR_UNSUPPORTED, "n_recent=%d: %zu bytes of recent slots exceed the %zu bytes of shared "
+                    "memory the page roll stages them in", w->n_recent, (size_t)w->n_recent * (size_t)w->D * 2,
+                    kMaxOptinSmem);
     LQ_TRY(check_ptr(w->k_rot, "k_rot"));
     LQ_TRY(check_ptr(w->k_pre, "k_pre"));
     LQ_TRY(check_ptr(w->v, "v"));
@@ -448,6 +456,6 @@ loopvq_status loopvq_dequant_debug(const loopvq_cache *cc, int layer, int t, int
 
 const char *loopvq_last_error(void) { return g_err; }
 
-int loopvq_abi_version(void) { return 2; }
+int loopvq_abi_version(void) { return 3; }
 
 }  // extern "C"

@@ -17,7 +17,9 @@
 // staged in shared memory in the canonical K-major layout without swizzle: 8-row x 16-byte core
 // matrices, the K-direction neighbour 128 bytes on (leading byte offset), the next 8 rows KB*128
 // bytes on (stride byte offset).  One thread issues the MMAs and commits to an mbarrier; every wait
-// on it is bounded in time, and a timeout writes 0xFFFFFFFF words instead of codes.
+// on it is bounded in time (loopvq_set_wait_limit_ns); a CTA whose wait runs out sets the fault word
+// that loopvq_fault_check reports, waits (bounded) for the work it already issued, writes 0xFF code bytes
+// for its unfinished tokens and releases its tensor memory.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -64,15 +66,31 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
-// Wait for the mbarrier phase with the given parity; false after ~2 s.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity) {
+// Non-blocking test of the mbarrier phase (try_wait may suspend the thread for a while first).
+__device__ __forceinline__ bool mbar_test(uint32_t mbar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait for the mbarrier phase with the given parity; false once limit_ns have passed.  A limit of 0
+// tests the phase once without blocking.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t mbar, uint32_t parity, uint64_t limit_ns) {
+    if (limit_ns == 0) return mbar_test(mbar, parity);
     if (mbar_try(mbar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try(mbar, parity)) return true;
-        if (globaltimer() - t0 > 2000000000ull) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
     }
 }
+
+// Bound on the wait for work already issued, before a CTA that gave up releases its tensor memory.
+constexpr uint64_t kDrainNs = 2000000000ull;
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -204,6 +222,8 @@ struct EncodeTcArgs {
     const int16_t *tperm;
     const uint16_t *tsig;
     int B;
+    unsigned int *fault;      // per-GPU fault word: kFaultEncodeWait is set when a wait runs out
+    unsigned long long wait_ns;
 };
 
 // Shared-memory plan (bytes): B operands for K and V (256 x KD bf16 each), A operands for K and V
@@ -493,9 +513,18 @@ __global__ void __launch_bounds__(256, 2) encode_tc_kernel(const EncodeTcArgs a)
                 tc::mma_commit(mbar);
             }
             // every thread waits (bounded); the CTA continues only if all of them saw the MMAs complete
-            ok = __syncthreads_and(tc::mbar_wait_bounded(mbar, phase) ? 1 : 0) != 0;
+            ok = __syncthreads_and(tc::mbar_wait_bounded(mbar, phase, a.wait_ns) ? 1 : 0) != 0;
+            if (!ok) {
+                // give up: record the fault, and let the contraction already issued finish (bounded) before
+                // its shared-memory operands and tensor memory are released
+                if (tid == 0) {
+                    atomicOr(a.fault, kFaultEncodeWait);
+                    tc::mbar_wait_bounded(mbar, phase, tc::kDrainNs);
+                }
+                __syncthreads();
+                break;
+            }
             phase ^= 1u;
-            if (!ok) break;
             tc::tc_fence_after();
             // ---- exact arg-max of the row: maximum over both halves, then the first column equal to it
             const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -597,6 +626,8 @@ cudaError_t launch_encode_tc(const loopvq_cache &cc, int layer, int block, const
     a.nb = nb;
     a.tok0 = tok0;
     a.ntok = ntok;
+    a.wait_ns = wait_limit_ns();
+    if (cudaError_t ef = fault_word_for_current_device(&a.fault); ef != cudaSuccess) return ef;
     if (ncb_of(cc) == 1) {
         if (cc.D == 128 && cc.c == 4 && cc.Tc == 4) return launch_tc_ct<128, 4, 4, false>(a, s);
         if (cc.D == 128 && cc.c == 8 && cc.Tc == 4) return launch_tc_ct<128, 8, 4, false>(a, s);
@@ -640,6 +671,8 @@ cudaError_t launch_tasq_encode_tc(const loopvq_cache &cc, const loopvq_tasq &tq,
     a.nb = nb;
     a.tok0 = tok0;
     a.ntok = ntok;
+    a.wait_ns = wait_limit_ns();
+    if (cudaError_t ef = fault_word_for_current_device(&a.fault); ef != cudaSuccess) return ef;
     a.tw = tq.w + ((size_t)layer * cc.T + t0) * cc.Hkv * cc.D;
     a.tperm = tq.perm + ((size_t)layer * NB + block) * cc.Hkv * (cc.D / 2);
     a.tsig = tq.sigma + ((size_t)layer * cc.T + t0) * cc.B * cc.Nmax;

@@ -42,6 +42,14 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_floa
 // Sets the thread-local message returned by loopvq_last_error().
 void set_last_error(const char *msg);
 
+// Bits of the per-GPU fault word (faults.cu), reported by loopvq_fault_check.
+constexpr unsigned int kFaultEncodeWait = 1u;   // a tensor-core encode's bounded wait ran out
+constexpr unsigned int kFaultWindowFull = 2u;   // a window roll found the coded cache full
+// Device address of the fault word on the current device (looked up once per device).
+cudaError_t fault_word_for_current_device(unsigned int **out);
+// Bound on each wait of the tensor-core encoder for its own contraction (loopvq_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
+
 // Raises a kernel's dynamic shared-memory limit on the current device to at least `bytes`.  The
 // attribute is set on the first such request (or a larger one) per kernel and device only, so steady
 // launches make no attribute call: less host time per call, and nothing but launches inside a CUDA

@@ -10,9 +10,10 @@
 // the recent tokens oldest first.  Keys are kept rotated (for attention) and before RoPE (for the
 // encoder).  The per-sequence counters fill (slots in use) and coded_end (end of the coded tokens)
 // live on the device, so a decode step never waits for the host:
-//   advance: full windows encode their oldest page into the coded cache (every layer and block,
-//            one launch), move the recent slots down by 8 (one launch) and update the counters;
-//            then every sequence reserves the new token's slot.
+//   advance: full windows whose coded cache has room for a page encode their oldest page into it
+//            (every layer and block, one launch), move the recent slots down by 8 (one launch) and
+//            update the counters; then every sequence reserves the new token's slot.  A full window
+//            without room does not roll and sets the fault word (LOOPVQ_ERR_OVERFLOW).
 //   append:  the new token's K (rotated and not) and V of one (layer, loop step) go to slot fill-1.
 //   attend:  the coded kernel over [n_s, coded_end), whose merge kernel also attends to the window
 //            slots and combines both parts through their log-sum-exps (two launches in all).
@@ -28,6 +29,12 @@ struct WinEncArgs {
     int L, T, NB, B, Hkv, K, Nmax, W, n_sink;
 };
 
+// A sequence rolls when its window is full and the coded cache has room for the page; the three
+// kernels of an advance all take this decision from the same counters.
+__device__ __forceinline__ bool rolls(const int32_t *fill, const int32_t *coded_end, int b, int W, int Nmax) {
+    return __ldg(fill + b) >= W && __ldg(coded_end + b) + 8 <= Nmax;
+}
+
 // One thread per index word of the oldest recent page: token i < 8 of the page, pair-group p.
 // Grid: (ceil(8 NP / 128), L * NB * Hkv, B); the CTA's (layer, block, head) share a codebook.
 template <int D, int C, int TC>
@@ -36,7 +43,7 @@ __global__ void __launch_bounds__(128) window_page_encode_kernel(const WinEncArg
     constexpr int NP = D / (2 * C);
     extern __shared__ __align__(16) float ecb[];             // [2][K][G] fp32
     const int b = blockIdx.z;
-    if (__ldg(a.fill + b) < a.W) return;                     // only full windows roll (uniform per CTA)
+    if (!rolls(a.fill, a.coded_end, b, a.W, a.Nmax)) return; // uniform per CTA
     const int h = blockIdx.y % a.Hkv;
     const int lb = blockIdx.y / a.Hkv;
     const int block = lb % a.NB, layer = lb / a.NB;
@@ -47,8 +54,7 @@ __global__ void __launch_bounds__(128) window_page_encode_kernel(const WinEncArg
     const int wl = blockIdx.x * blockDim.x + threadIdx.x;
     if (wl >= 8 * NP) return;
     const int i = wl / NP, p = wl % NP;
-    const int n = __ldg(a.coded_end + b) + i;                // token position of the word
-    if (n < 0 || n >= a.Nmax) return;                        // outside the coded cache: not written
+    const int n = __ldg(a.coded_end + b) + i;                // token position of the word (< Nmax: it rolls)
     const int slot = a.n_sink + i;
     const size_t tstride = (size_t)a.B * a.Hkv * a.W * D;    // one loop step of the window
     float z[4][G];
@@ -74,11 +80,12 @@ __global__ void __launch_bounds__(128) window_page_encode_kernel(const WinEncArg
 // Grid: (L * T * Hkv, B); the rows are staged whole in shared memory, so the overlapping copy
 // reads every slot before any is written.
 __global__ void __launch_bounds__(256) window_shift_kernel(uint16_t *k_rot, uint16_t *k_pre, uint16_t *v,
-                                                           const int32_t *fill, int B, int Hkv, int D, int W,
-                                                           int n_sink, int n_recent) {
+                                                           const int32_t *fill, const int32_t *coded_end, int B,
+                                                           int Hkv, int D, int W, int n_sink, int n_recent,
+                                                           int Nmax) {
     extern __shared__ __align__(16) uint4 stage[];
     const int b = blockIdx.y;
-    if (__ldg(fill + b) < W) return;
+    if (!rolls(fill, coded_end, b, W, Nmax)) return;
     const int lt = blockIdx.x / Hkv, h = blockIdx.x % Hkv;
     const size_t row = (((size_t)lt * B + b) * Hkv + h) * (size_t)W * D;
     const int n16 = n_recent * D / 8;                        // 16-byte words moved
@@ -93,11 +100,18 @@ __global__ void __launch_bounds__(256) window_shift_kernel(uint16_t *k_rot, uint
     }
 }
 
-__global__ void window_counters_kernel(int32_t *fill, int32_t *coded_end, int B, int W) {
+// A full window whose coded cache has no room for the page does not roll: its counters stay, and the
+// fault word records it (loopvq_fault_check reports LOOPVQ_ERR_OVERFLOW).
+__global__ void window_counters_kernel(int32_t *fill, int32_t *coded_end, int B, int W, int Nmax,
+                                       unsigned int *fault) {
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= B) return;
     int f = fill[b];
     if (f >= W) {
+        if (coded_end[b] + 8 > Nmax) {
+            atomicOr(fault, kFaultWindowFull);
+            return;
+        }
         f -= 8;
         coded_end[b] += 8;
     }
@@ -174,10 +188,13 @@ cudaError_t launch_window_advance(const loopvq_window &w, const loopvq_cache &cc
     const size_t smem = (size_t)w.n_recent * w.D * 2;
     e = ensure_dynamic_smem((const void *)window_shift_kernel, smem);
     if (e != cudaSuccess) return e;
-    window_shift_kernel<<<dim3(w.L * w.T * w.Hkv, w.B), 256, smem, s>>>(w.k_rot, w.k_pre, w.v, w.fill, w.B, w.Hkv,
-                                                                         w.D, W, w.n_sink, w.n_recent);
+    unsigned int *fault = nullptr;
+    if ((e = fault_word_for_current_device(&fault)) != cudaSuccess) return e;
+    window_shift_kernel<<<dim3(w.L * w.T * w.Hkv, w.B), 256, smem, s>>>(w.k_rot, w.k_pre, w.v, w.fill, w.coded_end,
+                                                                         w.B, w.Hkv, w.D, W, w.n_sink, w.n_recent,
+                                                                         cc.Nmax);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    window_counters_kernel<<<(w.B + 127) / 128, 128, 0, s>>>(w.fill, w.coded_end, w.B, W);
+    window_counters_kernel<<<(w.B + 127) / 128, 128, 0, s>>>(w.fill, w.coded_end, w.B, W, cc.Nmax, fault);
     return cudaGetLastError();
 }
 

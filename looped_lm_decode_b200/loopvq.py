@@ -15,7 +15,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libloopvq.so")
 
-LOOPVQ_OK, LOOPVQ_ERR_INVALID_ARG, LOOPVQ_ERR_UNSUPPORTED, LOOPVQ_ERR_WORKSPACE, LOOPVQ_ERR_CUDA = range(5)
+(LOOPVQ_OK, LOOPVQ_ERR_INVALID_ARG, LOOPVQ_ERR_UNSUPPORTED, LOOPVQ_ERR_WORKSPACE, LOOPVQ_ERR_CUDA, LOOPVQ_ERR_TIMEOUT,
+ LOOPVQ_ERR_OVERFLOW) = range(7)
 LOOPVQ_BF16, LOOPVQ_FP32 = 0, 1
 
 EXPORTS = ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "loopvq_rope_elems",
@@ -25,7 +26,8 @@ EXPORTS = ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "l
            "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn", "loopvq_merge2",
            "loopvq_window_slots", "loopvq_window_advance", "loopvq_window_append",
            "loopvq_window_workspace_bytes", "loopvq_window_decode_attn", "loopvq_tasq_w_elems",
-           "loopvq_tasq_perm_elems", "loopvq_tasq_sigma_elems", "loopvq_tasq_encode", "loopvq_tasq_decode_attn")
+           "loopvq_tasq_perm_elems", "loopvq_tasq_sigma_elems", "loopvq_tasq_encode", "loopvq_tasq_decode_attn",
+           "loopvq_fault_check", "loopvq_set_wait_limit_ns", "loopvq_wait_limit_ns")
 
 
 class CacheDesc(C.Structure):
@@ -119,6 +121,12 @@ def lib():
         L.loopvq_last_error.argtypes = []
         L.loopvq_last_error.restype = C.c_char_p
         L.loopvq_abi_version.restype = i
+        L.loopvq_fault_check.argtypes = [vp]
+        L.loopvq_fault_check.restype = i
+        L.loopvq_set_wait_limit_ns.argtypes = [C.c_uint64]
+        L.loopvq_set_wait_limit_ns.restype = None
+        L.loopvq_wait_limit_ns.argtypes = []
+        L.loopvq_wait_limit_ns.restype = C.c_uint64
         _lib = L
     return _lib
 
@@ -126,6 +134,21 @@ def lib():
 def _check(status):
     if status != LOOPVQ_OK:
         raise LoopVQError(status, lib().loopvq_last_error().decode())
+
+
+def fault_check(stream=None):
+    """loopvq_fault_check: synchronise the stream, then raise LoopVQError if a kernel on this GPU recorded a
+    fault (an encode wait that ran out, a window roll without room) since the last check."""
+    _check(lib().loopvq_fault_check(_stream(stream)))
+
+
+def set_wait_limit_ns(ns: int):
+    """loopvq_set_wait_limit_ns: bound on each wait of the tensor-core encoder (process-wide)."""
+    lib().loopvq_set_wait_limit_ns(int(ns))
+
+
+def wait_limit_ns() -> int:
+    return int(lib().loopvq_wait_limit_ns())
 
 
 def _ptr(t):

@@ -24,7 +24,7 @@ def test_every_declared_symbol_is_exported():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(LQ.EXPORTS)
-    assert lib.loopvq_abi_version() == 2
+    assert lib.loopvq_abi_version() == 3
 
 
 def _cache(**kw):
@@ -178,6 +178,23 @@ def test_window_validation_before_launch():
     w.Hq, w.fill = c.Hq, None
     assert lib.loopvq_window_advance(C.byref(w), c.ref(), None) == 1
     assert lib.loopvq_window_workspace_bytes(C.byref(w), c.ref(), 1024) == 0
+    # the page roll stages the recent slots of one (layer, loop step, sequence, head) in shared memory:
+    # 1024 x 128 bf16 = 256 KiB is more than a CTA can have, so the advance is refused before any launch
+    w.fill, w.n_recent = 0x70000, 1024
+    assert lib.loopvq_window_advance(C.byref(w), c.ref(), None) == 2
+    assert b"shared memory" in lib.loopvq_last_error()
+    w.n_recent = 904                                         # 904 x 128 x 2 = 231424 bytes: fits
+    assert lib.loopvq_window_slots(C.byref(w)) == 8 + 904 + 8
+
+
+def test_wait_limit_is_process_wide_and_settable():
+    lib = LQ.lib()
+    old = LQ.wait_limit_ns()
+    assert old == 2_000_000_000
+    LQ.set_wait_limit_ns(0)
+    assert LQ.wait_limit_ns() == 0
+    LQ.set_wait_limit_ns(old)
+    assert lib.loopvq_wait_limit_ns() == old
 
 
 def test_per_group_codebook_sizes_and_validation():
