@@ -27,13 +27,16 @@
 //  * The lane's 4 partial scores are reduce-scattered over the 8 lanes of its t (3 exchanges); each
 //    lane finishes one token.  The softmax maximum is one value per warp, lazy (it moves, with an exact
 //    rescale, only when a score exceeds it by more than 8 in log2 units).
-//  * Values on the tensor cores, one mma.sync m16n8k16 (bf16 in, fp32 accumulate) per (token, group
-//    quad): the k dimension is (token slot t, channel e) of one token per lane group, so a lane's B
-//    fragment is exactly its gathered 8-byte value entry (channels 0-1 and 2-3 of group 8u + g, no
-//    conversion or re-pairing).  A row g holds, at channel g % 4, the token's weight split into a bf16
-//    hi part (rows 0-3) or lo part (rows 4-7), which represents the fp32 weight to about 2^-16
-//    relative; the two rows are added at the end.  The 16 MMAs of a tile are issued token-major, so
-//    consecutive ones write different accumulators.
+//  * Values on the tensor cores with mma.sync m16n8k16 (bf16 in, fp32 accumulate), 8 per 16-token tile:
+//    one per (token octet, group octet u).  The k dimension is (token slot, channel parity) over slots t
+//    and t + 4 of the octet, the A rows g and g + 8 are channels 0-1 and 2-3 of group 8u + g, so a lane's
+//    A quad is exactly its two gathered 8-byte value entries (tokens t and t + 4, as loaded: no moves or
+//    permutes).  B column g < 4 holds, at channel parity g & 1, the token's weight split into a bf16 hi
+//    part (g < 2) or lo part, which represents the fp32 weight to about 2^-16 relative; columns 4-7 are
+//    zero.  Lanes t = 0 and 1 accumulate the hi and lo parts of the same channels, added at the end.
+//    (The first version put the weights in A with one token per MMA: 16 MMAs per tile with half the A
+//    rows zero, whose A quads had to be assembled from separate registers; 7% slower at ctx32k.  TaSQ
+//    keys keep that form, which measured faster there.)
 //  * Index words arrive through a per-warp ring of 1 KiB stages in shared memory filled with 16-byte
 //    cp.async copies (lane L copies chunks L and L + 32 of the tile); each lane reads its 8 words with
 //    conflict-free 4-byte loads.
@@ -160,10 +163,18 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             // this warp's run of 16-token tiles [i0, i1) of the piece
             const int i0 = (int)((long long)warp * n16 / WARPS), i1 = (int)((long long)(warp + 1) * n16 / WARPS);
             const int kown = 2 * (g & 1) + ((g >> 1) & 1);  // the token (0..3) this lane finishes
-            // A row g: part g >> 2 (0: bytes 0-1 of x, 1: bytes 2-3) at channel e = g & 3
-            const uint32_t part_lo = (g & 4) ? 0x4432u : 0x4410u, part_hi = (g & 4) ? 0x3244u : 0x1044u;
-            const uint32_t sel0 = (g & 2) ? 0x4444u : ((g & 1) ? part_hi : part_lo);
-            const uint32_t sel2 = (g & 2) ? ((g & 1) ? part_hi : part_lo) : 0x4444u;
+            // Value products (below), selectors of the packed weight x = {hi part: bytes 0-1, lo part: 2-3}.
+            // Plain keys: B column g < 4 takes part g >> 1 in half g & 1, columns 4..7 are zero.  TaSQ keys:
+            // A row g takes part g >> 2 at channel g & 3, in a0 for channels 0-1 and a2 for 2-3.
+            uint32_t sel0, sel2;
+            if constexpr (TQ) {
+                const uint32_t part_lo = (g & 4) ? 0x4432u : 0x4410u, part_hi = (g & 4) ? 0x3244u : 0x1044u;
+                sel0 = (g & 2) ? 0x4444u : ((g & 1) ? part_hi : part_lo);
+                sel2 = (g & 2) ? ((g & 1) ? part_hi : part_lo) : 0x4444u;
+            } else {
+                sel0 = g >= 4 ? 0x4444u : ((g & 2) ? ((g & 1) ? 0x3244u : 0x4432u) : ((g & 1) ? 0x1044u : 0x4410u));
+                sel2 = 0u;
+            }
             // index copies: lane L takes chunks L (four-tile L / 16) and L + 32 (four-tile L / 16 + 2)
             const int kc = lane >> 4;
             const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP;
@@ -386,61 +397,101 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                         l *= corr;
                         const float2 c2 = f2(corr, corr);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {              // rows 8..15 (z, w) stay zero
+                        for (int j = 0; j < 4; ++j) {
                             const float2 lo2 = __fmul2_rn(f2(acc[j].x, acc[j].y), c2);
                             acc[j].x = lo2.x;
                             acc[j].y = lo2.y;
+                            if constexpr (!TQ) {                // with TaSQ keys rows 8..15 (z, w) stay zero
+                                const float2 hi2 = __fmul2_rn(f2(acc[j].z, acc[j].w), c2);
+                                acc[j].z = hi2.x;
+                                acc[j].w = hi2.y;
+                            }
                         }
                         m = tmax;
                     }
                     const float p = ex2(sk - m);
                     l += p;
 
-                    // ---- weights: token k's {bf16 hi, bf16 lo} from lane 4 g'(k) + t; A row g = (part g >> 2,
-                    // channel g & 3): a0 holds the part at channel 0 or 1, a2 at channel 2 or 3, else zero
-                    uint32_t ak0[4], ak2[4];
+                    // ---- weights: token k's {bf16 hi, bf16 lo} (about 2^-16 of the fp32 weight together) from
+                    // the lane 4 g'(k) + t that finished it
+                    uint32_t xk[4];
                     {
                         const float hv = __uint_as_float(__float_as_uint(p) & 0xffff0000u);
                         const uint32_t x = cvt_bf16x2(p - hv, hv);        // upper: lo part, lower: hi part
-                        const uint32_t xk[4] = {__shfl_sync(0xffffffffu, x, t), __shfl_sync(0xffffffffu, x, 8 + t),
-                                                __shfl_sync(0xffffffffu, x, 4 + t), __shfl_sync(0xffffffffu, x, 12 + t)};
+                        xk[0] = __shfl_sync(0xffffffffu, x, t);
+                        xk[1] = __shfl_sync(0xffffffffu, x, 8 + t);
+                        xk[2] = __shfl_sync(0xffffffffu, x, 4 + t);
+                        xk[3] = __shfl_sync(0xffffffffu, x, 12 + t);
+                    }
+                    if constexpr (!TQ) {
+                        // ---- values: A rows g, g + 8 = channels 0-1, 2-3 of group 8u + g; k = (token slot, channel
+                        // parity) over slots t (k 2t, 2t + 1) and t + 4 (k 2t + 8, 2t + 9) of a token octet, so the
+                        // lane's A quad is its two gathered 8-byte entries as loaded; B column g < 4 = (part g >> 1,
+                        // parity g & 1) holds the slot's weight part at that parity
+                        uint32_t bw[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) bw[k] = __byte_perm(xk[k], 0u, sel0);
+#pragma unroll
+                        for (int o = 0; o < 2; ++o) {
+                            uint2 v[2][4];
+#pragma unroll
+                            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    v[j][u] = lds64(smem, __byte_perm((u & 1) ? wb[2 * o + j] : wa[2 * o + j], colv,
+                                                                      (u < 2) ? 0x7624u : 0x7634u));
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                mma_bf16_16816(acc[u], v[0][u].x, v[0][u].y, v[1][u].x, v[1][u].y, bw[2 * o],
+                                               bw[2 * o + 1]);
+                        }
+                    } else {
+                        // ---- values with TaSQ keys: k = (token slot t, channel e) of one token per MMA, B = the
+                        // lane's gathered entry, A row g = (part g >> 2, channel g & 3)
+                        uint2 v[4][4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                v[k][u] = lds64(smem, __byte_perm((u & 1) ? wb[k] : wa[k], colv, (u < 2) ? 0x7624u : 0x7634u));
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            ak0[k] = __byte_perm(xk[k], 0u, sel0);
-                            ak2[k] = __byte_perm(xk[k], 0u, sel2);
+                            const uint32_t a0 = __byte_perm(xk[k], 0u, sel0), a2 = __byte_perm(xk[k], 0u, sel2);
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) mma_bf16_16816(acc[u], a0, 0u, a2, 0u, v[k][u].x, v[k][u].y);
                         }
                     }
-
-                    // ---- values: k-slot 2t + e (e < 2: word .x, channel e) and 2t + 8 + e (word .y, channel
-                    // 2 + e) of the lane's token; column g = group 8u + g
-                    uint2 v[4][4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            v[k][u] = lds64(smem, __byte_perm((u & 1) ? wb[k] : wa[k], colv, (u < 2) ? 0x7624u : 0x7634u));
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) mma_bf16_16816(acc[u], ak0[k], 0u, ak2[k], 0u, v[k][u].x, v[k][u].y);
                 }
             }
             cp_async_wait<0>();
 
-            // ---- the warp's record: lane (g < 4, t) holds channel g of groups 8u + 2t, 8u + 2t + 1 (hi
-            // parts; the lo parts come from lane + 16)
+            // ---- the warp's record
             {
                 float lsum = l;
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
                 lsum *= 0.5f;                              // every token is finished by two lanes
+                if constexpr (!TQ) {
+                    // lane (g, 0) holds the hi parts of channels 0-3 of group 8u + g, lane (g, 1) the lo parts
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {              // rows g + 4 (lo parts) to lanes g < 4
-                    const float vx = acc[u].x + __shfl_xor_sync(0xffffffffu, acc[u].x, 16);
-                    const float vy = acc[u].y + __shfl_xor_sync(0xffffffffu, acc[u].y, 16);
-                    if (g < 4) {
-                        rec[4 * (8 * u + 2 * t) + g] = vx;
-                        rec[4 * (8 * u + 2 * t + 1) + g] = vy;
+                    for (int u = 0; u < 4; ++u) {
+                        float4 c = acc[u];
+                        c.x += __shfl_xor_sync(0xffffffffu, c.x, 1);
+                        c.y += __shfl_xor_sync(0xffffffffu, c.y, 1);
+                        c.z += __shfl_xor_sync(0xffffffffu, c.z, 1);
+                        c.w += __shfl_xor_sync(0xffffffffu, c.w, 1);
+                        if (t == 0) *reinterpret_cast<float4 *>(rec + 4 * (8 * u + g)) = c;
+                    }
+                } else {
+                    // lane (g < 4, t) holds channel g of groups 8u + 2t, 8u + 2t + 1 (hi parts; lo parts in lane + 16)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float vx = acc[u].x + __shfl_xor_sync(0xffffffffu, acc[u].x, 16);
+                        const float vy = acc[u].y + __shfl_xor_sync(0xffffffffu, acc[u].y, 16);
+                        if (g < 4) {
+                            rec[4 * (8 * u + 2 * t) + g] = vx;
+                            rec[4 * (8 * u + 2 * t + 1) + g] = vy;
+                        }
                     }
                 }
                 if (lane == 0) {
