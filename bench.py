@@ -36,10 +36,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from synth import (WORKLOADS, lengths, random_indices, queries, bf16_bits_to_f32, codebook, codebooks,  # noqa: E402
-                   tasq_weights, tasq_perm)
+                   tasq_weights, tasq_perm, kv_loops)
 
 METRIC = "LoopVQ decode-attn µs/step & GB/s at 32K ctx, 0.5 bit; % of roofline"
 SMEM_BYTES_PER_CLK_SM = 128
+FP32_FLOPS_PER_CLK_SM = 256          # 128 fp32 lanes x one fused multiply-add
 N_SM = 148
 
 
@@ -258,8 +259,9 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
     }
 
 
-def workload_desc(w):
+def workload_desc(w, world=1):
     return {
+        "parallelism": "replicas" if world > 1 else "single GPU",
         "workload": f"{w.name}: looped decoder, {w.L} layers x {w.T} loop steps (blocks of {w.Tc}), "
                     f"{w.Hkv} KV / {w.Hq} q heads, D={w.D}, c={w.c} (G={w.G}, K={w.K}, {8 / w.G:g} bit), "
                     f"batch {w.B}, cache {w.Nmax} tokens",
@@ -289,6 +291,27 @@ def call_bytes(w, lens):
 def gather_bytes(w, lens):
     """Shared-memory gather bytes of one call: D bf16 key and D bf16 value per token and KV head."""
     return int(np.sum(lens)) * w.Hkv * 2 * w.D * 2
+
+
+def call_flops(w, lens):
+    """Algorithmic fp32 work of one call: per token and KV head, the RoPE rotation of the rebuilt key
+    (3D) once, then per query head its score (2D) and its value sum (2D): 7D with one query head,
+    3D + 4D per query head with several."""
+    return int(np.sum(lens)) * w.Hkv * (3 * w.D + 4 * w.D * (w.Hq // w.Hkv))
+
+
+def floors(w, lens, sm_mhz, hbm_gbs):
+    """The three per-call floors (µs) and the peaks behind them: HBM (algorithmic bytes at the measured
+    copy bandwidth), shared-memory gathers (128 B/clk/SM x 148 SMs x the sampled SM clock) and fp32
+    (128 lanes x 2 flops/clk/SM x 148 SMs x the clock).  The largest binds."""
+    smem_gbs = SMEM_BYTES_PER_CLK_SM * N_SM * sm_mhz * 1e6 / 1e9
+    fp32_tflops = FP32_FLOPS_PER_CLK_SM * N_SM * sm_mhz * 1e6 / 1e12
+    cb, gb, fl = call_bytes(w, lens), gather_bytes(w, lens), call_flops(w, lens)
+    return {
+        "hbm": {"us": cb / (hbm_gbs * 1e9) * 1e6, "per_call": cb, "peak": hbm_gbs, "unit": "GB/s"},
+        "smem": {"us": gb / (smem_gbs * 1e9) * 1e6, "per_call": gb, "peak": smem_gbs, "unit": "GB/s"},
+        "fp32": {"us": fl / (fp32_tflops * 1e12) * 1e6, "per_call": fl, "peak": fp32_tflops, "unit": "TFLOP/s"},
+    }
 
 
 class Clocks:
@@ -393,27 +416,153 @@ def cpu_sample(w, seconds, layer=0, t=1):
     return total_s, nbytes, units
 
 
+def cpu_model():
+    """CPU model name of the host (first /proc/cpuinfo entry)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_threads():
+    """Cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_sample_all_cores(w, seconds_1core_per_unit, threads, budget_s, layer=0, t=1):
+    """The checker's decode on `threads` host cores at once: (sequence, query head) units of one call, one
+    per thread at a time.  The checker's ctypes calls release the GIL, so the threads run on separate
+    cores.  The number of units is bounded so the run takes about budget_s; inputs are regenerated before
+    the clock starts."""
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import oracle as O
+    lens = lengths(w)
+    m = t % w.Tc
+    order = [(b, hq) for b in range(w.B) for hq in range(w.Hq)]
+    nunits = max(threads, int(threads * budget_s / max(seconds_1core_per_unit, 1e-3)))
+    nunits = min(nunits, len(order))
+    units = [_cpu_inputs(w, layer, t, b, hq) + (b, hq) for b, hq in order[:nunits]]
+
+    def one(u):
+        q, ik, iv, Ek, Ev, b, hq = u
+        if w.tasq:
+            h = hq // (w.Hq // w.Hkv)
+            n = len(ik)
+            O.tasq_decode(q, ik, iv, Ek, Ev, _tasq_params(w)[1][layer, t // w.Tc, h], _tasq_params(w)[0][layer, t, h],
+                          np.ones(n), w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        else:
+            (O.decode_pg if w.ncb > 1 else O.decode)(q, ik, iv, Ek, Ev, w.c, w.Tc, m, w.theta, 1 / math.sqrt(w.D))
+        return len(ik) * 2 * (w.D // w.c)
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        t0 = time.perf_counter()
+        nbytes = sum(ex.map(one, units))
+        wall = time.perf_counter() - t0
+    return wall, nbytes, nunits
+
+
+def _unpack_codes(words, Nmax, NP):
+    """Index words of one (layer, block, sequence, KV head) -> [Nmax][2NP] K and V codes (the word
+    layout of include/loopvq.h: tiles of 4 tokens, [Nmax/4][NP][4]; bytes K p, K p+NP, V p, V p+NP)."""
+    wd = words.reshape(Nmax // 4, NP, 4).transpose(0, 2, 1).reshape(Nmax, NP).astype(np.uint32)
+    k = np.concatenate([wd & 0xFF, (wd >> 8) & 0xFF], axis=1).astype(np.uint8)
+    v = np.concatenate([(wd >> 16) & 0xFF, (wd >> 24) & 0xFF], axis=1).astype(np.uint8)
+    return k, v
+
+
+def cpu_encode_and_ties(w, cache, threads, budget_s, layer=0, blk=0):
+    """The checker's encode of sampled tokens of one (layer, block) on `threads` cores, timed and
+    extrapolated to the whole (layer, block) unit (labelled as such), and the GPU's codes for the same
+    tokens compared with it: a code that differs counts as a near-tie when the two fp64 distances differ
+    by at most 1e-5 relative, anything else as a mismatch.  Runs after the timed region."""
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import oracle as O
+    if w.tasq:
+        return None, {"checked": 0, "note": "TaSQ codes are checked by the GPU tests, not here"}
+    NP = w.D // (2 * w.c)
+    # sample: one (sequence, KV head) per thread, a run of tokens each, keys and values
+    chunk = min(4096, w.Nmax)
+    pairs = [((i * 7) % w.B, (i * 5) % w.Hkv) for i in range(threads)]
+    jobs = []
+    for j, (b, h) in enumerate(pairs):
+        tok0 = (j * 997) % max(1, w.Nmax - chunk)
+        toks = range(tok0, tok0 + chunk)
+        for kv in range(2):
+            x = kv_loops(w, layer, kv, blk * w.Tc, blk * w.Tc + w.Tc - 1, [b], toks, [h])[:, 0, :, 0, :]
+            E = bf16_bits_to_f32(_codebook(w, layer, blk, kv, h))
+            jobs.append((b, h, kv, tok0, np.ascontiguousarray(bf16_bits_to_f32(x)), np.ascontiguousarray(E)))
+    enc = O.encode_pg if w.ncb > 1 else O.encode
+
+    def one(job):
+        return enc(job[4], job[5], w.c)
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        t0 = time.perf_counter()
+        refs = list(ex.map(one, jobs))
+        wall = time.perf_counter() - t0
+    vec_sample = len(jobs) * chunk * (w.D // w.c)
+    vec_unit = 2 * w.B * w.Nmax * w.Hkv * (w.D // w.c)
+    enc_line = {"ms_per_layer_block": wall * vec_unit / vec_sample * 1e3, "cores": threads, "extrapolated": True,
+                "sample": f"{len(jobs)} runs of {chunk} tokens (one sequence and KV head each, K and V) of "
+                          f"layer {layer}, block {blk}: {vec_sample} coupled vectors timed in {wall:.2f} s on "
+                          f"{threads} threads, scaled to the {vec_unit} vectors of the (layer, block)"}
+    # the GPU codes of the same tokens
+    checked = ties = other = 0
+    per_bh = w.Nmax * NP
+    for (b, h, kv, tok0, x, E), ref in zip(jobs, refs):
+        base = ((layer * w.NB + blk) * w.B + b) * w.Hkv + h
+        words = cache.idx[base * per_bh:(base + 1) * per_bh].cpu().numpy().view(np.uint32)
+        ck, cv = _unpack_codes(words, w.Nmax, NP)
+        gpu = (ck if kv == 0 else cv)[tok0:tok0 + chunk]
+        checked += gpu.size
+        for i, g in zip(*np.nonzero(gpu != ref)):
+            if w.ncb > 1:
+                dg = O.dist64_pg(x, E, w.c, int(i), int(g), int(gpu[i, g]))
+                do = O.dist64_pg(x, E, w.c, int(i), int(g), int(ref[i, g]))
+            else:
+                dg = O.dist64(x, E, w.c, int(i), int(g), int(gpu[i, g]))
+                do = O.dist64(x, E, w.c, int(i), int(g), int(ref[i, g]))
+            if abs(dg - do) <= 1e-5 * max(dg, do):
+                ties += 1
+            else:
+                other += 1
+    return enc_line, {"checked": checked, "near_ties": ties, "mismatches": other,
+                      "rule": "a differing code is a near-tie when its fp64 distance is within 1e-5 relative "
+                              "of the checker's; any other difference is a mismatch"}
+
+
 def run_reference(args):
     """The CPU checker as the reference arm: each step decodes a bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
+    nthr = host_threads()
     per_step = max(0.1, min(2.0, 60.0 / max(1, args.steps + args.warmup)))
+    s1, _, u1 = cpu_sample(w, min(per_step, 2.0))            # one unit's single-thread time sizes the steps
+    per_unit = s1 / max(u1, 1)
     for _ in range(args.warmup):
-        cpu_sample(w, per_step)
+        cpu_sample_all_cores(w, per_unit, nthr, per_step)
     tot_s, tot_b, tot_u = 0.0, 0, 0
     for _ in range(args.steps):
-        s, b, u = cpu_sample(w, per_step)
+        s, b, u = cpu_sample_all_cores(w, per_unit, nthr, per_step)
         tot_s, tot_b, tot_u = tot_s + s, tot_b + b, tot_u + u
     gbs = tot_b / tot_s / 1e9
-    sample = (f"{tot_u} (sequence, query head) units of the layer-0, loop-step-2 call over {args.steps} steps; "
-              f"fp64 dequant, RoPE and softmax per unit; single thread")
+    sample = (f"{tot_u} (sequence, query head) units of the layer-0, loop-step-2 call over {args.steps} steps, "
+              f"one unit per thread at a time on {nthr} threads; fp64 dequant, RoPE and softmax per unit")
     line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_desc(w),
-            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "data": "synthetic", "config": workload_desc(w, int(os.environ.get("WORLD_SIZE", "1"))),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": nthr, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -563,23 +712,30 @@ def main():
         step_bytes = cb * ncall
         value = job_throughput(world, step_bytes, ms_step)
         hbm_peak, peak_kind = peaks()
-        achieved = cb / (avg_call_ms * 1e-3) / 1e9
         sm_mhz = clk.get("sm_mhz") or 1965.0
-        smem_peak = SMEM_BYTES_PER_CLK_SM * N_SM * sm_mhz * 1e6 / 1e9
-        smem_achieved = gb / (avg_call_ms * 1e-3) / 1e9
+        fl = floors(w, lens_np, sm_mhz, hbm_peak)
+        bound = max(fl, key=lambda k: fl[k]["us"])
+        call_us = avg_call_ms * 1e3
+        scale_unit = {"GB/s": 1e9, "TFLOP/s": 1e12}
+        achieved = fl[bound]["per_call"] / (call_us * 1e-6) / scale_unit[fl[bound]["unit"]]
+        floor_line = {k: {"floor_us": v["us"], "frac": v["us"] / call_us, "peak": v["peak"], "unit": v["unit"],
+                          "per_call": v["per_call"]} for k, v in fl.items()}
+        floor_line["hbm"]["peak_kind"] = f"{peak_kind} copy bandwidth"
+        floor_line["smem"]["peak_kind"] = f"derived: {SMEM_BYTES_PER_CLK_SM} B/clk/SM x {N_SM} SMs x median SM clock"
+        floor_line["fp32"]["peak_kind"] = (f"derived: {FP32_FLOPS_PER_CLK_SM} flop/clk/SM x {N_SM} SMs x median SM "
+                                           "clock; algorithmic flops 3D + 4D per query head per token and KV head")
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": dict(workload_desc(w), parallelism=("replicas" if world > 1 else "single GPU")),
+            "config": workload_desc(w, world),
             "us_per_step": ms_step * 1e3, "us_per_call": avg_call_ms * 1e3, "calls_per_step": ncall,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": profiled_traffic(w), "peak_kind": peak_kind,
+            "roofline": {"bound": bound, "achieved": achieved, "peak": fl[bound]["peak"], "unit": fl[bound]["unit"],
+                         "frac": achieved / fl[bound]["peak"], "traffic": profiled_traffic(w),
+                         "peak_kind": floor_line[bound]["peak_kind"],
                          "kernel": f"one loopvq_decode_attn call ({decode_kernel_name(w)}_kernel + merge_kernel)",
-                         "bytes_per_launch": cb},
-            "smem_gather": {"achieved": smem_achieved, "peak": smem_peak, "unit": "GB/s",
-                            "frac": smem_achieved / smem_peak, "bytes_per_launch": gb,
-                            "peak_kind": f"derived: {SMEM_BYTES_PER_CLK_SM} B/clk/SM x {N_SM} SMs x median SM clock"},
+                         "per_launch": fl[bound]["per_call"], "bytes_per_launch": cb,
+                         "floors": floor_line},
             "clocks": clk,
             "e2e": {"value": job_throughput(world, step_bytes, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -599,10 +755,19 @@ def main():
             if compare["windowed"] is not None:
                 line["windowed"] = compare["windowed"]
         if world == 1 and not args.no_cpu_baseline:
-            s, nb, u = cpu_sample(w, args.cpu_seconds)
-            line["cpu_baseline"] = {"value": nb / s / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"{u} (sequence, query head) units of the layer-0, loop-step-2 call, "
-                                              f"{s:.1f} s single-threaded"}
+            s1, nb1, u1 = cpu_sample(w, args.cpu_seconds)
+            nthr = host_threads()
+            sa, nba, ua = cpu_sample_all_cores(w, s1 / max(u1, 1), nthr, args.cpu_seconds)
+            enc_cpu, ties = cpu_encode_and_ties(w, cache, nthr, args.cpu_seconds)
+            line["cpu_baseline"] = {
+                "value": nb1 / s1 / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "cpu_model": cpu_model(),
+                "sample": f"{u1} (sequence, query head) units of the layer-0, loop-step-2 call, {s1:.1f} s "
+                          f"single-threaded",
+                "all_cores": {"value": nba / sa / 1e9, "unit": "GB/s", "cores": nthr,
+                              "sample": f"{ua} units of the same call on {nthr} threads (one unit per thread at a "
+                                        f"time), {sa:.1f} s wall"},
+                "encode": enc_cpu}
+            line["near_ties"] = ties
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
