@@ -139,7 +139,9 @@ size_t loopvq_decode_workspace_bytes(const loopvq_cache *cache, int max_len);
  * out       fp32 [B][Hq][D]; len_b == 0 gives zeros.
  * lse       fp32 [B][Hq] natural-log log-sum-exp, -inf for len_b == 0; may be NULL.
  * workspace device scratch of at least loopvq_decode_workspace_bytes(cache, max_len)
- *           bytes, 16-byte aligned; its contents on entry do not matter.
+ *           bytes, 16-byte aligned; its contents on entry do not matter.  Calls
+ *           that share a workspace must be ordered on the GPU (one stream, or
+ *           events).
  */
 loopvq_status loopvq_decode_attn(const loopvq_cache *cache, int layer, int t,
                                  const uint16_t *q, const int32_t *lens, int max_len,

@@ -19,8 +19,8 @@ namespace loopvq {
 // the shared memory left over serves as L1 for the RoPE rows); with one codebook per channel group,
 // one CTA of 16 warps per SM (128 KiB of tables).  Measured at ctx32k: a second wave, or three CTAs
 // per SM at 80 registers, is 3 to 10 % slower.  decode_mha_kernel runs two CTAs of 8 warps per SM
-// (2-deep index ring per warp): with fp32 key tables this is as fast as one CTA of 16 warps at ctx32k
-// and 4% faster on the short deep32 calls; a 3-deep ring is 2% slower.
+// (2-deep index ring per warp): one CTA of 16 warps is 3% slower at ctx32k and 8% at ctx4k, a 3-deep
+// ring 1% slower.
 
 static constexpr int kSms = 148;                           // B200; more CTAs than fit only add a wave
 static constexpr int kWords = 1;                           // index words per lane per iteration (4-token tiles)
@@ -33,9 +33,13 @@ static constexpr KernelShape kernel_shape(bool pg, int qpk) {
     return pg ? KernelShape{16, 1, 4} : KernelShape{8, 2, 2};
 }
 
-static size_t ring_smem_bytes(bool pg, int qpk) {
+// Tables, the per-thread index queue and, with at most 2 query heads per KV head, the slot records
+// (decode_split_kernel keeps its tables across the pieces of one KV head then).
+static size_t ring_smem_bytes(bool pg, int qpk, int D) {
     const KernelShape k = kernel_shape(pg, qpk);
-    return (pg ? 131072 : 65536) + (size_t)k.depth * k.warps * 32 * 16 * kWords;
+    const size_t nslot = (size_t)k.warps * (32 / (D / 8));
+    const size_t recs = qpk <= 2 ? nslot * qpk * (D + 4) * sizeof(float) : 0;
+    return (pg ? 131072 : 65536) + (size_t)k.depth * k.warps * 32 * 16 * kWords + recs;
 }
 
 // decode_mha_kernel (one query head per KV head, D = 128, groups of 4 channels, one shared codebook)
@@ -123,8 +127,8 @@ static cudaError_t launch_t(const DecodeArgs &a, const DecodePlan &plan, cudaStr
     constexpr KernelShape K = kernel_shape(PG, QPK);
     constexpr int NSLOT = K.warps * (32 / (D / 8));
     const size_t red = (size_t)NSLOT * QPK * (D + 4) * sizeof(float);
-    const size_t smem = ring_smem_bytes(PG, QPK);
-    if (red > smem) return cudaErrorInvalidConfiguration;   // the slot records reuse slices and queue
+    const size_t smem = ring_smem_bytes(PG, QPK, D);
+    if (red > smem) return cudaErrorInvalidConfiguration;   // the slot records fit (own area or the tables)
     // TaSQ with one query head per KV head carries the rotated query from tile to tile (XR): its
     // table values sit at permuted columns, 8 scalar loads per tile.  The plain kernels load the
     // table row one iteration ahead, which measured faster for them (143 vs 150 us at ctx32k).

@@ -269,6 +269,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     constexpr int STRIDE = NSLOT * TT;                     // tokens between two iterations of a slot
     constexpr int QB = NT * 16 * NW;                       // bytes of one prefetch-queue stage
     constexpr uint32_t TBL = PG ? 131072u : 65536u;        // bytes of the staged K/V tables
+    // With at most 2 query heads per KV head the slot records get their own shared memory after the
+    // index queue, so a CTA keeps its tables across pieces of one KV head (its next piece is usually the
+    // next sequence of the same head); otherwise they reuse the tables, which are staged every piece.
+    constexpr bool KEEP = QPK <= 2;
+    constexpr uint32_t REC_OFF = TBL + (uint32_t)DEPTH * QB;
     static_assert(C == 4 || C == 8 || C == 16 || C == 32, "c");
     static_assert(NL >= 8 && NL <= 16, "slot width");
 
@@ -311,6 +316,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
     }
     const int ch = gp * C + half * 4;                      // first of this lane's 4 low channels
 
+    int staged_h = -1;                                     // the KV head whose slices the tables hold
     // the pieces of this CTA, segment by segment
     while (pos < x_end && h < a.Hkv) {
         int len, st, base;
@@ -361,7 +367,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
                 cp_async_commit();
             }
 
-            if constexpr (!PG) {
+            const bool restage = !KEEP || h != staged_h;   // CTA-uniform
+            staged_h = h;
+            if (!restage) {
+            } else if constexpr (!PG) {
             // stage the K and V slices as bank-private replicas (rows >= K zeroed)
             {
                 const uint16_t *sk = a.slk + (size_t)h * a.K * C;
@@ -714,11 +723,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_split_kernel(const De
             cp_async_wait<0>();
 
             // ---- combine the slots of this CTA, write the split's partial result
-            __syncthreads();                                       // slices and queue no longer needed
+            __syncthreads();                                       // the queue (and without KEEP the slices) no longer needed
             constexpr int RS = D + 4;                              // floats per (slot, query head) record
             // l_ sums the weights of the tokens this lane finished: add the other token positions of the slot
             constexpr int TOKBITS = (TT == 8) ? 3 : 2;
-            float *red = reinterpret_cast<float *>(smem);
+            float *red = reinterpret_cast<float *>(smem + (KEEP ? REC_OFF : 0u));
 #pragma unroll
             for (int j = 0; j < QPK; ++j) {
                 float lsum = l_[j];

@@ -8,11 +8,14 @@
 //
 // Design (B200, sm_100a):
 //  * The tile space, pieces and partial records are those of decode_split_kernel (decode_kernel.cuh),
-//    and its merge kernel combines the records.  The slices are staged as bank-private replicas, the K
-//    slice converted to fp32: row r holds K entry r as 16 bytes of fp32 in 8 replicas (a lane reads
-//    replica lane % 8 with one 16-byte load, so the 8 lanes of a quarter-warp wavefront hit distinct
-//    banks) and V entry r as 8 bytes of bf16 in 16 replicas (replica lane % 16).  The key side thus needs
-//    no bf16 unpacking; fp32 keys measured 6% faster than bf16 keys with their unpacks.
+//    and its merge kernel combines the records.  The slices are staged as bank-private replicas: row r
+//    holds K entry r as 8 bytes of bf16 in 16 replicas and V entry r likewise (a lane reads replica
+//    lane % 16, so the 16 lanes of a half-warp wavefront hit distinct banks).  Each gathered key entry is
+//    widened to fp32 by one m16n8k8 tensor-core product with the identity (lane-local, exact), so the
+//    key side needs no ALU unpacking and gathers 256 bytes per token and KV head instead of the 512 of
+//    fp32 tables (4% faster at ctx32k than fp32 tables, once the value side below was in place; 6%
+//    slower before it).  With TaSQ keys the K slice is staged in fp32 (16 bytes in 8 replicas), which
+//    measured faster there.
 //  * A warp takes a contiguous run of 16-token tiles of the piece.  Lane (g, t) = (lane / 4, lane % 4)
 //    owns the tokens t, t + 4, t + 8, t + 12 of each tile and the two pair-groups g and g + 8: the
 //    channel groups g, g + 8 (low channels) and g + 16, g + 24 (their RoPE partners), 8 RoPE pairs.
@@ -23,7 +26,7 @@
 //    that is one fused multiply-add per component and step.  For the 4 low-frequency pairs the same
 //    recurrence is run in the difference form D_{j+1} = D_j - 4 sin^2(2w) X_j, X_{j+1} = X_j + D_{j+1}
 //    (Reinsch), whose coefficient keeps full relative precision as w -> 0.  Both are set from the
-//    table every 32 tiles, which bounds the rounding drift to 128 steps.
+//    table every 64 tiles, which bounds the rounding drift to 256 steps (every 32 measured 1% slower).
 //  * The lane's 4 partial scores are reduce-scattered over the 8 lanes of its t (3 exchanges); each
 //    lane finishes one token.  The softmax maximum is one value per warp, lazy (it moves, with an exact
 //    rescale, only when a score exceeds it by more than 8 in log2 units).
@@ -49,6 +52,17 @@
 #include "decode_kernel.cuh"
 
 namespace loopvq {
+
+// Four bf16 channels (two packed words) widened to fp32 on the tensor core: an m16n8k8 product with the
+// identity as B returns each lane's own A elements, so lane (g, t) gets (a0.lo, a0.hi, a1.lo, a1.hi).
+// `eye` is the lane's identity fragment, B[2t][g] and B[2t + 1][g].
+__device__ __forceinline__ float4 widen_bf16x4(uint2 e, uint32_t eye) {
+    float4 c;
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, {%7, %7, %7, %7};"
+        : "=f"(c.x), "=f"(c.y), "=f"(c.z), "=f"(c.w)
+        : "r"(e.x), "r"(e.y), "r"(eye), "f"(0.f));
+    return c;
+}
 
 __device__ __forceinline__ uint32_t cvt_bf16x2(float hi_elem, float lo_elem) {
     uint32_t r;
@@ -89,7 +103,7 @@ template <int WARPS, int MINB, int DEPTH, bool TQ = false>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const DecodeArgs a) {
     constexpr int D = 128, NP = 16;                        // pair-groups = index words per token
     constexpr int NT = WARPS * 32;
-    constexpr int ANCHOR = 32;                             // tiles between two settings from the table
+    constexpr int ANCHOR = 64;                             // tiles between two settings from the table
     using S = MhaSmem<WARPS, DEPTH>;
 
     extern __shared__ __align__(128) unsigned char smem[];
@@ -104,7 +118,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
     int h = (int)(range_info[3] >> 32), b = (int)(range_info[3] & 0xffffffffLL);
 
     const int g = lane >> 2, t = lane & 3;
-    const uint32_t colk = (uint32_t)((lane & 7) * 16);      // the lane's fp32 K replica
+    // the lane's K replica: bf16 (8 bytes, replica lane % 16) with plain keys, fp32 (16 bytes, replica
+    // lane % 8) with TaSQ keys
+    const uint32_t colk = TQ ? (uint32_t)((lane & 7) * 16) : (uint32_t)((lane & 15) * 8);
+    const uint32_t eye = ((2 * (lane & 3) == (lane >> 2)) ? 0x3F80u : 0u) |
+                         ((2 * (lane & 3) + 1 == (lane >> 2)) ? 0x3F800000u : 0u);
     const uint32_t colv = (uint32_t)((lane & 15) * 8) + 128u;   // and its V replica
     const uint32_t smem_base = (uint32_t)__cvta_generic_to_shared(smem);
     const uint32_t ring = smem_base + S::kRing + (uint32_t)warp * DEPTH * 1024u;
@@ -150,10 +168,15 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                         ek = __ldg(reinterpret_cast<const uint2 *>(sk + (size_t)r * 4));
                         ev = __ldg(reinterpret_cast<const uint2 *>(sv + (size_t)r * 4));
                     }
-                    const float4 kf = make_float4(bf16lo(ek.x), bf16hi(ek.x), bf16lo(ek.y), bf16hi(ek.y));
                     unsigned char *row = smem + r * 256;
+                    if constexpr (TQ) {
+                        const float4 kf = make_float4(bf16lo(ek.x), bf16hi(ek.x), bf16lo(ek.y), bf16hi(ek.y));
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) *reinterpret_cast<float4 *>(row + ((k + r) & 7) * 16) = kf;
+                        for (int k = 0; k < 8; ++k) *reinterpret_cast<float4 *>(row + ((k + r) & 7) * 16) = kf;
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + ((k + r) & 15) * 8) = ek;
+                    }
 #pragma unroll
                     for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + 128 + ((k + r) & 15) * 8) = ev;
                 }
@@ -321,10 +344,18 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                     float s[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const float4 e0 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wa[k], colk, 0x7604));
-                        const float4 e1 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wa[k], colk, 0x7614));
-                        const float4 e2 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wb[k], colk, 0x7604));
-                        const float4 e3 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wb[k], colk, 0x7614));
+                        float4 e0, e1, e2, e3;
+                        if constexpr (TQ) {
+                            e0 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wa[k], colk, 0x7604));
+                            e1 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wa[k], colk, 0x7614));
+                            e2 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wb[k], colk, 0x7604));
+                            e3 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wb[k], colk, 0x7614));
+                        } else {
+                            e0 = widen_bf16x4(lds64(smem, __byte_perm(wa[k], colk, 0x7604)), eye);
+                            e1 = widen_bf16x4(lds64(smem, __byte_perm(wa[k], colk, 0x7614)), eye);
+                            e2 = widen_bf16x4(lds64(smem, __byte_perm(wb[k], colk, 0x7604)), eye);
+                            e3 = widen_bf16x4(lds64(smem, __byte_perm(wb[k], colk, 0x7614)), eye);
+                        }
                         if constexpr (TQ) {
                             // entries (u_f, u_{f+D/2}, u_f', u_{f'+D/2}): one packed FMA per pair
                             float2 sc2 = __fmul2_rn(xq[0], f2(e0.x, e0.y));
