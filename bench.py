@@ -477,22 +477,42 @@ def _unpack_codes(words, Nmax, NP):
     return k, v
 
 
-def cpu_encode_and_ties(w, cache, threads, budget_s, layer=0, blk=0):
+def tie_sample(w, threads):
+    """The tokens the encode baseline and the tie count use: one (sequence, KV head) per thread, a run of
+    `chunk` tokens each."""
+    chunk = min(4096, w.Nmax)
+    return chunk, [((j * 7) % w.B, (j * 5) % w.Hkv, (j * 997) % max(1, w.Nmax - chunk)) for j in range(threads)]
+
+
+def gpu_sample_codes(w, cache, threads, layer=0, blk=0):
+    """The GPU's key and value codes of the tie sample's tokens, copied to the host.  Taken right after the
+    cache is encoded: the windowed comparison later rolls window pages into the same cache, which replaces
+    the codes of the tokens it rolls."""
+    NP = w.D // (2 * w.c)
+    chunk, sample = tie_sample(w, threads)
+    per_bh = w.Nmax * NP
+    codes = {}
+    for b, h, tok0 in sample:
+        base = ((layer * w.NB + blk) * w.B + b) * w.Hkv + h
+        words = cache.idx[base * per_bh:(base + 1) * per_bh].cpu().numpy().view(np.uint32)
+        ck, cv = _unpack_codes(words, w.Nmax, NP)
+        codes[(b, h, tok0)] = (ck[tok0:tok0 + chunk].copy(), cv[tok0:tok0 + chunk].copy())
+    return codes
+
+
+def cpu_encode_and_ties(w, gpu_codes, threads, budget_s, layer=0, blk=0):
     """The checker's encode of sampled tokens of one (layer, block) on `threads` cores, timed and
     extrapolated to the whole (layer, block) unit (labelled as such), and the GPU's codes for the same
-    tokens compared with it: a code that differs counts as a near-tie when the two fp64 distances differ
-    by at most 1e-5 relative, anything else as a mismatch.  Runs after the timed region."""
+    tokens (`gpu_sample_codes`) compared with it: a code that differs counts as a near-tie when the two
+    fp64 distances differ by at most 1e-5 relative, anything else as a mismatch.  Runs after the timed
+    region."""
     from concurrent.futures import ThreadPoolExecutor
     from oracle import oracle as O
     if w.tasq:
         return None, {"checked": 0, "note": "TaSQ codes are checked by the GPU tests, not here"}
-    NP = w.D // (2 * w.c)
-    # sample: one (sequence, KV head) per thread, a run of tokens each, keys and values
-    chunk = min(4096, w.Nmax)
-    pairs = [((i * 7) % w.B, (i * 5) % w.Hkv) for i in range(threads)]
+    chunk, sample = tie_sample(w, threads)
     jobs = []
-    for j, (b, h) in enumerate(pairs):
-        tok0 = (j * 997) % max(1, w.Nmax - chunk)
+    for b, h, tok0 in sample:
         toks = range(tok0, tok0 + chunk)
         for kv in range(2):
             x = kv_loops(w, layer, kv, blk * w.Tc, blk * w.Tc + w.Tc - 1, [b], toks, [h])[:, 0, :, 0, :]
@@ -515,12 +535,8 @@ def cpu_encode_and_ties(w, cache, threads, budget_s, layer=0, blk=0):
                           f"{threads} threads, scaled to the {vec_unit} vectors of the (layer, block)"}
     # the GPU codes of the same tokens
     checked = ties = other = 0
-    per_bh = w.Nmax * NP
     for (b, h, kv, tok0, x, E), ref in zip(jobs, refs):
-        base = ((layer * w.NB + blk) * w.B + b) * w.Hkv + h
-        words = cache.idx[base * per_bh:(base + 1) * per_bh].cpu().numpy().view(np.uint32)
-        ck, cv = _unpack_codes(words, w.Nmax, NP)
-        gpu = (ck if kv == 0 else cv)[tok0:tok0 + chunk]
+        gpu = gpu_codes[(b, h, tok0)][kv]
         checked += gpu.size
         for i, g in zip(*np.nonzero(gpu != ref)):
             if w.ncb > 1:
@@ -698,6 +714,9 @@ def main():
     h2d = q_host.numel() * q_host.element_size() + lens_host.numel() * 4
     d2h = out_host.numel() * 4 + lse_host.numel() * 4
 
+    tie_codes = None
+    if world == 1 and not args.no_cpu_baseline and not w.tasq:
+        tie_codes = gpu_sample_codes(w, cache, host_threads())
     compare = None
     if not args.no_compare and rank == 0:
         compare = bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream)
@@ -758,7 +777,7 @@ def main():
             s1, nb1, u1 = cpu_sample(w, args.cpu_seconds)
             nthr = host_threads()
             sa, nba, ua = cpu_sample_all_cores(w, s1 / max(u1, 1), nthr, args.cpu_seconds)
-            enc_cpu, ties = cpu_encode_and_ties(w, cache, nthr, args.cpu_seconds)
+            enc_cpu, ties = cpu_encode_and_ties(w, tie_codes, nthr, args.cpu_seconds)
             line["cpu_baseline"] = {
                 "value": nb1 / s1 / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "cpu_model": cpu_model(),
                 "sample": f"{u1} (sequence, query head) units of the layer-0, loop-step-2 call, {s1:.1f} s "
