@@ -14,8 +14,7 @@
 //    widened to fp32 by one m16n8k8 tensor-core product with the identity (lane-local, exact), so the
 //    key side needs no ALU unpacking and gathers 256 bytes per token and KV head instead of the 512 of
 //    fp32 tables (4% faster at ctx32k than fp32 tables, once the value side below was in place; 6%
-//    slower before it).  With TaSQ keys the K slice is staged in fp32 (16 bytes in 8 replicas), which
-//    measured faster there.
+//    slower before it; with TaSQ keys 9% faster together with the value layout below, slower alone).
 //  * A warp takes a contiguous run of 16-token tiles of the piece.  Lane (g, t) = (lane / 4, lane % 4)
 //    owns the tokens t, t + 4, t + 8, t + 12 of each tile and the two pair-groups g and g + 8: the
 //    channel groups g, g + 8 (low channels) and g + 16, g + 24 (their RoPE partners), 8 RoPE pairs.
@@ -38,12 +37,11 @@
 //    part (g < 2) or lo part, which represents the fp32 weight to about 2^-16 relative; columns 4-7 are
 //    zero.  Lanes t = 0 and 1 accumulate the hi and lo parts of the same channels, added at the end.
 //    (The first version put the weights in A with one token per MMA: 16 MMAs per tile with half the A
-//    rows zero, whose A quads had to be assembled from separate registers; 7% slower at ctx32k.  TaSQ
-//    keys keep that form, which measured faster there.)
+//    rows zero, whose A quads had to be assembled from separate registers; 7% slower at ctx32k.)
 //  * Index words arrive through a per-warp ring of 1 KiB stages in shared memory filled with 16-byte
 //    cp.async copies (lane L copies chunks L and L + 32 of the tile); each lane reads its 8 words with
 //    conflict-free 4-byte loads.
-//  * TaSQ keys (TQ, LoopVQ paper App. B): word p's key codes are TaSQ groups 2p and 2p + 1, whose fp32
+//  * TaSQ keys (TQ, LoopVQ paper App. B): word p's key codes are TaSQ groups 2p and 2p + 1, whose
 //    entries hold the RoPE pairs of the head's pair order interleaved.  The lane's 8 pairs come from
 //    that order, so all of them run the difference form; their rotated query is divided by the channel
 //    weight, and the finished score is multiplied by the token's scale, read one tile ahead.
@@ -118,9 +116,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
     int h = (int)(range_info[3] >> 32), b = (int)(range_info[3] & 0xffffffffLL);
 
     const int g = lane >> 2, t = lane & 3;
-    // the lane's K replica: bf16 (8 bytes, replica lane % 16) with plain keys, fp32 (16 bytes, replica
-    // lane % 8) with TaSQ keys
-    const uint32_t colk = TQ ? (uint32_t)((lane & 7) * 16) : (uint32_t)((lane & 15) * 8);
+    // the lane's K replica (8 bytes of bf16, replica lane % 16)
+    const uint32_t colk = (uint32_t)((lane & 15) * 8);
     const uint32_t eye = ((2 * (lane & 3) == (lane >> 2)) ? 0x3F80u : 0u) |
                          ((2 * (lane & 3) + 1 == (lane >> 2)) ? 0x3F800000u : 0u);
     const uint32_t colv = (uint32_t)((lane & 15) * 8) + 128u;   // and its V replica
@@ -153,11 +150,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             const int n16 = (n4 + 3) >> 2;
             __syncthreads();                               // the previous piece's tables and records are done
 
-            // stage: row r = K entry r in fp32, 8 replicas of 16 bytes at [0, 128); V entry r in bf16,
-            // 16 replicas of 8 bytes at [128, 256).  The slices depend on the KV head only, so a piece of
-            // the head already staged (the next sequence of the same head) keeps them.  Thread r reads
-            // entry r once and writes its replicas starting at replica r mod 8 (16), so the lanes of each
-            // quarter-warp (half-warp) store write distinct banks.
+            // stage: row r = K entry r in bf16, 16 replicas of 8 bytes at [0, 128); V entry r likewise at
+            // [128, 256).  The slices depend on the KV head only, so a piece of the head already staged (the
+            // next sequence of the same head) keeps them.  Thread r reads entry r once and writes its
+            // replicas starting at replica r mod 16, so the lanes of each half-warp store write distinct
+            // banks.
             const bool restage = h != staged_h;
             if (restage) {
                 const uint16_t *sk = a.slk + (size_t)h * a.K * 4;
@@ -169,14 +166,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                         ev = __ldg(reinterpret_cast<const uint2 *>(sv + (size_t)r * 4));
                     }
                     unsigned char *row = smem + r * 256;
-                    if constexpr (TQ) {
-                        const float4 kf = make_float4(bf16lo(ek.x), bf16hi(ek.x), bf16lo(ek.y), bf16hi(ek.y));
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) *reinterpret_cast<float4 *>(row + ((k + r) & 7) * 16) = kf;
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + ((k + r) & 15) * 8) = ek;
-                    }
+                    for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + ((k + r) & 15) * 8) = ek;
 #pragma unroll
                     for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + 128 + ((k + r) & 15) * 8) = ev;
                 }
@@ -186,18 +177,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             // this warp's run of 16-token tiles [i0, i1) of the piece
             const int i0 = (int)((long long)warp * n16 / WARPS), i1 = (int)((long long)(warp + 1) * n16 / WARPS);
             const int kown = 2 * (g & 1) + ((g >> 1) & 1);  // the token (0..3) this lane finishes
-            // Value products (below), selectors of the packed weight x = {hi part: bytes 0-1, lo part: 2-3}.
-            // Plain keys: B column g < 4 takes part g >> 1 in half g & 1, columns 4..7 are zero.  TaSQ keys:
-            // A row g takes part g >> 2 at channel g & 3, in a0 for channels 0-1 and a2 for 2-3.
-            uint32_t sel0, sel2;
-            if constexpr (TQ) {
-                const uint32_t part_lo = (g & 4) ? 0x4432u : 0x4410u, part_hi = (g & 4) ? 0x3244u : 0x1044u;
-                sel0 = (g & 2) ? 0x4444u : ((g & 1) ? part_hi : part_lo);
-                sel2 = (g & 2) ? ((g & 1) ? part_hi : part_lo) : 0x4444u;
-            } else {
-                sel0 = g >= 4 ? 0x4444u : ((g & 2) ? ((g & 1) ? 0x3244u : 0x4432u) : ((g & 1) ? 0x1044u : 0x4410u));
-                sel2 = 0u;
-            }
+            // Value products (below), selector of the packed weight x = {hi part: bytes 0-1, lo part: 2-3}:
+            // B column g < 4 takes part g >> 1 in half g & 1, columns 4..7 are zero.
+            const uint32_t sel0 =
+                g >= 4 ? 0x4444u : ((g & 2) ? ((g & 1) ? 0x3244u : 0x4432u) : ((g & 1) ? 0x1044u : 0x4410u));
             // index copies: lane L takes chunks L (four-tile L / 16) and L + 32 (four-tile L / 16 + 2)
             const int kc = lane >> 4;
             const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP;
@@ -344,18 +327,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                     float s[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        float4 e0, e1, e2, e3;
-                        if constexpr (TQ) {
-                            e0 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wa[k], colk, 0x7604));
-                            e1 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wa[k], colk, 0x7614));
-                            e2 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wb[k], colk, 0x7604));
-                            e3 = *reinterpret_cast<const float4 *>(smem + __byte_perm(wb[k], colk, 0x7614));
-                        } else {
-                            e0 = widen_bf16x4(lds64(smem, __byte_perm(wa[k], colk, 0x7604)), eye);
-                            e1 = widen_bf16x4(lds64(smem, __byte_perm(wa[k], colk, 0x7614)), eye);
-                            e2 = widen_bf16x4(lds64(smem, __byte_perm(wb[k], colk, 0x7604)), eye);
-                            e3 = widen_bf16x4(lds64(smem, __byte_perm(wb[k], colk, 0x7614)), eye);
-                        }
+                        const float4 e0 = widen_bf16x4(lds64(smem, __byte_perm(wa[k], colk, 0x7604)), eye);
+                        const float4 e1 = widen_bf16x4(lds64(smem, __byte_perm(wa[k], colk, 0x7614)), eye);
+                        const float4 e2 = widen_bf16x4(lds64(smem, __byte_perm(wb[k], colk, 0x7604)), eye);
+                        const float4 e3 = widen_bf16x4(lds64(smem, __byte_perm(wb[k], colk, 0x7614)), eye);
                         if constexpr (TQ) {
                             // entries (u_f, u_{f+D/2}, u_f', u_{f'+D/2}): one packed FMA per pair
                             float2 sc2 = __fmul2_rn(xq[0], f2(e0.x, e0.y));
@@ -432,11 +407,9 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                             const float2 lo2 = __fmul2_rn(f2(acc[j].x, acc[j].y), c2);
                             acc[j].x = lo2.x;
                             acc[j].y = lo2.y;
-                            if constexpr (!TQ) {                // with TaSQ keys rows 8..15 (z, w) stay zero
-                                const float2 hi2 = __fmul2_rn(f2(acc[j].z, acc[j].w), c2);
-                                acc[j].z = hi2.x;
-                                acc[j].w = hi2.y;
-                            }
+                            const float2 hi2 = __fmul2_rn(f2(acc[j].z, acc[j].w), c2);
+                            acc[j].z = hi2.x;
+                            acc[j].w = hi2.y;
                         }
                         m = tmax;
                     }
@@ -454,43 +427,26 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                         xk[2] = __shfl_sync(0xffffffffu, x, 4 + t);
                         xk[3] = __shfl_sync(0xffffffffu, x, 12 + t);
                     }
-                    if constexpr (!TQ) {
-                        // ---- values: A rows g, g + 8 = channels 0-1, 2-3 of group 8u + g; k = (token slot, channel
-                        // parity) over slots t (k 2t, 2t + 1) and t + 4 (k 2t + 8, 2t + 9) of a token octet, so the
-                        // lane's A quad is its two gathered 8-byte entries as loaded; B column g < 4 = (part g >> 1,
-                        // parity g & 1) holds the slot's weight part at that parity
-                        uint32_t bw[4];
+                    // ---- values: A rows g, g + 8 = channels 0-1, 2-3 of group 8u + g; k = (token slot, channel
+                    // parity) over slots t (k 2t, 2t + 1) and t + 4 (k 2t + 8, 2t + 9) of a token octet, so the
+                    // lane's A quad is its two gathered 8-byte entries as loaded; B column g < 4 = (part g >> 1,
+                    // parity g & 1) holds the slot's weight part at that parity
+                    uint32_t bw[4];
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) bw[k] = __byte_perm(xk[k], 0u, sel0);
+                    for (int k = 0; k < 4; ++k) bw[k] = __byte_perm(xk[k], 0u, sel0);
 #pragma unroll
-                        for (int o = 0; o < 2; ++o) {
-                            uint2 v[2][4];
+                    for (int o = 0; o < 2; ++o) {
+                        uint2 v[2][4];
 #pragma unroll
-                            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                                for (int u = 0; u < 4; ++u)
-                                    v[j][u] = lds64(smem, __byte_perm((u & 1) ? wb[2 * o + j] : wa[2 * o + j], colv,
-                                                                      (u < 2) ? 0x7624u : 0x7634u));
+                        for (int j = 0; j < 2; ++j)
 #pragma unroll
                             for (int u = 0; u < 4; ++u)
-                                mma_bf16_16816(acc[u], v[0][u].x, v[0][u].y, v[1][u].x, v[1][u].y, bw[2 * o],
-                                               bw[2 * o + 1]);
-                        }
-                    } else {
-                        // ---- values with TaSQ keys: k = (token slot t, channel e) of one token per MMA, B = the
-                        // lane's gathered entry, A row g = (part g >> 2, channel g & 3)
-                        uint2 v[4][4];
+                                v[j][u] = lds64(smem, __byte_perm((u & 1) ? wb[2 * o + j] : wa[2 * o + j], colv,
+                                                                  (u < 2) ? 0x7624u : 0x7634u));
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                v[k][u] = lds64(smem, __byte_perm((u & 1) ? wb[k] : wa[k], colv, (u < 2) ? 0x7624u : 0x7634u));
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t a0 = __byte_perm(xk[k], 0u, sel0), a2 = __byte_perm(xk[k], 0u, sel2);
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) mma_bf16_16816(acc[u], a0, 0u, a2, 0u, v[k][u].x, v[k][u].y);
-                        }
+                        for (int u = 0; u < 4; ++u)
+                            mma_bf16_16816(acc[u], v[0][u].x, v[0][u].y, v[1][u].x, v[1][u].y, bw[2 * o],
+                                           bw[2 * o + 1]);
                     }
                 }
             }
@@ -502,28 +458,15 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
                 lsum *= 0.5f;                              // every token is finished by two lanes
-                if constexpr (!TQ) {
-                    // lane (g, 0) holds the hi parts of channels 0-3 of group 8u + g, lane (g, 1) the lo parts
+                // lane (g, 0) holds the hi parts of channels 0-3 of group 8u + g, lane (g, 1) the lo parts
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        float4 c = acc[u];
-                        c.x += __shfl_xor_sync(0xffffffffu, c.x, 1);
-                        c.y += __shfl_xor_sync(0xffffffffu, c.y, 1);
-                        c.z += __shfl_xor_sync(0xffffffffu, c.z, 1);
-                        c.w += __shfl_xor_sync(0xffffffffu, c.w, 1);
-                        if (t == 0) *reinterpret_cast<float4 *>(rec + 4 * (8 * u + g)) = c;
-                    }
-                } else {
-                    // lane (g < 4, t) holds channel g of groups 8u + 2t, 8u + 2t + 1 (hi parts; lo parts in lane + 16)
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float vx = acc[u].x + __shfl_xor_sync(0xffffffffu, acc[u].x, 16);
-                        const float vy = acc[u].y + __shfl_xor_sync(0xffffffffu, acc[u].y, 16);
-                        if (g < 4) {
-                            rec[4 * (8 * u + 2 * t) + g] = vx;
-                            rec[4 * (8 * u + 2 * t + 1) + g] = vy;
-                        }
-                    }
+                for (int u = 0; u < 4; ++u) {
+                    float4 c = acc[u];
+                    c.x += __shfl_xor_sync(0xffffffffu, c.x, 1);
+                    c.y += __shfl_xor_sync(0xffffffffu, c.y, 1);
+                    c.z += __shfl_xor_sync(0xffffffffu, c.z, 1);
+                    c.w += __shfl_xor_sync(0xffffffffu, c.w, 1);
+                    if (t == 0) *reinterpret_cast<float4 *>(rec + 4 * (8 * u + g)) = c;
                 }
                 if (lane == 0) {
                     rec[D] = lsum > 0.f ? m : -CUDART_INF_F;
