@@ -86,11 +86,11 @@ def job_throughput(world, bytes_per_step_per_rank, ms_per_step_max):
 
 def decode_kernel_name(w):
     """The split kernel a decode call of workload w runs: decode_mha_kernel for one query head per KV
-    head at D = 128 with groups of 4 channels (plain or TaSQ keys), decode_gqa_kernel for 4 query heads
-    per KV head at D = 128 with groups of 8 (plain keys), both with a shared codebook;
-    decode_split_kernel otherwise."""
+    head at D = 128 with groups of 4 channels (plain or TaSQ keys) or of 16 (plain keys),
+    decode_gqa_kernel for 4 query heads per KV head at D = 128 with groups of 8 (plain keys), all with a
+    shared codebook; decode_split_kernel otherwise."""
     if w.D == 128 and w.ncb == 1:
-        if w.c == 4 and w.Hq == w.Hkv:
+        if w.Hq == w.Hkv and (w.c == 4 or (w.c == 16 and not w.tasq)):
             return "decode_mha"                   # plain or TaSQ keys
         if w.c == 8 and w.Hq == 4 * w.Hkv and not w.tasq:
             return "decode_gqa"

@@ -42,14 +42,15 @@ static size_t ring_smem_bytes(bool pg, int qpk, int D) {
     return (pg ? 131072 : 65536) + (size_t)k.depth * k.warps * 32 * 16 * kWords + recs;
 }
 
-// decode_mha_kernel (one query head per KV head, D = 128, groups of 4 channels, one shared codebook)
+// decode_mha_kernel (one query head per KV head, D = 128, groups of 4 channels or of 16, one shared
+// codebook)
 // runs the step-4 RoPE recurrence in plain form on the frequencies f < D/4 and in difference form on
 // f >= D/4; it needs |sin 4w_f| >= 0.04 on the first (the recurrence's rounding grows as 1/|sin 4w|),
 // 4w_f <= 1 on the second, and table rows 2 and 4.  With the base 1e4: min |sin 4w| = 0.046 (f = 31).
 static constexpr int kMhaWarps = 8, kMhaMinBlocks = 2, kMhaDepth = 2;
 
 static bool mha_applies(const loopvq_cache &cc) {
-    if (cc.D != 128 || cc.c != 4 || cc.Hq != cc.Hkv || ncb_of(cc) != 1 || cc.Nmax < 8) return false;
+    if (cc.D != 128 || (cc.c != 4 && cc.c != 16) || cc.Hq != cc.Hkv || ncb_of(cc) != 1 || cc.Nmax < 8) return false;
     for (int f = 0; f < 64; ++f) {
         const double w = pow((double)cc.theta, -2.0 * f / 128.0);
         if (f < 32 ? fabs(sin(4.0 * w)) < 0.04 : 4.0 * w > 1.0) return false;
@@ -82,10 +83,10 @@ static cudaError_t launch_gqa(const DecodeArgs &a, const DecodePlan &plan, cudaS
     return launch_merge<128>(a, s);
 }
 
-template <bool TQ>
+template <bool TQ, int C>
 static cudaError_t launch_mha(const DecodeArgs &a, const DecodePlan &plan, cudaStream_t s) {
-    using S = MhaSmem<kMhaWarps, kMhaDepth>;
-    auto kern = decode_mha_kernel<kMhaWarps, kMhaMinBlocks, kMhaDepth, TQ>;
+    using S = MhaSmem<kMhaWarps, kMhaDepth, 64u * (128 / (2 * C))>;
+    auto kern = decode_mha_kernel<kMhaWarps, kMhaMinBlocks, kMhaDepth, TQ, C>;
     cudaError_t e = ensure_dynamic_smem((const void *)kern, S::kBytes);
     if (e != cudaSuccess) return e;
     if (plan.ncta > 0) {
@@ -232,7 +233,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
         a.tperm = tq->perm + ((size_t)layer * NB + beta) * cc.Hkv * (cc.D / 2);
         a.tsig = tq->sigma + ((size_t)layer * cc.T + t) * cc.B * cc.Nmax;
         if (ncb_of(cc) != 1) return cudaErrorInvalidValue;
-        if (plan.mha) return launch_mha<true>(a, plan, s);
+        if (plan.mha && cc.c == 4) return launch_mha<true, 4>(a, plan, s);
         if (cc.D == 128 && cc.c == 4) return dispatch_tq_qpk<128, 4>(qpk, a, plan, s);
         if (cc.D == 128 && cc.c == 8) return dispatch_tq_qpk<128, 8>(qpk, a, plan, s);
         if (cc.D == 64 && cc.c == 4) return dispatch_tq_qpk<64, 4>(qpk, a, plan, s);
@@ -240,7 +241,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
         return cudaErrorInvalidValue;
     }
     const bool pg = ncb_of(cc) > 1;
-    if (plan.mha) return launch_mha<false>(a, plan, s);
+    if (plan.mha) return cc.c == 4 ? launch_mha<false, 4>(a, plan, s) : launch_mha<false, 16>(a, plan, s);
     if (plan.gqa) return launch_gqa(a, plan, s);
     if (cc.D == 128) return pg ? dispatch_c<128, true>(cc.c, qpk, a, plan, s) : dispatch_c<128, false>(cc.c, qpk, a, plan, s);
     if (cc.D == 64) return pg ? dispatch_c<64, true>(cc.c, qpk, a, plan, s) : dispatch_c<64, false>(cc.c, qpk, a, plan, s);

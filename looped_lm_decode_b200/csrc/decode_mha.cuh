@@ -41,6 +41,12 @@
 //  * Index words arrive through a per-warp ring of 1 KiB stages in shared memory filled with 16-byte
 //    cp.async copies (lane L copies chunks L and L + 32 of the tile); each lane reads its 8 words with
 //    conflict-free 4-byte loads.
+//  * Groups of 16 channels (C = 16: the per-loop-step coding the LoopVQ paper compares against, Sec. 5.1,
+//    "CQ") keep every lane's work: pair-group g's channels are quarter g % 4 of code group 4g / 16, its
+//    RoPE partners the same quarter of group 4g / 16 + NP, and pair-group g + 8 is two groups on, so a
+//    lane reads words g / 4 and g / 4 + 2 instead of g and g + 8 and gathers its 8 bytes at quarter g % 4
+//    of the 32-byte entry.  Entries are staged in 4 replicas (replica t), rows stay 256 bytes, and the
+//    ring stage is NP = 4 words per token (256 bytes per 16-token tile).
 //  * TaSQ keys (TQ, LoopVQ paper App. B): word p's key codes are TaSQ groups 2p and 2p + 1, whose
 //    entries hold the RoPE pairs of the head's pair order interleaved.  The lane's 8 pairs come from
 //    that order, so all of them run the difference form; their rotated query is divided by the channel
@@ -81,12 +87,13 @@ __device__ __forceinline__ void cp_async16_zfill(uint32_t dst_smem, const void *
                  : "memory");
 }
 
-// Shared memory of the kernel: K/V replicas, then the index ring, then the warp records.
-template <int WARPS, int DEPTH>
+// Shared memory of the kernel: K/V replicas, then the index ring (stages of SB bytes), then the warp
+// records.
+template <int WARPS, int DEPTH, uint32_t SB>
 struct MhaSmem {
     static constexpr uint32_t kTables = 65536u;
     static constexpr uint32_t kRing = kTables;
-    static constexpr uint32_t kRingBytes = (uint32_t)WARPS * DEPTH * 1024u;
+    static constexpr uint32_t kRingBytes = (uint32_t)WARPS * DEPTH * SB;
     static constexpr uint32_t kRec = kRing + kRingBytes;
     static constexpr uint32_t kRecFloats = 128 + 4;
     static constexpr uint32_t kBytes = kRec + (uint32_t)WARPS * kRecFloats * 4u;
@@ -97,12 +104,14 @@ struct MhaSmem {
 // interleaved; the lane keeps one rotated query pair (re, im) per pair, divided by the channel weight,
 // runs the difference-form recurrence on every pair, and multiplies each finished score by its token's
 // scale sigma.
-template <int WARPS, int MINB, int DEPTH, bool TQ = false>
+template <int WARPS, int MINB, int DEPTH, bool TQ = false, int C = 4>
 __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const DecodeArgs a) {
-    constexpr int D = 128, NP = 16;                        // pair-groups = index words per token
+    static_assert(C == 4 || (C == 16 && !TQ), "groups of 4 channels, or of 16 with plain keys");
+    constexpr int D = 128, NP = D / (2 * C);               // index words per token
+    constexpr uint32_t SB = 64u * NP;                      // bytes of one 16-token ring stage
     constexpr int NT = WARPS * 32;
     constexpr int ANCHOR = 64;                             // tiles between two settings from the table
-    using S = MhaSmem<WARPS, DEPTH>;
+    using S = MhaSmem<WARPS, DEPTH, SB>;
 
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ long long range_info[4];
@@ -116,13 +125,14 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
     int h = (int)(range_info[3] >> 32), b = (int)(range_info[3] & 0xffffffffLL);
 
     const int g = lane >> 2, t = lane & 3;
-    // the lane's K replica (8 bytes of bf16, replica lane % 16)
-    const uint32_t colk = (uint32_t)((lane & 15) * 8);
+    // the lane's K column: C = 4, replica lane % 16 of the 8-byte entry; C = 16, quarter g % 4 of the
+    // 32-byte entry in replica t (the 16 lanes of a half-warp read 16 distinct 8-byte slots of a row)
+    const uint32_t colk = C == 4 ? (uint32_t)((lane & 15) * 8) : (uint32_t)(t * 32 + (g & 3) * 8);
     const uint32_t eye = ((2 * (lane & 3) == (lane >> 2)) ? 0x3F80u : 0u) |
                          ((2 * (lane & 3) + 1 == (lane >> 2)) ? 0x3F800000u : 0u);
-    const uint32_t colv = (uint32_t)((lane & 15) * 8) + 128u;   // and its V replica
+    const uint32_t colv = colk + 128u;                     // and its V column
     const uint32_t smem_base = (uint32_t)__cvta_generic_to_shared(smem);
-    const uint32_t ring = smem_base + S::kRing + (uint32_t)warp * DEPTH * 1024u;
+    const uint32_t ring = smem_base + S::kRing + (uint32_t)warp * DEPTH * SB;
     float *rec = reinterpret_cast<float *>(smem + S::kRec) + warp * S::kRecFloats;
 
     // recurrence coefficients of the lane's pairs: high pairs f = 4g + e (2 cos 4w), low pairs
@@ -157,19 +167,40 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             // banks.
             const bool restage = h != staged_h;
             if (restage) {
-                const uint16_t *sk = a.slk + (size_t)h * a.K * 4;
-                const uint16_t *sv = a.slv + (size_t)h * a.K * 4;
+                const uint16_t *sk = a.slk + (size_t)h * a.K * C;
+                const uint16_t *sv = a.slv + (size_t)h * a.K * C;
                 for (int r = tid; r < 256; r += NT) {
-                    uint2 ek = make_uint2(0u, 0u), ev = make_uint2(0u, 0u);
-                    if (r < a.K) {
-                        ek = __ldg(reinterpret_cast<const uint2 *>(sk + (size_t)r * 4));
-                        ev = __ldg(reinterpret_cast<const uint2 *>(sv + (size_t)r * 4));
-                    }
                     unsigned char *row = smem + r * 256;
+                    if constexpr (C == 4) {
+                        uint2 ek = make_uint2(0u, 0u), ev = make_uint2(0u, 0u);
+                        if (r < a.K) {
+                            ek = __ldg(reinterpret_cast<const uint2 *>(sk + (size_t)r * 4));
+                            ev = __ldg(reinterpret_cast<const uint2 *>(sv + (size_t)r * 4));
+                        }
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + ((k + r) & 15) * 8) = ek;
+                        for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + ((k + r) & 15) * 8) = ek;
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + 128 + ((k + r) & 15) * 8) = ev;
+                        for (int k = 0; k < 16; ++k) *reinterpret_cast<uint2 *>(row + 128 + ((k + r) & 15) * 8) = ev;
+                    } else {
+                        // 32-byte entries, 4 replicas each in [0, 128) (K) and [128, 256) (V)
+                        uint4 e[4] = {};
+                        if (r < a.K) {
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                e[j] = __ldg(reinterpret_cast<const uint4 *>(sk + (size_t)r * 16) + j);
+                                e[2 + j] = __ldg(reinterpret_cast<const uint4 *>(sv + (size_t)r * 16) + j);
+                            }
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t o = (uint32_t)((k + r) & 3) * 32u;
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                *reinterpret_cast<uint4 *>(row + o + 16 * j) = e[j];
+                                *reinterpret_cast<uint4 *>(row + 128 + o + 16 * j) = e[2 + j];
+                            }
+                        }
+                    }
                 }
                 staged_h = h;
             }
@@ -181,24 +212,30 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             // B column g < 4 takes part g >> 1 in half g & 1, columns 4..7 are zero.
             const uint32_t sel0 =
                 g >= 4 ? 0x4444u : ((g & 2) ? ((g & 1) ? 0x3244u : 0x4432u) : ((g & 1) ? 0x1044u : 0x4410u));
-            // index copies: lane L takes chunks L (four-tile L / 16) and L + 32 (four-tile L / 16 + 2)
-            const int kc = lane >> 4;
+            // index copies: a stage is 4 NP chunks of 16 bytes (the 4 tokens of one four-tile and word),
+            // in memory order; lane L takes chunk L (four-tile L / NP) and, with C = 4, chunk L + 32
+            // (four-tile L / NP + 2).  With C = 16 the 16 chunks go to lanes 0..15.
+            const int kc = lane / NP;
+            const bool copier = C == 4 || lane < 16;
             const uint32_t *idx_b = a.idx + ((size_t)b * a.Hkv + h) * (size_t)a.Nmax * NP;
-            const char *src = reinterpret_cast<const char *>(idx_b + ((size_t)((tok_begin >> 2) + 4 * i0 + kc) * NP + (lane & 15)) * 4);
+            const char *src = reinterpret_cast<const char *>(idx_b + (size_t)((tok_begin >> 2) + 4 * i0) * NP * 4) + lane * 16;
             const uint32_t dst = ring + (uint32_t)lane * 16u;
             int crem = n4 - 4 * i0, ctl = i1 - i0;         // four-tiles of the piece / tiles of the warp, from the copy on
             auto copy_tile = [&](uint32_t soff) {
-                const bool f0 = ctl > 0 && crem > kc, f1 = ctl > 0 && crem > kc + 2;
                 // a chunk outside the piece reads nothing (source size 0) from a valid address
-                cp_async16_zfill(dst + soff, f0 ? src : reinterpret_cast<const char *>(a.idx), f0);
-                cp_async16_zfill(dst + soff + 512u, f1 ? src + 512 : reinterpret_cast<const char *>(a.idx), f1);
+                const bool f0 = ctl > 0 && crem > kc;
+                if (copier) cp_async16_zfill(dst + soff, f0 ? src : reinterpret_cast<const char *>(a.idx), f0);
+                if constexpr (C == 4) {
+                    const bool f1 = ctl > 0 && crem > kc + 2;
+                    cp_async16_zfill(dst + soff + 512u, f1 ? src + 512 : reinterpret_cast<const char *>(a.idx), f1);
+                }
                 cp_async_commit();
-                src += 1024;
+                src += SB;
                 crem -= 4;
                 --ctl;
             };
 #pragma unroll
-            for (int d = 0; d < DEPTH; ++d) copy_tile((uint32_t)d * 1024u);
+            for (int d = 0; d < DEPTH; ++d) copy_tile((uint32_t)d * SB);
 
             float4 acc[4];
 #pragma unroll
@@ -227,7 +264,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
             };
             float sig_next = 0.f;
             if constexpr (TQ) sig_next = load_sig(nrel);
-            const unsigned char *wrd = smem + S::kRing + (uint32_t)warp * DEPTH * 1024u + 4u * (4 * g + t);
+            // the lane's words: token t of pair-group g's word 4g / C and of pair-group g + 8's word
+            const unsigned char *wrd = smem + S::kRing + (uint32_t)warp * DEPTH * SB + 4u * (4 * (4 * g / C) + t);
             uint32_t soff = 0;
             if (restage) __syncthreads();                  // tables staged (the condition is CTA-uniform)
 
@@ -319,8 +357,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                     uint32_t wa[4], wb[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        wa[k] = wp[64 * k];                // four-tile k, pair-group g, token t
-                        wb[k] = wp[64 * k + 32];           // pair-group g + 8
+                        wa[k] = wp[4 * NP * k];            // four-tile k, pair-group g, token t
+                        wb[k] = wp[4 * NP * k + 128 / C];  // pair-group g + 8: word 4g / C + 32 / C
                     }
 
                     // ---- keys: gather, rebuild, score the lane's 4 tokens over its 8 pairs
@@ -376,7 +414,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) decode_mha_kernel(const Deco
                     // the stage's words are in registers: refill it with the tile DEPTH ahead
                     __syncwarp();
                     copy_tile(soff);
-                    soff = soff + 1024u == DEPTH * 1024u ? 0u : soff + 1024u;
+                    soff = soff + SB == DEPTH * SB ? 0u : soff + SB;
 
                     // ---- reduce-scatter over the 8 lanes of this t: lane (g, t) ends with token kown
                     float sk;
