@@ -31,7 +31,7 @@
 //    (lane L copies chunk L of the tile) and are read with conflict-free 4-byte loads.
 #pragma once
 
-#include "decode_mha.cuh"
+#include "decode_kernel.cuh"
 
 namespace loopvq {
 

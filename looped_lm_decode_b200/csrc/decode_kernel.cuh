@@ -97,6 +97,28 @@ __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// 16-byte copy that reads `full ? 16 : 0` bytes from src and zero-fills the rest of the destination
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst_smem, const void *src, bool full) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(full ? 16 : 0)
+                 : "memory");
+}
+
+// two fp32 values rounded to bf16 and packed: hi_elem in the upper half, lo_elem in the lower
+__device__ __forceinline__ uint32_t cvt_bf16x2(float hi_elem, float lo_elem) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi_elem), "f"(lo_elem));
+    return r;
+}
+
+// d += A B, m16n8k16, bf16 operands, fp32 accumulators (warp-level tensor-core product)
+__device__ __forceinline__ void mma_bf16_16816(float4 &d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d.x), "+f"(d.y), "+f"(d.z), "+f"(d.w)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 

@@ -68,25 +68,6 @@ __device__ __forceinline__ float4 widen_bf16x4(uint2 e, uint32_t eye) {
     return c;
 }
 
-__device__ __forceinline__ uint32_t cvt_bf16x2(float hi_elem, float lo_elem) {
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi_elem), "f"(lo_elem));
-    return r;
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float4 &d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d.x), "+f"(d.y), "+f"(d.z), "+f"(d.w)
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst_smem, const void *src, bool full) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(full ? 16 : 0)
-                 : "memory");
-}
-
 // Shared memory of the kernel: K/V replicas, then the index ring (stages of SB bytes), then the warp
 // records.
 template <int WARPS, int DEPTH, uint32_t SB>
