@@ -120,11 +120,12 @@ def test_decode_parity_small(name, lens_kind):
             assert ok, f"{name} layer {layer} t {t}: {msg}"
 
 
-@pytest.mark.parametrize("name", ["ctx", "gqa"])
+@pytest.mark.parametrize("name", ["ctx", "gqa", "cq16"])
 @pytest.mark.parametrize("gain", [8.0, 0.0])
 def test_decode_peaky_and_flat_queries(name, gain):
     """q x 8 makes the softmax peaky (large max-rescale traffic); q = 0 gives the mean of values.  "ctx"
-    runs the one-head-per-KV-head kernel, "gqa" the 4-heads-per-KV-head kernel."""
+    runs the one-head-per-KV-head kernel, "cq16" the same kernel with groups of 16 channels, "gqa" the
+    4-heads-per-KV-head kernel."""
     w = SMALL[name]
     cache = make_cache(w)
     codes = _upload_random_codes(w, cache)
@@ -137,7 +138,7 @@ def test_decode_peaky_and_flat_queries(name, gain):
     assert ok, msg
 
 
-@pytest.mark.parametrize("name", ["ctx", "gqa"])
+@pytest.mark.parametrize("name", ["ctx", "gqa", "cq16"])
 def test_decode_edge_lengths(name):
     w = SMALL[name].replace(B=8)
     N = w.Nmax
@@ -162,9 +163,10 @@ def test_decode_edge_lengths(name):
 
 
 @pytest.mark.parametrize("w", [WORKLOADS["ctx4k"].replace(L=1, B=3, Hkv=2, Hq=2, Nmax=20),
+                               WORKLOADS["ctx4k"].replace(L=1, B=3, Hkv=2, Hq=2, Nmax=20, c=16, Tc=1),
                                WORKLOADS["gqa16k"].replace(L=1, B=3, Hkv=1, Hq=4, Nmax=12),
                                WORKLOADS["ctx4k"].replace(L=1, B=2, Hkv=1, Hq=1, Nmax=4)],
-                         ids=["mha-nmax20", "gqa-nmax12", "mha-nmax4"])
+                         ids=["mha-nmax20", "mha-c16-nmax20", "gqa-nmax12", "mha-nmax4"])
 def test_decode_short_caches(w):
     """Caches shorter than a 16-token tile (and one below the 8 positions the one- and four-head kernels
     need, which takes the general kernel): partial tiles, zero-filled index copies, RoPE rows near Nmax."""
