@@ -229,14 +229,20 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
     ws_w = torch.empty(max(LQ.window_workspace_bytes(win, cache, w.Nmax), 16), dtype=torch.uint8, device=dev)
     out_c = torch.empty_like(out_b)
     lse_c = torch.empty_like(lse_b)
-    def wstep(st):
+    def wstep(st):                                    # the token appended by the windowed call itself
         LQ.window_advance(win, cache, stream=st)
         for t in range(w.T):
             for layer in range(w.L):
-                i = t * w.L + layer
+                LQ.window_append_decode_attn(win, cache, layer, t, tok[0], tok[1], tok[2], qs[t * w.L + layer],
+                                             w.Nmax, out=out_c, lse=lse_c, workspace=ws_w, stream=st)
+
+    def wstep_separate(st):                           # the same step with a separate append launch
+        LQ.window_advance(win, cache, stream=st)
+        for t in range(w.T):
+            for layer in range(w.L):
                 LQ.window_append(win, layer, t, tok[0], tok[1], tok[2], stream=st)
-                LQ.window_decode_attn(win, cache, layer, t, qs[i], w.Nmax, out=out_c, lse=lse_c, workspace=ws_w,
-                                      stream=st)
+                LQ.window_decode_attn(win, cache, layer, t, qs[t * w.L + layer], w.Nmax, out=out_c, lse=lse_c,
+                                      workspace=ws_w, stream=st)
 
     def wcalls(st):                                   # the attention calls of a step alone
         for t in range(w.T):
@@ -246,16 +252,20 @@ def bf16_and_window(w, cache, lens, lens_np, max_len, qs, ws, stream, reps=3):
 
     nsteps = 16                                       # two page rolls for every sequence
     win_step_ms = replay_ms(graph_of(wstep), nsteps, stream)      # the window state lives on the device
+    win_step_sep_ms = replay_ms(graph_of(wstep_separate), nsteps, stream)
     win_call_ms = replay_ms(graph_of(wcalls), 2, stream) / (w.T * w.L)
     del win
 
     return {
         "bf16_cache": bf16_line,
-        "windowed": {"us_per_call": win_call_ms * 1e3, "us_per_step": win_step_ms * 1e3, "steps": nsteps,
+        "windowed": {"us_per_call": win_call_ms * 1e3, "us_per_step": win_step_ms * 1e3,
+                     "us_per_step_separate_append": win_step_sep_ms * 1e3, "steps": nsteps,
                      "sink": n_sink, "recent": n_recent,
                      "calls": "per step: loopvq_window_advance (page roll every 8 steps), then per (loop step, "
-                              "layer) loopvq_window_append + loopvq_window_decode_attn (coded split kernel + merge "
-                              "kernel, which also attends to the window slots)"},
+                              "layer) loopvq_window_append_decode_attn (coded split kernel + merge kernel, which "
+                              "writes the new token into the window and attends to the window slots); "
+                              "us_per_step_separate_append: the same step with loopvq_window_append + "
+                              "loopvq_window_decode_attn"},
     }
 
 

@@ -348,6 +348,22 @@ loopvq_status loopvq_window_decode_attn(const loopvq_window *w, const loopvq_cac
                                         float *lse, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * loopvq_window_append followed by loopvq_window_decode_attn, in the decode
+ * call's two launches: the merge kernel writes the new token into slot
+ * fill_b - 1 of (layer, t) (rotated key, key before RoPE, value, as
+ * loopvq_window_append does) and attends to it together with the other
+ * window slots.  Results and window contents equal those of the two calls.
+ * k_rot, k_pre, v: bf16 [B][Hkv][D], 16-byte aligned, as for
+ * loopvq_window_append; the other arguments as for loopvq_window_decode_attn.
+ * Call after loopvq_window_advance; concurrent calls for the same (layer, t)
+ * race on the window slot.
+ */
+loopvq_status loopvq_window_append_decode_attn(const loopvq_window *w, const loopvq_cache *cache, int layer, int t,
+                                               const uint16_t *k_rot, const uint16_t *k_pre, const uint16_t *v,
+                                               const uint16_t *q, int max_coded, float scale, float *out,
+                                               float *lse, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Explicit reconstruction for checking (eq. 5): for sequence b, tokens
  * tok0 .. tok0+ntok-1 and every KV head, the loop-step-t reconstruction of
  * keys (kv = 0) or values (kv = 1); keys are rotated by RoPE at their

@@ -406,9 +406,10 @@ size_t loopvq_window_workspace_bytes(const loopvq_window *w, const loopvq_cache 
     return loopvq::window_ws_bytes(*w, *cc, max_coded);
 }
 
-loopvq_status loopvq_window_decode_attn(const loopvq_window *w, const loopvq_cache *cc, int layer, int t,
-                                        const uint16_t *q, int max_coded, float scale, float *out, float *lse,
-                                        void *workspace, size_t ws_bytes, void *stream) {
+static loopvq_status window_decode(const char *name, const loopvq_window *w, const loopvq_cache *cc, int layer, int t,
+                                   const uint16_t *k_rot, const uint16_t *k_pre, const uint16_t *v, const uint16_t *q,
+                                   int max_coded, float scale, float *out, float *lse, void *workspace, size_t ws_bytes,
+                                   void *stream) {
     g_err[0] = 0;
     LQ_TRY(check_window(w, cc));
     LQ_TRY(check_ptr(cc->idx, "idx"));
@@ -416,6 +417,11 @@ loopvq_status loopvq_window_decode_attn(const loopvq_window *w, const loopvq_cac
     LQ_TRY(check_ptr(cc->rope, "rope"));
     LQ_TRY(check_ptr(q, "q"));
     LQ_TRY(check_ptr(out, "out"));
+    if (k_rot || k_pre || v) {
+        LQ_TRY(check_ptr(k_rot, "k_rot"));
+        LQ_TRY(check_ptr(k_pre, "k_pre"));
+        LQ_TRY(check_ptr(v, "v"));
+    }
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(LOOPVQ_ERR_INVALID_ARG, "lse not 4-byte aligned");
     if (layer < 0 || layer >= cc->L) return fail(LOOPVQ_ERR_INVALID_ARG, "layer=%d out of [0, %d)", layer, cc->L);
     if (t < 0 || t >= cc->T) return fail(LOOPVQ_ERR_INVALID_ARG, "t=%d out of [0, %d)", t, cc->T);
@@ -429,9 +435,28 @@ loopvq_status loopvq_window_decode_attn(const loopvq_window *w, const loopvq_cac
                     workspace ? ws_bytes : (size_t)0);
     if (!aligned16(workspace)) return fail(LOOPVQ_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
     cudaError_t e = loopvq::launch_window_decode(*w, *cc, layer, t, q, max_coded, scale, out, lse, workspace,
-                                                 (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "loopvq_window_decode_attn");
+                                                 (cudaStream_t)stream, k_rot, k_pre, v);
+    if (e != cudaSuccess) return cuda_fail(e, name);
     return LOOPVQ_OK;
+}
+
+loopvq_status loopvq_window_decode_attn(const loopvq_window *w, const loopvq_cache *cc, int layer, int t,
+                                        const uint16_t *q, int max_coded, float scale, float *out, float *lse,
+                                        void *workspace, size_t ws_bytes, void *stream) {
+    return window_decode("loopvq_window_decode_attn", w, cc, layer, t, nullptr, nullptr, nullptr, q, max_coded, scale,
+                         out, lse, workspace, ws_bytes, stream);
+}
+
+loopvq_status loopvq_window_append_decode_attn(const loopvq_window *w, const loopvq_cache *cc, int layer, int t,
+                                               const uint16_t *k_rot, const uint16_t *k_pre, const uint16_t *v,
+                                               const uint16_t *q, int max_coded, float scale, float *out, float *lse,
+                                               void *workspace, size_t ws_bytes, void *stream) {
+    if (!k_rot || !k_pre || !v) {
+        g_err[0] = 0;
+        return fail(LOOPVQ_ERR_INVALID_ARG, "k_rot, k_pre and v are required");
+    }
+    return window_decode("loopvq_window_append_decode_attn", w, cc, layer, t, k_rot, k_pre, v, q, max_coded, scale,
+                         out, lse, workspace, ws_bytes, stream);
 }
 
 loopvq_status loopvq_dequant_debug(const loopvq_cache *cc, int layer, int t, int kv, int b, int tok0, int ntok,

@@ -7,6 +7,7 @@
 #include <math.h>
 
 #include "decode_kernel.cuh"
+#include "decode_merge.cuh"
 #include "decode_gqa.cuh"
 #include "decode_mha.cuh"
 
@@ -198,7 +199,7 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
                           const uint16_t *q, const int32_t *starts, int start_all, const int32_t *lens, int max_len,
                           float scale, float *out, float *lse, void *workspace, cudaStream_t s,
                           const loopvq_tasq *tq, const uint16_t *wk, const uint16_t *wv, const int32_t *wfill,
-                          int W) {
+                          int W, const WindowAppend *app) {
     DecodeArgs a{};
     const int beta = t / cc.Tc;
     a.idx = cc.idx + idx_base(cc, layer, beta, 0, 0);
@@ -226,6 +227,14 @@ cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int la
     a.wv = wv;
     a.wfill = wfill;
     a.W = W;
+    if (app != nullptr) {
+        a.nk = app->k_rot;
+        a.nkp = app->k_pre;
+        a.nv = app->v;
+        a.wk_w = app->w_k_rot;
+        a.wkp_w = app->w_k_pre;
+        a.wv_w = app->w_v;
+    }
     const int qpk = cc.Hq / cc.Hkv;
     if (tq) {
         const int NB = cc.T / cc.Tc;

@@ -76,11 +76,18 @@ struct DecodePlan {
     size_t ws_bytes;    // workspace needed
 };
 DecodePlan plan_decode(const loopvq_cache &cc, int max_len, bool tasq = false);
+// A window token appended by the windowed decode's merge kernel: its rows [B][Hkv][D] and the window
+// arrays of (layer, t) it is written to.
+struct WindowAppend {
+    const uint16_t *k_rot, *k_pre, *v;
+    uint16_t *w_k_rot, *w_k_pre, *w_v;
+};
 cudaError_t launch_decode(const loopvq_cache &cc, const DecodePlan &plan, int layer, int t,
                           const uint16_t *q, const int32_t *starts, int start_all, const int32_t *lens, int max_len,
                           float scale, float *out, float *lse, void *workspace, cudaStream_t s,
                           const loopvq_tasq *tq = nullptr, const uint16_t *wk = nullptr,
-                          const uint16_t *wv = nullptr, const int32_t *wfill = nullptr, int W = 0);
+                          const uint16_t *wv = nullptr, const int32_t *wfill = nullptr, int W = 0,
+                          const WindowAppend *app = nullptr);
 cudaError_t launch_tasq_encode(const loopvq_cache &cc, const loopvq_tasq &tq, int layer, int block, const void *xk,
                                const void *xv, int x_dtype, const int64_t *strides, int b0, int nb, int tok0, int ntok,
                                cudaStream_t s);
@@ -99,6 +106,8 @@ cudaError_t launch_window_append(const loopvq_window &w, int layer, int t, const
                                  const uint16_t *k_pre, const uint16_t *v, cudaStream_t s);
 size_t window_ws_bytes(const loopvq_window &w, const loopvq_cache &cc, int max_coded);
 cudaError_t launch_window_decode(const loopvq_window &w, const loopvq_cache &cc, int layer, int t, const uint16_t *q,
-                                 int max_coded, float scale, float *out, float *lse, void *ws, cudaStream_t s);
+                                 int max_coded, float scale, float *out, float *lse, void *ws, cudaStream_t s,
+                                 const uint16_t *k_rot = nullptr, const uint16_t *k_pre = nullptr,
+                                 const uint16_t *v = nullptr);
 
 }  // namespace loopvq

@@ -215,14 +215,18 @@ size_t window_ws_bytes(const loopvq_window &w, const loopvq_cache &cc, int max_c
 }
 
 // The coded kernel over tokens [n_sink, coded_end_b); its merge kernel attends to the window slots
-// [0, fill_b) of (layer, t) itself and folds them into the log-sum-exp merge (decode_kernel.cuh).
+// [0, fill_b) of (layer, t) itself and folds them into the log-sum-exp merge (decode_kernel.cuh).  With
+// k_rot, k_pre, v given, slot fill_b - 1 is the token they hold, which the merge kernel also writes into
+// the window (the work of launch_window_append, without its launch).
 cudaError_t launch_window_decode(const loopvq_window &w, const loopvq_cache &cc, int layer, int t, const uint16_t *q,
-                                 int max_coded, float scale, float *out, float *lse, void *ws, cudaStream_t s) {
+                                 int max_coded, float scale, float *out, float *lse, void *ws, cudaStream_t s,
+                                 const uint16_t *k_rot, const uint16_t *k_pre, const uint16_t *v) {
     const int W = window_slots(w);
     const size_t off = ((size_t)layer * w.T + t) * w.B * w.Hkv * W * w.D;
     const DecodePlan pc = plan_decode(cc, max_coded);
+    const WindowAppend app{k_rot, k_pre, v, w.k_rot + off, w.k_pre + off, w.v + off};
     return launch_decode(cc, pc, layer, t, q, nullptr, w.n_sink, w.coded_end, max_coded, scale, out, lse, ws, s,
-                         nullptr, w.k_rot + off, w.v + off, w.fill, W);
+                         nullptr, w.k_rot + off, w.v + off, w.fill, W, k_rot != nullptr ? &app : nullptr);
 }
 
 }  // namespace loopvq

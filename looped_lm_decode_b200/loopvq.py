@@ -25,7 +25,8 @@ EXPORTS = ("loopvq_idx_words", "loopvq_codebook_elems", "loopvq_slice_elems", "l
            "loopvq_decode_attn_noalloc", "loopvq_noalloc_scratch_bytes", "loopvq_decode_attn_range",
            "loopvq_bf16_decode_workspace_bytes", "loopvq_bf16_decode_attn", "loopvq_merge2",
            "loopvq_window_slots", "loopvq_window_advance", "loopvq_window_append",
-           "loopvq_window_workspace_bytes", "loopvq_window_decode_attn", "loopvq_tasq_w_elems",
+           "loopvq_window_workspace_bytes", "loopvq_window_decode_attn", "loopvq_window_append_decode_attn",
+           "loopvq_tasq_w_elems",
            "loopvq_tasq_perm_elems", "loopvq_tasq_sigma_elems", "loopvq_tasq_encode", "loopvq_tasq_decode_attn",
            "loopvq_fault_check", "loopvq_set_wait_limit_ns", "loopvq_wait_limit_ns")
 
@@ -106,6 +107,8 @@ def lib():
         L.loopvq_window_workspace_bytes.restype = sz
         L.loopvq_window_decode_attn.argtypes = [PW, P, i, i, vp, i, f, vp, vp, vp, sz, vp]
         L.loopvq_window_decode_attn.restype = i
+        L.loopvq_window_append_decode_attn.argtypes = [PW, P, i, i, vp, vp, vp, vp, i, f, vp, vp, vp, sz, vp]
+        L.loopvq_window_append_decode_attn.restype = i
         PT = C.POINTER(TasqDesc)
         for name in ("loopvq_tasq_w_elems", "loopvq_tasq_perm_elems", "loopvq_tasq_sigma_elems"):
             getattr(L, name).argtypes = [P]
@@ -419,6 +422,25 @@ def window_decode_attn(win: Window, cache: Cache, layer: int, t: int, q, max_cod
     _check(lib().loopvq_window_decode_attn(win.ref(), cache.ref(), layer, t, _ptr(q), max_coded, scale, _ptr(out),
                                            _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                            _stream(stream)))
+    return out, lse
+
+
+def window_append_decode_attn(win: Window, cache: Cache, layer: int, t: int, k_rot, k_pre, v, q, max_coded: int,
+                              scale: float = 0.0, out=None, lse=None, workspace=None, stream=None):
+    """window_append then window_decode_attn, in the decode call's launches (the merge kernel writes the
+    token k_rot, k_pre, v, bf16 [B][Hkv][D], into slot fill - 1 and attends to it)."""
+    B, Hq, D = cache.B, cache.Hq, cache.D
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(window_workspace_bytes(win, cache, max_coded), 16), dtype=torch.uint8,
+                                device=dev)
+    _check(lib().loopvq_window_append_decode_attn(win.ref(), cache.ref(), layer, t, _ptr(k_rot), _ptr(k_pre), _ptr(v),
+                                                  _ptr(q), max_coded, scale, _ptr(out), _ptr(lse), _ptr(workspace),
+                                                  workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
 
 

@@ -168,6 +168,14 @@ def test_window_validation_before_launch():
                                          None) == 1
     assert lib.loopvq_window_append(C.byref(w), 2, 0, fake, fake, fake, None) == 1
     assert lib.loopvq_window_append(C.byref(w), 0, 0, fake, C.c_void_p(0x20008), fake, None) == 1
+    # the fused call: a missing or misaligned token, a short workspace, a bad layer, all before any launch
+    fused = lib.loopvq_window_append_decode_attn
+    assert fused(C.byref(w), c.ref(), 0, 0, fake, None, fake, fake, 1024, 0.0, fake, None, fake, need, None) == 1
+    assert b"required" in lib.loopvq_last_error()
+    assert fused(C.byref(w), c.ref(), 0, 0, fake, C.c_void_p(0x20008), fake, fake, 1024, 0.0, fake, None, fake, need,
+                 None) == 1
+    assert fused(C.byref(w), c.ref(), 0, 0, fake, fake, fake, fake, 1024, 0.0, fake, None, fake, need - 1, None) == 3
+    assert fused(C.byref(w), c.ref(), c.L, 0, fake, fake, fake, fake, 1024, 0.0, fake, None, fake, need, None) == 1
     w.n_recent = 60                                          # not a multiple of 8
     assert lib.loopvq_window_slots(C.byref(w)) == 0
     assert lib.loopvq_window_advance(C.byref(w), c.ref(), None) == 1

@@ -253,11 +253,14 @@ def _raw(w, n):
     return k, kr, v                                                   # [L][T][B][n][Hkv][D] bits
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["append-then-attend", "fused"])
 @pytest.mark.parametrize("name", list(LIFE))
-def test_window_life_cycle(name):
+def test_window_life_cycle(name, fused):
     """Prefill, then decode steps that roll the window twice: every attention call equals one softmax
     over the bf16 window tokens and the coded tokens, and every rolled page's codes equal the checker's
-    encode of the original pre-RoPE keys and values."""
+    encode of the original pre-RoPE keys and values.  "fused": the checked (layer, t) take their token
+    through loopvq_window_append_decode_attn, so later calls, and the page rolls, read what its merge
+    kernel wrote into the window."""
     w = LIFE[name]
     n_s, n_r = 8, 16
     P0, steps = 40, 20                                                # prefill length, decode steps
@@ -290,11 +293,17 @@ def test_window_life_cycle(name):
         LQ.window_advance(win, cache)
         for layer in range(w.L):
             for t in range(w.T):
-                LQ.window_append(win, layer, t, _dev_bits(kr[layer, t, :, n]), _dev_bits(kp[layer, t, :, n]),
-                                 _dev_bits(vv[layer, t, :, n]))
+                if not (fused and (layer, t) in checks):
+                    LQ.window_append(win, layer, t, _dev_bits(kr[layer, t, :, n]), _dev_bits(kp[layer, t, :, n]),
+                                     _dev_bits(vv[layer, t, :, n]))
         for layer, t in checks:
             qb = queries(w, layer, t, gain=1.0 + 0.25 * step)
-            out, lse = LQ.window_decode_attn(win, cache, layer, t, _dev_bits(qb), w.Nmax)
+            if fused:
+                out, lse = LQ.window_append_decode_attn(win, cache, layer, t, _dev_bits(kr[layer, t, :, n]),
+                                                        _dev_bits(kp[layer, t, :, n]), _dev_bits(vv[layer, t, :, n]),
+                                                        _dev_bits(qb), w.Nmax)
+            else:
+                out, lse = LQ.window_decode_attn(win, cache, layer, t, _dev_bits(qb), w.Nmax)
             torch.cuda.synchronize()
             blk, m = t // w.Tc, t % w.Tc
             qpk = w.Hq // w.Hkv
@@ -332,3 +341,40 @@ def test_window_life_cycle(name):
                                   np_codebook_f32(w, layer, blk, 1, h), w.c)
                     np.testing.assert_array_equal(ck[n_s:coded_end], rk)
                     np.testing.assert_array_equal(cv[n_s:coded_end], rv)
+
+
+@pytest.mark.parametrize("name", list(LIFE))
+def test_fused_append_equals_append_then_attend(name):
+    """From the same window state, loopvq_window_append_decode_attn gives bit for bit the outputs of
+    loopvq_window_append followed by loopvq_window_decode_attn, and leaves the same window."""
+    w = LIFE[name]
+    cache = make_cache(w)
+    for layer in range(w.L):
+        for blk in range(w.NB):
+            for b in range(w.B):
+                for h in range(w.Hkv):
+                    ik = random_indices(w, layer, blk, 0, b, h, range(w.Nmax))
+                    iv = random_indices(w, layer, blk, 1, b, h, range(w.Nmax))
+                    words_view(cache, layer, blk, b, h).copy_(torch.from_numpy(pack_words(ik, iv, cache.NP).view(np.int32)))
+    win = LQ.Window(cache, n_sink=8, n_recent=16)
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    for buf in (win.k_rot, win.k_pre, win.v):
+        buf.copy_(torch.randn(buf.shape, generator=gen, device="cuda").to(torch.bfloat16))
+    win.fill.copy_(torch.tensor([win.W - 5, 9, win.W][:w.B], dtype=torch.int32))
+    win.coded_end.copy_(torch.tensor([60, 32, 100][:w.B], dtype=torch.int32))
+    new = [torch.randn((w.B, w.Hkv, w.D), generator=gen, device="cuda").to(torch.bfloat16) for _ in range(3)]
+    saved = [x.clone() for x in (win.k_rot, win.k_pre, win.v)]
+    for layer, t in ((0, 0), (w.L - 1, w.T - 1)):
+        q = _dev_bits(queries(w, layer, t))
+        for x, y in zip((win.k_rot, win.k_pre, win.v), saved):
+            x.copy_(y)
+        LQ.window_append(win, layer, t, *new)
+        o1, l1 = LQ.window_decode_attn(win, cache, layer, t, q, w.Nmax)
+        after = [x.clone() for x in (win.k_rot, win.k_pre, win.v)]
+        for x, y in zip((win.k_rot, win.k_pre, win.v), saved):
+            x.copy_(y)
+        o2, l2 = LQ.window_append_decode_attn(win, cache, layer, t, *new, q, w.Nmax)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), (layer, t)
+        for x, y in zip((win.k_rot, win.k_pre, win.v), after):
+            assert torch.equal(x, y), (layer, t)
