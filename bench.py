@@ -114,7 +114,7 @@ def kernel_sources_hash(kern):
     csrc = os.path.join(ROOT, "looped_lm_decode_b200", "csrc")
     h = hashlib.sha256()
     heads = {"decode_mha": ("decode_mha.cuh", "decode_kernel.cuh"),
-             "decode_gqa": ("decode_gqa.cuh", "decode_kernel.cuh")}.get(kern, ("decode_kernel.cuh",))
+             "decode_gqa": ("decode_gqa.cuh", "decode_kernel.cuh")}.get(kern, ("decode_split.cuh", "decode_kernel.cuh"))
     for src in heads:
         with open(os.path.join(csrc, src), "rb") as f:
             h.update(_code_only(f.read()))

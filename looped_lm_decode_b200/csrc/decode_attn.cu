@@ -1,5 +1,6 @@
 // Decode attention over the loop-axis coded cache, one loop step of one layer:
-// launch planning and dispatch.  The kernels are in decode_kernel.cuh.
+// launch planning and dispatch.  The kernels are in decode_split.cuh, decode_mha.cuh, decode_gqa.cuh and
+// decode_merge.cuh, on the shared tile space of decode_kernel.cuh.
 //
 // LoopVQ paper, Sec. 4.3 "Attention": the quantized tokens are divided into
 // splits processed by separate thread blocks, and the partial outputs of all
@@ -8,6 +9,7 @@
 
 #include "decode_kernel.cuh"
 #include "decode_merge.cuh"
+#include "decode_split.cuh"
 #include "decode_gqa.cuh"
 #include "decode_mha.cuh"
 

@@ -9,7 +9,7 @@
 //
 // Design (B200, sm_100a):
 //  * The tile space, pieces, partial records and merge are those of decode_split_kernel
-//    (decode_kernel.cuh).  The slices are staged as bank-private replicas: the K entry converted to
+//    (decode_kernel.cuh, decode_merge.cuh).  The slices are staged as bank-private replicas: the K entry converted to
 //    fp32 (32 bytes) with its two halves in 8 replicas each (row r of [0, 64 KiB): first halves at
 //    [0, 128), second at [128, 256); a lane reads replica lane % 8), the V entry in bf16 (16 bytes) in 16
 //    replicas (row r of [64 KiB, 128 KiB); replica lane % 16), so the 8 lanes of each quarter-warp

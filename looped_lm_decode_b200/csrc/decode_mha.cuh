@@ -8,7 +8,7 @@
 //
 // Design (B200, sm_100a):
 //  * The tile space, pieces and partial records are those of decode_split_kernel (decode_kernel.cuh),
-//    and its merge kernel combines the records.  The slices are staged as bank-private replicas: row r
+//    and the merge kernel (decode_merge.cuh) combines the records.  The slices are staged as bank-private replicas: row r
 //    holds K entry r as 8 bytes of bf16 in 16 replicas and V entry r likewise (a lane reads replica
 //    lane % 16, so the 16 lanes of a half-warp wavefront hit distinct banks).  Each gathered key entry is
 //    widened to fp32 by one m16n8k8 tensor-core product with the identity (lane-local, exact), so the

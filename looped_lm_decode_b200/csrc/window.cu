@@ -215,7 +215,7 @@ size_t window_ws_bytes(const loopvq_window &w, const loopvq_cache &cc, int max_c
 }
 
 // The coded kernel over tokens [n_sink, coded_end_b); its merge kernel attends to the window slots
-// [0, fill_b) of (layer, t) itself and folds them into the log-sum-exp merge (decode_kernel.cuh).  With
+// [0, fill_b) of (layer, t) itself and folds them into the log-sum-exp merge (decode_merge.cuh).  With
 // k_rot, k_pre, v given, slot fill_b - 1 is the token they hold, which the merge kernel also writes into
 // the window (the work of launch_window_append, without its launch).
 cudaError_t launch_window_decode(const loopvq_window &w, const loopvq_cache &cc, int layer, int t, const uint16_t *q,
