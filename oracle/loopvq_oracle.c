@@ -94,7 +94,7 @@ void ora_encode(const float *x, int Tc, int N, int D, int c, const float *E, int
     }
 }
 
-/* fp64 squared distance between coupled vector (n, g) and entry r; used to judge near-ties. */
+/* fp64 squared distance between coupled vector (n, g) and entry r; used to classify near-ties. */
 double ora_dist64(const float *x, int Tc, int N, int D, int c, const float *E, int n, int g, int r)
 {
     const int G = c * Tc;

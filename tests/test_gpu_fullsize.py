@@ -9,8 +9,8 @@ Bulk inputs come from the CUDA generator; the checker regenerates the inputs of
 each row on the CPU from the same counters.  The checker's calls run on host
 threads (its ctypes calls release the GIL).  Encode checks cover every token of two
 (sequence, KV head) pairs of the deep32 and ctx32k launches; the near-ties found
-(codes that differ with fp64 distances within 1e-5 relative) are written to
-gpurun_out/near_ties.json when that folder exists, and printed.
+(codes that differ with fp64 distances within 1e-5 relative) are printed, and written to
+near_ties.json in the directory LOOPVQ_RECORD_DIR names, when it is set.
 """
 import json
 import math
@@ -29,15 +29,14 @@ from tests.helpers import unpack_words, words_view, np_codebook_f32, attn_tolera
 
 pytestmark = pytest.mark.gpu
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 THREADS = max(1, len(os.sched_getaffinity(0)))
 SAMPLES = {"ctx32k": [(0, 0), (3, 7), (7, 15)], "ctx4k": [(0, 0), (31, 15)], "gqa16k": [(0, 0), (63, 13)],
            "deep32": [(1, 39), (0, 17)], "ctx32k_cq": [(0, 0), (6, 11)], "ctx32k_pg": [(2, 3), (7, 15)]}
 
 
 def _record_ties(key, value):
-    out = os.path.join(ROOT, "gpurun_out")
-    if not os.path.isdir(out):
+    out = os.environ.get("LOOPVQ_RECORD_DIR", "")
+    if not out or not os.path.isdir(out):
         return
     path = os.path.join(out, "near_ties.json")
     data = {}

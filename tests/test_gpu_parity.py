@@ -4,7 +4,7 @@ Bars: codes bit-exact (a mismatch is allowed only as a near-tie whose two fp64
 distances differ by < 1e-5 relative, and is counted); reconstruction bit-exact;
 attention max|out - ref| <= 2e-3 * ||ref||_inf per call tensor and
 |lse - lse_ref| <= 1e-3.  Inputs are seeded synthetic data from synth/; the
-checker never sees anything the GPU produced except the outputs it judges.
+checker never sees anything the GPU produced except the outputs it is compared with.
 """
 import math
 
